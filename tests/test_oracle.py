@@ -1,0 +1,321 @@
+"""Pins for the CPU oracle: each test ties it to something other than itself.
+
+Pins: the page-1 density table (golden), closed forms of the block counts,
+brute-force loops on tiny shapes, torch's CPU SDPA in fp64 (a different
+library routine), closed-form outputs (one visible key, all-equal scores,
+a two-key softcap case), the tiled recurrence, and degenerate cases.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import attention as OA
+from oracle import blockmask as OB
+from oracle import bruteforce as BF
+from oracle import masks as OM
+from oracle import online as OO
+
+
+def _rand(shape, seed, scale=1.0):
+    g = np.random.default_rng(seed)
+    return g.standard_normal(shape) * scale
+
+
+# ---------------------------------------------------------------- block tables
+
+def test_page1_density_table(golden):
+    """Token and block densities printed on page 1 (results table)."""
+    for pattern, seq, window, tok_pct, blk_pct in golden("page1_density_table.txt"):
+        L = int(seq)
+        if pattern == "causal":
+            tok, blk = OB.densities(OM.CAUSAL, L, L)
+        else:
+            tok, blk = OB.densities(OM.SLIDING_WINDOW_CAUSAL, L, L, window=int(window))
+        assert f"{100 * tok:.2f}" == tok_pct, (pattern, seq, window, tok)
+        assert f"{100 * blk:.2f}" == blk_pct, (pattern, seq, window, blk)
+
+
+@pytest.mark.parametrize("nq", [1, 2, 5, 64])
+def test_causal_block_counts_closed_form(nq):
+    """L = S = 128 nq: nq(nq+1)/2 live blocks; the diagonal ones are the partial ones."""
+    t = OB.block_tables(OM.CAUSAL, 128 * nq, 128 * nq)
+    assert int(t["kv_num_blocks"].sum()) == nq
+    assert int(t["full_kv_num_blocks"].sum()) == nq * (nq - 1) // 2
+    for i in range(nq):
+        assert t["kv_num_blocks"][i] == 1 and t["kv_indices"][i, 0] == i
+        assert list(t["full_kv_indices"][i, :i]) == list(range(i))
+
+
+@pytest.mark.parametrize("nq,w", [(64, 256), (64, 1024), (40, 128), (64, 64), (30, 100)])
+def test_window_block_counts_closed_form(nq, w):
+    """Row i covers keys (q - W, q]; for W a multiple of 128 that is W/128 full blocks
+    below the diagonal block, the oldest of them cut by the window (partial);
+    for W < 128 the diagonal block and the one before it, both partial."""
+    t = OB.block_tables(OM.SLIDING_WINDOW_CAUSAL, 128 * nq, 128 * nq, window=w)
+    for i in range(nq):
+        if w % 128 == 0:
+            nb = w // 128
+            exp_partial = [j for j in (i - nb, i) if j >= 0]
+            exp_full = list(range(max(0, i - nb + 1), i))
+        elif w < 128:
+            exp_partial = [j for j in (i - 1, i) if j >= 0]
+            exp_full = []
+        else:  # 128 < W < 256, not a multiple: keys back to q - W + 1 reach block i - 2
+            exp_partial = [j for j in (i - 2, i - 1, i) if j >= 0]
+            exp_full = []
+        got_p = list(t["kv_indices"][i, : t["kv_num_blocks"][i]])
+        got_f = list(t["full_kv_indices"][i, : t["full_kv_num_blocks"][i]])
+        assert got_p == exp_partial, (i, got_p, exp_partial)
+        assert got_f == exp_full, (i, got_f, exp_full)
+
+
+def test_window_32k_total_live_blocks():
+    """3 live blocks per row except the first two rows: 3 * 256 - 3 = 765 of 65536."""
+    t = OB.block_tables(OM.SLIDING_WINDOW_CAUSAL, 32768, 32768, window=256)
+    live = t["kv_num_blocks"].sum() + t["full_kv_num_blocks"].sum()
+    assert live == 3 * 256 - 3
+    assert t["full_kv_num_blocks"].sum() == 255
+
+
+def test_block_tables_unused_entries_are_zero():
+    t = OB.block_tables(OM.SLIDING_WINDOW_CAUSAL, 1000, 1000, window=200)
+    for i in range(t["n_q_blocks"]):
+        assert not t["kv_indices"][i, t["kv_num_blocks"][i]:].any()
+        assert not t["full_kv_indices"][i, t["full_kv_num_blocks"][i]:].any()
+
+
+@pytest.mark.parametrize("kind,L,S,w", [
+    (OM.CAUSAL, 300, 300, None), (OM.CAUSAL, 130, 260, None), (OM.CAUSAL, 260, 129, None),
+    (OM.SLIDING_WINDOW_CAUSAL, 385, 385, 70), (OM.SLIDING_WINDOW_CAUSAL, 256, 200, 150),
+    (OM.DOCUMENT_CAUSAL, 384, 384, None), (OM.CAUSAL, 1, 1, None), (OM.CAUSAL, 5, 0, None)])
+def test_block_classification_bruteforce(kind, L, S, w):
+    """Vectorised classification equals a per-pair loop, including ragged tails."""
+    doc = None
+    if kind == OM.DOCUMENT_CAUSAL:
+        rng = np.random.default_rng(5)
+        doc = rng.integers(0, 3, size=max(L, S))   # unsorted ids on purpose
+    live, full, _ = OB.classify(kind, L, S, w, doc)
+    for i in range(live.shape[0]):
+        for j in range(live.shape[1]):
+            c = BF.classify_block(kind, i, j, L, S, w, doc)
+            assert (c != "empty") == live[i, j], (i, j, c)
+            assert (c == "full") == full[i, j], (i, j, c)
+
+
+# ---------------------------------------------------------------- attention
+
+def _oracle(q, k, v, kind, **kw):
+    return OA.attention_head(q, k, v, kind, **kw)
+
+
+@pytest.mark.parametrize("L,S,D", [(1, 1, 64), (7, 7, 64), (128, 128, 64), (129, 129, 64),
+                                   (200, 256, 64), (256, 200, 64), (33, 40, 128)])
+@pytest.mark.parametrize("kind", [OM.CAUSAL, OM.SLIDING_WINDOW_CAUSAL, OM.DOCUMENT_CAUSAL])
+def test_attention_bruteforce_tiny(L, S, D, kind):
+    """Vectorised fp64 oracle equals pure-Python loops (scores, mask, softmax, LSE)."""
+    if L * S * D > 256 * 200 * 64 // 2 and kind != OM.CAUSAL:
+        pytest.skip("keep the pure-Python loops short")
+    q, k, v = _rand((L, D), 1), _rand((S, D), 2), _rand((S, D), 3)
+    w = 37 if kind == OM.SLIDING_WINDOW_CAUSAL else None
+    doc = None
+    if kind == OM.DOCUMENT_CAUSAL:
+        doc = np.sort(np.random.default_rng(4).integers(0, 4, size=max(L, S)))
+    sk = 1 if L % 2 else 0
+    out, lse = _oracle(q, k, v, kind, window=w, doc_id=doc, score_kind=sk, softcap=3.0)
+    bo, bl = BF.attention_head(q.tolist(), k.tolist(), v.tolist(), kind, w,
+                               None if doc is None else doc.tolist(), sk, 3.0)
+    np.testing.assert_allclose(out, np.array(bo).reshape(out.shape), rtol=0, atol=1e-12)
+    bl = np.array(bl)
+    assert np.array_equal(np.isinf(lse), np.isinf(bl))
+    fin = np.isfinite(bl)
+    np.testing.assert_allclose(lse[fin], bl[fin], rtol=0, atol=1e-12)
+
+
+def test_rows_of_p_sum_to_one():
+    """With V = 1 every live row's output is sum_j P_ij = 1 (up to the rounding
+    of a sum of at most 300 fp64 terms, 300 * 2**-53 < 4e-14)."""
+    L = 300
+    q, k = _rand((L, 64), 10), _rand((L, 64), 11)
+    v = np.ones((L, 64))
+    for kind, w in ((OM.CAUSAL, None), (OM.SLIDING_WINDOW_CAUSAL, 50)):
+        out, _ = _oracle(q, k, v, kind, window=w)
+        assert np.abs(out - 1.0).max() <= 4e-14
+
+
+def test_single_visible_key_returns_its_value():
+    """Query 0 under every causal rule, and the first token of each document,
+    see exactly one key: the output is that key's V, bit for bit."""
+    L = 6000
+    q, k, v = _rand((L, 64), 20), _rand((L, 64), 21), _rand((L, 64), 22)
+    rows = np.array([0, 2048, 5000])
+    doc = W.doc_id_from_starts(L, [2048, 5000]).numpy()
+    out, lse = _oracle(q, k, v, OM.DOCUMENT_CAUSAL, doc_id=doc, rows=rows)
+    for r, o in zip(rows, out):
+        assert np.array_equal(o, v[r])
+    for kind, w in ((OM.CAUSAL, None), (OM.SLIDING_WINDOW_CAUSAL, 256)):
+        out, lse = _oracle(q, k, v, kind, window=w, rows=np.array([0]))
+        assert np.array_equal(out[0], v[0])
+        assert lse[0] == pytest.approx(float(q[0] @ k[0]) / 8.0, abs=1e-13)
+
+
+def test_equal_scores_closed_form():
+    """K = 0 makes every score 0: out is the mean of the visible V rows and
+    lse = ln(number of visible keys), for each mask rule."""
+    L = 700
+    q, v = _rand((L, 64), 30), _rand((L, 64), 31)
+    k = np.zeros((L, 64))
+    starts = [0, 100, 333, 600]
+    doc = W.doc_id_from_starts(L, starts[1:]).numpy()
+    csum = np.cumsum(v, axis=0)
+    for kind, w in ((OM.CAUSAL, None), (OM.SLIDING_WINDOW_CAUSAL, 64), (OM.DOCUMENT_CAUSAL, None)):
+        out, lse = _oracle(q, k, v, kind, window=w, doc_id=doc)
+        for i in range(L):
+            if kind == OM.CAUSAL:
+                lo = 0
+            elif kind == OM.SLIDING_WINDOW_CAUSAL:
+                lo = max(0, i - w + 1)
+            else:
+                lo = max(s for s in starts if s <= i)
+            n = i - lo + 1
+            mean = (csum[i] - (csum[lo - 1] if lo > 0 else 0)) / n
+            assert np.abs(out[i] - mean).max() <= 1e-13
+            assert abs(lse[i] - math.log(n)) <= 1e-13
+
+
+def test_softcap_two_key_closed_form():
+    """One key with scaled score 15 ln 3 (capped by c=30 to exactly 15, since
+    tanh(ln 3 / 2) = 1/2) and one key with score 0: the weights are
+    e^15 : 1.  Capping the unscaled score, dropping c, or skipping the cap
+    all give different weights."""
+    D = 64
+    scale = 1.0 / 8.0
+    x = 15.0 * math.log(3.0)
+    q = np.zeros((2, D)); q[1, 0] = 1.0
+    k = np.zeros((2, D)); k[0, 0] = x / scale
+    v = np.zeros((2, D)); v[0, 1] = 1.0; v[1, 2] = 1.0
+    out, lse = _oracle(q, k, v, OM.CAUSAL, score_kind=1, softcap=30.0)
+    w0 = math.exp(15.0) / (math.exp(15.0) + 1.0)
+    assert out[1, 1] == pytest.approx(w0, abs=1e-14)
+    assert out[1, 2] == pytest.approx(1.0 - w0, abs=1e-14)
+    assert lse[1] == pytest.approx(math.log(math.exp(15.0) + 1.0), abs=1e-12)
+
+
+def test_softcap_infinite_cap_is_identity():
+    L = 257
+    q, k, v = _rand((L, 64), 40, 2.0), _rand((L, 64), 41, 2.0), _rand((L, 64), 42)
+    a, la = _oracle(q, k, v, OM.CAUSAL)
+    b, lb = _oracle(q, k, v, OM.CAUSAL, score_kind=1, softcap=1e30)
+    assert np.abs(a - b).max() <= 1e-12 and np.abs(la - lb).max() <= 1e-12
+
+
+def test_special_case_reductions():
+    """W >= S turns the window rule into causal; one document is causal."""
+    L = 400
+    q, k, v = _rand((L, 64), 50), _rand((L, 64), 51), _rand((L, 64), 52)
+    c, lc = _oracle(q, k, v, OM.CAUSAL)
+    w, lw = _oracle(q, k, v, OM.SLIDING_WINDOW_CAUSAL, window=L)
+    d, ld = _oracle(q, k, v, OM.DOCUMENT_CAUSAL, doc_id=np.zeros(L, dtype=np.int64))
+    assert np.array_equal(c, w) and np.array_equal(lc, lw)
+    assert np.array_equal(c, d) and np.array_equal(lc, ld)
+    tc = OB.block_tables(OM.CAUSAL, L, L)
+    tw = OB.block_tables(OM.SLIDING_WINDOW_CAUSAL, L, L, window=10 ** 6)
+    for key in ("kv_num_blocks", "kv_indices", "full_kv_num_blocks", "full_kv_indices"):
+        assert np.array_equal(tc[key], tw[key])
+
+
+def test_fully_masked_rows_give_zero_and_minus_inf():
+    """Window rule with L > S + W - 1: rows q >= S + W - 1 see no key."""
+    L, S, w = 300, 100, 50
+    q, k, v = _rand((L, 64), 60), _rand((S, 64), 61), _rand((S, 64), 62)
+    out, lse = _oracle(q, k, v, OM.SLIDING_WINDOW_CAUSAL, window=w)
+    dead = np.arange(L) >= S + w - 1
+    assert np.all(out[dead] == 0.0) and np.all(np.isneginf(lse[dead]))
+    assert np.all(np.isfinite(lse[~dead]))
+    out0, lse0 = _oracle(q, k[:0], v[:0], OM.CAUSAL)
+    assert np.all(out0 == 0.0) and np.all(np.isneginf(lse0))
+
+
+@pytest.mark.parametrize("kind,w", [(OM.CAUSAL, None), (OM.SLIDING_WINDOW_CAUSAL, 100),
+                                    (OM.DOCUMENT_CAUSAL, None)])
+def test_matches_torch_sdpa_fp64(golden, kind, w):
+    """torch's CPU SDPA in float64 given the same boolean mask (True = use the
+    pair) agrees with the oracle to fp64 rounding; the SDPA tutorial's section 1
+    measured SDPA against a naive implementation at 7.22e-16 / 1.11e-15 (golden)."""
+    bound = max(float(r[2]) for r in golden("sdpa_fp64_equivalence.txt"))
+    g = torch.Generator().manual_seed(0)
+    q, k, v = (torch.randn(2, 8, 512, 64, generator=g, dtype=torch.float64) for _ in range(3))
+    L = 512
+    doc = np.sort(np.random.default_rng(1).integers(0, 5, size=L))
+    mask = torch.from_numpy(OM.mask_rows(kind, np.arange(L), L, w, doc))
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask)
+    worst = 0.0
+    for b in range(2):
+        for h in range(8):
+            o, _ = _oracle(q[b, h], k[b, h], v[b, h], kind, window=w, doc_id=doc)
+            worst = max(worst, float(np.abs(o - ref[b, h].numpy()).max()))
+    assert worst <= 10 * bound, worst
+
+
+def test_sdpa_fully_masked_row_is_zero():
+    """SDPA returns 0 (not NaN) for an all-False mask row (SDPA tutorial
+    section 4); the oracle's reading for such rows agrees."""
+    g = torch.Generator().manual_seed(3)
+    q, k, v = (torch.randn(1, 1, 4, 8, generator=g, dtype=torch.float64) for _ in range(3))
+    mask = torch.zeros(1, 1, 4, 4, dtype=torch.bool)
+    mask[..., 1:, 0] = True
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask)
+    assert torch.all(ref[0, 0, 0] == 0)
+    # oracle with window 1 and S shifted: row 0 of a window rule over keys 1.. sees nothing
+    out, lse = _oracle(q[0, 0].numpy(), k[0, 0, :0].numpy(), v[0, 0, :0].numpy(), OM.CAUSAL)
+    assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+# ---------------------------------------------------------------- tiled recurrence
+
+def test_tiled_softmax_matches_plain(golden):
+    """Running-max softmax over 4096 values vs plain softmax (page 3 table)."""
+    x = _rand((4096,), 70)     # N(0,1): softmax entries ~1/4096, as on the page
+    plain = np.exp(x - x.max()) / np.exp(x - x.max()).sum()
+    for tile, max_err, _ in golden("tiled_softmax_errors.txt"):
+        got = OO.softmax_tiled_1d(x, int(tile))
+        err = np.abs(got - plain).max()
+        assert err < 1e-9          # the page's acceptance threshold
+        assert err <= 100 * float(max_err) + 1e-17
+
+
+@pytest.mark.parametrize("kind,w,sk", [(OM.CAUSAL, None, 0), (OM.SLIDING_WINDOW_CAUSAL, 300, 1),
+                                       (OM.DOCUMENT_CAUSAL, None, 0)])
+def test_tiled_attention_matches_dense(kind, w, sk):
+    L = 1000
+    q, k, v = _rand((L, 64), 80), _rand((L, 64), 81), _rand((L, 64), 82)
+    doc = W.doc_id_from_starts(L, [200, 640]).numpy()
+    a, la = OA.attention_head(q, k, v, kind, window=w, doc_id=doc, score_kind=sk, softcap=5.0)
+    b, lb = OO.attention_head_tiled(q, k, v, kind, window=w, doc_id=doc, score_kind=sk, softcap=5.0)
+    assert np.abs(a - b).max() <= 1e-14
+    assert np.abs(la - lb).max() <= 1e-13
+
+
+def test_row_subset_equals_full():
+    L = 600
+    q, k, v = _rand((L, 64), 90), _rand((L, 64), 91), _rand((L, 64), 92)
+    full, lf = OA.attention_head(q, k, v, OM.CAUSAL)
+    rows = np.array([5, 599, 128, 0, 300])
+    sub, ls = OA.attention_head(q, k, v, OM.CAUSAL, rows=rows)
+    # BLAS may block a different row set differently: equal up to fp64 rounding
+    assert np.abs(full[rows] - sub).max() <= 1e-14 and np.abs(lf[rows] - ls).max() <= 1e-13
+
+
+def test_workload_generators_are_seeded():
+    a = W.make_qkv(W.C1_CAUSAL_256)
+    b = W.make_qkv(W.C1_CAUSAL_256)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y) and x.dtype == torch.bfloat16
+    d = W.make_doc_id(W.C4_DOC_SEEDED)
+    n_docs = int(d.max()) + 1
+    assert 4 <= n_docs <= 16 and d.shape == (8192,)
+    assert torch.all(d[1:] >= d[:-1])
+    f = W.make_doc_id(W.C4_DOC_FIXED)
+    assert int(f[2047]) == 0 and int(f[2048]) == 1 and int(f[4999]) == 1 and int(f[5000]) == 2
