@@ -1,0 +1,54 @@
+// Host-side entry points shared by both operations: status strings, device
+// queries and the device error word of the forward workspace.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "fa_internal.h"
+
+namespace fa {
+
+int num_sms_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  static std::mutex mu;
+  static int cache[kMaxDevices] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace fa
+
+extern "C" const char* fa_status_string(int32_t status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+extern "C" int32_t fa_num_sms(void) { return fa::num_sms_current_device(); }
+
+extern "C" fa_status fa_get_last_device_error(void* workspace, void* stream) {
+  if (workspace == nullptr) return FA_ERR_INVALID_ARG;
+  cudaStream_t s = fa::as_stream(stream);
+  FA_CUDA_CHECK(cudaStreamSynchronize(s));
+  int32_t word = 0;
+  FA_CUDA_CHECK(cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s));
+  FA_CUDA_CHECK(cudaStreamSynchronize(s));
+  if (word != 0) {
+    FA_CUDA_CHECK(cudaMemsetAsync(workspace, 0, sizeof(word), s));
+    FA_CUDA_CHECK(cudaStreamSynchronize(s));
+    if (word & fa::kDevErrTimeout) return FA_ERR_TIMEOUT;
+  }
+  return FA_OK;
+}

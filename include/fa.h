@@ -1,0 +1,188 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) block-sparse attention library (libfa.so).
+ *
+ * Two operations, following the FlexAttention how-to
+ * ("FlexAttention on Apple Silicon: block mask how-to", dreaming.press):
+ *
+ *   fa_create_block_mask  ~ create_block_mask(mask_mod, B=None, H=None, Q_LEN, KV_LEN)
+ *                           ("Mask 1: causal", "Mask 2: sliding-window causal",
+ *                            "Mask 3: document-packed"): classifies every 128x128 block of
+ *                           the (Q_LEN x KV_LEN) score grid as empty, full or partial and
+ *                           writes per-row block lists; one mask is broadcast over batch
+ *                           and heads.
+ *   fa_flex_attention_fwd ~ flex_attention(q, k, v, block_mask=, score_mod=)
+ *                           ("Setup", "Bonus: a score_mod for soft-capping"):
+ *                           out = softmax(Q K^T * scale + mask / score_mod) V computed tile by
+ *                           tile on the tensor cores with an online softmax; empty blocks are
+ *                           never touched.  The attention definition is the one of the SDPA
+ *                           tutorial (qiita GeneLab_999, section 1).
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are DEVICE pointers owned by the caller (for instance
+ *    torch tensors).  The library never allocates device memory.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Argument errors are detected on the host before any launch and
+ *    returned as a status; nothing is launched then.
+ *  - Layouts are C-contiguous.  Q is (B, H, L, D); K and V are (B, H, S, D); out
+ *    is (B, H, L, D) in the input dtype; lse is (B, H, L) float32.  D is 64 or 128.
+ *  - Mask semantics: "true" means the (q, kv) pair is used (the SDPA boolean-mask
+ *    convention, SDPA tutorial section 4).  Indices are absolute positions, so for
+ *    L != S the causal diagonal is upper-left aligned.  Positions past L or S are
+ *    never live.
+ *  - A query row with no live key returns out = 0 and lse = -inf (SDPA returns 0
+ *    for such rows, SDPA tutorial section 4).
+ *  - Device pointers passed to fa_flex_attention_fwd must be 16-byte aligned.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,  /* bad pointer, size, enum value or mismatched shapes */
+  FA_ERR_UNSUPPORTED = 2,  /* valid request outside what this build implements (e.g. D=96) */
+  FA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (no device, launch error ...) */
+  FA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (reported by
+                              fa_get_last_device_error) */
+} fa_status;
+
+typedef enum {
+  FA_MASK_CAUSAL = 0,                /* q_idx >= kv_idx                                   */
+  FA_MASK_SLIDING_WINDOW_CAUSAL = 1, /* q_idx >= kv_idx && q_idx - kv_idx < window        */
+  FA_MASK_DOCUMENT_CAUSAL = 2        /* q_idx >= kv_idx && doc_id[q_idx] == doc_id[kv_idx] */
+} fa_mask_kind;
+
+typedef enum {
+  FA_SCORE_NONE = 0,
+  FA_SCORE_TANH_SOFTCAP = 1          /* score -> softcap * tanh(score / softcap), on the scaled score */
+} fa_score_kind;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/* Block size of the mask tables; the only value this build accepts. */
+#define FA_BLOCK 128
+/* Largest Q_LEN / KV_LEN accepted (8192 blocks of 128). */
+#define FA_MAX_LEN (8192 * 128)
+
+/*
+ * Block tables of one mask, broadcast over batch and heads.
+ *
+ * The caller allocates the five arrays on the device and stores their pointers
+ * here BEFORE calling fa_create_block_mask, which fills both the arrays and the
+ * scalar fields.  Sizes: nQ = ceil(q_len / 128), nKV = ceil(kv_len / 128)
+ * (fa_block_mask_dims computes them).
+ *
+ *   kv_num_blocks[nQ]           number of PARTIAL blocks of q-block row i
+ *   kv_indices[nQ * nKV]        row i: its partial kv-block indices, ascending, then 0s
+ *   full_kv_num_blocks[nQ]      number of FULL blocks of row i
+ *   full_kv_indices[nQ * nKV]   row i: its full kv-block indices, ascending, then 0s
+ *   q_order[nQ]                 q-block rows sorted by descending live-block count
+ *                               (ties by ascending row): the order in which the forward
+ *                               kernel's persistent scheduler hands out work
+ *
+ * A FULL block has all 128 x 128 pairs in range and allowed (the kernel skips the
+ * mask there); a PARTIAL block has some but not all pairs live (the kernel evaluates
+ * the mask per element); EMPTY blocks appear in neither list and are never read.
+ * `doc_id` is kept (not copied): it must stay valid while the mask is used.
+ */
+typedef struct fa_block_mask {
+  int32_t* kv_num_blocks;
+  int32_t* kv_indices;
+  int32_t* full_kv_num_blocks;
+  int32_t* full_kv_indices;
+  int32_t* q_order;
+  int32_t q_len;
+  int32_t kv_len;
+  int32_t block;
+  int32_t n_q_blocks;
+  int32_t n_kv_blocks;
+  int32_t kind;           /* fa_mask_kind */
+  int32_t window;         /* sliding window W (kind 1), else 0 */
+  const int32_t* doc_id;  /* device int32[max(q_len, kv_len)] (kind 2), else NULL */
+} fa_block_mask;
+
+/* nQ and nKV of a (q_len, kv_len) mask with the given block size.
+ * Returns FA_ERR_INVALID_ARG for negative lengths, block != 128, lengths above
+ * FA_MAX_LEN or NULL outputs.  Host only, no CUDA call. */
+FA_API fa_status fa_block_mask_dims(int32_t q_len, int32_t kv_len, int32_t block,
+                             int32_t* n_q_blocks, int32_t* n_kv_blocks);
+
+/*
+ * Build the block tables of a mask rule (FlexAttention how-to, "Mask 1..3").
+ *   kind    fa_mask_kind.
+ *   window  W >= 1 for FA_MASK_SLIDING_WINDOW_CAUSAL (ignored otherwise).
+ *   doc_id  device int32 array of length max(q_len, kv_len) for
+ *           FA_MASK_DOCUMENT_CAUSAL (one id per position, indexed by both q_idx and
+ *           kv_idx as in the how-to's document_id tensor); ignored otherwise. Any
+ *           int32 values are allowed (they need not be sorted).
+ *   q_len, kv_len  >= 0 and <= FA_MAX_LEN;  block must be 128.
+ *   bm      in: the five device array pointers (non-NULL when nQ > 0);
+ *           out: every field filled.
+ * Launches two kernels on `stream`; the tables are ready when the stream reaches
+ * that point.  Returns FA_ERR_INVALID_ARG (nothing launched) on bad arguments,
+ * FA_ERR_CUDA if a launch fails.
+ */
+FA_API fa_status fa_create_block_mask(int32_t kind, int32_t window, const int32_t* doc_id,
+                               int32_t q_len, int32_t kv_len, int32_t block,
+                               fa_block_mask* bm, void* stream);
+
+/* Bytes of the device workspace fa_flex_attention_fwd needs (a small constant).
+ * The caller allocates it, ZEROES IT ONCE, and may then reuse it for every call on
+ * one stream; calls that run concurrently must use distinct workspaces. */
+FA_API size_t fa_fwd_workspace_bytes(void);
+
+/*
+ * Block-sparse attention forward.
+ *   q         device (B, H, L, D), dtype `dtype`.
+ *   k, v      device (B, H, S, D), dtype `dtype`.
+ *   dtype     FA_BF16 or FA_FP16 (Q, K, V and out share it; accumulation is fp32).
+ *   B, H, L, S, D   sizes; D in {64, 128}; L == bm->q_len and S == bm->kv_len.
+ *             B*H == 0 or L == 0 is a no-op returning FA_OK.
+ *   bm        tables from fa_create_block_mask (device arrays stay owned by the caller).
+ *   score_kind, softcap   FA_SCORE_NONE, or FA_SCORE_TANH_SOFTCAP with softcap > 0.
+ *   scale     multiplier of Q K^T; <= 0 selects 1/sqrt(D).
+ *   out       device (B, H, L, D), dtype `dtype`.
+ *   lse       device (B, H, L) float32: natural-log softmax denominator
+ *             m + ln(sum exp(s - m)); may be NULL.
+ *   workspace device buffer of fa_fwd_workspace_bytes() bytes (see there).
+ * The kernel is persistent (one CTA per SM) and processes (batch*head, q-block) work
+ * units in the order of bm->q_order.  Returns FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED
+ * (nothing launched) or FA_ERR_CUDA.  Device-side timeouts are reported by
+ * fa_get_last_device_error.
+ */
+FA_API fa_status fa_flex_attention_fwd(const void* q, const void* k, const void* v, int32_t dtype,
+                                int32_t B, int32_t H, int32_t L, int32_t S, int32_t D,
+                                const fa_block_mask* bm, int32_t score_kind, float softcap,
+                                float scale, void* out, float* lse, void* workspace,
+                                void* stream);
+
+/* Synchronises `stream`, then reads and clears the error word that the forward
+ * kernel keeps in `workspace`.  Returns FA_ERR_TIMEOUT if a bounded device wait gave
+ * up since the last query (the outputs of that call are then invalid), FA_ERR_CUDA
+ * if the stream reports an error, FA_OK otherwise. */
+FA_API fa_status fa_get_last_device_error(void* workspace, void* stream);
+
+/* Static, human-readable name of a status code. */
+FA_API const char* fa_status_string(int32_t status);
+
+/* Number of SMs the forward kernel's persistent grid uses on the current device
+ * (0 if no device).  Informational. */
+FA_API int32_t fa_num_sms(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* FA_H_ */

@@ -1,0 +1,83 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the binding
+(C-ABI) and compare with the CPU fp64 oracle on the same seeded inputs.
+
+Tolerances (floating point, against the fp64 oracle, bf16/fp16 inputs with
+fp32 accumulation): max |out err| <= 2e-2, mean |out err| <= 2e-3,
+max |lse err| <= 1e-3 (absolute, natural log).  Integer tables are bit-exact.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import workloads as W
+from oracle import attention as OA
+
+MAX_ERR = 2e-2
+MEAN_ERR = 2e-3
+LSE_ERR = 1e-3
+
+
+def run_gpu(q, k, v, kind, window=0, doc_id=None, score_kind=0, softcap=0.0, scale=0.0):
+    """q, k, v CPU tensors -> (out, lse) CPU tensors from the CUDA path."""
+    import block_sparse_attention_create_b200 as fa
+    dev = "cuda"
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    dd = doc_id.to(dev) if doc_id is not None else None
+    bm = fa.create_block_mask(kind, q.shape[2], k.shape[2], window=window, doc_id=dd, device=dev)
+    out, lse = fa.flex_attention(qd, kd, vd, bm, score_mod=score_kind, softcap=softcap,
+                                 scale=scale, return_lse=True)
+    torch.cuda.synchronize()
+    assert fa.last_device_error() == fa.FA_OK
+    return out.cpu(), lse.cpu()
+
+
+def oracle_rows(q, k, v, b, h, rows, kind, window=0, doc_id=None, score_kind=0, softcap=0.0,
+                scale=0.0):
+    return OA.attention_head(q[b, h], k[b, h], v[b, h], kind, window=window or None,
+                             doc_id=None if doc_id is None else doc_id.numpy(),
+                             score_kind=score_kind, softcap=softcap,
+                             scale=scale if scale > 0 else None, rows=rows)
+
+
+def compare(out_gpu, lse_gpu, out_ref, lse_ref, what=""):
+    """Element-by-element comparison; returns a dict of the error figures."""
+    og = out_gpu.double().numpy()
+    err = np.abs(og - out_ref)
+    lg = lse_gpu.double().numpy()
+    inf_ref = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lg), inf_ref), f"{what}: -inf LSE rows differ"
+    lerr = np.abs(lg[~inf_ref] - lse_ref[~inf_ref]) if (~inf_ref).any() else np.zeros(1)
+    res = {"max": float(err.max()) if err.size else 0.0,
+           "mean": float(err.mean()) if err.size else 0.0,
+           "lse_max": float(lerr.max())}
+    assert np.isfinite(og).all(), f"{what}: non-finite output"
+    assert res["max"] <= MAX_ERR, f"{what}: max |err| {res['max']:.3e}"
+    assert res["mean"] <= MEAN_ERR, f"{what}: mean |err| {res['mean']:.3e}"
+    assert res["lse_max"] <= LSE_ERR, f"{what}: max |lse err| {res['lse_max']:.3e}"
+    return res
+
+
+def sample_rows(L, seed, n_random=192, head=192, tail=128):
+    g = np.random.default_rng(seed)
+    rows = set(range(min(head, L))) | set(range(max(0, L - tail), L))
+    rows |= set(g.integers(0, L, size=min(n_random, L)).tolist())
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def check_workload(w: W.Workload, heads=None, rows=None, seed=0):
+    """Full-size GPU run of a workload; oracle on the given heads and rows."""
+    q, k, v = W.make_qkv(w)
+    doc = W.make_doc_id(w)
+    out, lse = run_gpu(q, k, v, w.mask_kind, w.window, doc, w.score_kind, w.softcap)
+    if heads is None:
+        heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    if rows is None:
+        rows = np.arange(w.L)
+    results = []
+    for (b, h) in heads:
+        o_ref, l_ref = oracle_rows(q, k, v, b, h, rows, w.mask_kind, w.window, doc, w.score_kind,
+                                   w.softcap)
+        results.append(compare(out[b, h][rows], lse[b, h][rows], o_ref, l_ref,
+                               f"{w.name} b{b} h{h}"))
+    return results

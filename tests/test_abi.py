@@ -1,0 +1,155 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, the ctypes struct mirrors the C layout, and host-side argument
+validation rejects bad calls before any CUDA call is made."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+@pytest.fixture(scope="module")
+def fa():
+    from block_sparse_attention_create_b200 import build
+    build.build()
+    import block_sparse_attention_create_b200 as m
+    return m
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_two_operations():
+    syms = declared_symbols()
+    assert "fa_create_block_mask" in syms and "fa_flex_attention_fwd" in syms
+
+
+def test_library_exports_every_declared_symbol(fa):
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(fa_\w+)", out))
+    for s in declared_symbols():
+        assert s in exported, s
+        assert hasattr(fa._lib, s)
+    assert set(fa.EXPORTED) == set(declared_symbols())
+
+
+def test_struct_layout_matches_c(fa):
+    """Compile a C probe against include/fa.h and compare offsets with ctypes."""
+    fields = [f for f, _ in fa.fa_block_mask._fields_]
+    src = "#include <stdio.h>\n#include <stddef.h>\n#include \"fa.h\"\nint main(void){\n"
+    src += 'printf("%zu\\n", sizeof(fa_block_mask));\n'
+    for f in fields:
+        src += f'printf("%zu\\n", offsetof(fa_block_mask, {f}));\n'
+    src += "return 0;}\n"
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "probe.c")
+        exe = os.path.join(d, "probe")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-I", os.path.dirname(HEADER), c, "-o", exe], check=True)
+        vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True,
+                                               check=True).stdout.split()]
+    assert vals[0] == ctypes.sizeof(fa.fa_block_mask)
+    for f, off in zip(fields, vals[1:]):
+        assert getattr(fa.fa_block_mask, f).offset == off, f
+
+
+def test_enum_values_match_header(fa):
+    text = open(HEADER).read()
+    for name in ("FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
+                 "FA_ERR_TIMEOUT", "FA_MASK_CAUSAL", "FA_MASK_SLIDING_WINDOW_CAUSAL",
+                 "FA_MASK_DOCUMENT_CAUSAL", "FA_SCORE_NONE", "FA_SCORE_TANH_SOFTCAP",
+                 "FA_BF16", "FA_FP16"):
+        m = re.search(rf"\b{name}\s*=\s*(\d+)", text)
+        assert m and int(m.group(1)) == getattr(fa, name), name
+
+
+def test_status_strings(fa):
+    assert fa.fa_status_string(0) == b"FA_OK"
+    assert fa.fa_status_string(4) == b"FA_ERR_TIMEOUT"
+    assert fa.fa_status_string(99) == b"FA_ERR_UNKNOWN"
+
+
+def test_block_mask_dims(fa):
+    assert fa.block_mask_dims(32768, 32768) == (256, 256)
+    assert fa.block_mask_dims(129, 1) == (2, 1)
+    assert fa.block_mask_dims(0, 0) == (0, 0)
+    nq, nkv = ctypes.c_int32(), ctypes.c_int32()
+    assert fa.fa_block_mask_dims(-1, 5, 128, ctypes.byref(nq), ctypes.byref(nkv)) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_block_mask_dims(5, 5, 64, ctypes.byref(nq), ctypes.byref(nkv)) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_block_mask_dims(fa.FA_MAX_LEN + 1, 5, 128, ctypes.byref(nq),
+                                 ctypes.byref(nkv)) == fa.FA_ERR_INVALID_ARG
+
+
+def test_create_block_mask_rejects_bad_arguments(fa):
+    bm = fa.fa_block_mask()
+    null = ctypes.c_void_p(0)
+    # unknown kind, bad window, missing doc ids, NULL struct, NULL arrays
+    assert fa.fa_create_block_mask(7, 0, null, 256, 256, 128, ctypes.byref(bm), null) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_create_block_mask(1, 0, null, 256, 256, 128, ctypes.byref(bm), null) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_create_block_mask(2, 0, null, 256, 256, 128, ctypes.byref(bm), null) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_create_block_mask(0, 0, null, 256, 256, 128, None, null) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_create_block_mask(0, 0, null, 256, 256, 128, ctypes.byref(bm), null) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_create_block_mask(0, 0, null, 256, 256, 100, ctypes.byref(bm), null) == fa.FA_ERR_INVALID_ARG
+    # an empty mask is valid and launches nothing
+    assert fa.fa_create_block_mask(0, 0, null, 0, 0, 128, ctypes.byref(bm), null) == fa.FA_OK
+    assert (bm.q_len, bm.n_q_blocks, bm.block) == (0, 0, 128)
+
+
+def _fwd(fa, bm, **kw):
+    args = dict(q=1024, k=1024, v=1024, dtype=0, B=1, H=1, L=256, S=256, D=64, sk=0, cap=0.0,
+                scale=0.0, out=1024, lse=0, ws=1024)
+    args.update(kw)
+    vp = ctypes.c_void_p
+    return fa.fa_flex_attention_fwd(vp(args["q"]), vp(args["k"]), vp(args["v"]), args["dtype"],
+                                    args["B"], args["H"], args["L"], args["S"], args["D"],
+                                    ctypes.byref(bm) if bm is not None else None, args["sk"],
+                                    args["cap"], args["scale"], vp(args["out"]), vp(args["lse"]),
+                                    vp(args["ws"]), vp(0))
+
+
+def test_fwd_rejects_bad_arguments_on_host(fa):
+    """Every case below is refused before any CUDA call (the pointers are fake)."""
+    bm = fa.fa_block_mask()
+    bm.q_len, bm.kv_len, bm.block, bm.n_q_blocks, bm.n_kv_blocks = 256, 256, 128, 2, 2
+    bm.kv_num_blocks = bm.full_kv_num_blocks = bm.q_order = 4096
+    E = fa.FA_ERR_INVALID_ARG
+    assert _fwd(fa, None) == E
+    assert _fwd(fa, bm, ws=0) == E
+    assert _fwd(fa, bm, dtype=5) == E
+    assert _fwd(fa, bm, L=128) == E                 # L != mask q_len
+    assert _fwd(fa, bm, S=512) == E                 # S != mask kv_len
+    assert _fwd(fa, bm, sk=1, cap=0.0) == E         # softcap needs c > 0
+    assert _fwd(fa, bm, sk=1, cap=float("inf")) == E
+    assert _fwd(fa, bm, sk=3) == E
+    assert _fwd(fa, bm, scale=float("nan")) == E
+    assert _fwd(fa, bm, B=-1) == E
+    assert _fwd(fa, bm, D=96) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd(fa, bm, q=1030) == E                # not 16-byte aligned
+    assert _fwd(fa, bm, out=0) == E
+    assert _fwd(fa, bm, k=0) == E
+    # B*H == 0 or L == 0: nothing to do
+    assert _fwd(fa, bm, B=0) == fa.FA_OK
+    bm0 = fa.fa_block_mask()
+    bm0.q_len, bm0.kv_len, bm0.block = 0, 256, 128
+    assert _fwd(fa, bm0, L=0) == fa.FA_OK
+
+
+def test_workspace_size(fa):
+    assert fa.fa_fwd_workspace_bytes() >= 4
+
+
+def test_product_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "block_sparse_attention_create_b200")
+    pat = re.compile(r"^\s*(import\s+oracle|from\s+oracle\b)", re.M)
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith(".py"):
+                assert not pat.search(open(os.path.join(dirpath, f)).read()), f

@@ -1,0 +1,159 @@
+"""Forward parity on the GPU: the CUDA path (through the C-ABI binding) against
+the fp64 CPU oracle on the same seeded inputs, element by element.
+
+Small shapes are compared on every row of every head (they span several 128-row
+tiles and ragged tails); the full-size workloads run at their real sizes on the
+GPU, in the launch configuration the benchmark times, and are compared on
+sampled heads and rows (each row's result is independent of the others)."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from parity import check_workload, compare, oracle_rows, run_gpu, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_compare(q, k, v, kind, window=0, doc=None, sk=0, cap=0.0, scale=0.0):
+    out, lse = run_gpu(q, k, v, kind, window, doc, sk, cap, scale)
+    B, H, L = q.shape[0], q.shape[1], q.shape[2]
+    res = []
+    for b in range(B):
+        for h in range(H):
+            o_ref, l_ref = oracle_rows(q, k, v, b, h, np.arange(L), kind, window, doc, sk, cap, scale)
+            res.append(compare(out[b, h], lse[b, h], o_ref, l_ref, f"b{b} h{h}"))
+    return out, lse, res
+
+
+def test_small_causal_workload_all_rows():
+    w = W.C1_CAUSAL_256
+    res = check_workload(w)
+    assert len(res) == w.B * w.H
+
+
+@pytest.mark.parametrize("w", (W.C2_CAUSAL_8192,) + W.C2_WINDOWS, ids=lambda w: w.name)
+def test_8192_sweep_sampled(w):
+    rows = sample_rows(w.L, seed=1)
+    check_workload(w, heads=[(0, 0), (0, w.H - 1)], rows=rows)
+
+
+def test_32k_window_sampled():
+    w = W.C3_SWA256_32K
+    rows = sample_rows(w.L, seed=2, n_random=256)
+    check_workload(w, heads=[(0, 0), (0, 5)], rows=rows)
+
+
+@pytest.mark.parametrize("w", (W.C4_DOC_FIXED, W.C4_DOC_SEEDED), ids=lambda w: w.name)
+def test_document_sampled(w):
+    rows = sample_rows(w.L, seed=3)
+    rows = np.union1d(rows, np.array([2047, 2048, 2049, 4999, 5000, 5001]))
+    check_workload(w, heads=[(0, 0), (0, 15)], rows=rows)
+
+
+def test_softcap_d128_sampled():
+    w = W.C5_SWA1024_SOFTCAP
+    rows = sample_rows(w.L, seed=4, n_random=128, head=128, tail=64)
+    check_workload(w, heads=[(0, 0), (1, 15)], rows=rows)
+
+
+@pytest.mark.parametrize("L,S", [(200, 200), (333, 333), (300, 1000), (1000, 300), (1, 1),
+                                 (1, 129), (129, 1), (257, 64)])
+@pytest.mark.parametrize("kind,window", [(0, 0), (1, 100), (2, 0)])
+def test_ragged_shapes_all_rows(L, S, kind, window):
+    q, k, v = W.random_qkv(2, 2, L, S, 64, torch.bfloat16, seed=L * 7 + S)
+    doc = None
+    if kind == 2:
+        g = torch.Generator().manual_seed(L + S)
+        doc = torch.randint(0, 3, (max(L, S),), generator=g, dtype=torch.int32)
+    _full_compare(q, k, v, kind, window, doc)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("D", [64, 128])
+def test_dtypes_and_head_dims(dtype, D):
+    q, k, v = W.random_qkv(1, 3, 640, 640, D, dtype, seed=D + (dtype == torch.float16))
+    _full_compare(q, k, v, 0)
+    _full_compare(q, k, v, 1, window=300, sk=1, cap=5.0)
+
+
+def test_softcap_and_custom_scale():
+    q, k, v = W.random_qkv(1, 2, 512, 512, 64, torch.bfloat16, seed=11, scale=2.0)
+    _full_compare(q, k, v, 0, sk=1, cap=3.0)
+    _full_compare(q, k, v, 1, window=200, scale=0.3)
+
+
+def test_fully_masked_rows_zero_and_minus_inf():
+    """Window rule with L > S + W - 1: rows q >= S + W - 1 see no key."""
+    q, k, v = W.random_qkv(1, 2, 700, 100, 64, torch.bfloat16, seed=12)
+    out, lse, _ = _full_compare(q, k, v, 1, window=50)
+    assert torch.all(out[:, :, 149:] == 0) and torch.all(torch.isneginf(lse[:, :, 149:]))
+    q, k, v = W.random_qkv(1, 1, 300, 0, 64, torch.bfloat16, seed=13)
+    out, lse = run_gpu(q, k, v, 0)
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_single_visible_key_is_bit_exact():
+    """Row 0 (every rule) and the first token of each document see one key:
+    P = 1 exactly, so out must equal that key's V bit for bit."""
+    w = W.C4_DOC_FIXED
+    q, k, v = W.make_qkv(w)
+    doc = W.make_doc_id(w)
+    out, _ = run_gpu(q, k, v, w.mask_kind, 0, doc)
+    for r in (0, 2048, 5000):
+        assert torch.equal(out[0, :, r], v[0, :, r])
+    q, k, v = W.random_qkv(1, 4, 300, 300, 128, torch.bfloat16, seed=14)
+    for kind, window in ((0, 0), (1, 64)):
+        out, _ = run_gpu(q, k, v, kind, window)
+        assert torch.equal(out[0, :, 0], v[0, :, 0])
+
+
+def test_online_rescale_path():
+    """Scores that grow by far more than 2^8 between blocks processed later force
+    the deferred O rescale: keys far in the past score highest, and the
+    diagonal (partial) block is processed first."""
+    L, D = 1024, 64
+    g = torch.Generator().manual_seed(15)
+    q = torch.zeros(1, 2, L, D)
+    q[..., 0] = 4.0
+    q += 0.1 * torch.randn(q.shape, generator=g)
+    k = 0.1 * torch.randn(1, 2, L, D, generator=g)
+    k[..., 0] += torch.linspace(20.0, 0.0, L)
+    v = torch.randn(1, 2, L, D, generator=g)
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    _full_compare(q, k, v, 0)
+    _full_compare(q, k, v, 2, doc=torch.tensor([0] * 300 + [1] * 724, dtype=torch.int32))
+
+
+def test_many_units_persistent_schedule():
+    """More work units than (CTAs x slots): every worker takes several units."""
+    q, k, v = W.random_qkv(4, 16, 2048, 2048, 64, torch.bfloat16, seed=16)
+    out, lse = run_gpu(q, k, v, 0)
+    rows = sample_rows(2048, seed=5, n_random=64, head=64, tail=64)
+    for (b, h) in ((0, 0), (1, 7), (3, 15)):
+        o_ref, l_ref = oracle_rows(q, k, v, b, h, rows, 0)
+        compare(out[b, h][rows], lse[b, h][rows], o_ref, l_ref, f"b{b} h{h}")
+
+
+def test_deterministic_and_stream_safe():
+    import block_sparse_attention_create_b200 as fa
+    q, k, v = (t.cuda() for t in W.random_qkv(1, 4, 1000, 1000, 64, torch.bfloat16, seed=17))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        bm = fa.create_block_mask(1, 1000, 1000, window=300, device="cuda", stream=s)
+        a = fa.flex_attention(q, k, v, bm, stream=s)
+        b = fa.flex_attention(q, k, v, bm, stream=s)
+    s.synchronize()
+    assert torch.equal(a, b)
+    assert fa.last_device_error(stream=s) == fa.FA_OK
+
+
+def test_empty_batch_and_zero_length_are_noops():
+    import block_sparse_attention_create_b200 as fa
+    q = torch.empty(0, 2, 256, 64, dtype=torch.bfloat16, device="cuda")
+    bm = fa.create_block_mask(0, 256, 256, device="cuda")
+    out = fa.flex_attention(q, q, q, bm)
+    assert out.shape == q.shape
+    q0 = torch.empty(1, 2, 0, 64, dtype=torch.bfloat16, device="cuda")
+    bm0 = fa.create_block_mask(0, 0, 0, device="cuda")
+    assert fa.flex_attention(q0, q0, q0, bm0).shape == q0.shape
