@@ -1,0 +1,398 @@
+"""Benchmark of the block-sparse attention hot path on B200.
+
+A step is one pass of the whole path over one batch of synthetic input:
+fa_create_block_mask (block classification + schedule order) followed by
+fa_flex_attention_fwd.  Default workload: sliding-window causal W=256,
+B=1 H=8 L=S=32768 D=64 bf16 (the FlexAttention vs SDPA M1 Max benchmark's
+longest case, qiita kiarina, "検証結果").
+
+Prints one JSON line (rank 0).  `value` is live-block TFLOP/s of whole steps
+(4 * D * 128^2 FLOPs per live block per batch*head: the two matmuls over the
+blocks the mask keeps; skipped blocks count nothing), summed over ranks and
+divided by the max-over-ranks device time.  L2 is flushed (a 512 MiB write)
+between timed steps, outside the timed region.
+
+--impl reference times the CPU fp64 oracle (the only reference there is) on a
+bounded row sample of the same workload, on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "fwd ms & live-block TFLOP/s (frac of BF16 TC peak) at S=32768 W=256"
+UNIT = "TFLOP/s"
+# Page-1 FlexAttention forward on M1 Max at this workload: 75.27 ms (context only).
+PAGE_FWD_MS = {"swa256_L32768_B1_H8_D64_bf16": 75.27, "causal_L8192_B1_H8_D64_bf16": 231.22,
+               "swa64_L8192_B1_H8_D64_bf16": 11.75, "swa256_L8192_B1_H8_D64_bf16": 19.14,
+               "swa1024_L8192_B1_H8_D64_bf16": 56.24, "swa4096_L8192_B1_H8_D64_bf16": 169.24}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def live_blocks_per_row(w: W.Workload):
+    """Live 128x128 blocks of every q-block row, from the GPU-independent closed
+    forms of the mask (causal / window) or a pass over the document ids."""
+    nq = -(-w.L // 128)
+    nkv = -(-w.S // 128)
+    out = np.zeros(nq, dtype=np.int64)
+    doc = W.make_doc_id(w)
+    doc = doc.numpy() if doc is not None else None
+    for i in range(nq):
+        q0, q1 = i * 128, min(w.L, i * 128 + 128) - 1
+        for j in range(nkv):
+            k0, k1 = j * 128, min(w.S, j * 128 + 128) - 1
+            if k0 > q1:
+                break
+            if w.mask_kind == W.MASK_SLIDING_WINDOW_CAUSAL and k1 < q0 - w.window + 1:
+                continue
+            if w.mask_kind == W.MASK_DOCUMENT_CAUSAL:
+                dq = set(doc[q0:q1 + 1].tolist())
+                if not dq.intersection(doc[k0:k1 + 1].tolist()):
+                    continue
+            out[i] += 1
+    return out
+
+
+def work_figures(w: W.Workload):
+    per_row = live_blocks_per_row(w)
+    live = int(per_row.sum())
+    flops = 4.0 * w.D * 128 * 128 * live * w.B * w.H
+    esz = 2
+    bytes_ = (w.B * w.H * (w.L * w.D * esz * 2 + w.S * w.D * esz * 2 + w.L * 4)
+              + per_row.size * (3 + 2 * (-(-w.S // 128))) * 4)
+    return {"live_blocks": live, "per_row": per_row, "flops": flops, "bytes": bytes_}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the GPU is busy."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "utilization.gpu")
+
+    def __init__(self, index, enabled=True):
+        self.index = index
+        self.enabled = enabled
+        self.proc = None
+
+    def __enter__(self):
+        if not self.enabled:
+            return self
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons, busy = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                util = float(f[9])
+                clk = float(f[1])
+                mx = float(f[2])
+            except ValueError:
+                continue
+            if util < 50:
+                continue
+            busy += 1
+            sm.append(clk)
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples_under_load": busy}
+
+
+def run_ours(args, w: W.Workload, rank, world, device):
+    import block_sparse_attention_create_b200 as fa
+    torch.cuda.set_device(device)
+    q, k, v = W.make_qkv(w)
+    doc = W.make_doc_id(w)
+    qd, kd, vd = q.to(device), k.to(device), v.to(device)
+    dd = doc.to(device) if doc is not None else None
+    out = torch.empty_like(qd)
+    lse = torch.empty(w.B, w.H, w.L, dtype=torch.float32, device=device)
+    bm = fa.BlockMask(w.L, w.S, device)
+    ws = fa.workspace(device)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    def step():
+        fa.create_block_mask(w.mask_kind, w.L, w.S, window=w.window, doc_id=dd, out=bm,
+                             stream=stream)
+        fa.flex_attention(qd, kd, vd, bm, score_mod=w.score_kind, softcap=w.softcap, out=out,
+                          lse=lse, ws=ws, stream=stream)
+
+    fig = work_figures(w)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert fa.last_device_error(device) == fa.FA_OK
+
+    # keep the GPU at load clocks for ~1 s inside the sampling window, untimed
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(device.index if device.index is not None else 0,
+                      enabled=not args.profile) as clk:
+        t_end = time.time() + (0.0 if args.profile else 1.0)
+        while time.time() < t_end:
+            for _ in range(50):
+                step()
+            torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            fa.create_block_mask(w.mask_kind, w.L, w.S, window=w.window, doc_id=dd, out=bm,
+                                 stream=stream)
+            mids[i].record(stream)
+            fa.flex_attention(qd, kd, vd, bm, score_mod=w.score_kind, softcap=w.softcap,
+                              out=out, lse=lse, ws=ws, stream=stream)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+    assert fa.last_device_error(device) == fa.FA_OK
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    fwd_ms = [m.elapsed_time(e) for m, e in zip(mids, ends)]
+    mask_ms = [s.elapsed_time(m) for s, m in zip(starts, mids)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end to end through the public API: pinned host inputs in, results out
+    e2e = ({"ms": float("nan"), "h2d": 0, "d2h": 0} if args.profile
+           else run_e2e(args, w, fa, q, k, v, doc, device, world))
+    return {"fig": fig, "total_ms": total_ms, "step_ms": step_ms, "fwd_ms": fwd_ms,
+            "mask_ms": mask_ms, "clocks": clk.summary(), "e2e": e2e}
+
+
+def run_e2e(args, w, fa, q, k, v, doc, device, world):
+    hq, hk, hv = (t.pin_memory() for t in (q, k, v))
+    hdoc = doc.pin_memory() if doc is not None else None
+    hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    hlse = torch.empty(w.B, w.H, w.L, dtype=torch.float32).pin_memory()
+    qd, kd, vd = (torch.empty(t.shape, dtype=t.dtype, device=device) for t in (q, k, v))
+    dd = torch.empty(doc.shape, dtype=doc.dtype, device=device) if doc is not None else None
+    out = torch.empty_like(qd)
+    lse = torch.empty(w.B, w.H, w.L, dtype=torch.float32, device=device)
+    bm = fa.BlockMask(w.L, w.S, device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        qd.copy_(hq, non_blocking=True)
+        kd.copy_(hk, non_blocking=True)
+        vd.copy_(hv, non_blocking=True)
+        if dd is not None:
+            dd.copy_(hdoc, non_blocking=True)
+        fa.create_block_mask(w.mask_kind, w.L, w.S, window=w.window, doc_id=dd, out=bm,
+                             stream=stream)
+        fa.flex_attention(qd, kd, vd, bm, score_mod=w.score_kind, softcap=w.softcap, out=out,
+                          lse=lse, stream=stream)
+        hout.copy_(out, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + (
+        hdoc.numel() * 4 if hdoc is not None else 0)
+    d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
+    return {"ms": ms, "h2d": h2d, "d2h": d2h}
+
+
+def oracle_sample(w: W.Workload, rows, fig):
+    """Time the oracle on `rows` of head (0, 0); returns (seconds, live FLOPs credited)."""
+    from oracle import attention as OA
+    q, k, v = W.make_qkv(w)
+    doc = W.make_doc_id(w)
+    t0 = time.perf_counter()
+    OA.attention_head(q[0, 0], k[0, 0], v[0, 0], w.mask_kind, window=w.window or None,
+                      doc_id=None if doc is None else doc.numpy(), score_kind=w.score_kind,
+                      softcap=w.softcap, rows=rows)
+    dt = time.perf_counter() - t0
+    credited = sum(4.0 * w.D * 128 * int(fig["per_row"][r // 128]) for r in rows)
+    return dt, credited
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=W.C3_SWA256_32K.name, choices=sorted(W.BY_NAME))
+    ap.add_argument("--cpu-rows", type=int, default=2048,
+                    help="oracle rows timed for cpu_baseline (bounded sample)")
+    ap.add_argument("--profile", action="store_true",
+                    help="short run for profilers: warm-up and timed steps only (no clock "
+                         "window, no end-to-end leg, no CPU baseline); not a bench value")
+    args = ap.parse_args()
+    w = W.BY_NAME[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    peaks, peaks_src = load_peaks()
+    fig = work_figures(w)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        rows_per_step = 64
+        g = np.random.default_rng(0)
+        for _ in range(args.warmup):
+            oracle_sample(w, np.sort(g.integers(0, w.L, rows_per_step)), fig)
+        tot_s, tot_f = 0.0, 0.0
+        for _ in range(args.steps):
+            dt, fl = oracle_sample(w, np.sort(g.integers(0, w.L, rows_per_step)), fig)
+            tot_s += dt
+            tot_f += fl
+        value = tot_f / tot_s / 1e12
+        ms_step = fig["flops"] / (value * 1e12) * 1e3
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {**w.describe(), "parallelism": "none (host cores)"},
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(),
+                                 "kind": "oracle",
+                                 "sample": f"{rows_per_step} random query rows of head (0,0) per "
+                                           "step; ms_per_step extrapolates to the whole workload"},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    r = run_ours(args, w, rank, world, device)
+
+    total_flops = fig["flops"] * args.steps * world
+    value = total_flops / (r["total_ms"] * 1e-3) / 1e12
+    fwd_avg = statistics.mean(r["fwd_ms"])
+    fwd_med = statistics.median(r["fwd_ms"])
+    fwd_tflops = fig["flops"] / (fwd_avg * 1e-3) / 1e12
+    fwd_gbs = fig["bytes"] / (fwd_avg * 1e-3) / 1e9
+    hbm_peak = peaks["hbm_gbs"]
+    tc_peak = peaks["bf16_tflops"]
+    e2e_value = fig["flops"] * args.steps * world / (r["e2e"]["ms"] * 1e-3) / 1e12
+    tensor_frac = fwd_tflops / tc_peak
+    hbm_frac = fwd_gbs / hbm_peak
+    bound = "hbm" if hbm_frac >= tensor_frac else "tensor"
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": fwd_gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": hbm_frac, "traffic": None}
+    else:
+        roof = {"bound": "tensor", "achieved": fwd_tflops, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": tensor_frac, "traffic": None}
+    roof["peak_source"] = f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"
+    roof["kernel"] = "fwd_kernel (fa_flex_attention_fwd)"
+    page_ms = PAGE_FWD_MS.get(w.name)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": r["total_ms"] / args.steps,
+            "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": (value / (fig["flops"] / (page_ms * 1e-3) / 1e12)) if page_ms else None,
+            "dtype": w.dtype_name, "data": "synthetic",
+            "config": {**w.describe(), "parallelism": f"replicas x{world}" if world > 1 else "none",
+                       "l2": "flushed between timed steps (512 MiB write, untimed)",
+                       "step": "fa_create_block_mask + fa_flex_attention_fwd"},
+            "fwd_ms": fwd_avg, "fwd_ms_median": fwd_med, "fwd_tflops": fwd_tflops,
+            "fwd_tensor_frac": tensor_frac, "fwd_hbm_gbs": fwd_gbs, "fwd_hbm_frac": hbm_frac,
+            "mask_build_ms": statistics.mean(r["mask_ms"]),
+            "live_blocks_per_head": fig["live_blocks"], "live_gflop": fig["flops"] / 1e9,
+            "algorithmic_mb": fig["bytes"] / 1e6,
+            "roofline": roof,
+            "gpu_launches": 3 * args.steps,
+            "clocks": r["clocks"],
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": r["e2e"]["h2d"],
+                    "d2h_bytes_per_step": r["e2e"]["d2h"],
+                    "ms_per_step": r["e2e"]["ms"] / args.steps}}
+    if rank == 0 and world == 1 and not args.profile:
+        rows = np.sort(np.random.default_rng(1).choice(w.L, size=min(args.cpu_rows, w.L),
+                                                       replace=False))
+        dt, credited = oracle_sample(w, rows, fig)
+        line["cpu_baseline"] = {"value": credited / dt / 1e12, "unit": UNIT, "cores": cpu_threads(),
+                                "kind": "oracle",
+                                "sample": f"{len(rows)} random query rows of head (0,0), "
+                                          f"{dt:.1f} s; live-block FLOPs of those rows credited"}
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

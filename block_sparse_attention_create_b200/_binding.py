@@ -1,0 +1,222 @@
+"""ctypes binding of libfa.so, the B200 block-sparse attention library.
+
+Argument marshalling only: every step of the computation runs in the library's
+CUDA kernels.  The C-ABI names are re-exported unchanged (``fa_create_block_mask``,
+``fa_flex_attention_fwd``, ...); ``create_block_mask`` and ``flex_attention`` are
+thin conveniences that allocate the output tensors with torch and pass pointers,
+mirroring the FlexAttention calls of the how-to
+("FlexAttention on Apple Silicon: block mask how-to", dreaming.press, "Setup").
+
+There is no fallback: if libfa.so is missing or cannot be loaded, importing this
+module raises ImportError.  Build it with
+``python -m block_sparse_attention_create_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa.so")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+FA_MASK_CAUSAL, FA_MASK_SLIDING_WINDOW_CAUSAL, FA_MASK_DOCUMENT_CAUSAL = range(3)
+FA_SCORE_NONE, FA_SCORE_TANH_SOFTCAP = range(2)
+FA_BF16, FA_FP16 = range(2)
+FA_BLOCK = 128
+FA_MAX_LEN = 8192 * 128
+
+# Every symbol include/fa.h declares.
+EXPORTED = ("fa_block_mask_dims", "fa_create_block_mask", "fa_fwd_workspace_bytes",
+            "fa_flex_attention_fwd", "fa_get_last_device_error", "fa_status_string",
+            "fa_num_sms")
+
+
+class fa_block_mask(ctypes.Structure):
+    """Mirror of ``struct fa_block_mask`` in include/fa.h."""
+    _fields_ = [
+        ("kv_num_blocks", ctypes.c_void_p),
+        ("kv_indices", ctypes.c_void_p),
+        ("full_kv_num_blocks", ctypes.c_void_p),
+        ("full_kv_indices", ctypes.c_void_p),
+        ("q_order", ctypes.c_void_p),
+        ("q_len", ctypes.c_int32),
+        ("kv_len", ctypes.c_int32),
+        ("block", ctypes.c_int32),
+        ("n_q_blocks", ctypes.c_int32),
+        ("n_kv_blocks", ctypes.c_int32),
+        ("kind", ctypes.c_int32),
+        ("window", ctypes.c_int32),
+        ("doc_id", ctypes.c_void_p),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m block_sparse_attention_create_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    i32, vp, f32 = ctypes.c_int32, ctypes.c_void_p, ctypes.c_float
+    lib.fa_block_mask_dims.argtypes = [i32, i32, i32, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    lib.fa_block_mask_dims.restype = i32
+    lib.fa_create_block_mask.argtypes = [i32, i32, vp, i32, i32, i32, ctypes.POINTER(fa_block_mask), vp]
+    lib.fa_create_block_mask.restype = i32
+    lib.fa_fwd_workspace_bytes.argtypes = []
+    lib.fa_fwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa_flex_attention_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                          ctypes.POINTER(fa_block_mask), i32, f32, f32, vp, vp, vp, vp]
+    lib.fa_flex_attention_fwd.restype = i32
+    lib.fa_get_last_device_error.argtypes = [vp, vp]
+    lib.fa_get_last_device_error.restype = i32
+    lib.fa_status_string.argtypes = [i32]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_num_sms.argtypes = []
+    lib.fa_num_sms.restype = i32
+    return lib
+
+
+_lib = _load()
+
+# ---- the C-ABI, same names --------------------------------------------------
+fa_block_mask_dims = _lib.fa_block_mask_dims
+fa_create_block_mask = _lib.fa_create_block_mask
+fa_fwd_workspace_bytes = _lib.fa_fwd_workspace_bytes
+fa_flex_attention_fwd = _lib.fa_flex_attention_fwd
+fa_get_last_device_error = _lib.fa_get_last_device_error
+fa_status_string = _lib.fa_status_string
+fa_num_sms = _lib.fa_num_sms
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {fa_status_string(status).decode()}")
+
+
+def _check(status: int, what: str):
+    if status != FA_OK:
+        raise FAError(status, what)
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def block_mask_dims(q_len: int, kv_len: int, block: int = FA_BLOCK):
+    nq, nkv = ctypes.c_int32(), ctypes.c_int32()
+    _check(fa_block_mask_dims(q_len, kv_len, block, ctypes.byref(nq), ctypes.byref(nkv)),
+           "fa_block_mask_dims")
+    return nq.value, nkv.value
+
+
+class BlockMask:
+    """Device block tables of one mask (broadcast over batch and heads).
+
+    Holds the torch tensors the library fills and the ctypes struct that points
+    at them; reuse one BlockMask across forwards, as the how-to recommends.
+    """
+
+    def __init__(self, q_len: int, kv_len: int, device, block: int = FA_BLOCK):
+        nq, nkv = block_mask_dims(q_len, kv_len, block)
+        i32 = dict(dtype=torch.int32, device=device)
+        self.kv_num_blocks = torch.zeros(nq, **i32)
+        self.kv_indices = torch.zeros(nq, nkv, **i32)
+        self.full_kv_num_blocks = torch.zeros(nq, **i32)
+        self.full_kv_indices = torch.zeros(nq, nkv, **i32)
+        self.q_order = torch.zeros(2 * nq, **i32)   # schedule: (row, partial | full << 16)
+        self.doc_id: Optional[torch.Tensor] = None
+        self.struct = fa_block_mask()
+        self.struct.kv_num_blocks = self.kv_num_blocks.data_ptr()
+        self.struct.kv_indices = self.kv_indices.data_ptr()
+        self.struct.full_kv_num_blocks = self.full_kv_num_blocks.data_ptr()
+        self.struct.full_kv_indices = self.full_kv_indices.data_ptr()
+        self.struct.q_order = self.q_order.data_ptr()
+        self.q_len, self.kv_len, self.n_q_blocks, self.n_kv_blocks = q_len, kv_len, nq, nkv
+
+    def tables(self):
+        """Host copies of the integer tables (for inspection and tests)."""
+        return {k: getattr(self, k).cpu().numpy() for k in
+                ("kv_num_blocks", "kv_indices", "full_kv_num_blocks", "full_kv_indices", "q_order")}
+
+
+def create_block_mask(kind: int, q_len: int, kv_len: int, window: int = 0,
+                      doc_id: Optional[torch.Tensor] = None, device="cuda",
+                      stream: Optional[torch.cuda.Stream] = None, out: Optional[BlockMask] = None
+                      ) -> BlockMask:
+    """fa_create_block_mask on fresh (or the given) device tables."""
+    bm = out if out is not None else BlockMask(q_len, kv_len, device)
+    if doc_id is not None:
+        if doc_id.dtype != torch.int32 or not doc_id.is_cuda or not doc_id.is_contiguous():
+            raise ValueError("doc_id must be a contiguous int32 CUDA tensor")
+        if doc_id.numel() < max(q_len, kv_len):
+            raise ValueError("doc_id must hold max(q_len, kv_len) ids")
+        bm.doc_id = doc_id
+    _check(fa_create_block_mask(kind, window, _ptr(doc_id), q_len, kv_len, FA_BLOCK,
+                                ctypes.byref(bm.struct), _stream_handle(stream)),
+           "fa_create_block_mask")
+    return bm
+
+
+_workspaces = {}
+
+
+def workspace(device) -> torch.Tensor:
+    """A zeroed forward workspace per device (reused by every call on that device)."""
+    dev = torch.device(device)
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    ws = _workspaces.get(key)
+    if ws is None:
+        ws = torch.zeros(int(fa_fwd_workspace_bytes()), dtype=torch.uint8, device=f"cuda:{key}")
+        _workspaces[key] = ws
+    return ws
+
+
+_DTYPES = {torch.bfloat16: FA_BF16, torch.float16: FA_FP16}
+
+
+def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask: BlockMask,
+                   score_mod: int = FA_SCORE_NONE, softcap: float = 0.0, scale: float = 0.0,
+                   out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                   return_lse: bool = False, ws: Optional[torch.Tensor] = None,
+                   stream: Optional[torch.cuda.Stream] = None):
+    """fa_flex_attention_fwd on torch tensors q (B,H,L,D), k/v (B,H,S,D)."""
+    if q.dtype not in _DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share dtype bf16 or fp16")
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("q, k, v must be contiguous 4-D CUDA tensors")
+    B, H, L, D = q.shape
+    S = k.shape[2]
+    if k.shape != (B, H, S, D) or v.shape != (B, H, S, D):
+        raise ValueError("k and v must be (B, H, S, D) with the q's B, H, D")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty(B, H, L, dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(q.device)
+    _check(fa_flex_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], B, H, L, S, D,
+                                 ctypes.byref(block_mask.struct), score_mod, float(softcap),
+                                 float(scale), _ptr(out), _ptr(lse), _ptr(ws),
+                                 _stream_handle(stream)),
+           "fa_flex_attention_fwd")
+    return (out, lse) if return_lse else out
+
+
+def last_device_error(device=None, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """fa_get_last_device_error on the per-device workspace; returns the status."""
+    dev = device if device is not None else torch.cuda.current_device()
+    return fa_get_last_device_error(_ptr(workspace(dev)), _stream_handle(stream))
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

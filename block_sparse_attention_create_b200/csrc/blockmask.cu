@@ -146,14 +146,18 @@ classify_rows_kernel(int kind, int window, const int32_t* __restrict__ doc, int 
   }
 }
 
-// q_order: rows by descending live count, ties by ascending row.  Keys
-// (n_kv - count) << 13 | row are unique, so a bitonic sort of them in shared
-// memory gives one deterministic order.
+// Schedule table q_order[2 * n_q]: rank k (rows by descending live count, ties by
+// ascending row) -> [2k] = row, [2k+1] = partial count | full count << 16.  Keys
+// (n_kv - count) << 13 | row are unique, so every sort of them gives the same
+// order: up to 2048 rows each thread ranks its rows by counting smaller keys;
+// above that a bitonic sort in shared memory.
 __global__ void __launch_bounds__(kOrderThreads)
 order_rows_kernel(int n_q, int n_kv, int n_pow2, const int32_t* __restrict__ kv_num,
-                  const int32_t* __restrict__ full_num, int32_t* __restrict__ q_order) {
+                  const int32_t* __restrict__ full_num, int32_t* __restrict__ sched) {
   extern __shared__ uint32_t keys[];
-  for (int t = threadIdx.x; t < n_pow2; t += blockDim.x) {
+  const bool rank_sort = n_q <= 2048;
+  const int n_keys = rank_sort ? n_q : n_pow2;
+  for (int t = threadIdx.x; t < n_keys; t += blockDim.x) {
     if (t < n_q) {
       const int cnt = kv_num[t] + full_num[t];
       keys[t] = (static_cast<uint32_t>(n_kv - cnt) << 13) | static_cast<uint32_t>(t);
@@ -162,6 +166,16 @@ order_rows_kernel(int n_q, int n_kv, int n_pow2, const int32_t* __restrict__ kv_
     }
   }
   __syncthreads();
+  if (rank_sort) {
+    for (int t = threadIdx.x; t < n_q; t += blockDim.x) {
+      const uint32_t key = keys[t];
+      int rank = 0;
+      for (int j = 0; j < n_q; ++j) rank += keys[j] < key ? 1 : 0;
+      sched[2 * rank] = t;
+      sched[2 * rank + 1] = kv_num[t] | (full_num[t] << 16);
+    }
+    return;
+  }
   for (int k = 2; k <= n_pow2; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
       for (int t = threadIdx.x; t < n_pow2; t += blockDim.x) {
@@ -178,7 +192,11 @@ order_rows_kernel(int n_q, int n_kv, int n_pow2, const int32_t* __restrict__ kv_
       __syncthreads();
     }
   }
-  for (int t = threadIdx.x; t < n_q; t += blockDim.x) q_order[t] = static_cast<int32_t>(keys[t] & 0x1FFFu);
+  for (int t = threadIdx.x; t < n_q; t += blockDim.x) {
+    const int row = static_cast<int>(keys[t] & 0x1FFFu);
+    sched[2 * t] = row;
+    sched[2 * t + 1] = kv_num[row] | (full_num[row] << 16);
+  }
 }
 
 }  // namespace
@@ -229,7 +247,8 @@ extern "C" fa_status fa_create_block_mask(int32_t kind, int32_t window, const in
   FA_CUDA_CHECK(cudaGetLastError());
   int n_pow2 = 1;
   while (n_pow2 < nq) n_pow2 <<= 1;
-  order_rows_kernel<<<1, kOrderThreads, n_pow2 * sizeof(uint32_t), s>>>(
+  const size_t order_smem = (nq <= 2048 ? nq : n_pow2) * sizeof(uint32_t);
+  order_rows_kernel<<<1, kOrderThreads, order_smem, s>>>(
       nq, nkv, n_pow2, bm->kv_num_blocks, bm->full_kv_num_blocks, bm->q_order);
   FA_CUDA_CHECK(cudaGetLastError());
   return FA_OK;

@@ -67,6 +67,8 @@ struct Cfg {
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kBlockN * D * 2;
   static constexpr int kStages = (D == 64) ? 8 : 4;
+  // Q tiles per slot: two at D=64, so the next unit's Q loads while this one runs.
+  static constexpr int kQBuf = (D == 64) ? 2 : 1;
   static constexpr uint32_t kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t s_col(int slot) { return 128u * slot; }
   __host__ __device__ static constexpr uint32_t o_col(int slot) { return 256u + static_cast<uint32_t>(D) * slot; }
@@ -74,10 +76,10 @@ struct Cfg {
 
 template <int D>
 struct __align__(1024) Smem {
-  uint8_t q[kNumSlots][Cfg<D>::kTileBytes];
+  uint8_t q[kNumSlots][Cfg<D>::kQBuf][Cfg<D>::kTileBytes];
   uint8_t kv[Cfg<D>::kStages][Cfg<D>::kTileBytes];
-  uint64_t q_full[kNumSlots];
-  uint64_t q_empty[kNumSlots];
+  uint64_t q_full[kNumSlots][Cfg<D>::kQBuf];
+  uint64_t q_empty[kNumSlots][Cfg<D>::kQBuf];
   uint64_t s_full[kNumSlots];
   uint64_t p_full[kNumSlots];
   uint64_t o_full[kNumSlots];
@@ -90,17 +92,16 @@ struct __align__(1024) Smem {
 };
 
 struct Params {
-  const int32_t* kv_num;
   const int32_t* kv_idx;
-  const int32_t* full_num;
   const int32_t* full_idx;
-  const int32_t* q_order;
+  const int32_t* sched;  // per rank k: [2k] = q-block row, [2k+1] = partial | full << 16
   const int32_t* doc_id;
   void* out;
   float* lse;
   int32_t* err;
   int BH, L, S, n_kv, num_units;
   int mask_kind, window, softcap_on, is_bf16;
+  int split_p;       // P fed to the PV product as two 16-bit terms (hi + lo)
   float scale_log2;  // scale * log2(e)
   float cap_k;       // 2 * scale * log2(e) / c : exp2(s * cap_k) = e^(2 s scale / c)
   float cap_a;       // c * log2(e)
@@ -108,65 +109,70 @@ struct Params {
 };
 
 // ---------------------------------------------------------------- scheduling
-// Work unit u -> (q-block rank u / BH in q_order, batch*head u % BH).  Units are
-// dealt to the grid's (CTA, slot) workers in rounds, alternating direction
-// ("snake"), so the heaviest rows of the LPT order spread over all workers.
+// Work unit u -> (rank u / BH of the LPT-ordered schedule table, batch*head u % BH).
+// Units are dealt to the grid's (CTA, slot) workers in rounds, alternating
+// direction ("snake"), so the heaviest rows of the LPT order spread over all
+// workers.  Every role of a CTA walks the same sequence.
 struct Unit {
   int bh, qblk, np, n;
 };
 
-__device__ __forceinline__ Unit decode_unit(const Params& p, int u) {
-  const int k = u / p.BH;
-  Unit x;
-  x.bh = u - k * p.BH;
-  x.qblk = __ldg(p.q_order + k);
-  x.np = __ldg(p.kv_num + x.qblk);
-  x.n = x.np + __ldg(p.full_num + x.qblk);
-  return x;
+__device__ __forceinline__ int2 ldg_nc_v2(const int32_t* ptr) {
+  int2 v;
+  asm volatile("ld.global.nc.v2.s32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(ptr));
+  return v;
+}
+__device__ __forceinline__ int ldg_nc(const int32_t* ptr) {
+  int v;
+  asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(ptr));
+  return v;
 }
 
-// kv-block index of the j-th block of the unit: partial blocks first, then full ones.
-__device__ __forceinline__ int block_index(const Params& p, const Unit& x, int j, bool& full) {
-  const size_t row = static_cast<size_t>(x.qblk) * p.n_kv;
-  if (j < x.np) {
-    full = false;
-    return __ldg(p.kv_idx + row + j);
+// Unit sequence of one worker with a one-unit lookahead: the schedule entry of
+// the next unit is requested when the current one is handed out, so its global
+// load latency overlaps a whole unit of work.
+struct UnitIter {
+  int worker, workers, round, num_units, BH;
+  const int32_t* sched;
+  int nu;   // next unit id, -1 when exhausted
+  int2 nx;  // its schedule entry (load in flight)
+
+  __device__ __forceinline__ void init(const Params& p, int slot) {
+    worker = static_cast<int>(blockIdx.x) * kNumSlots + slot;
+    workers = static_cast<int>(gridDim.x) * kNumSlots;
+    round = 0;
+    num_units = p.num_units;
+    BH = p.BH;
+    sched = p.sched;
+    fetch();
   }
-  full = true;
-  return __ldg(p.full_idx + row + (j - x.np));
-}
-
-struct Sched {
-  int worker, workers, round;
-  __device__ __forceinline__ int next(int num_units) {
+  __device__ __forceinline__ void fetch() {
     const int u = round * workers + ((round & 1) ? (workers - 1 - worker) : worker);
     ++round;
-    return u < num_units ? u : -1;
+    nu = u < num_units ? u : -1;
+    if (nu >= 0) nx = ldg_nc_v2(sched + 2 * (nu / BH));
+  }
+  __device__ __forceinline__ bool pop(Unit& x) {
+    if (nu < 0) return false;
+    const int k = nu / BH;
+    x.bh = nu - k * BH;
+    x.qblk = nx.x;
+    x.np = nx.y & 0xFFFF;
+    x.n = x.np + (nx.y >> 16);
+    fetch();
+    return true;
+  }
+  __device__ __forceinline__ bool pop_nonempty(Unit& x) {
+    while (pop(x))
+      if (x.n > 0) return true;
+    return false;
   }
 };
 
-struct SlotState {
-  Sched sched;
-  Unit unit;
-  int j;      // current block within the unit
-  int units;  // non-empty units finished on this slot
-  bool active;
-};
-
-__device__ __forceinline__ bool next_nonempty(SlotState& st, const Params& p) {
-  while (true) {
-    const int u = st.sched.next(p.num_units);
-    if (u < 0) {
-      st.active = false;
-      return false;
-    }
-    st.unit = decode_unit(p, u);
-    if (st.unit.n > 0) {
-      st.j = 0;
-      st.active = true;
-      return true;
-    }
-  }
+// kv-block index of the j-th block of the unit: partial blocks first, then full ones.
+__device__ __forceinline__ int block_index(const Params& p, const Unit& x, int j) {
+  const size_t row = static_cast<size_t>(x.qblk) * p.n_kv;
+  return j < x.np ? ldg_nc(p.kv_idx + row + j) : ldg_nc(p.full_idx + row + (j - x.np));
 }
 
 // ---------------------------------------------------------------- bounded wait
@@ -199,15 +205,36 @@ __device__ __forceinline__ bool wait_warp(Smem<D>& sm, uint64_t* bar, uint32_t p
 }
 
 // ---------------------------------------------------------------- roles
+// TMA producer: the whole warp walks the MMA warp's consumption order (per slot:
+// Q, K_0, then V_j, K_{j+1} ...; slots interleaved the way the MMA warp visits
+// them) and lane 0 issues the copies.  Block indices are fetched 32 at a time,
+// one per lane, and the first chunk of the slot's next unit is requested when
+// its current unit starts.
+struct ProdSlot {
+  UnitIter it;
+  Unit cur, nxt;
+  bool has_cur, has_nxt;
+  int j;           // block of `cur` whose V is loaded next
+  int units;       // non-empty units started on this slot
+  int chunk;       // 32-block chunk of cur's list held in `idx`
+  int idx, nxt_idx;
+};
+
+__device__ __forceinline__ int chunk_index(const Params& p, const Unit& x, int chunk, int lane) {
+  const int jj = chunk * 32 + lane;
+  return jj < x.n ? block_index(p, x, jj) : 0;
+}
+
 template <int D>
 __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
                               const CUtensorMap* tk, const CUtensorMap* tv) {
   using C = Cfg<D>;
+  const int lane = threadIdx.x & 31;
   const uint64_t pol_kv = policy_evict_last();
   const uint64_t pol_q = policy_evict_first();
-  SlotState st[kNumSlots];
+  ProdSlot st[kNumSlots];
   int kv_cnt = 0;
-  int q_armed[kNumSlots] = {};
+  int q_armed[kNumSlots][C::kQBuf] = {};
   bool ok = true;
 
   auto load_tile = [&](const CUtensorMap* map, int row0, int bh, uint8_t* dst, uint64_t* bar,
@@ -215,32 +242,60 @@ __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* t
 #pragma unroll
     for (int c = 0; c < C::kChunks; ++c) tma_load_3d(dst + c * kChunkBytes, map, bar, c * 64, row0, bh, pol);
   };
-  auto load_kv = [&](const CUtensorMap* map, SlotState& s) -> bool {
+  auto kv_block = [&](ProdSlot& s, int j) -> int {
+    const int chunk = j >> 5;
+    if (chunk != s.chunk) {
+      s.idx = chunk_index(p, s.cur, chunk, lane);
+      s.chunk = chunk;
+    }
+    return __shfl_sync(0xffffffffu, s.idx, j & 31);
+  };
+  auto load_kv = [&](const CUtensorMap* map, ProdSlot& s, int j) -> bool {
     const int stage = kv_cnt % C::kStages;
     const uint32_t phase = (kv_cnt / C::kStages) & 1;
-    if (!wait_bar(sm, &sm.kv_empty[stage], phase ^ 1, p)) return false;
-    mbar_arrive_expect_tx(&sm.kv_full[stage], C::kTileBytes);
-    bool full;
-    const int kvb = block_index(p, s.unit, s.j, full);
-    load_tile(map, kvb * kBlockN, s.unit.bh, sm.kv[stage], &sm.kv_full[stage], pol_kv);
+    const int kvb = kv_block(s, j);
+    if (!wait_warp(sm, &sm.kv_empty[stage], phase ^ 1, p)) return false;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sm.kv_full[stage], C::kTileBytes);
+      load_tile(map, kvb * kBlockN, s.cur.bh, sm.kv[stage], &sm.kv_full[stage], pol_kv);
+    }
+    __syncwarp();
     ++kv_cnt;
     return true;
   };
-  auto load_q = [&](int slot) -> bool {
-    SlotState& s = st[slot];
-    if (!wait_bar(sm, &sm.q_empty[slot], (s.units & 1) ^ 1, p)) return false;
-    mbar_arrive_expect_tx(&sm.q_full[slot], C::kTileBytes);
-    load_tile(tq, s.unit.qblk * kBlockN, s.unit.bh, sm.q[slot], &sm.q_full[slot], pol_q);
-    ++q_armed[slot];
-    return true;
+  // Make `nxt` current (its first index chunk is already in flight) and look one unit ahead.
+  auto advance = [&](ProdSlot& s) {
+    s.has_cur = s.has_nxt;
+    s.cur = s.nxt;
+    s.idx = s.nxt_idx;
+    s.chunk = 0;
+    s.j = 0;
+    s.has_nxt = s.it.pop_nonempty(s.nxt);
+    if (s.has_nxt) s.nxt_idx = chunk_index(p, s.nxt, 0, lane);
+  };
+  auto start_unit = [&](int slot) -> bool {  // Q and K_0 of the current unit
+    ProdSlot& s = st[slot];
+    const int b = s.units % C::kQBuf;
+    const uint32_t phase = (s.units / C::kQBuf) & 1;
+    if (!wait_warp(sm, &sm.q_empty[slot][b], phase ^ 1, p)) return false;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sm.q_full[slot][b], C::kTileBytes);
+      load_tile(tq, s.cur.qblk * kBlockN, s.cur.bh, sm.q[slot][b], &sm.q_full[slot][b], pol_q);
+    }
+    __syncwarp();
+    ++q_armed[slot][b];
+    ++s.units;
+    return load_kv(tk, s, 0);
   };
 
+#pragma unroll
   for (int s = 0; s < kNumSlots; ++s) {
-    st[s].sched = Sched{static_cast<int>(blockIdx.x) * kNumSlots + s,
-                        static_cast<int>(gridDim.x) * kNumSlots, 0};
+    st[s].it.init(p, s);
     st[s].units = 0;
-    q_armed[s] = 0;
-    if (ok && next_nonempty(st[s], p)) ok = load_q(s) && load_kv(tk, st[s]);
+    st[s].has_nxt = st[s].it.pop_nonempty(st[s].nxt);
+    if (st[s].has_nxt) st[s].nxt_idx = chunk_index(p, st[s].nxt, 0, lane);
+    advance(st[s]);
+    if (ok && st[s].has_cur) ok = start_unit(s);
   }
   bool any = true;
   while (ok && any) {
@@ -248,20 +303,20 @@ __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* t
 #pragma unroll
     for (int s = 0; s < kNumSlots; ++s) {
       if (!ok) break;
-      if (!st[s].active) continue;
+      if (!st[s].has_cur) continue;
       any = true;
-      ok = load_kv(tv, st[s]);
+      ok = load_kv(tv, st[s], st[s].j);
       if (!ok) break;
       ++st[s].j;
-      if (st[s].j < st[s].unit.n) {
-        ok = load_kv(tk, st[s]);
+      if (st[s].j < st[s].cur.n) {
+        ok = load_kv(tk, st[s], st[s].j);
       } else {
-        ++st[s].units;
-        if (next_nonempty(st[s], p)) ok = load_q(s) && load_kv(tk, st[s]);
+        advance(st[s]);
+        if (st[s].has_cur) ok = start_unit(s);
       }
     }
   }
-  if (!ok) {
+  if (!ok && lane == 0) {
     // Drain: wait (bounded) for every TMA copy this warp armed, so that no copy
     // lands in shared memory after the CTA has exited.
     const uint64_t t0 = globaltimer_ns();
@@ -272,14 +327,28 @@ __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* t
              globaltimer_ns() - t0 < p.timeout_ns) {
       }
     }
-    for (int s = 0; s < kNumSlots; ++s) {
-      if (q_armed[s] == 0) continue;
-      while (!mbar_try_wait(&sm.q_full[s], (q_armed[s] - 1) & 1) &&
-             globaltimer_ns() - t0 < p.timeout_ns) {
+    for (int s = 0; s < kNumSlots; ++s)
+      for (int b = 0; b < C::kQBuf; ++b) {
+        if (q_armed[s][b] == 0) continue;
+        while (!mbar_try_wait(&sm.q_full[s][b], (q_armed[s][b] - 1) & 1) &&
+               globaltimer_ns() - t0 < p.timeout_ns) {
+        }
       }
-    }
   }
+  __syncwarp();
 }
+
+// MMA issuer: one thread issues every tcgen05.mma of the CTA.  Per slot and block
+// j it issues PV_{j-1} then S_j, so each slot alternates between the tensor core
+// and its softmax warpgroup while the other slot fills the gap.
+struct MmaSlot {
+  UnitIter it;
+  Unit cur;
+  bool active;
+  int j;      // block whose PV is issued next
+  int units;  // non-empty units started on this slot
+  int blk;    // blocks finished on this slot (p_full phase)
+};
 
 template <int D>
 __device__ void mma_role(Smem<D>& sm, const Params& p, uint32_t tmem) {
@@ -287,19 +356,20 @@ __device__ void mma_role(Smem<D>& sm, const Params& p, uint32_t tmem) {
   const int lane = threadIdx.x & 31;
   const uint32_t idesc_s = idesc_f16_f32(p.is_bf16 != 0, 128, 128, false);
   const uint32_t idesc_pv = idesc_f16_f32(p.is_bf16 != 0, 128, D, true);
-  SlotState st[kNumSlots];
-  int blk[kNumSlots] = {};
+  MmaSlot st[kNumSlots];
   int kv_cnt = 0;
   bool ok = true;
 
-  auto issue_s = [&](int slot) -> bool {
-    SlotState& s = st[slot];
-    if (s.j == 0 && !wait_warp(sm, &sm.q_full[slot], s.units & 1, p)) return false;
+  auto issue_s = [&](int slot, int j) -> bool {
+    MmaSlot& s = st[slot];
+    const int b = (s.units - 1) % C::kQBuf;  // Q buffer of the current unit
+    if (j == 0 && !wait_warp(sm, &sm.q_full[slot][b], ((s.units - 1) / C::kQBuf) & 1, p))
+      return false;
     const int stage = kv_cnt % C::kStages;
     if (!wait_warp(sm, &sm.kv_full[stage], (kv_cnt / C::kStages) & 1, p)) return false;
     tc_fence_after();
     if (lane == 0) {
-      const uint32_t qa = smem_u32(sm.q[slot]);
+      const uint32_t qa = smem_u32(sm.q[slot][b]);
       const uint32_t ka = smem_u32(sm.kv[stage]);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
@@ -309,16 +379,17 @@ __device__ void mma_role(Smem<D>& sm, const Params& p, uint32_t tmem) {
       }
       umma_commit(&sm.kv_empty[stage]);
       umma_commit(&sm.s_full[slot]);
-      if (s.j == s.unit.n - 1) umma_commit(&sm.q_empty[slot]);
+      if (j == s.cur.n - 1) umma_commit(&sm.q_empty[slot][b]);
     }
     __syncwarp();
     ++kv_cnt;
     return true;
   };
   auto issue_pv = [&](int slot) -> bool {
-    SlotState& s = st[slot];
-    if (!wait_warp(sm, &sm.p_full[slot], blk[slot] & 1, p)) return false;
-    if (s.j == 0 && !wait_warp(sm, &sm.o_empty[slot], (s.units & 1) ^ 1, p)) return false;
+    MmaSlot& s = st[slot];
+    if (!wait_warp(sm, &sm.p_full[slot], s.blk & 1, p)) return false;
+    // O of this slot is free once the epilogue of its previous unit has read it
+    if (s.j == 0 && !wait_warp(sm, &sm.o_empty[slot], ((s.units - 1) & 1) ^ 1, p)) return false;
     const int stage = kv_cnt % C::kStages;
     if (!wait_warp(sm, &sm.kv_full[stage], (kv_cnt / C::kStages) & 1, p)) return false;
     tc_fence_after();
@@ -330,21 +401,35 @@ __device__ void mma_role(Smem<D>& sm, const Params& p, uint32_t tmem) {
                 sdesc_sw128(va + kk * 2048, kChunkBytes, 1024), idesc_pv,
                 (s.j > 0 || kk > 0) ? 1u : 0u);
       }
+      if (p.split_p) {
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk)
+          umma_ts(tmem + C::o_col(slot), tmem + C::s_col(slot) + 64 + kk * 8,
+                  sdesc_sw128(va + kk * 2048, kChunkBytes, 1024), idesc_pv, 1u);
+      }
       umma_commit(&sm.kv_empty[stage]);
-      if (s.j == s.unit.n - 1) umma_commit(&sm.o_full[slot]);
+      if (s.j == s.cur.n - 1) umma_commit(&sm.o_full[slot]);
     }
     __syncwarp();
     ++kv_cnt;
-    ++blk[slot];
+    ++s.blk;
     return true;
   };
+  auto start_unit = [&](int slot) -> bool {
+    MmaSlot& s = st[slot];
+    s.active = s.it.pop_nonempty(s.cur);
+    if (!s.active) return true;
+    s.j = 0;
+    ++s.units;
+    return issue_s(slot, 0);
+  };
 
+#pragma unroll
   for (int s = 0; s < kNumSlots; ++s) {
-    st[s].sched = Sched{static_cast<int>(blockIdx.x) * kNumSlots + s,
-                        static_cast<int>(gridDim.x) * kNumSlots, 0};
+    st[s].it.init(p, s);
     st[s].units = 0;
-    blk[s] = 0;
-    if (ok && next_nonempty(st[s], p)) ok = issue_s(s);
+    st[s].blk = 0;
+    if (ok) ok = start_unit(s);
   }
   bool any = true;
   while (ok && any) {
@@ -357,12 +442,7 @@ __device__ void mma_role(Smem<D>& sm, const Params& p, uint32_t tmem) {
       ok = issue_pv(s);
       if (!ok) break;
       ++st[s].j;
-      if (st[s].j < st[s].unit.n) {
-        ok = issue_s(s);
-      } else {
-        ++st[s].units;
-        if (next_nonempty(st[s], p)) ok = issue_s(s);
-      }
+      ok = st[s].j < st[s].cur.n ? issue_s(s, st[s].j) : start_unit(s);
     }
   }
   if (!ok) {
@@ -384,6 +464,19 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi, bool bf16) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ void unpack2(uint32_t v, bool bf16, float& lo, float& hi) {
+  if (bf16) {
+    lo = __uint_as_float(v << 16);
+    hi = __uint_as_float(v & 0xFFFF0000u);
+  } else {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&v));
+    lo = f.x;
+    hi = f.y;
+  }
+}
+
+// Softmax warpgroup of one slot: thread t owns row t of the slot's 128-row tile
+// (TMEM lane t), so row max and row sum need no shuffles.
 template <int D>
 __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int slot) {
   using C = Cfg<D>;
@@ -393,14 +486,15 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
   const uint32_t t_s = tmem + C::s_col(slot) + lane_off;
   const uint32_t t_o = tmem + C::o_col(slot) + lane_off;
   const bool bf16 = p.is_bf16 != 0;
-  Sched sched{static_cast<int>(blockIdx.x) * kNumSlots + slot,
-              static_cast<int>(gridDim.x) * kNumSlots, 0};
+  // Factor that turns the value kept in x[] into log2 units: the raw score is
+  // kept (and scaled inside the exponent's FFMA) unless a score_mod rewrote it.
+  const float xs = p.softcap_on ? 1.f : p.scale_log2;
+  UnitIter it;
+  it.init(p, slot);
   int blk = 0, units = 0;
+  Unit un;
 
-  while (true) {
-    const int u = sched.next(p.num_units);
-    if (u < 0) break;
-    const Unit un = decode_unit(p, u);
+  while (it.pop(un)) {
     const int row = un.qblk * kBlockN + t;
     const bool valid = row < p.L;
     const size_t orow = static_cast<size_t>(un.bh) * p.L + row;
@@ -417,11 +511,12 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
     // live keys of this row: kv in [lo, hi] (and, for documents, doc_id[kv] == dq)
     const int hi = min(row, p.S - 1);
     const int lo = p.mask_kind == FA_MASK_SLIDING_WINDOW_CAUSAL ? max(row - p.window + 1, 0) : 0;
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f;  // running max (log2 units) and running sum
+    int kvb = block_index(p, un, 0);
 
     for (int j = 0; j < un.n; ++j) {
-      bool full;
-      const int kvb = block_index(p, un, j, full);
+      const bool full = j >= un.np;
+      const int kvb_next = j + 1 < un.n ? block_index(p, un, j + 1) : 0;
       if (!wait_warp(sm, &sm.s_full[slot], blk & 1, p)) return;
       tc_fence_after();
       float x[128];
@@ -434,16 +529,12 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
 #pragma unroll
         for (int i = 0; i < 128; ++i) x[i] = __uint_as_float(xr[i]);
       }
-      // scores in log2 units: x = log2(e) * score_mod(s * scale)
-      if (p.softcap_on) {
+      if (p.softcap_on) {  // x = log2(e) * c * tanh(s * scale / c)
 #pragma unroll
         for (int i = 0; i < 128; ++i) {
           const float e = ex2_approx(x[i] * p.cap_k);            // e^(2y), y = s * scale / c
           x[i] = p.cap_a - 2.f * p.cap_a * rcp_approx(e + 1.f);  // c * log2(e) * tanh(y)
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) x[i] *= p.scale_log2;
       }
       if (!full) {  // PARTIAL block: evaluate the mask rule per element
         const int a = lo - kvb * kBlockN;  // live columns: a <= i <= b
@@ -472,10 +563,17 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
             if (i < a || i > b) x[i] = -INFINITY;
         }
       }
-      float mb = x[0];
+      // row max: 16 independent chains, then a tree
+      float mx[16];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mb = fmaxf(mb, x[i]);
-      const float m_new = fmaxf(m, mb);
+      for (int i = 0; i < 16; ++i) mx[i] = x[i];
+#pragma unroll
+      for (int i = 16; i < 128; ++i) mx[i & 15] = fmaxf(mx[i & 15], x[i]);
+#pragma unroll
+      for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+      const float m_new = fmaxf(m, mx[0] * xs);
       // Deferred rescale: keep the stale max unless the new one exceeds it by more
       // than 2^8; exact, because l and O always use the same max.
       float alpha = 1.f;
@@ -488,21 +586,34 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         }
         m = m_new;
       }
-      const float mu = (m == -INFINITY) ? 0.f : m;
-      float sum = 0.f;
+      const float neg_mu = (m == -INFINITY) ? 0.f : -m;
+      // P = exp2(x * xs - m) as 16-bit pairs: P_hi = round(p) over S columns 0-63 and,
+      // when split, P_lo = round(p - P_hi) over columns 64-127 (both PV products are
+      // accumulated, so P carries ~16 significant bits instead of 8).
+      float sums[8];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[32];
+      for (int i = 0; i < 8; ++i) sums[i] = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(x[c * 64 + 2 * i] - mu);
-          const float p1 = ex2_approx(x[c * 64 + 2 * i + 1] - mu);
-          sum += p0 + p1;
-          pk[i] = pack2(p0, p1, bf16);
+      for (int c = 0; c < 4; ++c) {
+        uint32_t ph[16], pl[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2_approx(fmaf(x[c * 32 + 2 * i], xs, neg_mu));
+          const float p1 = ex2_approx(fmaf(x[c * 32 + 2 * i + 1], xs, neg_mu));
+          sums[i & 7] += p0 + p1;
+          ph[i] = pack2(p0, p1, bf16);
+          float h0, h1;
+          unpack2(ph[i], bf16, h0, h1);
+          pl[i] = pack2(p0 - h0, p1 - h1, bf16);
         }
-        tmem_st32(t_s + c * 32, pk);  // P (16-bit pairs) over the first 64 S columns
+        tmem_st16(t_s + c * 16, ph);
+        if (p.split_p) tmem_st16(t_s + 64 + c * 16, pl);
       }
-      l += sum;
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) sums[i] += sums[i + w];
+      l += sums[0];
       if (__any_sync(0xffffffffu, rescale_o)) {
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
@@ -518,6 +629,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
       tc_fence_before();
       mbar_arrive(&sm.p_full[slot]);
       ++blk;
+      kvb = kvb_next;
     }
 
     // epilogue: O / l -> out, LSE
@@ -557,8 +669,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kNumSlots; ++s) {
-      mbar_init(&sm.q_full[s], 1);
-      mbar_init(&sm.q_empty[s], 1);
+      for (int b = 0; b < Cfg<D>::kQBuf; ++b) {
+        mbar_init(&sm.q_full[s][b], 1);
+        mbar_init(&sm.q_empty[s][b], 1);
+      }
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.p_full[s], 128);
       mbar_init(&sm.o_full[s], 1);
@@ -597,7 +711,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
   }
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == kProducerWarp) {
-    if ((threadIdx.x & 31) == 0) producer_role<D>(sm, p, &tmap_q, &tmap_k, &tmap_v);
+    producer_role<D>(sm, p, &tmap_q, &tmap_k, &tmap_v);
   } else if (warp == kMmaWarp) {
     mma_role<D>(sm, p, tmem);
   }
@@ -713,11 +827,9 @@ extern "C" fa_status fa_flex_attention_fwd(const void* q, const void* k, const v
 
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
   Params prm{};
-  prm.kv_num = bm->kv_num_blocks;
   prm.kv_idx = bm->kv_indices;
-  prm.full_num = bm->full_kv_num_blocks;
   prm.full_idx = bm->full_kv_indices;
-  prm.q_order = bm->q_order;
+  prm.sched = bm->q_order;
   prm.doc_id = bm->doc_id;
   prm.out = out;
   prm.lse = lse;
@@ -734,6 +846,7 @@ extern "C" fa_status fa_flex_attention_fwd(const void* q, const void* k, const v
   prm.scale_log2 = sc * kLog2e;
   prm.cap_k = prm.softcap_on ? 2.f * sc * kLog2e / softcap : 0.f;
   prm.cap_a = prm.softcap_on ? softcap * kLog2e : 0.f;
+  prm.split_p = 1;
   prm.timeout_ns = 2000000000ull;
   const cudaStream_t s = as_stream(stream);
   if (D == 64) return launch<64>(q, k, v, dtype == FA_BF16, prm.BH, L, S, prm, s);

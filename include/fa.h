@@ -79,7 +79,7 @@ typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
 /*
  * Block tables of one mask, broadcast over batch and heads.
  *
- * The caller allocates the five arrays on the device and stores their pointers
+ * The caller allocates the five arrays on the device (8-byte aligned) and stores their pointers
  * here BEFORE calling fa_create_block_mask, which fills both the arrays and the
  * scalar fields.  Sizes: nQ = ceil(q_len / 128), nKV = ceil(kv_len / 128)
  * (fa_block_mask_dims computes them).
@@ -88,9 +88,11 @@ typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
  *   kv_indices[nQ * nKV]        row i: its partial kv-block indices, ascending, then 0s
  *   full_kv_num_blocks[nQ]      number of FULL blocks of row i
  *   full_kv_indices[nQ * nKV]   row i: its full kv-block indices, ascending, then 0s
- *   q_order[nQ]                 q-block rows sorted by descending live-block count
- *                               (ties by ascending row): the order in which the forward
- *                               kernel's persistent scheduler hands out work
+ *   q_order[2 * nQ]             the forward kernel's schedule: rank k lists the q-block
+ *                               rows by descending live-block count (ties by ascending
+ *                               row); q_order[2k] = row, q_order[2k+1] = its partial
+ *                               count | full count << 16.  The persistent scheduler hands
+ *                               out work in this order (heaviest rows first).
  *
  * A FULL block has all 128 x 128 pairs in range and allowed (the kernel skips the
  * mask there); a PARTIAL block has some but not all pairs live (the kernel evaluates

@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 import tempfile
 
 import pytest
@@ -17,8 +18,8 @@ HEADER = os.path.join(ROOT, "include", "fa.h")
 def fa():
     from block_sparse_attention_create_b200 import build
     build.build()
-    import block_sparse_attention_create_b200 as m
-    return m
+    from block_sparse_attention_create_b200 import _binding
+    return _binding
 
 
 def declared_symbols():
@@ -144,6 +145,19 @@ def test_fwd_rejects_bad_arguments_on_host(fa):
 
 def test_workspace_size(fa):
     assert fa.fa_fwd_workspace_bytes() >= 4
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """With libfa.so absent the binding raises instead of falling back."""
+    import shutil
+    pkg = os.path.join(ROOT, "block_sparse_attention_create_b200")
+    dst = tmp_path / "block_sparse_attention_create_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "_build", "__pycache__"))
+    code = ("import sys; sys.path.insert(0, %r); import block_sparse_attention_create_b200 as fa\n"
+            "try:\n    fa.flex_attention\nexcept ImportError as e:\n    print('raised', e)\n"
+            % str(tmp_path))
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True)
+    assert "raised" in out.stdout and "libfa.so is missing" in out.stdout, out.stdout + out.stderr
 
 
 def test_product_never_imports_the_oracle():

@@ -23,12 +23,16 @@ def _check(kind, L, S, window=0, doc=None):
     ref = OB.block_tables(kind, L, S, window or None, None if doc is None else doc.numpy())
     for key in ("kv_num_blocks", "kv_indices", "full_kv_num_blocks", "full_kv_indices"):
         assert np.array_equal(got[key].reshape(ref[key].shape), ref[key]), key
-    # q_order: a permutation of the rows, by descending live count, ties ascending
+    # schedule: a permutation of the rows, by descending live count, ties ascending,
+    # each with its partial / full counts
     cnt = ref["kv_num_blocks"] + ref["full_kv_num_blocks"]
-    order = got["q_order"]
+    order = got["q_order"][0::2]
+    packed = got["q_order"][1::2]
     assert sorted(order.tolist()) == list(range(len(cnt)))
     keys = [(-int(cnt[i]), int(i)) for i in order]
     assert keys == sorted(keys)
+    assert np.array_equal(packed & 0xFFFF, ref["kv_num_blocks"][order])
+    assert np.array_equal(packed >> 16, ref["full_kv_num_blocks"][order])
 
 
 @pytest.mark.parametrize("w", W.ALL, ids=lambda w: w.name)
