@@ -62,6 +62,13 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: O is rescaled only when max grows > 2^8
 
+// TMEM layouts (512 columns, lanes = the 128 rows of a tile):
+//  D = 64  ("separate P"): S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384)
+//          O0 [384,448) O1 [448,512).  The softmax frees S as soon as it has read
+//          it, so S_{j+1} is computed on the tensor core while softmax j runs.
+//  D = 128 ("aliased P"):  S0/P0 [0,128) S1/P1 [128,256) O0 [256,384) O1 [384,512).
+//          P overwrites the S it came from (hi in columns 0-63, lo in 64-127), so
+//          S_{j+1} waits for PV_j; the other slot covers that gap.
 template <int D>
 struct Cfg {
   static constexpr int kChunks = D / 64;
@@ -69,9 +76,15 @@ struct Cfg {
   static constexpr int kStages = (D == 64) ? 8 : 4;
   // Q tiles per slot: two at D=64, so the next unit's Q loads while this one runs.
   static constexpr int kQBuf = (D == 64) ? 2 : 1;
+  static constexpr bool kSepP = (D == 64);
   static constexpr uint32_t kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t s_col(int slot) { return 128u * slot; }
-  __host__ __device__ static constexpr uint32_t o_col(int slot) { return 256u + static_cast<uint32_t>(D) * slot; }
+  __host__ __device__ static constexpr uint32_t p_col(int slot) {
+    return kSepP ? 256u + 64u * slot : 128u * slot;
+  }
+  __host__ __device__ static constexpr uint32_t o_col(int slot) {
+    return kSepP ? 384u + 64u * slot : 256u + static_cast<uint32_t>(D) * slot;
+  }
 };
 
 template <int D>
@@ -81,7 +94,9 @@ struct __align__(1024) Smem {
   uint64_t q_full[kNumSlots][Cfg<D>::kQBuf];
   uint64_t q_empty[kNumSlots][Cfg<D>::kQBuf];
   uint64_t s_full[kNumSlots];
+  uint64_t s_empty[kNumSlots];  // separate-P layout: softmax has read S
   uint64_t p_full[kNumSlots];
+  uint64_t pv_done[kNumSlots];  // separate-P layout: PV_j finished (P buffer and O stable)
   uint64_t o_full[kNumSlots];
   uint64_t o_empty[kNumSlots];
   uint64_t kv_full[Cfg<D>::kStages];
@@ -204,20 +219,39 @@ __device__ __forceinline__ bool wait_warp(Smem<D>& sm, uint64_t* bar, uint32_t p
   return __all_sync(0xffffffffu, wait_bar(sm, bar, parity, p));
 }
 
+// Wait polled by lane 0 only (the lane elect_one_sync picks in a converged warp);
+// the outcome is broadcast to the warp.  For the producer and MMA warps, whose
+// dependent work is issued by that lane.
+template <int D>
+__device__ __forceinline__ bool wait_lane0(Smem<D>& sm, uint64_t* bar, uint32_t parity, const Params& p) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(sm, bar, parity, p);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
 // ---------------------------------------------------------------- roles
+// The producer and the MMA warp keep one state record per slot.  Every function
+// that touches a slot's record takes the slot as a template parameter, so the
+// records live in registers (a runtime slot index would put them in local memory).
+
 // TMA producer: the whole warp walks the MMA warp's consumption order (per slot:
 // Q, K_0, then V_j, K_{j+1} ...; slots interleaved the way the MMA warp visits
-// them) and lane 0 issues the copies.  Block indices are fetched 32 at a time,
-// one per lane, and the first chunk of the slot's next unit is requested when
-// its current unit starts.
+// them) and one elected lane issues the copies.  Block indices are fetched 32 at
+// a time, one per lane, and the first chunk of the slot's next unit is requested
+// when its current unit starts.
 struct ProdSlot {
   UnitIter it;
   Unit cur, nxt;
   bool has_cur, has_nxt;
-  int j;           // block of `cur` whose V is loaded next
-  int units;       // non-empty units started on this slot
-  int chunk;       // 32-block chunk of cur's list held in `idx`
+  int j;      // block of `cur` whose V is loaded next
+  int units;  // non-empty units started on this slot
+  int chunk;  // 32-block chunk of cur's list held in `idx`
   int idx, nxt_idx;
+};
+
+struct ProdShared {
+  int kv_cnt;  // tiles issued into the K/V ring (both slots)
+  uint64_t pol_kv, pol_q;
 };
 
 __device__ __forceinline__ int chunk_index(const Params& p, const Unit& x, int chunk, int lane) {
@@ -226,121 +260,136 @@ __device__ __forceinline__ int chunk_index(const Params& p, const Unit& x, int c
 }
 
 template <int D>
+__device__ __forceinline__ void load_tile(const CUtensorMap* map, int row0, int bh, uint8_t* dst,
+                                          uint64_t* bar, uint64_t pol) {
+#pragma unroll
+  for (int c = 0; c < Cfg<D>::kChunks; ++c)
+    tma_load_3d(dst + c * kChunkBytes, map, bar, c * 64, row0, bh, pol);
+}
+
+template <int D>
+__device__ __forceinline__ bool prod_load_kv(Smem<D>& sm, const Params& p, const CUtensorMap* map,
+                                             ProdSlot& s, int j, ProdShared& ps, int lane) {
+  using C = Cfg<D>;
+  const int stage = ps.kv_cnt % C::kStages;
+  const uint32_t phase = (ps.kv_cnt / C::kStages) & 1;
+  const int chunk = j >> 5;
+  if (chunk != s.chunk) {
+    s.idx = chunk_index(p, s.cur, chunk, lane);
+    s.chunk = chunk;
+  }
+  const int kvb = __shfl_sync(0xffffffffu, s.idx, j & 31);
+  if (!wait_lane0(sm, &sm.kv_empty[stage], phase ^ 1, p)) return false;
+  if (elect_one_sync()) {
+    mbar_arrive_expect_tx(&sm.kv_full[stage], C::kTileBytes);
+    load_tile<D>(map, kvb * kBlockN, s.cur.bh, sm.kv[stage], &sm.kv_full[stage], ps.pol_kv);
+  }
+  __syncwarp();
+  ++ps.kv_cnt;
+  return true;
+}
+
+// Make `nxt` current (its first index chunk is already in flight) and look one unit ahead.
+__device__ __forceinline__ void prod_advance(ProdSlot& s, const Params& p, int lane) {
+  s.has_cur = s.has_nxt;
+  s.cur = s.nxt;
+  s.idx = s.nxt_idx;
+  s.chunk = 0;
+  s.j = 0;
+  s.has_nxt = s.it.pop_nonempty(s.nxt);
+  if (s.has_nxt) s.nxt_idx = chunk_index(p, s.nxt, 0, lane);
+}
+
+// Q and K_0 of the slot's current unit.
+template <int D, int SLOT>
+__device__ __forceinline__ bool prod_start_unit(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
+                                                const CUtensorMap* tk, ProdSlot& s, ProdShared& ps,
+                                                int lane) {
+  using C = Cfg<D>;
+  const int b = s.units % C::kQBuf;
+  const uint32_t phase = (s.units / C::kQBuf) & 1;
+  if (!wait_lane0(sm, &sm.q_empty[SLOT][b], phase ^ 1, p)) return false;
+  if (elect_one_sync()) {
+    mbar_arrive_expect_tx(&sm.q_full[SLOT][b], C::kTileBytes);
+    load_tile<D>(tq, s.cur.qblk * kBlockN, s.cur.bh, sm.q[SLOT][b], &sm.q_full[SLOT][b], ps.pol_q);
+  }
+  __syncwarp();
+  ++s.units;
+  return prod_load_kv<D>(sm, p, tk, s, 0, ps, lane);
+}
+
+template <int D, int SLOT>
+__device__ __forceinline__ bool prod_init(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
+                                          const CUtensorMap* tk, ProdSlot& s, ProdShared& ps, int lane) {
+  s.it.init(p, SLOT);
+  s.units = 0;
+  s.has_nxt = s.it.pop_nonempty(s.nxt);
+  if (s.has_nxt) s.nxt_idx = chunk_index(p, s.nxt, 0, lane);
+  prod_advance(s, p, lane);
+  return s.has_cur ? prod_start_unit<D, SLOT>(sm, p, tq, tk, s, ps, lane) : true;
+}
+
+// V_j of the current block, then K_{j+1} (or the next unit's Q and K_0).
+template <int D, int SLOT>
+__device__ __forceinline__ bool prod_step(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
+                                          const CUtensorMap* tk, const CUtensorMap* tv, ProdSlot& s,
+                                          ProdShared& ps, int lane, bool& any) {
+  if (!s.has_cur) return true;
+  any = true;
+  if (!prod_load_kv<D>(sm, p, tv, s, s.j, ps, lane)) return false;
+  ++s.j;
+  if (s.j < s.cur.n) return prod_load_kv<D>(sm, p, tk, s, s.j, ps, lane);
+  prod_advance(s, p, lane);
+  return s.has_cur ? prod_start_unit<D, SLOT>(sm, p, tq, tk, s, ps, lane) : true;
+}
+
+template <int D>
 __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
                               const CUtensorMap* tk, const CUtensorMap* tv) {
   using C = Cfg<D>;
+  static_assert(kNumSlots == 2, "the producer loop visits two slots");
   const int lane = threadIdx.x & 31;
-  const uint64_t pol_kv = policy_evict_last();
-  const uint64_t pol_q = policy_evict_first();
-  ProdSlot st[kNumSlots];
-  int kv_cnt = 0;
-  int q_armed[kNumSlots][C::kQBuf] = {};
-  bool ok = true;
-
-  auto load_tile = [&](const CUtensorMap* map, int row0, int bh, uint8_t* dst, uint64_t* bar,
-                       uint64_t pol) {
-#pragma unroll
-    for (int c = 0; c < C::kChunks; ++c) tma_load_3d(dst + c * kChunkBytes, map, bar, c * 64, row0, bh, pol);
-  };
-  auto kv_block = [&](ProdSlot& s, int j) -> int {
-    const int chunk = j >> 5;
-    if (chunk != s.chunk) {
-      s.idx = chunk_index(p, s.cur, chunk, lane);
-      s.chunk = chunk;
-    }
-    return __shfl_sync(0xffffffffu, s.idx, j & 31);
-  };
-  auto load_kv = [&](const CUtensorMap* map, ProdSlot& s, int j) -> bool {
-    const int stage = kv_cnt % C::kStages;
-    const uint32_t phase = (kv_cnt / C::kStages) & 1;
-    const int kvb = kv_block(s, j);
-    if (!wait_warp(sm, &sm.kv_empty[stage], phase ^ 1, p)) return false;
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&sm.kv_full[stage], C::kTileBytes);
-      load_tile(map, kvb * kBlockN, s.cur.bh, sm.kv[stage], &sm.kv_full[stage], pol_kv);
-    }
-    __syncwarp();
-    ++kv_cnt;
-    return true;
-  };
-  // Make `nxt` current (its first index chunk is already in flight) and look one unit ahead.
-  auto advance = [&](ProdSlot& s) {
-    s.has_cur = s.has_nxt;
-    s.cur = s.nxt;
-    s.idx = s.nxt_idx;
-    s.chunk = 0;
-    s.j = 0;
-    s.has_nxt = s.it.pop_nonempty(s.nxt);
-    if (s.has_nxt) s.nxt_idx = chunk_index(p, s.nxt, 0, lane);
-  };
-  auto start_unit = [&](int slot) -> bool {  // Q and K_0 of the current unit
-    ProdSlot& s = st[slot];
-    const int b = s.units % C::kQBuf;
-    const uint32_t phase = (s.units / C::kQBuf) & 1;
-    if (!wait_warp(sm, &sm.q_empty[slot][b], phase ^ 1, p)) return false;
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&sm.q_full[slot][b], C::kTileBytes);
-      load_tile(tq, s.cur.qblk * kBlockN, s.cur.bh, sm.q[slot][b], &sm.q_full[slot][b], pol_q);
-    }
-    __syncwarp();
-    ++q_armed[slot][b];
-    ++s.units;
-    return load_kv(tk, s, 0);
-  };
-
-#pragma unroll
-  for (int s = 0; s < kNumSlots; ++s) {
-    st[s].it.init(p, s);
-    st[s].units = 0;
-    st[s].has_nxt = st[s].it.pop_nonempty(st[s].nxt);
-    if (st[s].has_nxt) st[s].nxt_idx = chunk_index(p, st[s].nxt, 0, lane);
-    advance(st[s]);
-    if (ok && st[s].has_cur) ok = start_unit(s);
-  }
+  ProdShared ps;
+  ps.kv_cnt = 0;
+  ps.pol_kv = policy_evict_last();
+  ps.pol_q = policy_evict_first();
+  ProdSlot s0, s1;
+  bool ok = prod_init<D, 0>(sm, p, tq, tk, s0, ps, lane);
+  if (ok) ok = prod_init<D, 1>(sm, p, tq, tk, s1, ps, lane);
   bool any = true;
   while (ok && any) {
     any = false;
-#pragma unroll
-    for (int s = 0; s < kNumSlots; ++s) {
-      if (!ok) break;
-      if (!st[s].has_cur) continue;
-      any = true;
-      ok = load_kv(tv, st[s], st[s].j);
-      if (!ok) break;
-      ++st[s].j;
-      if (st[s].j < st[s].cur.n) {
-        ok = load_kv(tk, st[s], st[s].j);
-      } else {
-        advance(st[s]);
-        if (st[s].has_cur) ok = start_unit(s);
-      }
-    }
+    ok = prod_step<D, 0>(sm, p, tq, tk, tv, s0, ps, lane, any);
+    if (ok) ok = prod_step<D, 1>(sm, p, tq, tk, tv, s1, ps, lane, any);
   }
-  if (!ok && lane == 0) {
+  if (!ok && elect_one_sync()) {
     // Drain: wait (bounded) for every TMA copy this warp armed, so that no copy
     // lands in shared memory after the CTA has exited.
     const uint64_t t0 = globaltimer_ns();
     for (int stage = 0; stage < C::kStages; ++stage) {
-      const int fills = kv_cnt / C::kStages + (stage < kv_cnt % C::kStages ? 1 : 0);
+      const int fills = ps.kv_cnt / C::kStages + (stage < ps.kv_cnt % C::kStages ? 1 : 0);
       if (fills == 0) continue;
       while (!mbar_try_wait(&sm.kv_full[stage], (fills - 1) & 1) &&
              globaltimer_ns() - t0 < p.timeout_ns) {
       }
     }
-    for (int s = 0; s < kNumSlots; ++s)
+    for (int slot = 0; slot < kNumSlots; ++slot) {
+      const int units = slot == 0 ? s0.units : s1.units;
       for (int b = 0; b < C::kQBuf; ++b) {
-        if (q_armed[s][b] == 0) continue;
-        while (!mbar_try_wait(&sm.q_full[s][b], (q_armed[s][b] - 1) & 1) &&
+        const int fills = units > b ? (units - 1 - b) / C::kQBuf + 1 : 0;
+        if (fills == 0) continue;
+        while (!mbar_try_wait(&sm.q_full[slot][b], (fills - 1) & 1) &&
                globaltimer_ns() - t0 < p.timeout_ns) {
         }
       }
+    }
   }
   __syncwarp();
 }
 
-// MMA issuer: one thread issues every tcgen05.mma of the CTA.  Per slot and block
-// j it issues PV_{j-1} then S_j, so each slot alternates between the tensor core
-// and its softmax warpgroup while the other slot fills the gap.
+// MMA issuer: one elected thread issues every tcgen05.mma of the CTA.  Per slot and
+// block j it issues PV_{j-1} then S_j, so each slot alternates between the tensor
+// core and its softmax warpgroup while the other slot fills the gap.
 struct MmaSlot {
   UnitIter it;
   Unit cur;
@@ -350,104 +399,421 @@ struct MmaSlot {
   int blk;    // blocks finished on this slot (p_full phase)
 };
 
+struct MmaShared {
+  int kv_cnt;
+  uint32_t tmem, idesc_s, idesc_pv;
+  bool split;
+};
+
+template <int D, int SLOT>
+__device__ __forceinline__ bool mma_issue_s(Smem<D>& sm, const Params& p, MmaSlot& s, int j,
+                                            MmaShared& ms) {
+  using C = Cfg<D>;
+  const int b = (s.units - 1) % C::kQBuf;  // Q buffer of the current unit
+  if (j == 0 && !wait_lane0(sm, &sm.q_full[SLOT][b], ((s.units - 1) / C::kQBuf) & 1, p)) return false;
+  const int stage = ms.kv_cnt % C::kStages;
+  if (!wait_lane0(sm, &sm.kv_full[stage], (ms.kv_cnt / C::kStages) & 1, p)) return false;
+  tc_fence_after();
+  // descriptors are warp-uniform: computed by every lane, issued by one
+  const uint64_t qd = sdesc_sw128(smem_u32(sm.q[SLOT][b]), 16, 1024);
+  const uint64_t kd = sdesc_sw128(smem_u32(sm.kv[stage]), 16, 1024);
+  const uint32_t d_s = ms.tmem + C::s_col(SLOT);
+  const bool last = j == s.cur.n - 1;
+  if (elect_one_sync()) {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      // K step kk: 32 bytes into the 128-byte swizzled row, chunk kk / 4
+      const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+      umma_ss(d_s, qd + off, kd + off, ms.idesc_s, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&sm.kv_empty[stage]);
+    umma_commit(&sm.s_full[SLOT]);
+    if (last) umma_commit(&sm.q_empty[SLOT][b]);
+  }
+  __syncwarp();
+  ++ms.kv_cnt;
+  return true;
+}
+
+template <int D, int SLOT>
+__device__ __forceinline__ bool mma_issue_pv(Smem<D>& sm, const Params& p, MmaSlot& s, MmaShared& ms) {
+  using C = Cfg<D>;
+  if (!wait_lane0(sm, &sm.p_full[SLOT], s.blk & 1, p)) return false;
+  // O of this slot is free once the epilogue of its previous unit has read it
+  if (s.j == 0 && !wait_lane0(sm, &sm.o_empty[SLOT], ((s.units - 1) & 1) ^ 1, p)) return false;
+  const int stage = ms.kv_cnt % C::kStages;
+  if (!wait_lane0(sm, &sm.kv_full[stage], (ms.kv_cnt / C::kStages) & 1, p)) return false;
+  tc_fence_after();
+  const uint64_t vd = sdesc_sw128(smem_u32(sm.kv[stage]), kChunkBytes, 1024);
+  const uint32_t d_o = ms.tmem + C::o_col(SLOT);
+  const uint32_t a_p = ms.tmem + C::s_col(SLOT);
+  const uint32_t acc0 = s.j > 0 ? 1u : 0u;
+  const bool last = s.j == s.cur.n - 1;
+  if (elect_one_sync()) {
+    // K step kk covers 16 rows of V (2048 bytes, two 8-row swizzle atoms)
+#pragma unroll
+    for (int kk = 0; kk < kBlockN / 16; ++kk)
+      umma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * 128), ms.idesc_pv,
+              kk > 0 ? 1u : acc0);
+    if (ms.split) {
+#pragma unroll
+      for (int kk = 0; kk < kBlockN / 16; ++kk)
+        umma_ts(d_o, a_p + 64 + kk * 8, vd + static_cast<uint64_t>(kk * 128), ms.idesc_pv, 1u);
+    }
+    umma_commit(&sm.kv_empty[stage]);
+    if (last) umma_commit(&sm.o_full[SLOT]);
+  }
+  __syncwarp();
+  ++ms.kv_cnt;
+  ++s.blk;
+  return true;
+}
+
+template <int D, int SLOT>
+__device__ __forceinline__ bool mma_start_unit(Smem<D>& sm, const Params& p, MmaSlot& s, MmaShared& ms) {
+  s.active = s.it.pop_nonempty(s.cur);
+  if (!s.active) return true;
+  s.j = 0;
+  ++s.units;
+  return mma_issue_s<D, SLOT>(sm, p, s, 0, ms);
+}
+
+template <int D, int SLOT>
+__device__ __forceinline__ bool mma_step(Smem<D>& sm, const Params& p, MmaSlot& s, MmaShared& ms,
+                                         bool& any) {
+  if (!s.active) return true;
+  any = true;
+  if (!mma_issue_pv<D, SLOT>(sm, p, s, ms)) return false;
+  ++s.j;
+  return s.j < s.cur.n ? mma_issue_s<D, SLOT>(sm, p, s, s.j, ms)
+                       : mma_start_unit<D, SLOT>(sm, p, s, ms);
+}
+
 template <int D>
 __device__ void mma_role(Smem<D>& sm, const Params& p, uint32_t tmem) {
-  using C = Cfg<D>;
-  const int lane = threadIdx.x & 31;
-  const uint32_t idesc_s = idesc_f16_f32(p.is_bf16 != 0, 128, 128, false);
-  const uint32_t idesc_pv = idesc_f16_f32(p.is_bf16 != 0, 128, D, true);
-  MmaSlot st[kNumSlots];
-  int kv_cnt = 0;
-  bool ok = true;
-
-  auto issue_s = [&](int slot, int j) -> bool {
-    MmaSlot& s = st[slot];
-    const int b = (s.units - 1) % C::kQBuf;  // Q buffer of the current unit
-    if (j == 0 && !wait_warp(sm, &sm.q_full[slot][b], ((s.units - 1) / C::kQBuf) & 1, p))
-      return false;
-    const int stage = kv_cnt % C::kStages;
-    if (!wait_warp(sm, &sm.kv_full[stage], (kv_cnt / C::kStages) & 1, p)) return false;
-    tc_fence_after();
-    if (lane == 0) {
-      const uint32_t qa = smem_u32(sm.q[slot][b]);
-      const uint32_t ka = smem_u32(sm.kv[stage]);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-        umma_ss(tmem + C::s_col(slot), sdesc_sw128(qa + off, 16, 1024),
-                sdesc_sw128(ka + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-      }
-      umma_commit(&sm.kv_empty[stage]);
-      umma_commit(&sm.s_full[slot]);
-      if (j == s.cur.n - 1) umma_commit(&sm.q_empty[slot][b]);
-    }
-    __syncwarp();
-    ++kv_cnt;
-    return true;
-  };
-  auto issue_pv = [&](int slot) -> bool {
-    MmaSlot& s = st[slot];
-    if (!wait_warp(sm, &sm.p_full[slot], s.blk & 1, p)) return false;
-    // O of this slot is free once the epilogue of its previous unit has read it
-    if (s.j == 0 && !wait_warp(sm, &sm.o_empty[slot], ((s.units - 1) & 1) ^ 1, p)) return false;
-    const int stage = kv_cnt % C::kStages;
-    if (!wait_warp(sm, &sm.kv_full[stage], (kv_cnt / C::kStages) & 1, p)) return false;
-    tc_fence_after();
-    if (lane == 0) {
-      const uint32_t va = smem_u32(sm.kv[stage]);
-#pragma unroll
-      for (int kk = 0; kk < kBlockN / 16; ++kk) {
-        umma_ts(tmem + C::o_col(slot), tmem + C::s_col(slot) + kk * 8,
-                sdesc_sw128(va + kk * 2048, kChunkBytes, 1024), idesc_pv,
-                (s.j > 0 || kk > 0) ? 1u : 0u);
-      }
-      if (p.split_p) {
-#pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk)
-          umma_ts(tmem + C::o_col(slot), tmem + C::s_col(slot) + 64 + kk * 8,
-                  sdesc_sw128(va + kk * 2048, kChunkBytes, 1024), idesc_pv, 1u);
-      }
-      umma_commit(&sm.kv_empty[stage]);
-      if (s.j == s.cur.n - 1) umma_commit(&sm.o_full[slot]);
-    }
-    __syncwarp();
-    ++kv_cnt;
-    ++s.blk;
-    return true;
-  };
-  auto start_unit = [&](int slot) -> bool {
-    MmaSlot& s = st[slot];
-    s.active = s.it.pop_nonempty(s.cur);
-    if (!s.active) return true;
-    s.j = 0;
-    ++s.units;
-    return issue_s(slot, 0);
-  };
-
-#pragma unroll
-  for (int s = 0; s < kNumSlots; ++s) {
-    st[s].it.init(p, s);
-    st[s].units = 0;
-    st[s].blk = 0;
-    if (ok) ok = start_unit(s);
-  }
+  static_assert(kNumSlots == 2, "the MMA loop visits two slots");
+  MmaShared ms;
+  ms.kv_cnt = 0;
+  ms.tmem = tmem;
+  ms.idesc_s = idesc_f16_f32(p.is_bf16 != 0, 128, 128, false);
+  ms.idesc_pv = idesc_f16_f32(p.is_bf16 != 0, 128, D, true);
+  ms.split = p.split_p != 0;
+  MmaSlot s0, s1;
+  s0.it.init(p, 0);
+  s1.it.init(p, 1);
+  s0.units = s1.units = 0;
+  s0.blk = s1.blk = 0;
+  bool ok = mma_start_unit<D, 0>(sm, p, s0, ms);
+  if (ok) ok = mma_start_unit<D, 1>(sm, p, s1, ms);
   bool any = true;
   while (ok && any) {
     any = false;
-#pragma unroll
-    for (int s = 0; s < kNumSlots; ++s) {
-      if (!ok) break;
-      if (!st[s].active) continue;
-      any = true;
-      ok = issue_pv(s);
-      if (!ok) break;
-      ++st[s].j;
-      ok = st[s].j < st[s].cur.n ? issue_s(s, st[s].j) : start_unit(s);
-    }
+    ok = mma_step<D, 0>(sm, p, s0, ms, any);
+    if (ok) ok = mma_step<D, 1>(sm, p, s1, ms, any);
   }
   if (!ok) {
-    // Drain every MMA this thread issued before TMEM is released.
-    if (lane == 0) umma_commit(&sm.drain);
+    // Drain every MMA this warp issued before TMEM is released.
+    if (elect_one_sync()) umma_commit(&sm.drain);
+    __syncwarp();
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&sm.drain, 0) && globaltimer_ns() - t0 < p.timeout_ns) {
+    }
+  }
+}
+
+// ---------------------------------------------------------------- separate-P roles
+// With P in its own TMEM columns each slot runs a stream of S ops one block ahead
+// of its stream of PV ops.  The MMA warp and the producer walk the same rounds:
+//   start:   S(slot 0, block 0), S(slot 1, block 0)
+//   round r: S(slot 0, r+1), S(slot 1, r+1), PV(slot 0, r), PV(slot 1, r)
+// where a slot's blocks run over its non-empty units back to back.  S ops consume
+// K tiles (and the unit's Q at block 0), PV ops consume V tiles, in that order.
+
+// A position in a slot's block stream (producer side: with block indices).
+struct ProdCursor {
+  UnitIter it;
+  Unit cur, nxt;
+  bool has_cur, has_nxt;
+  int j;      // block of `cur`
+  int units;  // non-empty units entered
+  int chunk;  // 32-block chunk of cur's list held in `idx`
+  int idx, nxt_idx;
+};
+
+__device__ __forceinline__ void pc_enter_next(ProdCursor& c, const Params& p, int lane) {
+  c.has_cur = c.has_nxt;
+  c.cur = c.nxt;
+  c.idx = c.nxt_idx;
+  c.chunk = 0;
+  c.j = 0;
+  if (c.has_cur) ++c.units;
+  c.has_nxt = c.it.pop_nonempty(c.nxt);
+  if (c.has_nxt) c.nxt_idx = chunk_index(p, c.nxt, 0, lane);
+}
+
+__device__ __forceinline__ void pc_init(ProdCursor& c, const Params& p, int slot, int lane) {
+  c.it.init(p, slot);
+  c.units = 0;
+  c.has_nxt = c.it.pop_nonempty(c.nxt);
+  if (c.has_nxt) c.nxt_idx = chunk_index(p, c.nxt, 0, lane);
+  pc_enter_next(c, p, lane);
+}
+
+// Move to the next block of the stream; true if that entered a new unit.
+__device__ __forceinline__ bool pc_step(ProdCursor& c, const Params& p, int lane) {
+  ++c.j;
+  if (c.j < c.cur.n) return false;
+  pc_enter_next(c, p, lane);
+  return true;
+}
+
+__device__ __forceinline__ int pc_block(ProdCursor& c, const Params& p, int lane) {
+  const int chunk = c.j >> 5;
+  if (chunk != c.chunk) {
+    c.idx = chunk_index(p, c.cur, chunk, lane);
+    c.chunk = chunk;
+  }
+  return __shfl_sync(0xffffffffu, c.idx, c.j & 31);
+}
+
+template <int D>
+__device__ __forceinline__ bool sep_load_tile(Smem<D>& sm, const Params& p, const CUtensorMap* map,
+                                              int kvb, int bh, ProdShared& ps) {
+  using C = Cfg<D>;
+  const int stage = ps.kv_cnt % C::kStages;
+  const uint32_t phase = (ps.kv_cnt / C::kStages) & 1;
+  if (!wait_lane0(sm, &sm.kv_empty[stage], phase ^ 1, p)) return false;
+  if (elect_one_sync()) {
+    mbar_arrive_expect_tx(&sm.kv_full[stage], C::kTileBytes);
+    load_tile<D>(map, kvb * kBlockN, bh, sm.kv[stage], &sm.kv_full[stage], ps.pol_kv);
+  }
+  __syncwarp();
+  ++ps.kv_cnt;
+  return true;
+}
+
+// Loads for one S op at the K cursor: the unit's Q when at block 0, then K.
+template <int D, int SLOT>
+__device__ __forceinline__ bool sep_prod_s(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
+                                           const CUtensorMap* tk, ProdCursor& c, ProdShared& ps,
+                                           int lane) {
+  using C = Cfg<D>;
+  if (c.j == 0) {
+    const int u = c.units - 1;
+    const int b = u % C::kQBuf;
+    if (!wait_lane0(sm, &sm.q_empty[SLOT][b], ((u / C::kQBuf) & 1) ^ 1, p)) return false;
+    if (elect_one_sync()) {
+      mbar_arrive_expect_tx(&sm.q_full[SLOT][b], C::kTileBytes);
+      load_tile<D>(tq, c.cur.qblk * kBlockN, c.cur.bh, sm.q[SLOT][b], &sm.q_full[SLOT][b], ps.pol_q);
+    }
+    __syncwarp();
+  }
+  const int kvb = pc_block(c, p, lane);
+  return sep_load_tile<D>(sm, p, tk, kvb, c.cur.bh, ps);
+}
+
+// The V load of a slot's PV op r reads the block its K load of round r - 1 read,
+// so the K cursor leaves a one-entry record {bh, block} behind for it.
+struct PendingV {
+  int bh, kvb;
+  bool valid;
+};
+
+template <int D, int SLOT>
+__device__ __forceinline__ bool sep_prod_round_s(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
+                                                 const CUtensorMap* tk, ProdCursor& c, PendingV& pv,
+                                                 ProdShared& ps, int lane) {
+  if (!c.has_cur) {
+    pv.valid = false;
+    return true;
+  }
+  pv.bh = c.cur.bh;
+  pv.kvb = pc_block(c, p, lane);
+  pv.valid = true;
+  pc_step(c, p, lane);
+  return c.has_cur ? sep_prod_s<D, SLOT>(sm, p, tq, tk, c, ps, lane) : true;
+}
+
+template <int D>
+__device__ void producer_role_sep(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
+                                  const CUtensorMap* tk, const CUtensorMap* tv) {
+  using C = Cfg<D>;
+  static_assert(kNumSlots == 2, "the producer loop visits two slots");
+  const int lane = threadIdx.x & 31;
+  ProdShared ps;
+  ps.kv_cnt = 0;
+  ps.pol_kv = policy_evict_last();
+  ps.pol_q = policy_evict_first();
+  ProdCursor k0, k1;
+  PendingV v0, v1;
+  pc_init(k0, p, 0, lane);
+  pc_init(k1, p, 1, lane);
+  bool ok = true;
+  if (k0.has_cur) ok = sep_prod_s<D, 0>(sm, p, tq, tk, k0, ps, lane);
+  if (ok && k1.has_cur) ok = sep_prod_s<D, 1>(sm, p, tq, tk, k1, ps, lane);
+  while (ok && (k0.has_cur || k1.has_cur)) {
+    ok = sep_prod_round_s<D, 0>(sm, p, tq, tk, k0, v0, ps, lane);
+    if (ok) ok = sep_prod_round_s<D, 1>(sm, p, tq, tk, k1, v1, ps, lane);
+    if (ok && v0.valid) ok = sep_load_tile<D>(sm, p, tv, v0.kvb, v0.bh, ps);
+    if (ok && v1.valid) ok = sep_load_tile<D>(sm, p, tv, v1.kvb, v1.bh, ps);
+  }
+  if (!ok && elect_one_sync()) {
+    const uint64_t t0 = globaltimer_ns();
+    for (int stage = 0; stage < C::kStages; ++stage) {
+      const int fills = ps.kv_cnt / C::kStages + (stage < ps.kv_cnt % C::kStages ? 1 : 0);
+      if (fills == 0) continue;
+      while (!mbar_try_wait(&sm.kv_full[stage], (fills - 1) & 1) &&
+             globaltimer_ns() - t0 < p.timeout_ns) {
+      }
+    }
+    for (int slot = 0; slot < kNumSlots; ++slot) {
+      const int units = slot == 0 ? k0.units : k1.units;
+      for (int b = 0; b < C::kQBuf; ++b) {
+        const int fills = units > b ? (units - 1 - b) / C::kQBuf + 1 : 0;
+        if (fills == 0) continue;
+        while (!mbar_try_wait(&sm.q_full[slot][b], (fills - 1) & 1) &&
+               globaltimer_ns() - t0 < p.timeout_ns) {
+        }
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// MMA-side position in a slot's block stream.
+struct MmaCursor {
+  UnitIter it;
+  Unit cur;
+  bool active;
+  int j;      // block of `cur`
+  int units;  // non-empty units entered
+  int ops;    // ops issued on this stream (barrier phase)
+};
+
+__device__ __forceinline__ void mc_enter_next(MmaCursor& c) {
+  c.active = c.it.pop_nonempty(c.cur);
+  c.j = 0;
+  if (c.active) ++c.units;
+}
+__device__ __forceinline__ void mc_init(MmaCursor& c, const Params& p, int slot) {
+  c.it.init(p, slot);
+  c.units = 0;
+  c.ops = 0;
+  mc_enter_next(c);
+}
+__device__ __forceinline__ void mc_step(MmaCursor& c) {
+  ++c.ops;
+  if (++c.j >= c.cur.n) mc_enter_next(c);
+}
+
+template <int D, int SLOT>
+__device__ __forceinline__ bool sep_mma_s(Smem<D>& sm, const Params& p, MmaCursor& c, MmaShared& ms) {
+  using C = Cfg<D>;
+  const int u = c.units - 1;
+  const int b = u % C::kQBuf;
+  // the softmax must have read the previous S of this slot
+  if (c.ops > 0 && !wait_lane0(sm, &sm.s_empty[SLOT], (c.ops - 1) & 1, p)) return false;
+  if (c.j == 0 && !wait_lane0(sm, &sm.q_full[SLOT][b], (u / C::kQBuf) & 1, p)) return false;
+  const int stage = ms.kv_cnt % C::kStages;
+  if (!wait_lane0(sm, &sm.kv_full[stage], (ms.kv_cnt / C::kStages) & 1, p)) return false;
+  tc_fence_after();
+  const uint64_t qd = sdesc_sw128(smem_u32(sm.q[SLOT][b]), 16, 1024);
+  const uint64_t kd = sdesc_sw128(smem_u32(sm.kv[stage]), 16, 1024);
+  const uint32_t d_s = ms.tmem + C::s_col(SLOT);
+  const bool last = c.j == c.cur.n - 1;
+  if (elect_one_sync()) {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+      umma_ss(d_s, qd + off, kd + off, ms.idesc_s, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(&sm.kv_empty[stage]);
+    umma_commit(&sm.s_full[SLOT]);
+    if (last) umma_commit(&sm.q_empty[SLOT][b]);
+  }
+  __syncwarp();
+  ++ms.kv_cnt;
+  return true;
+}
+
+// The PV op of round r is the block the S op of round r - 1 covered: the S cursor
+// leaves {first, last, unit number} behind for it.
+struct PendingPV {
+  bool valid, first, last;
+  int units;  // non-empty units entered when that block was current
+  int ops;    // PV ops issued on this slot
+};
+
+template <int D, int SLOT>
+__device__ __forceinline__ bool sep_mma_pv(Smem<D>& sm, const Params& p, PendingPV& v, MmaShared& ms) {
+  using C = Cfg<D>;
+  if (!wait_lane0(sm, &sm.p_full[SLOT], v.ops & 1, p)) return false;
+  // O of this slot is free once the epilogue of its previous unit has read it
+  if (v.first && v.units > 1 && !wait_lane0(sm, &sm.o_empty[SLOT], (v.units - 2) & 1, p))
+    return false;
+  const int stage = ms.kv_cnt % C::kStages;
+  if (!wait_lane0(sm, &sm.kv_full[stage], (ms.kv_cnt / C::kStages) & 1, p)) return false;
+  tc_fence_after();
+  const uint64_t vd = sdesc_sw128(smem_u32(sm.kv[stage]), kChunkBytes, 1024);
+  const uint32_t d_o = ms.tmem + C::o_col(SLOT);
+  const uint32_t a_p = ms.tmem + C::p_col(SLOT);
+  const uint32_t acc0 = v.first ? 0u : 1u;
+  const bool last = v.last;
+  if (elect_one_sync()) {
+#pragma unroll
+    for (int kk = 0; kk < kBlockN / 16; ++kk)
+      umma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * 128), ms.idesc_pv,
+              kk > 0 ? 1u : acc0);
+    umma_commit(&sm.kv_empty[stage]);
+    umma_commit(&sm.pv_done[SLOT]);
+    if (last) umma_commit(&sm.o_full[SLOT]);
+  }
+  __syncwarp();
+  ++ms.kv_cnt;
+  ++v.ops;
+  return true;
+}
+
+template <int D, int SLOT>
+__device__ __forceinline__ bool sep_mma_round_s(Smem<D>& sm, const Params& p, MmaCursor& c,
+                                                PendingPV& v, MmaShared& ms) {
+  if (!c.active) {
+    v.valid = false;
+    return true;
+  }
+  v.valid = true;
+  v.first = c.j == 0;
+  v.last = c.j == c.cur.n - 1;
+  v.units = c.units;
+  mc_step(c);
+  return c.active ? sep_mma_s<D, SLOT>(sm, p, c, ms) : true;
+}
+
+template <int D>
+__device__ void mma_role_sep(Smem<D>& sm, const Params& p, uint32_t tmem) {
+  static_assert(kNumSlots == 2, "the MMA loop visits two slots");
+  MmaShared ms;
+  ms.kv_cnt = 0;
+  ms.tmem = tmem;
+  ms.idesc_s = idesc_f16_f32(p.is_bf16 != 0, 128, 128, false);
+  ms.idesc_pv = idesc_f16_f32(p.is_bf16 != 0, 128, D, true);
+  ms.split = false;
+  MmaCursor s0, s1;  // S streams of the two slots
+  PendingPV v0, v1;  // their PV streams, one block behind
+  v0.ops = v1.ops = 0;
+  mc_init(s0, p, 0);
+  mc_init(s1, p, 1);
+  bool ok = true;
+  if (s0.active) ok = sep_mma_s<D, 0>(sm, p, s0, ms);
+  if (ok && s1.active) ok = sep_mma_s<D, 1>(sm, p, s1, ms);
+  while (ok && (s0.active || s1.active)) {
+    ok = sep_mma_round_s<D, 0>(sm, p, s0, v0, ms);
+    if (ok) ok = sep_mma_round_s<D, 1>(sm, p, s1, v1, ms);
+    if (ok && v0.valid) ok = sep_mma_pv<D, 0>(sm, p, v0, ms);
+    if (ok && v1.valid) ok = sep_mma_pv<D, 1>(sm, p, v1, ms);
+  }
+  if (!ok) {
+    if (elect_one_sync()) umma_commit(&sm.drain);
     __syncwarp();
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(&sm.drain, 0) && globaltimer_ns() - t0 < p.timeout_ns) {
@@ -475,6 +841,59 @@ __device__ __forceinline__ void unpack2(uint32_t v, bool bf16, float& lo, float&
   }
 }
 
+// 64 consecutive S columns of this thread's row (TMEM lane) into registers.
+__device__ __forceinline__ void load_s_half(uint32_t taddr, float (&x)[64]) {
+  uint32_t xr[64];
+  tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(xr));
+  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32));
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(xr[i]);
+}
+
+// Mask rule on 64 columns of a PARTIAL block: column i (key kv0 + i) is live iff
+// a <= i <= b (causal / window interval, clipped to the keys that exist) and, for
+// documents, doc_id[kv0 + i] == dq.  Dead entries become -inf.
+__device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int a, int b, int kv0,
+                                           int dq) {
+  if (p.mask_kind == FA_MASK_DOCUMENT_CAUSAL) {
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint32_t same = 0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int kv = kv0 + c * 32 + i;
+        const int d = kv < p.S ? __ldg(p.doc_id + kv) : dq + 1;
+        same |= (d == dq ? 1u : 0u) << i;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int ii = c * 32 + i;
+        if (ii < a || ii > b || !((same >> i) & 1u)) x[ii] = -INFINITY;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 64; ++i)
+      if (i < a || i > b) x[i] = -INFINITY;
+  }
+}
+
+// Max of 64 values: 8 chains of three-input maxima, then a tree.
+__device__ __forceinline__ float row_max64(const float (&x)[64]) {
+  float mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = fmaxf(x[i], x[i + 8]);
+#pragma unroll
+  for (int i = 16; i < 64; i += 16)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) mx[c] = fmax3(mx[c], x[i + c], x[i + 8 + c]);
+  mx[0] = fmax3(mx[0], mx[1], mx[2]);
+  mx[3] = fmax3(mx[3], mx[4], mx[5]);
+  mx[6] = fmaxf(mx[6], mx[7]);
+  return fmax3(mx[0], mx[3], mx[6]);
+}
+
 // Softmax warpgroup of one slot: thread t owns row t of the slot's 128-row tile
 // (TMEM lane t), so row max and row sum need no shuffles.
 template <int D>
@@ -484,11 +903,13 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
   const int wq = t >> 5;                    // TMEM lane quarter of this warp
   const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
   const uint32_t t_s = tmem + C::s_col(slot) + lane_off;
+  const uint32_t t_p = tmem + C::p_col(slot) + lane_off;
   const uint32_t t_o = tmem + C::o_col(slot) + lane_off;
   const bool bf16 = p.is_bf16 != 0;
   // Factor that turns the value kept in x[] into log2 units: the raw score is
   // kept (and scaled inside the exponent's FFMA) unless a score_mod rewrote it.
   const float xs = p.softcap_on ? 1.f : p.scale_log2;
+  const bool split = p.split_p != 0 && !C::kSepP;
   UnitIter it;
   it.init(p, slot);
   int blk = 0, units = 0;
@@ -519,61 +940,31 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
       const int kvb_next = j + 1 < un.n ? block_index(p, un, j + 1) : 0;
       if (!wait_warp(sm, &sm.s_full[slot], blk & 1, p)) return;
       tc_fence_after();
-      float x[128];
-      {
-        uint32_t xr[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tmem_ld32(t_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(xr + c * 32));
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 128; ++i) x[i] = __uint_as_float(xr[i]);
+      // Pass 1: the block's row max from the raw scores (a PARTIAL block's masked
+      // entries excluded).  The softcap is monotone, so the max of the capped scores
+      // is the cap of the raw max.  Pass 2 then turns each half of 64 keys into P with
+      // that one max: P_hi of half h goes to P columns [32h, 32h + 32); with the
+      // split, P_lo goes to columns 64 + [32h, 32h + 32), held in registers until
+      // half 1 has been read (in the aliased layout those columns are still S).
+      const int a = lo - kvb * kBlockN;  // live columns of the block: a <= i <= b
+      const int b = hi - kvb * kBlockN;
+      float rmax = -INFINITY;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float x[64];
+        load_s_half(t_s + h * 64, x);
+        if (!full) apply_mask(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq);
+        rmax = fmaxf(rmax, row_max64(x));
       }
-      if (p.softcap_on) {  // x = log2(e) * c * tanh(s * scale / c)
-#pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const float e = ex2_approx(x[i] * p.cap_k);            // e^(2y), y = s * scale / c
-          x[i] = p.cap_a - 2.f * p.cap_a * rcp_approx(e + 1.f);  // c * log2(e) * tanh(y)
-        }
-      }
-      if (!full) {  // PARTIAL block: evaluate the mask rule per element
-        const int a = lo - kvb * kBlockN;  // live columns: a <= i <= b
-        const int b = hi - kvb * kBlockN;
-        if (p.mask_kind == FA_MASK_DOCUMENT_CAUSAL) {
-          const int kv0 = kvb * kBlockN;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t same = 0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int kv = kv0 + c * 32 + i;
-              const int d = kv < p.S ? __ldg(p.doc_id + kv) : dq + 1;
-              same |= (d == dq ? 1u : 0u) << i;
-            }
-            asm volatile("" ::: "memory");  // keep one chunk of id loads in flight at a time
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int ii = c * 32 + i;
-              if (ii < a || ii > b || !((same >> i) & 1u)) x[ii] = -INFINITY;
-            }
-          }
+      float mb = rmax;
+      if (rmax != -INFINITY) {
+        if (p.softcap_on) {
+          mb = p.cap_a - 2.f * p.cap_a * rcp_approx(ex2_approx(rmax * p.cap_k) + 1.f);
         } else {
-#pragma unroll
-          for (int i = 0; i < 128; ++i)
-            if (i < a || i > b) x[i] = -INFINITY;
+          mb = rmax * xs;
         }
       }
-      // row max: 16 independent chains, then a tree
-      float mx[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) mx[i] = x[i];
-#pragma unroll
-      for (int i = 16; i < 128; ++i) mx[i & 15] = fmaxf(mx[i & 15], x[i]);
-#pragma unroll
-      for (int w = 8; w > 0; w >>= 1)
-#pragma unroll
-        for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
-      const float m_new = fmaxf(m, mx[0] * xs);
+      const float m_new = fmaxf(m, mb);
       // Deferred rescale: keep the stale max unless the new one exceeds it by more
       // than 2^8; exact, because l and O always use the same max.
       float alpha = 1.f;
@@ -587,33 +978,11 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         m = m_new;
       }
       const float neg_mu = (m == -INFINITY) ? 0.f : -m;
-      // P = exp2(x * xs - m) as 16-bit pairs: P_hi = round(p) over S columns 0-63 and,
-      // when split, P_lo = round(p - P_hi) over columns 64-127 (both PV products are
-      // accumulated, so P carries ~16 significant bits instead of 8).
-      float sums[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) sums[i] = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t ph[16], pl[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2_approx(fmaf(x[c * 32 + 2 * i], xs, neg_mu));
-          const float p1 = ex2_approx(fmaf(x[c * 32 + 2 * i + 1], xs, neg_mu));
-          sums[i & 7] += p0 + p1;
-          ph[i] = pack2(p0, p1, bf16);
-          float h0, h1;
-          unpack2(ph[i], bf16, h0, h1);
-          pl[i] = pack2(p0 - h0, p1 - h1, bf16);
-        }
-        tmem_st16(t_s + c * 16, ph);
-        if (p.split_p) tmem_st16(t_s + 64 + c * 16, pl);
+      if constexpr (C::kSepP) {
+        // the previous PV of this slot must be done before P is overwritten or O rescaled
+        if (blk > 0 && !wait_warp(sm, &sm.pv_done[slot], (blk - 1) & 1, p)) return;
+        tc_fence_after();
       }
-#pragma unroll
-      for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-        for (int i = 0; i < w; ++i) sums[i] += sums[i + w];
-      l += sums[0];
       if (__any_sync(0xffffffffu, rescale_o)) {
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
@@ -625,9 +994,67 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
           tmem_st32(t_o + c * 32, r);
         }
       }
+      uint32_t pl_hold[32];
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float x[64];
+        load_s_half(t_s + h * 64, x);
+        if (h == 1) {
+          if constexpr (C::kSepP) {  // all of S is read: the MMA warp may refill it
+            tc_fence_before();
+            __syncwarp();
+            if ((t & 31) == 0) mbar_arrive(&sm.s_empty[slot]);
+          }
+          if (split) tmem_st32(t_p + 64, pl_hold);
+        }
+        if (p.softcap_on) {  // x = log2(e) * c * tanh(s * scale / c)
+#pragma unroll
+          for (int i = 0; i < 64; i += 2) {
+            const float2 e = make_float2(ex2_approx(x[i] * p.cap_k), ex2_approx(x[i + 1] * p.cap_k));
+            const float2 r = make_float2(rcp_approx(e.x + 1.f), rcp_approx(e.y + 1.f));
+            const float2 v = fma2(r, make_float2(-2.f * p.cap_a, -2.f * p.cap_a),
+                                  make_float2(p.cap_a, p.cap_a));
+            x[i] = v.x;
+            x[i + 1] = v.y;
+          }
+        }
+        if (!full) apply_mask(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq);
+        // P = exp2(x * xs - m) as 16-bit pairs; with the split, P_hi = p truncated to
+        // bf16 and P_lo = round(p - P_hi), so P_hi + P_lo carries ~16 significant bits.
+        float2 sums[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sums[i] = make_float2(0.f, 0.f);
+        const float2 xs2 = make_float2(xs, xs), nm2 = make_float2(neg_mu, neg_mu);
+        uint32_t ph[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float2 a2 = fma2(make_float2(x[2 * i], x[2 * i + 1]), xs2, nm2);
+          const float2 pp = make_float2(ex2_approx(a2.x), ex2_approx(a2.y));
+          sums[i & 3] = add2(sums[i & 3], pp);
+          if (!split) {
+            ph[i] = pack2(pp.x, pp.y, bf16);
+          } else if (bf16) {
+            const uint32_t u0 = __float_as_uint(pp.x), u1 = __float_as_uint(pp.y);
+            ph[i] = __byte_perm(u0, u1, 0x7632);
+            const float2 lo2 = sub2(pp, make_float2(__uint_as_float(u0 & 0xFFFF0000u),
+                                                    __uint_as_float(u1 & 0xFFFF0000u)));
+            pl_hold[i] = pack2(lo2.x, lo2.y, true);
+          } else {
+            ph[i] = pack2(pp.x, pp.y, false);
+            float h0, h1;
+            unpack2(ph[i], false, h0, h1);
+            pl_hold[i] = pack2(pp.x - h0, pp.y - h1, false);
+          }
+        }
+        tmem_st32(t_p + h * 32, ph);
+        sums[0] = add2(add2(sums[0], sums[1]), add2(sums[2], sums[3]));
+        l += sums[0].x + sums[0].y;
+      }
+      if (split) tmem_st32(t_p + 96, pl_hold);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full[slot]);
+      __syncwarp();
+      if ((t & 31) == 0) mbar_arrive(&sm.p_full[slot]);
       ++blk;
       kvb = kvb_next;
     }
@@ -652,7 +1079,8 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
       }
     }
     tc_fence_before();
-    mbar_arrive(&sm.o_empty[slot]);
+    __syncwarp();
+    if ((t & 31) == 0) mbar_arrive(&sm.o_empty[slot]);
     if (valid && p.lse) p.lse[orow] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
     ++units;
   }
@@ -674,9 +1102,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
         mbar_init(&sm.q_empty[s][b], 1);
       }
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.p_full[s], 128);
+      mbar_init(&sm.s_empty[s], 4);
+      mbar_init(&sm.pv_done[s], 1);
+      mbar_init(&sm.p_full[s], 4);   // one arrival per softmax warp
       mbar_init(&sm.o_full[s], 1);
-      mbar_init(&sm.o_empty[s], 128);
+      mbar_init(&sm.o_empty[s], 4);
     }
     for (int i = 0; i < Cfg<D>::kStages; ++i) {
       mbar_init(&sm.kv_full[i], 1);
@@ -711,9 +1141,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
   }
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == kProducerWarp) {
-    producer_role<D>(sm, p, &tmap_q, &tmap_k, &tmap_v);
+    if constexpr (Cfg<D>::kSepP)
+      producer_role_sep<D>(sm, p, &tmap_q, &tmap_k, &tmap_v);
+    else
+      producer_role<D>(sm, p, &tmap_q, &tmap_k, &tmap_v);
   } else if (warp == kMmaWarp) {
-    mma_role<D>(sm, p, tmem);
+    if constexpr (Cfg<D>::kSepP)
+      mma_role_sep<D>(sm, p, tmem);
+    else
+      mma_role<D>(sm, p, tmem);
   }
   tc_fence_before();
   named_barrier_sync(1, kThreads);

@@ -78,9 +78,30 @@ def test_dtypes_and_head_dims(dtype, D):
 
 
 def test_softcap_and_custom_scale():
-    q, k, v = W.random_qkv(1, 2, 512, 512, 64, torch.bfloat16, seed=11, scale=2.0)
+    """x2-scaled inputs (|v| up to ~9, peaky softmax): bf16 at D=128 (P carried as
+    a hi + lo pair), fp16 at D=64 (P in fp16, 11 significant bits)."""
+    q, k, v = W.random_qkv(1, 2, 512, 512, 128, torch.bfloat16, seed=11, scale=2.0)
     _full_compare(q, k, v, 0, sk=1, cap=3.0)
     _full_compare(q, k, v, 1, window=200, scale=0.3)
+    q, k, v = W.random_qkv(1, 2, 512, 512, 64, torch.float16, seed=11, scale=2.0)
+    _full_compare(q, k, v, 0, sk=1, cap=3.0)
+    _full_compare(q, k, v, 1, window=200, scale=0.3)
+
+
+def test_d64_bf16_p_rounding_bound():
+    """At D=64 P enters the PV product rounded to bf16 (8 significant bits), so each
+    weight carries a relative error up to 2^-8 and the output error is bounded by
+    2^-8 * max|v| plus half an output ulp; check that bound on x2-scaled inputs,
+    where 2e-2 can be exceeded."""
+    q, k, v = W.random_qkv(1, 2, 512, 512, 64, torch.bfloat16, seed=11, scale=2.0)
+    out, lse = run_gpu(q, k, v, 1, 200, None, 0, 0.0, 0.3)
+    vmax = float(v.abs().max())
+    for h in range(2):
+        o_ref, l_ref = oracle_rows(q, k, v, 0, h, np.arange(512), 1, 200, None, 0, 0.0, 0.3)
+        err = np.abs(out[0, h].double().numpy() - o_ref)
+        bound = 2.0 ** -8 * vmax + 0.5 * np.abs(o_ref) * 2.0 ** -7
+        assert (err <= bound + 1e-3).all(), float((err - bound).max())
+        assert np.abs(lse[0, h].double().numpy() - l_ref).max() <= 1e-3
 
 
 def test_fully_masked_rows_zero_and_minus_inf():
