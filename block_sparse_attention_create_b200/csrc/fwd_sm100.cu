@@ -48,9 +48,9 @@ namespace {
 
 constexpr int kNumSlots = 2;
 constexpr int kSoftmaxWarps = 4 * kNumSlots;
-constexpr int kProducerWarp = kSoftmaxWarps;
-constexpr int kMmaWarp = kSoftmaxWarps + 1;
-constexpr int kThreads = (kSoftmaxWarps + 4) * 32;  // + one warpgroup: producer, MMA, 2 spare
+constexpr int kProducerWarp = kSoftmaxWarps;      // + slot: one TMA producer warp per slot
+constexpr int kMmaWarp = kSoftmaxWarps + kNumSlots;
+constexpr int kThreads = (kSoftmaxWarps + 4) * 32;  // + one warpgroup: 2 producers, MMA, 1 spare
 // Register split (per thread) after launch: 384 threads x 168 = 64512 registers at
 // launch; softmax warpgroups take 208, the control warpgroup 88:
 // 256 x 208 + 128 x 88 = 64512, and per SM sub-partition 208 + 208 + 88 <= 512.
@@ -73,7 +73,9 @@ template <int D>
 struct Cfg {
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kBlockN * D * 2;
-  static constexpr int kStages = (D == 64) ? 8 : 4;
+  // Per slot: a ring of K tiles and a ring of V tiles.
+  static constexpr int kKRing = (D == 64) ? 2 : 1;
+  static constexpr int kVRing = (D == 64) ? 2 : 1;
   // Q tiles per slot: two at D=64, so the next unit's Q loads while this one runs.
   static constexpr int kQBuf = (D == 64) ? 2 : 1;
   static constexpr bool kSepP = (D == 64);
@@ -90,17 +92,20 @@ struct Cfg {
 template <int D>
 struct __align__(1024) Smem {
   uint8_t q[kNumSlots][Cfg<D>::kQBuf][Cfg<D>::kTileBytes];
-  uint8_t kv[Cfg<D>::kStages][Cfg<D>::kTileBytes];
+  uint8_t k[kNumSlots][Cfg<D>::kKRing][Cfg<D>::kTileBytes];
+  uint8_t v[kNumSlots][Cfg<D>::kVRing][Cfg<D>::kTileBytes];
   uint64_t q_full[kNumSlots][Cfg<D>::kQBuf];
   uint64_t q_empty[kNumSlots][Cfg<D>::kQBuf];
+  uint64_t k_full[kNumSlots][Cfg<D>::kKRing];
+  uint64_t k_empty[kNumSlots][Cfg<D>::kKRing];
+  uint64_t v_full[kNumSlots][Cfg<D>::kVRing];
+  uint64_t v_empty[kNumSlots][Cfg<D>::kVRing];
   uint64_t s_full[kNumSlots];
   uint64_t s_empty[kNumSlots];  // separate-P layout: softmax has read S
   uint64_t p_full[kNumSlots];
   uint64_t pv_done[kNumSlots];  // separate-P layout: PV_j finished (P buffer and O stable)
   uint64_t o_full[kNumSlots];
   uint64_t o_empty[kNumSlots];
-  uint64_t kv_full[Cfg<D>::kStages];
-  uint64_t kv_empty[Cfg<D>::kStages];
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort_flag;
@@ -147,38 +152,34 @@ __device__ __forceinline__ int ldg_nc(const int32_t* ptr) {
 // the next unit is requested when the current one is handed out, so its global
 // load latency overlaps a whole unit of work.
 struct UnitIter {
-  int worker, workers, round, num_units, BH;
-  const int32_t* sched;
+  int worker, round;
   int nu;   // next unit id, -1 when exhausted
   int2 nx;  // its schedule entry (load in flight)
 
   __device__ __forceinline__ void init(const Params& p, int slot) {
     worker = static_cast<int>(blockIdx.x) * kNumSlots + slot;
-    workers = static_cast<int>(gridDim.x) * kNumSlots;
     round = 0;
-    num_units = p.num_units;
-    BH = p.BH;
-    sched = p.sched;
-    fetch();
+    fetch(p);
   }
-  __device__ __forceinline__ void fetch() {
+  __device__ __forceinline__ void fetch(const Params& p) {
+    const int workers = static_cast<int>(gridDim.x) * kNumSlots;
     const int u = round * workers + ((round & 1) ? (workers - 1 - worker) : worker);
     ++round;
-    nu = u < num_units ? u : -1;
-    if (nu >= 0) nx = ldg_nc_v2(sched + 2 * (nu / BH));
+    nu = u < p.num_units ? u : -1;
+    if (nu >= 0) nx = ldg_nc_v2(p.sched + 2 * (nu / p.BH));
   }
-  __device__ __forceinline__ bool pop(Unit& x) {
+  __device__ __forceinline__ bool pop(const Params& p, Unit& x) {
     if (nu < 0) return false;
-    const int k = nu / BH;
-    x.bh = nu - k * BH;
+    const int k = nu / p.BH;
+    x.bh = nu - k * p.BH;
     x.qblk = nx.x;
     x.np = nx.y & 0xFFFF;
     x.n = x.np + (nx.y >> 16);
-    fetch();
+    fetch(p);
     return true;
   }
-  __device__ __forceinline__ bool pop_nonempty(Unit& x) {
-    while (pop(x))
+  __device__ __forceinline__ bool pop_nonempty(const Params& p, Unit& x) {
+    while (pop(p, x))
       if (x.n > 0) return true;
     return false;
   }
@@ -230,306 +231,16 @@ __device__ __forceinline__ bool wait_lane0(Smem<D>& sm, uint64_t* bar, uint32_t 
 }
 
 // ---------------------------------------------------------------- roles
-// The producer and the MMA warp keep one state record per slot.  Every function
-// that touches a slot's record takes the slot as a template parameter, so the
-// records live in registers (a runtime slot index would put them in local memory).
+// Each slot has its own producer warp, its own ring of K tiles and its own ring of
+// V tiles; the MMA warp serves both slots, issuing whichever slot's next MMA is
+// ready.  A slot's blocks run over its non-empty units back to back (block i of
+// the slot's stream); K_i goes to K-ring stage i % kKRing, V_i to V-ring stage
+// i % kVRing, so producer and MMA warp agree on stages without a shared order.
+// Every function that touches per-slot state takes the slot as a template
+// parameter, so that state lives in registers.
 
-// TMA producer: the whole warp walks the MMA warp's consumption order (per slot:
-// Q, K_0, then V_j, K_{j+1} ...; slots interleaved the way the MMA warp visits
-// them) and one elected lane issues the copies.  Block indices are fetched 32 at
-// a time, one per lane, and the first chunk of the slot's next unit is requested
-// when its current unit starts.
-struct ProdSlot {
-  UnitIter it;
-  Unit cur, nxt;
-  bool has_cur, has_nxt;
-  int j;      // block of `cur` whose V is loaded next
-  int units;  // non-empty units started on this slot
-  int chunk;  // 32-block chunk of cur's list held in `idx`
-  int idx, nxt_idx;
-};
-
-struct ProdShared {
-  int kv_cnt;  // tiles issued into the K/V ring (both slots)
-  uint64_t pol_kv, pol_q;
-};
-
-__device__ __forceinline__ int chunk_index(const Params& p, const Unit& x, int chunk, int lane) {
-  const int jj = chunk * 32 + lane;
-  return jj < x.n ? block_index(p, x, jj) : 0;
-}
-
-template <int D>
-__device__ __forceinline__ void load_tile(const CUtensorMap* map, int row0, int bh, uint8_t* dst,
-                                          uint64_t* bar, uint64_t pol) {
-#pragma unroll
-  for (int c = 0; c < Cfg<D>::kChunks; ++c)
-    tma_load_3d(dst + c * kChunkBytes, map, bar, c * 64, row0, bh, pol);
-}
-
-template <int D>
-__device__ __forceinline__ bool prod_load_kv(Smem<D>& sm, const Params& p, const CUtensorMap* map,
-                                             ProdSlot& s, int j, ProdShared& ps, int lane) {
-  using C = Cfg<D>;
-  const int stage = ps.kv_cnt % C::kStages;
-  const uint32_t phase = (ps.kv_cnt / C::kStages) & 1;
-  const int chunk = j >> 5;
-  if (chunk != s.chunk) {
-    s.idx = chunk_index(p, s.cur, chunk, lane);
-    s.chunk = chunk;
-  }
-  const int kvb = __shfl_sync(0xffffffffu, s.idx, j & 31);
-  if (!wait_lane0(sm, &sm.kv_empty[stage], phase ^ 1, p)) return false;
-  if (elect_one_sync()) {
-    mbar_arrive_expect_tx(&sm.kv_full[stage], C::kTileBytes);
-    load_tile<D>(map, kvb * kBlockN, s.cur.bh, sm.kv[stage], &sm.kv_full[stage], ps.pol_kv);
-  }
-  __syncwarp();
-  ++ps.kv_cnt;
-  return true;
-}
-
-// Make `nxt` current (its first index chunk is already in flight) and look one unit ahead.
-__device__ __forceinline__ void prod_advance(ProdSlot& s, const Params& p, int lane) {
-  s.has_cur = s.has_nxt;
-  s.cur = s.nxt;
-  s.idx = s.nxt_idx;
-  s.chunk = 0;
-  s.j = 0;
-  s.has_nxt = s.it.pop_nonempty(s.nxt);
-  if (s.has_nxt) s.nxt_idx = chunk_index(p, s.nxt, 0, lane);
-}
-
-// Q and K_0 of the slot's current unit.
-template <int D, int SLOT>
-__device__ __forceinline__ bool prod_start_unit(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
-                                                const CUtensorMap* tk, ProdSlot& s, ProdShared& ps,
-                                                int lane) {
-  using C = Cfg<D>;
-  const int b = s.units % C::kQBuf;
-  const uint32_t phase = (s.units / C::kQBuf) & 1;
-  if (!wait_lane0(sm, &sm.q_empty[SLOT][b], phase ^ 1, p)) return false;
-  if (elect_one_sync()) {
-    mbar_arrive_expect_tx(&sm.q_full[SLOT][b], C::kTileBytes);
-    load_tile<D>(tq, s.cur.qblk * kBlockN, s.cur.bh, sm.q[SLOT][b], &sm.q_full[SLOT][b], ps.pol_q);
-  }
-  __syncwarp();
-  ++s.units;
-  return prod_load_kv<D>(sm, p, tk, s, 0, ps, lane);
-}
-
-template <int D, int SLOT>
-__device__ __forceinline__ bool prod_init(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
-                                          const CUtensorMap* tk, ProdSlot& s, ProdShared& ps, int lane) {
-  s.it.init(p, SLOT);
-  s.units = 0;
-  s.has_nxt = s.it.pop_nonempty(s.nxt);
-  if (s.has_nxt) s.nxt_idx = chunk_index(p, s.nxt, 0, lane);
-  prod_advance(s, p, lane);
-  return s.has_cur ? prod_start_unit<D, SLOT>(sm, p, tq, tk, s, ps, lane) : true;
-}
-
-// V_j of the current block, then K_{j+1} (or the next unit's Q and K_0).
-template <int D, int SLOT>
-__device__ __forceinline__ bool prod_step(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
-                                          const CUtensorMap* tk, const CUtensorMap* tv, ProdSlot& s,
-                                          ProdShared& ps, int lane, bool& any) {
-  if (!s.has_cur) return true;
-  any = true;
-  if (!prod_load_kv<D>(sm, p, tv, s, s.j, ps, lane)) return false;
-  ++s.j;
-  if (s.j < s.cur.n) return prod_load_kv<D>(sm, p, tk, s, s.j, ps, lane);
-  prod_advance(s, p, lane);
-  return s.has_cur ? prod_start_unit<D, SLOT>(sm, p, tq, tk, s, ps, lane) : true;
-}
-
-template <int D>
-__device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
-                              const CUtensorMap* tk, const CUtensorMap* tv) {
-  using C = Cfg<D>;
-  static_assert(kNumSlots == 2, "the producer loop visits two slots");
-  const int lane = threadIdx.x & 31;
-  ProdShared ps;
-  ps.kv_cnt = 0;
-  ps.pol_kv = policy_evict_last();
-  ps.pol_q = policy_evict_first();
-  ProdSlot s0, s1;
-  bool ok = prod_init<D, 0>(sm, p, tq, tk, s0, ps, lane);
-  if (ok) ok = prod_init<D, 1>(sm, p, tq, tk, s1, ps, lane);
-  bool any = true;
-  while (ok && any) {
-    any = false;
-    ok = prod_step<D, 0>(sm, p, tq, tk, tv, s0, ps, lane, any);
-    if (ok) ok = prod_step<D, 1>(sm, p, tq, tk, tv, s1, ps, lane, any);
-  }
-  if (!ok && elect_one_sync()) {
-    // Drain: wait (bounded) for every TMA copy this warp armed, so that no copy
-    // lands in shared memory after the CTA has exited.
-    const uint64_t t0 = globaltimer_ns();
-    for (int stage = 0; stage < C::kStages; ++stage) {
-      const int fills = ps.kv_cnt / C::kStages + (stage < ps.kv_cnt % C::kStages ? 1 : 0);
-      if (fills == 0) continue;
-      while (!mbar_try_wait(&sm.kv_full[stage], (fills - 1) & 1) &&
-             globaltimer_ns() - t0 < p.timeout_ns) {
-      }
-    }
-    for (int slot = 0; slot < kNumSlots; ++slot) {
-      const int units = slot == 0 ? s0.units : s1.units;
-      for (int b = 0; b < C::kQBuf; ++b) {
-        const int fills = units > b ? (units - 1 - b) / C::kQBuf + 1 : 0;
-        if (fills == 0) continue;
-        while (!mbar_try_wait(&sm.q_full[slot][b], (fills - 1) & 1) &&
-               globaltimer_ns() - t0 < p.timeout_ns) {
-        }
-      }
-    }
-  }
-  __syncwarp();
-}
-
-// MMA issuer: one elected thread issues every tcgen05.mma of the CTA.  Per slot and
-// block j it issues PV_{j-1} then S_j, so each slot alternates between the tensor
-// core and its softmax warpgroup while the other slot fills the gap.
-struct MmaSlot {
-  UnitIter it;
-  Unit cur;
-  bool active;
-  int j;      // block whose PV is issued next
-  int units;  // non-empty units started on this slot
-  int blk;    // blocks finished on this slot (p_full phase)
-};
-
-struct MmaShared {
-  int kv_cnt;
-  uint32_t tmem, idesc_s, idesc_pv;
-  bool split;
-};
-
-template <int D, int SLOT>
-__device__ __forceinline__ bool mma_issue_s(Smem<D>& sm, const Params& p, MmaSlot& s, int j,
-                                            MmaShared& ms) {
-  using C = Cfg<D>;
-  const int b = (s.units - 1) % C::kQBuf;  // Q buffer of the current unit
-  if (j == 0 && !wait_lane0(sm, &sm.q_full[SLOT][b], ((s.units - 1) / C::kQBuf) & 1, p)) return false;
-  const int stage = ms.kv_cnt % C::kStages;
-  if (!wait_lane0(sm, &sm.kv_full[stage], (ms.kv_cnt / C::kStages) & 1, p)) return false;
-  tc_fence_after();
-  // descriptors are warp-uniform: computed by every lane, issued by one
-  const uint64_t qd = sdesc_sw128(smem_u32(sm.q[SLOT][b]), 16, 1024);
-  const uint64_t kd = sdesc_sw128(smem_u32(sm.kv[stage]), 16, 1024);
-  const uint32_t d_s = ms.tmem + C::s_col(SLOT);
-  const bool last = j == s.cur.n - 1;
-  if (elect_one_sync()) {
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      // K step kk: 32 bytes into the 128-byte swizzled row, chunk kk / 4
-      const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
-      umma_ss(d_s, qd + off, kd + off, ms.idesc_s, kk > 0 ? 1u : 0u);
-    }
-    umma_commit(&sm.kv_empty[stage]);
-    umma_commit(&sm.s_full[SLOT]);
-    if (last) umma_commit(&sm.q_empty[SLOT][b]);
-  }
-  __syncwarp();
-  ++ms.kv_cnt;
-  return true;
-}
-
-template <int D, int SLOT>
-__device__ __forceinline__ bool mma_issue_pv(Smem<D>& sm, const Params& p, MmaSlot& s, MmaShared& ms) {
-  using C = Cfg<D>;
-  if (!wait_lane0(sm, &sm.p_full[SLOT], s.blk & 1, p)) return false;
-  // O of this slot is free once the epilogue of its previous unit has read it
-  if (s.j == 0 && !wait_lane0(sm, &sm.o_empty[SLOT], ((s.units - 1) & 1) ^ 1, p)) return false;
-  const int stage = ms.kv_cnt % C::kStages;
-  if (!wait_lane0(sm, &sm.kv_full[stage], (ms.kv_cnt / C::kStages) & 1, p)) return false;
-  tc_fence_after();
-  const uint64_t vd = sdesc_sw128(smem_u32(sm.kv[stage]), kChunkBytes, 1024);
-  const uint32_t d_o = ms.tmem + C::o_col(SLOT);
-  const uint32_t a_p = ms.tmem + C::s_col(SLOT);
-  const uint32_t acc0 = s.j > 0 ? 1u : 0u;
-  const bool last = s.j == s.cur.n - 1;
-  if (elect_one_sync()) {
-    // K step kk covers 16 rows of V (2048 bytes, two 8-row swizzle atoms)
-#pragma unroll
-    for (int kk = 0; kk < kBlockN / 16; ++kk)
-      umma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * 128), ms.idesc_pv,
-              kk > 0 ? 1u : acc0);
-    if (ms.split) {
-#pragma unroll
-      for (int kk = 0; kk < kBlockN / 16; ++kk)
-        umma_ts(d_o, a_p + 64 + kk * 8, vd + static_cast<uint64_t>(kk * 128), ms.idesc_pv, 1u);
-    }
-    umma_commit(&sm.kv_empty[stage]);
-    if (last) umma_commit(&sm.o_full[SLOT]);
-  }
-  __syncwarp();
-  ++ms.kv_cnt;
-  ++s.blk;
-  return true;
-}
-
-template <int D, int SLOT>
-__device__ __forceinline__ bool mma_start_unit(Smem<D>& sm, const Params& p, MmaSlot& s, MmaShared& ms) {
-  s.active = s.it.pop_nonempty(s.cur);
-  if (!s.active) return true;
-  s.j = 0;
-  ++s.units;
-  return mma_issue_s<D, SLOT>(sm, p, s, 0, ms);
-}
-
-template <int D, int SLOT>
-__device__ __forceinline__ bool mma_step(Smem<D>& sm, const Params& p, MmaSlot& s, MmaShared& ms,
-                                         bool& any) {
-  if (!s.active) return true;
-  any = true;
-  if (!mma_issue_pv<D, SLOT>(sm, p, s, ms)) return false;
-  ++s.j;
-  return s.j < s.cur.n ? mma_issue_s<D, SLOT>(sm, p, s, s.j, ms)
-                       : mma_start_unit<D, SLOT>(sm, p, s, ms);
-}
-
-template <int D>
-__device__ void mma_role(Smem<D>& sm, const Params& p, uint32_t tmem) {
-  static_assert(kNumSlots == 2, "the MMA loop visits two slots");
-  MmaShared ms;
-  ms.kv_cnt = 0;
-  ms.tmem = tmem;
-  ms.idesc_s = idesc_f16_f32(p.is_bf16 != 0, 128, 128, false);
-  ms.idesc_pv = idesc_f16_f32(p.is_bf16 != 0, 128, D, true);
-  ms.split = p.split_p != 0;
-  MmaSlot s0, s1;
-  s0.it.init(p, 0);
-  s1.it.init(p, 1);
-  s0.units = s1.units = 0;
-  s0.blk = s1.blk = 0;
-  bool ok = mma_start_unit<D, 0>(sm, p, s0, ms);
-  if (ok) ok = mma_start_unit<D, 1>(sm, p, s1, ms);
-  bool any = true;
-  while (ok && any) {
-    any = false;
-    ok = mma_step<D, 0>(sm, p, s0, ms, any);
-    if (ok) ok = mma_step<D, 1>(sm, p, s1, ms, any);
-  }
-  if (!ok) {
-    // Drain every MMA this warp issued before TMEM is released.
-    if (elect_one_sync()) umma_commit(&sm.drain);
-    __syncwarp();
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(&sm.drain, 0) && globaltimer_ns() - t0 < p.timeout_ns) {
-    }
-  }
-}
-
-// ---------------------------------------------------------------- separate-P roles
-// With P in its own TMEM columns each slot runs a stream of S ops one block ahead
-// of its stream of PV ops.  The MMA warp and the producer walk the same rounds:
-//   start:   S(slot 0, block 0), S(slot 1, block 0)
-//   round r: S(slot 0, r+1), S(slot 1, r+1), PV(slot 0, r), PV(slot 1, r)
-// where a slot's blocks run over its non-empty units back to back.  S ops consume
-// K tiles (and the unit's Q at block 0), PV ops consume V tiles, in that order.
-
-// A position in a slot's block stream (producer side: with block indices).
+// Producer-side position in a slot's block stream, with block indices fetched 32
+// at a time (one per lane) and the next unit's first chunk requested early.
 struct ProdCursor {
   UnitIter it;
   Unit cur, nxt;
@@ -540,6 +251,11 @@ struct ProdCursor {
   int idx, nxt_idx;
 };
 
+__device__ __forceinline__ int chunk_index(const Params& p, const Unit& x, int chunk, int lane) {
+  const int jj = chunk * 32 + lane;
+  return jj < x.n ? block_index(p, x, jj) : 0;
+}
+
 __device__ __forceinline__ void pc_enter_next(ProdCursor& c, const Params& p, int lane) {
   c.has_cur = c.has_nxt;
   c.cur = c.nxt;
@@ -547,24 +263,20 @@ __device__ __forceinline__ void pc_enter_next(ProdCursor& c, const Params& p, in
   c.chunk = 0;
   c.j = 0;
   if (c.has_cur) ++c.units;
-  c.has_nxt = c.it.pop_nonempty(c.nxt);
+  c.has_nxt = c.it.pop_nonempty(p, c.nxt);
   if (c.has_nxt) c.nxt_idx = chunk_index(p, c.nxt, 0, lane);
 }
 
 __device__ __forceinline__ void pc_init(ProdCursor& c, const Params& p, int slot, int lane) {
   c.it.init(p, slot);
   c.units = 0;
-  c.has_nxt = c.it.pop_nonempty(c.nxt);
+  c.has_nxt = c.it.pop_nonempty(p, c.nxt);
   if (c.has_nxt) c.nxt_idx = chunk_index(p, c.nxt, 0, lane);
   pc_enter_next(c, p, lane);
 }
 
-// Move to the next block of the stream; true if that entered a new unit.
-__device__ __forceinline__ bool pc_step(ProdCursor& c, const Params& p, int lane) {
-  ++c.j;
-  if (c.j < c.cur.n) return false;
-  pc_enter_next(c, p, lane);
-  return true;
+__device__ __forceinline__ void pc_step(ProdCursor& c, const Params& p, int lane) {
+  if (++c.j >= c.cur.n) pc_enter_next(c, p, lane);
 }
 
 __device__ __forceinline__ int pc_block(ProdCursor& c, const Params& p, int lane) {
@@ -577,242 +289,299 @@ __device__ __forceinline__ int pc_block(ProdCursor& c, const Params& p, int lane
 }
 
 template <int D>
-__device__ __forceinline__ bool sep_load_tile(Smem<D>& sm, const Params& p, const CUtensorMap* map,
-                                              int kvb, int bh, ProdShared& ps) {
-  using C = Cfg<D>;
-  const int stage = ps.kv_cnt % C::kStages;
-  const uint32_t phase = (ps.kv_cnt / C::kStages) & 1;
-  if (!wait_lane0(sm, &sm.kv_empty[stage], phase ^ 1, p)) return false;
+__device__ __forceinline__ void load_tile(const CUtensorMap* map, int row0, int bh, uint8_t* dst,
+                                          uint64_t* bar, uint64_t pol) {
+#pragma unroll
+  for (int c = 0; c < Cfg<D>::kChunks; ++c)
+    tma_load_3d(dst + c * kChunkBytes, map, bar, c * 64, row0, bh, pol);
+}
+
+// Arm `full` for one tile and issue its TMA copy, after `empty` shows the stage free.
+template <int D>
+__device__ __forceinline__ bool produce(Smem<D>& sm, const Params& p, const CUtensorMap* map,
+                                       int row0, int bh, uint8_t* dst, uint64_t* full,
+                                       uint64_t* empty, int fill, uint64_t pol) {
+  if (!wait_lane0(sm, empty, (fill & 1) ^ 1, p)) return false;
   if (elect_one_sync()) {
-    mbar_arrive_expect_tx(&sm.kv_full[stage], C::kTileBytes);
-    load_tile<D>(map, kvb * kBlockN, bh, sm.kv[stage], &sm.kv_full[stage], ps.pol_kv);
+    mbar_arrive_expect_tx(full, Cfg<D>::kTileBytes);
+    load_tile<D>(map, row0, bh, dst, full, pol);
   }
   __syncwarp();
-  ++ps.kv_cnt;
   return true;
 }
 
-// Loads for one S op at the K cursor: the unit's Q when at block 0, then K.
-template <int D, int SLOT>
-__device__ __forceinline__ bool sep_prod_s(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
-                                           const CUtensorMap* tk, ProdCursor& c, ProdShared& ps,
-                                           int lane) {
-  using C = Cfg<D>;
-  if (c.j == 0) {
-    const int u = c.units - 1;
-    const int b = u % C::kQBuf;
-    if (!wait_lane0(sm, &sm.q_empty[SLOT][b], ((u / C::kQBuf) & 1) ^ 1, p)) return false;
-    if (elect_one_sync()) {
-      mbar_arrive_expect_tx(&sm.q_full[SLOT][b], C::kTileBytes);
-      load_tile<D>(tq, c.cur.qblk * kBlockN, c.cur.bh, sm.q[SLOT][b], &sm.q_full[SLOT][b], ps.pol_q);
-    }
-    __syncwarp();
-  }
-  const int kvb = pc_block(c, p, lane);
-  return sep_load_tile<D>(sm, p, tk, kvb, c.cur.bh, ps);
-}
-
-// The V load of a slot's PV op r reads the block its K load of round r - 1 read,
-// so the K cursor leaves a one-entry record {bh, block} behind for it.
-struct PendingV {
-  int bh, kvb;
-  bool valid;
+struct ProdCounts {
+  int k, v;  // K / V tiles issued on this slot
 };
 
 template <int D, int SLOT>
-__device__ __forceinline__ bool sep_prod_round_s(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
-                                                 const CUtensorMap* tk, ProdCursor& c, PendingV& pv,
-                                                 ProdShared& ps, int lane) {
-  if (!c.has_cur) {
-    pv.valid = false;
-    return true;
+__device__ __forceinline__ bool produce_k(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
+                                          const CUtensorMap* tk, ProdCursor& c, ProdCounts& n,
+                                          int kvb, uint64_t pol_q, uint64_t pol_kv) {
+  using C = Cfg<D>;
+  if (c.j == 0) {  // the unit's Q tile first
+    const int u = c.units - 1;
+    const int b = u % C::kQBuf;
+    if (!produce<D>(sm, p, tq, c.cur.qblk * kBlockN, c.cur.bh, sm.q[SLOT][b], &sm.q_full[SLOT][b],
+                    &sm.q_empty[SLOT][b], u / C::kQBuf, pol_q))
+      return false;
   }
-  pv.bh = c.cur.bh;
-  pv.kvb = pc_block(c, p, lane);
-  pv.valid = true;
-  pc_step(c, p, lane);
-  return c.has_cur ? sep_prod_s<D, SLOT>(sm, p, tq, tk, c, ps, lane) : true;
+  const int st = n.k % C::kKRing;
+  if (!produce<D>(sm, p, tk, kvb * kBlockN, c.cur.bh, sm.k[SLOT][st], &sm.k_full[SLOT][st],
+                  &sm.k_empty[SLOT][st], n.k / C::kKRing, pol_kv))
+    return false;
+  ++n.k;
+  return true;
 }
 
-template <int D>
-__device__ void producer_role_sep(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
-                                  const CUtensorMap* tk, const CUtensorMap* tv) {
+template <int D, int SLOT>
+__device__ __forceinline__ bool produce_v(Smem<D>& sm, const Params& p, const CUtensorMap* tv,
+                                          ProdCounts& n, int kvb, int bh, uint64_t pol_kv) {
   using C = Cfg<D>;
-  static_assert(kNumSlots == 2, "the producer loop visits two slots");
+  const int st = n.v % C::kVRing;
+  if (!produce<D>(sm, p, tv, kvb * kBlockN, bh, sm.v[SLOT][st], &sm.v_full[SLOT][st],
+                  &sm.v_empty[SLOT][st], n.v / C::kVRing, pol_kv))
+    return false;
+  ++n.v;
+  return true;
+}
+
+// One producer warp per slot.  Separate-P layout: K runs one block ahead of V
+// (K_0, K_1, V_0, K_2, V_1, ...), matching S_{i+1} being issued during softmax i.
+// Aliased layout: K_i, V_i, K_{i+1}, ...
+template <int D, int SLOT>
+__device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
+                              const CUtensorMap* tk, const CUtensorMap* tv) {
+  using C = Cfg<D>;
   const int lane = threadIdx.x & 31;
-  ProdShared ps;
-  ps.kv_cnt = 0;
-  ps.pol_kv = policy_evict_last();
-  ps.pol_q = policy_evict_first();
-  ProdCursor k0, k1;
-  PendingV v0, v1;
-  pc_init(k0, p, 0, lane);
-  pc_init(k1, p, 1, lane);
+  const uint64_t pol_kv = policy_evict_last();
+  const uint64_t pol_q = policy_evict_first();
+  ProdCursor c;
+  ProdCounts n{0, 0};
+  pc_init(c, p, SLOT, lane);
   bool ok = true;
-  if (k0.has_cur) ok = sep_prod_s<D, 0>(sm, p, tq, tk, k0, ps, lane);
-  if (ok && k1.has_cur) ok = sep_prod_s<D, 1>(sm, p, tq, tk, k1, ps, lane);
-  while (ok && (k0.has_cur || k1.has_cur)) {
-    ok = sep_prod_round_s<D, 0>(sm, p, tq, tk, k0, v0, ps, lane);
-    if (ok) ok = sep_prod_round_s<D, 1>(sm, p, tq, tk, k1, v1, ps, lane);
-    if (ok && v0.valid) ok = sep_load_tile<D>(sm, p, tv, v0.kvb, v0.bh, ps);
-    if (ok && v1.valid) ok = sep_load_tile<D>(sm, p, tv, v1.kvb, v1.bh, ps);
+  if constexpr (C::kSepP) {
+    int pend_kvb = 0, pend_bh = 0;
+    bool pend = false;
+    if (c.has_cur) {
+      pend_kvb = pc_block(c, p, lane);
+      pend_bh = c.cur.bh;
+      pend = true;
+      ok = produce_k<D, SLOT>(sm, p, tq, tk, c, n, pend_kvb, pol_q, pol_kv);
+    }
+    while (ok && pend) {
+      pc_step(c, p, lane);
+      int next_kvb = 0, next_bh = 0;
+      const bool next = c.has_cur;
+      if (next) {
+        next_kvb = pc_block(c, p, lane);
+        next_bh = c.cur.bh;
+        ok = produce_k<D, SLOT>(sm, p, tq, tk, c, n, next_kvb, pol_q, pol_kv);
+      }
+      if (ok) ok = produce_v<D, SLOT>(sm, p, tv, n, pend_kvb, pend_bh, pol_kv);
+      pend = next;
+      pend_kvb = next_kvb;
+      pend_bh = next_bh;
+    }
+  } else {
+    while (ok && c.has_cur) {
+      const int kvb = pc_block(c, p, lane);
+      ok = produce_k<D, SLOT>(sm, p, tq, tk, c, n, kvb, pol_q, pol_kv);
+      if (ok) ok = produce_v<D, SLOT>(sm, p, tv, n, kvb, c.cur.bh, pol_kv);
+      pc_step(c, p, lane);
+    }
   }
   if (!ok && elect_one_sync()) {
+    // Drain: wait (bounded) for every TMA copy this warp armed, so that no copy
+    // lands in shared memory after the CTA has exited.
     const uint64_t t0 = globaltimer_ns();
-    for (int stage = 0; stage < C::kStages; ++stage) {
-      const int fills = ps.kv_cnt / C::kStages + (stage < ps.kv_cnt % C::kStages ? 1 : 0);
-      if (fills == 0) continue;
-      while (!mbar_try_wait(&sm.kv_full[stage], (fills - 1) & 1) &&
+    for (int st = 0; st < C::kKRing; ++st) {
+      const int fills = n.k / C::kKRing + (st < n.k % C::kKRing ? 1 : 0);
+      while (fills > 0 && !mbar_try_wait(&sm.k_full[SLOT][st], (fills - 1) & 1) &&
              globaltimer_ns() - t0 < p.timeout_ns) {
       }
     }
-    for (int slot = 0; slot < kNumSlots; ++slot) {
-      const int units = slot == 0 ? k0.units : k1.units;
-      for (int b = 0; b < C::kQBuf; ++b) {
-        const int fills = units > b ? (units - 1 - b) / C::kQBuf + 1 : 0;
-        if (fills == 0) continue;
-        while (!mbar_try_wait(&sm.q_full[slot][b], (fills - 1) & 1) &&
-               globaltimer_ns() - t0 < p.timeout_ns) {
-        }
+    for (int st = 0; st < C::kVRing; ++st) {
+      const int fills = n.v / C::kVRing + (st < n.v % C::kVRing ? 1 : 0);
+      while (fills > 0 && !mbar_try_wait(&sm.v_full[SLOT][st], (fills - 1) & 1) &&
+             globaltimer_ns() - t0 < p.timeout_ns) {
+      }
+    }
+    for (int b = 0; b < C::kQBuf; ++b) {
+      const int fills = c.units > b ? (c.units - 1 - b) / C::kQBuf + 1 : 0;
+      while (fills > 0 && !mbar_try_wait(&sm.q_full[SLOT][b], (fills - 1) & 1) &&
+             globaltimer_ns() - t0 < p.timeout_ns) {
       }
     }
   }
   __syncwarp();
 }
 
-// MMA-side position in a slot's block stream.
-struct MmaCursor {
+// MMA-side position in a slot's block stream (no block indices needed).
+struct MmaStream {
   UnitIter it;
   Unit cur;
   bool active;
   int j;      // block of `cur`
   int units;  // non-empty units entered
-  int ops;    // ops issued on this stream (barrier phase)
+  int i;      // position in the slot's block stream
 };
 
-__device__ __forceinline__ void mc_enter_next(MmaCursor& c) {
-  c.active = c.it.pop_nonempty(c.cur);
+__device__ __forceinline__ void ms_enter_next(MmaStream& c, const Params& p) {
+  c.active = c.it.pop_nonempty(p, c.cur);
   c.j = 0;
   if (c.active) ++c.units;
 }
-__device__ __forceinline__ void mc_init(MmaCursor& c, const Params& p, int slot) {
+__device__ __forceinline__ void ms_init(MmaStream& c, const Params& p, int slot) {
   c.it.init(p, slot);
   c.units = 0;
-  c.ops = 0;
-  mc_enter_next(c);
+  c.i = 0;
+  ms_enter_next(c, p);
 }
-__device__ __forceinline__ void mc_step(MmaCursor& c) {
-  ++c.ops;
-  if (++c.j >= c.cur.n) mc_enter_next(c);
+__device__ __forceinline__ void ms_step(MmaStream& c, const Params& p) {
+  ++c.i;
+  if (++c.j >= c.cur.n) ms_enter_next(c, p);
 }
 
+struct MmaShared {
+  uint32_t tmem, idesc_s, idesc_pv;
+  bool split;
+};
+
+// Probe shared by lanes: lane 0 tests the phase, the warp gets the answer.
+__device__ __forceinline__ bool probe(uint64_t* bar, uint32_t parity) {
+  uint32_t ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_test_wait(bar, parity) ? 1u : 0u;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// S_i = Q K_i^T for the slot's stream position `c`, if its inputs are ready.
+// `prev_done`: the S buffer may be overwritten (aliased layout: PV_{i-1} issued;
+// separate-P layout: the softmax has read S_{i-1}).
 template <int D, int SLOT>
-__device__ __forceinline__ bool sep_mma_s(Smem<D>& sm, const Params& p, MmaCursor& c, MmaShared& ms) {
+__device__ __forceinline__ bool try_s(Smem<D>& sm, const Params& p, MmaStream& c, MmaShared& ms) {
   using C = Cfg<D>;
   const int u = c.units - 1;
   const int b = u % C::kQBuf;
-  // the softmax must have read the previous S of this slot
-  if (c.ops > 0 && !wait_lane0(sm, &sm.s_empty[SLOT], (c.ops - 1) & 1, p)) return false;
-  if (c.j == 0 && !wait_lane0(sm, &sm.q_full[SLOT][b], (u / C::kQBuf) & 1, p)) return false;
-  const int stage = ms.kv_cnt % C::kStages;
-  if (!wait_lane0(sm, &sm.kv_full[stage], (ms.kv_cnt / C::kStages) & 1, p)) return false;
+  const int st = c.i % C::kKRing;
+  if constexpr (C::kSepP) {
+    if (c.i > 0 && !probe(&sm.s_empty[SLOT], (c.i - 1) & 1)) return false;
+  }
+  if (c.j == 0 && !probe(&sm.q_full[SLOT][b], (u / C::kQBuf) & 1)) return false;
+  if (!probe(&sm.k_full[SLOT][st], (c.i / C::kKRing) & 1)) return false;
   tc_fence_after();
+  // descriptors are warp-uniform: computed by every lane, issued by one
   const uint64_t qd = sdesc_sw128(smem_u32(sm.q[SLOT][b]), 16, 1024);
-  const uint64_t kd = sdesc_sw128(smem_u32(sm.kv[stage]), 16, 1024);
+  const uint64_t kd = sdesc_sw128(smem_u32(sm.k[SLOT][st]), 16, 1024);
   const uint32_t d_s = ms.tmem + C::s_col(SLOT);
   const bool last = c.j == c.cur.n - 1;
   if (elect_one_sync()) {
-#pragma unroll
+    // (fully unrolled at D=64, where the MMAs are short enough for issue cost to show)
+#pragma unroll(D == 64 ? 4 : 1)
     for (int kk = 0; kk < D / 16; ++kk) {
+      // K step kk: 32 bytes into the 128-byte swizzled row, chunk kk / 4
       const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
       umma_ss(d_s, qd + off, kd + off, ms.idesc_s, kk > 0 ? 1u : 0u);
     }
-    umma_commit(&sm.kv_empty[stage]);
+    umma_commit(&sm.k_empty[SLOT][st]);
     umma_commit(&sm.s_full[SLOT]);
     if (last) umma_commit(&sm.q_empty[SLOT][b]);
   }
   __syncwarp();
-  ++ms.kv_cnt;
+  ms_step(c, p);
   return true;
 }
 
-// The PV op of round r is the block the S op of round r - 1 covered: the S cursor
-// leaves {first, last, unit number} behind for it.
-struct PendingPV {
-  bool valid, first, last;
-  int units;  // non-empty units entered when that block was current
-  int ops;    // PV ops issued on this slot
-};
-
+// O += P_i V_i for the slot's stream position `c`, if its inputs are ready.
 template <int D, int SLOT>
-__device__ __forceinline__ bool sep_mma_pv(Smem<D>& sm, const Params& p, PendingPV& v, MmaShared& ms) {
+__device__ __forceinline__ bool try_pv(Smem<D>& sm, const Params& p, MmaStream& c, MmaShared& ms) {
   using C = Cfg<D>;
-  if (!wait_lane0(sm, &sm.p_full[SLOT], v.ops & 1, p)) return false;
+  const int st = c.i % C::kVRing;
+  if (!probe(&sm.p_full[SLOT], c.i & 1)) return false;
   // O of this slot is free once the epilogue of its previous unit has read it
-  if (v.first && v.units > 1 && !wait_lane0(sm, &sm.o_empty[SLOT], (v.units - 2) & 1, p))
-    return false;
-  const int stage = ms.kv_cnt % C::kStages;
-  if (!wait_lane0(sm, &sm.kv_full[stage], (ms.kv_cnt / C::kStages) & 1, p)) return false;
+  if (c.j == 0 && c.units > 1 && !probe(&sm.o_empty[SLOT], (c.units - 2) & 1)) return false;
+  if (!probe(&sm.v_full[SLOT][st], (c.i / C::kVRing) & 1)) return false;
   tc_fence_after();
-  const uint64_t vd = sdesc_sw128(smem_u32(sm.kv[stage]), kChunkBytes, 1024);
+  const uint64_t vd = sdesc_sw128(smem_u32(sm.v[SLOT][st]), kChunkBytes, 1024);
   const uint32_t d_o = ms.tmem + C::o_col(SLOT);
   const uint32_t a_p = ms.tmem + C::p_col(SLOT);
-  const uint32_t acc0 = v.first ? 0u : 1u;
-  const bool last = v.last;
+  const uint32_t acc0 = c.j > 0 ? 1u : 0u;
+  const bool last = c.j == c.cur.n - 1;
   if (elect_one_sync()) {
-#pragma unroll
+    // K step kk covers 16 rows of V (2048 bytes, two 8-row swizzle atoms)
+#pragma unroll(D == 64 ? 8 : 1)
     for (int kk = 0; kk < kBlockN / 16; ++kk)
       umma_ts(d_o, a_p + kk * 8, vd + static_cast<uint64_t>(kk * 128), ms.idesc_pv,
               kk > 0 ? 1u : acc0);
-    umma_commit(&sm.kv_empty[stage]);
-    umma_commit(&sm.pv_done[SLOT]);
+    if (ms.split) {
+#pragma unroll 1
+      for (int kk = 0; kk < kBlockN / 16; ++kk)
+        umma_ts(d_o, a_p + 64 + kk * 8, vd + static_cast<uint64_t>(kk * 128), ms.idesc_pv, 1u);
+    }
+    umma_commit(&sm.v_empty[SLOT][st]);
+    if constexpr (C::kSepP) umma_commit(&sm.pv_done[SLOT]);
     if (last) umma_commit(&sm.o_full[SLOT]);
   }
   __syncwarp();
-  ++ms.kv_cnt;
-  ++v.ops;
+  ms_step(c, p);
   return true;
 }
 
+// Per slot: its S stream and its PV stream (the PV stream trails).  In the aliased
+// layout S_{i+1} may only follow PV_i (the MMAs of one thread run in issue order,
+// so PV_i has read P before S_{i+1} overwrites it).
 template <int D, int SLOT>
-__device__ __forceinline__ bool sep_mma_round_s(Smem<D>& sm, const Params& p, MmaCursor& c,
-                                                PendingPV& v, MmaShared& ms) {
-  if (!c.active) {
-    v.valid = false;
-    return true;
-  }
-  v.valid = true;
-  v.first = c.j == 0;
-  v.last = c.j == c.cur.n - 1;
-  v.units = c.units;
-  mc_step(c);
-  return c.active ? sep_mma_s<D, SLOT>(sm, p, c, ms) : true;
+__device__ __forceinline__ bool mma_slot(Smem<D>& sm, const Params& p, MmaStream& cs,
+                                         MmaStream& cp, MmaShared& ms) {
+  bool progress = false;
+  if (cs.active && (Cfg<D>::kSepP || cs.i == cp.i)) progress |= try_s<D, SLOT>(sm, p, cs, ms);
+  if (cp.active && (!cs.active || cp.i < cs.i)) progress |= try_pv<D, SLOT>(sm, p, cp, ms);
+  return progress;
 }
 
 template <int D>
-__device__ void mma_role_sep(Smem<D>& sm, const Params& p, uint32_t tmem) {
-  static_assert(kNumSlots == 2, "the MMA loop visits two slots");
+__device__ void mma_role(Smem<D>& sm, const Params& p, uint32_t tmem) {
+  static_assert(kNumSlots == 2, "the MMA loop serves two slots");
   MmaShared ms;
-  ms.kv_cnt = 0;
   ms.tmem = tmem;
   ms.idesc_s = idesc_f16_f32(p.is_bf16 != 0, 128, 128, false);
   ms.idesc_pv = idesc_f16_f32(p.is_bf16 != 0, 128, D, true);
-  ms.split = false;
-  MmaCursor s0, s1;  // S streams of the two slots
-  PendingPV v0, v1;  // their PV streams, one block behind
-  v0.ops = v1.ops = 0;
-  mc_init(s0, p, 0);
-  mc_init(s1, p, 1);
+  ms.split = p.split_p != 0 && !Cfg<D>::kSepP;
+  MmaStream s0, p0, s1, p1;
+  ms_init(s0, p, 0);
+  ms_init(p0, p, 0);
+  ms_init(s1, p, 1);
+  ms_init(p1, p, 1);
   bool ok = true;
-  if (s0.active) ok = sep_mma_s<D, 0>(sm, p, s0, ms);
-  if (ok && s1.active) ok = sep_mma_s<D, 1>(sm, p, s1, ms);
-  while (ok && (s0.active || s1.active)) {
-    ok = sep_mma_round_s<D, 0>(sm, p, s0, v0, ms);
-    if (ok) ok = sep_mma_round_s<D, 1>(sm, p, s1, v1, ms);
-    if (ok && v0.valid) ok = sep_mma_pv<D, 0>(sm, p, v0, ms);
-    if (ok && v1.valid) ok = sep_mma_pv<D, 1>(sm, p, v1, ms);
+  uint64_t last_progress = 0;  // 0: progress since the last idle check
+  int idle = 0;
+  while (p0.active || p1.active) {
+    bool progress = mma_slot<D, 0>(sm, p, s0, p0, ms);
+    progress |= mma_slot<D, 1>(sm, p, s1, p1, ms);
+    if (progress) {
+      idle = 0;
+      last_progress = 0;
+      continue;
+    }
+    // nothing ready: back off briefly, and give up after the timeout
+    if (++idle >= 64) {
+      idle = 0;
+      const uint64_t now = globaltimer_ns();
+      if (last_progress == 0) last_progress = now;
+      if (sm.abort_flag) {
+        ok = false;
+        break;
+      }
+      if (now - last_progress > p.timeout_ns) {
+        sm.abort_flag = 1;
+        if ((threadIdx.x & 31) == 0) atomicOr(p.err, kDevErrTimeout);
+        ok = false;
+        break;
+      }
+    }
   }
   if (!ok) {
+    // Drain every MMA this warp issued before TMEM is released.
     if (elect_one_sync()) umma_commit(&sm.drain);
     __syncwarp();
     const uint64_t t0 = globaltimer_ns();
@@ -915,7 +684,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
   int blk = 0, units = 0;
   Unit un;
 
-  while (it.pop(un)) {
+  while (it.pop(p, un)) {
     const int row = un.qblk * kBlockN + t;
     const bool valid = row < p.L;
     const size_t orow = static_cast<size_t>(un.bh) * p.L + row;
@@ -1107,17 +876,21 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
       mbar_init(&sm.p_full[s], 4);   // one arrival per softmax warp
       mbar_init(&sm.o_full[s], 1);
       mbar_init(&sm.o_empty[s], 4);
-    }
-    for (int i = 0; i < Cfg<D>::kStages; ++i) {
-      mbar_init(&sm.kv_full[i], 1);
-      mbar_init(&sm.kv_empty[i], 1);
+      for (int i = 0; i < Cfg<D>::kKRing; ++i) {
+        mbar_init(&sm.k_full[s][i], 1);
+        mbar_init(&sm.k_empty[s][i], 1);
+      }
+      for (int i = 0; i < Cfg<D>::kVRing; ++i) {
+        mbar_init(&sm.v_full[s][i], 1);
+        mbar_init(&sm.v_empty[s][i], 1);
+      }
     }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == kProducerWarp && (threadIdx.x & 31) == 0) {
-    prefetch_tensormap(&tmap_q);
+    prefetch_tensormap(&tmap_q);  // the other producer warp shares the cached maps
     prefetch_tensormap(&tmap_k);
     prefetch_tensormap(&tmap_v);
   }
@@ -1141,15 +914,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
   }
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == kProducerWarp) {
-    if constexpr (Cfg<D>::kSepP)
-      producer_role_sep<D>(sm, p, &tmap_q, &tmap_k, &tmap_v);
-    else
-      producer_role<D>(sm, p, &tmap_q, &tmap_k, &tmap_v);
+    producer_role<D, 0>(sm, p, &tmap_q, &tmap_k, &tmap_v);
+  } else if (warp == kProducerWarp + 1) {
+    producer_role<D, 1>(sm, p, &tmap_q, &tmap_k, &tmap_v);
   } else if (warp == kMmaWarp) {
-    if constexpr (Cfg<D>::kSepP)
-      mma_role_sep<D>(sm, p, tmem);
-    else
-      mma_role<D>(sm, p, tmem);
+    mma_role<D>(sm, p, tmem);
   }
   tc_fence_before();
   named_barrier_sync(1, kThreads);
