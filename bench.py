@@ -42,6 +42,33 @@ PAGE_FWD_MS = {"swa256_L32768_B1_H8_D64_bf16": 75.27, "causal_L8192_B1_H8_D64_bf
                "swa64_L8192_B1_H8_D64_bf16": 11.75, "swa256_L8192_B1_H8_D64_bf16": 19.14,
                "swa1024_L8192_B1_H8_D64_bf16": 56.24, "swa4096_L8192_B1_H8_D64_bf16": 169.24}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one forward launch from an ncu capture, per workload,
+# with the hash of the kernel sources it was taken on: reported as roofline.traffic
+# only while the sources still hash to that value (null once the kernel changed).
+KERNEL_SOURCES = ("block_sparse_attention_create_b200/csrc/fwd_sm100.cu",
+                  "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
+NCU_TRAFFIC = {
+    "swa256_L32768_B1_H8_D64_bf16": {
+        "bytes": 101163264 + 6274048,
+        "sources_sha256": "29fc015b38e3672630f87c6944e33c9db5c9cfbfc7b5a530dd6e83a440efc772",
+        "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_full.md"},
+}
+
+
+def kernel_sources_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(w: W.Workload):
+    rec = NCU_TRAFFIC.get(w.name)
+    if rec is None or rec["sources_sha256"] != kernel_sources_hash():
+        return None
+    return rec["bytes"]
 
 
 def load_peaks():
@@ -294,7 +321,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=W.C3_SWA256_32K.name, choices=sorted(W.BY_NAME))
-    ap.add_argument("--cpu-rows", type=int, default=2048,
+    ap.add_argument("--cpu-rows", type=int, default=32768,
                     help="oracle rows timed for cpu_baseline (bounded sample)")
     ap.add_argument("--profile", action="store_true",
                     help="short run for profilers: warm-up and timed steps only (no clock "
@@ -354,10 +381,10 @@ def main():
     bound = "hbm" if hbm_frac >= tensor_frac else "tensor"
     if bound == "hbm":
         roof = {"bound": "hbm", "achieved": fwd_gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": hbm_frac, "traffic": None}
+                "frac": hbm_frac, "traffic": ncu_traffic(w)}
     else:
         roof = {"bound": "tensor", "achieved": fwd_tflops, "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": tensor_frac, "traffic": None}
+                "frac": tensor_frac, "traffic": ncu_traffic(w)}
     roof["peak_source"] = f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"
     roof["kernel"] = "fwd_kernel (fa_flex_attention_fwd)"
     page_ms = PAGE_FWD_MS.get(w.name)

@@ -616,6 +616,8 @@ __device__ __forceinline__ void load_s_half(uint32_t taddr, float (&x)[64]) {
   tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(xr));
   tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(xr + 32));
   tmem_wait_ld();
+  reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(xr));
+  reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(xr + 32));
 #pragma unroll
   for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(xr[i]);
 }
@@ -661,6 +663,52 @@ __device__ __forceinline__ float row_max64(const float (&x)[64]) {
   mx[3] = fmax3(mx[3], mx[4], mx[5]);
   mx[6] = fmaxf(mx[6], mx[7]);
   return fmax3(mx[0], mx[3], mx[6]);
+}
+
+// x = log2(e) * c * tanh(s * scale / c), the softcap in log2 units.
+__device__ __forceinline__ void softcap64(const Params& p, float (&x)[64]) {
+#pragma unroll
+  for (int i = 0; i < 64; i += 2) {
+    const float2 e = make_float2(ex2_approx(x[i] * p.cap_k), ex2_approx(x[i + 1] * p.cap_k));
+    const float2 r = make_float2(rcp_approx(e.x + 1.f), rcp_approx(e.y + 1.f));
+    const float2 v = fma2(r, make_float2(-2.f * p.cap_a, -2.f * p.cap_a), make_float2(p.cap_a, p.cap_a));
+    x[i] = v.x;
+    x[i + 1] = v.y;
+  }
+}
+
+// O *= alpha on this thread's row (all D columns), in TMEM.
+template <int D>
+__device__ __forceinline__ void rescale_o_rows(uint32_t t_o, float alpha) {
+#pragma unroll 1
+  for (int c = 0; c < D / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(t_o + c * 32, r);
+    tmem_wait_ld();
+    reg_fence32(r);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+    tmem_st32(t_o + c * 32, r);
+  }
+}
+
+// p = exp2(x * xs - m) for 64 keys, rounded to 16-bit pairs into ph[32]; returns the
+// sum of the fp32 p.
+__device__ __forceinline__ float exp_pack64(const float (&x)[64], float xs, float neg_mu, bool bf16,
+                                            uint32_t (&ph)[32]) {
+  float2 sums[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) sums[i] = make_float2(0.f, 0.f);
+  const float2 xs2 = make_float2(xs, xs), nm2 = make_float2(neg_mu, neg_mu);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const float2 a2 = fma2(make_float2(x[2 * i], x[2 * i + 1]), xs2, nm2);
+    const float2 pp = make_float2(ex2_approx(a2.x), ex2_approx(a2.y));
+    sums[i & 3] = add2(sums[i & 3], pp);
+    ph[i] = pack2(pp.x, pp.y, bf16);
+  }
+  sums[0] = add2(add2(sums[0], sums[1]), add2(sums[2], sums[3]));
+  return sums[0].x + sums[0].y;
 }
 
 // Softmax warpgroup of one slot: thread t owns row t of the slot's 128-row tile
@@ -709,117 +757,160 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
       const int kvb_next = j + 1 < un.n ? block_index(p, un, j + 1) : 0;
       if (!wait_warp(sm, &sm.s_full[slot], blk & 1, p)) return;
       tc_fence_after();
-      // Pass 1: the block's row max from the raw scores (a PARTIAL block's masked
-      // entries excluded).  The softcap is monotone, so the max of the capped scores
-      // is the cap of the raw max.  Pass 2 then turns each half of 64 keys into P with
-      // that one max: P_hi of half h goes to P columns [32h, 32h + 32); with the
-      // split, P_lo goes to columns 64 + [32h, 32h + 32), held in registers until
-      // half 1 has been read (in the aliased layout those columns are still S).
-      const int a = lo - kvb * kBlockN;  // live columns of the block: a <= i <= b
-      const int b = hi - kvb * kBlockN;
-      float rmax = -INFINITY;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        float x[64];
-        load_s_half(t_s + h * 64, x);
-        if (!full) apply_mask(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq);
-        rmax = fmaxf(rmax, row_max64(x));
-      }
-      float mb = rmax;
-      if (rmax != -INFINITY) {
-        if (p.softcap_on) {
-          mb = p.cap_a - 2.f * p.cap_a * rcp_approx(ex2_approx(rmax * p.cap_k) + 1.f);
-        } else {
-          mb = rmax * xs;
-        }
-      }
-      const float m_new = fmaxf(m, mb);
-      // Deferred rescale: keep the stale max unless the new one exceeds it by more
-      // than 2^8; exact, because l and O always use the same max.
-      float alpha = 1.f;
-      bool rescale_o = false;
-      if (m_new > m + kRescaleThreshold) {
-        if (m != -INFINITY) {
-          alpha = ex2_approx(m - m_new);
-          l *= alpha;
-          rescale_o = true;  // O already holds contributions of this row
-        }
-        m = m_new;
-      }
-      const float neg_mu = (m == -INFINITY) ? 0.f : -m;
       if constexpr (C::kSepP) {
-        // the previous PV of this slot must be done before P is overwritten or O rescaled
+        // Separate-P layout: the whole row of S (128 columns) comes into registers at
+        // once, S is released to the MMA warp right away, and P is written per half.
+        float x[128];
+        load_s_half(t_s, *reinterpret_cast<float(*)[64]>(x));
+        load_s_half(t_s + 64, *reinterpret_cast<float(*)[64]>(x + 64));
+        tc_fence_before();
+        __syncwarp();
+        if ((t & 31) == 0) mbar_arrive(&sm.s_empty[slot]);
+        if (p.softcap_on) softcap64(p, *reinterpret_cast<float(*)[64]>(x)), softcap64(p, *reinterpret_cast<float(*)[64]>(x + 64));
+        if (!full) {
+          const int a = lo - kvb * kBlockN;
+          const int b = hi - kvb * kBlockN;
+          apply_mask(p, *reinterpret_cast<float(*)[64]>(x), a, b, kvb * kBlockN, dq);
+          apply_mask(p, *reinterpret_cast<float(*)[64]>(x + 64), a - 64, b - 64, kvb * kBlockN + 64, dq);
+        }
+        const float mb = fmaxf(row_max64(*reinterpret_cast<float(*)[64]>(x)),
+                               row_max64(*reinterpret_cast<float(*)[64]>(x + 64))) * xs;
+        const float m_new = fmaxf(m, mb);
+        float alpha = 1.f;
+        bool rescale_o = false;
+        if (m_new > m + kRescaleThreshold) {
+          if (m != -INFINITY) {
+            alpha = ex2_approx(m - m_new);
+            l *= alpha;
+            rescale_o = true;
+          }
+          m = m_new;
+        }
+        const float neg_mu = (m == -INFINITY) ? 0.f : -m;
+        uint32_t ph[32];
+        l += exp_pack64(*reinterpret_cast<float(*)[64]>(x), xs, neg_mu, bf16, ph);
+        // The previous PV of this slot must be done before P is overwritten or O
+        // rescaled; waiting here, after the first half's exponentials, hides it.
         if (blk > 0 && !wait_warp(sm, &sm.pv_done[slot], (blk - 1) & 1, p)) return;
         tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, rescale_o)) {
+        if (__any_sync(0xffffffffu, rescale_o)) rescale_o_rows<D>(t_o, alpha);
+        tmem_st32(t_p, ph);
+        l += exp_pack64(*reinterpret_cast<float(*)[64]>(x + 64), xs, neg_mu, bf16, ph);
+        tmem_st32(t_p + 32, ph);
+      } else {
+      // Pass 1: the block's row max from the raw scores (a PARTIAL block's masked
+        // entries excluded).  The softcap is monotone, so the max of the capped scores
+        // is the cap of the raw max.  Pass 2 then turns each half of 64 keys into P with
+        // that one max: P_hi of half h goes to P columns [32h, 32h + 32); with the
+        // split, P_lo goes to columns 64 + [32h, 32h + 32), held in registers until
+        // half 1 has been read (in the aliased layout those columns are still S).
+        const int a = lo - kvb * kBlockN;  // live columns of the block: a <= i <= b
+        const int b = hi - kvb * kBlockN;
+        float rmax = -INFINITY;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_o + c * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(t_o + c * 32, r);
+        for (int h = 0; h < 2; ++h) {
+          float x[64];
+          load_s_half(t_s + h * 64, x);
+          if (!full) apply_mask(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq);
+          rmax = fmaxf(rmax, row_max64(x));
         }
-      }
-      uint32_t pl_hold[32];
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        float x[64];
-        load_s_half(t_s + h * 64, x);
-        if (h == 1) {
-          if constexpr (C::kSepP) {  // all of S is read: the MMA warp may refill it
-            tc_fence_before();
-            __syncwarp();
-            if ((t & 31) == 0) mbar_arrive(&sm.s_empty[slot]);
-          }
-          if (split) tmem_st32(t_p + 64, pl_hold);
-        }
-        if (p.softcap_on) {  // x = log2(e) * c * tanh(s * scale / c)
-#pragma unroll
-          for (int i = 0; i < 64; i += 2) {
-            const float2 e = make_float2(ex2_approx(x[i] * p.cap_k), ex2_approx(x[i + 1] * p.cap_k));
-            const float2 r = make_float2(rcp_approx(e.x + 1.f), rcp_approx(e.y + 1.f));
-            const float2 v = fma2(r, make_float2(-2.f * p.cap_a, -2.f * p.cap_a),
-                                  make_float2(p.cap_a, p.cap_a));
-            x[i] = v.x;
-            x[i + 1] = v.y;
-          }
-        }
-        if (!full) apply_mask(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq);
-        // P = exp2(x * xs - m) as 16-bit pairs; with the split, P_hi = p truncated to
-        // bf16 and P_lo = round(p - P_hi), so P_hi + P_lo carries ~16 significant bits.
-        float2 sums[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) sums[i] = make_float2(0.f, 0.f);
-        const float2 xs2 = make_float2(xs, xs), nm2 = make_float2(neg_mu, neg_mu);
-        uint32_t ph[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 a2 = fma2(make_float2(x[2 * i], x[2 * i + 1]), xs2, nm2);
-          const float2 pp = make_float2(ex2_approx(a2.x), ex2_approx(a2.y));
-          sums[i & 3] = add2(sums[i & 3], pp);
-          if (!split) {
-            ph[i] = pack2(pp.x, pp.y, bf16);
-          } else if (bf16) {
-            const uint32_t u0 = __float_as_uint(pp.x), u1 = __float_as_uint(pp.y);
-            ph[i] = __byte_perm(u0, u1, 0x7632);
-            const float2 lo2 = sub2(pp, make_float2(__uint_as_float(u0 & 0xFFFF0000u),
-                                                    __uint_as_float(u1 & 0xFFFF0000u)));
-            pl_hold[i] = pack2(lo2.x, lo2.y, true);
+        float mb = rmax;
+        if (rmax != -INFINITY) {
+          if (p.softcap_on) {
+            mb = p.cap_a - 2.f * p.cap_a * rcp_approx(ex2_approx(rmax * p.cap_k) + 1.f);
           } else {
-            ph[i] = pack2(pp.x, pp.y, false);
-            float h0, h1;
-            unpack2(ph[i], false, h0, h1);
-            pl_hold[i] = pack2(pp.x - h0, pp.y - h1, false);
+            mb = rmax * xs;
           }
         }
-        tmem_st32(t_p + h * 32, ph);
-        sums[0] = add2(add2(sums[0], sums[1]), add2(sums[2], sums[3]));
-        l += sums[0].x + sums[0].y;
+        const float m_new = fmaxf(m, mb);
+        // Deferred rescale: keep the stale max unless the new one exceeds it by more
+        // than 2^8; exact, because l and O always use the same max.
+        float alpha = 1.f;
+        bool rescale_o = false;
+        if (m_new > m + kRescaleThreshold) {
+          if (m != -INFINITY) {
+            alpha = ex2_approx(m - m_new);
+            l *= alpha;
+            rescale_o = true;  // O already holds contributions of this row
+          }
+          m = m_new;
+        }
+        const float neg_mu = (m == -INFINITY) ? 0.f : -m;
+        if constexpr (C::kSepP) {
+          // the previous PV of this slot must be done before P is overwritten or O rescaled
+          if (blk > 0 && !wait_warp(sm, &sm.pv_done[slot], (blk - 1) & 1, p)) return;
+          tc_fence_after();
+        }
+        if (__any_sync(0xffffffffu, rescale_o)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(t_o + c * 32, r);
+            tmem_wait_ld();
+            reg_fence32(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(t_o + c * 32, r);
+          }
+        }
+        uint32_t pl_hold[32];
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          float x[64];
+          load_s_half(t_s + h * 64, x);
+          if (h == 1) {
+            if constexpr (C::kSepP) {  // all of S is read: the MMA warp may refill it
+              tc_fence_before();
+              __syncwarp();
+              if ((t & 31) == 0) mbar_arrive(&sm.s_empty[slot]);
+            }
+            if (split) tmem_st32(t_p + 64, pl_hold);
+          }
+          if (p.softcap_on) {  // x = log2(e) * c * tanh(s * scale / c)
+#pragma unroll
+            for (int i = 0; i < 64; i += 2) {
+              const float2 e = make_float2(ex2_approx(x[i] * p.cap_k), ex2_approx(x[i + 1] * p.cap_k));
+              const float2 r = make_float2(rcp_approx(e.x + 1.f), rcp_approx(e.y + 1.f));
+              const float2 v = fma2(r, make_float2(-2.f * p.cap_a, -2.f * p.cap_a),
+                                    make_float2(p.cap_a, p.cap_a));
+              x[i] = v.x;
+              x[i + 1] = v.y;
+            }
+          }
+          if (!full) apply_mask(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq);
+          // P = exp2(x * xs - m) as 16-bit pairs; with the split, P_hi = p truncated to
+          // bf16 and P_lo = round(p - P_hi), so P_hi + P_lo carries ~16 significant bits.
+          float2 sums[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sums[i] = make_float2(0.f, 0.f);
+          const float2 xs2 = make_float2(xs, xs), nm2 = make_float2(neg_mu, neg_mu);
+          uint32_t ph[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float2 a2 = fma2(make_float2(x[2 * i], x[2 * i + 1]), xs2, nm2);
+            const float2 pp = make_float2(ex2_approx(a2.x), ex2_approx(a2.y));
+            sums[i & 3] = add2(sums[i & 3], pp);
+            if (!split) {
+              ph[i] = pack2(pp.x, pp.y, bf16);
+            } else if (bf16) {
+              const uint32_t u0 = __float_as_uint(pp.x), u1 = __float_as_uint(pp.y);
+              ph[i] = __byte_perm(u0, u1, 0x7632);
+              const float2 lo2 = sub2(pp, make_float2(__uint_as_float(u0 & 0xFFFF0000u),
+                                                      __uint_as_float(u1 & 0xFFFF0000u)));
+              pl_hold[i] = pack2(lo2.x, lo2.y, true);
+            } else {
+              ph[i] = pack2(pp.x, pp.y, false);
+              float h0, h1;
+              unpack2(ph[i], false, h0, h1);
+              pl_hold[i] = pack2(pp.x - h0, pp.y - h1, false);
+            }
+          }
+          tmem_st32(t_p + h * 32, ph);
+          sums[0] = add2(add2(sums[0], sums[1]), add2(sums[2], sums[3]));
+          l += sums[0].x + sums[0].y;
+        }
+        if (split) tmem_st32(t_p + 96, pl_hold);
       }
-      if (split) tmem_st32(t_p + 96, pl_hold);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -837,6 +928,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
       uint32_t r[32];
       tmem_ld32(t_o + c * 32, r);
       tmem_wait_ld();
+      reg_fence32(r);
       uint32_t pk[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i)
