@@ -23,17 +23,19 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfa.so")
 
-FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+(FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT,
+ FA_ERR_SCRATCH_TOO_SMALL) = range(6)
 FA_MASK_CAUSAL, FA_MASK_SLIDING_WINDOW_CAUSAL, FA_MASK_DOCUMENT_CAUSAL = range(3)
 FA_SCORE_NONE, FA_SCORE_TANH_SOFTCAP = range(2)
 FA_BF16, FA_FP16 = range(2)
 FA_BLOCK = 128
 FA_MAX_LEN = 8192 * 128
+FA_NOALLOC_SCRATCH_BYTES = 4 << 20
 
 # Every symbol include/fa.h declares.
 EXPORTED = ("fa_block_mask_dims", "fa_create_block_mask", "fa_fwd_workspace_bytes",
             "fa_flex_attention_fwd", "fa_get_last_device_error", "fa_status_string",
-            "fa_num_sms")
+            "fa_num_sms", "fa_flex_attention_fwd_noalloc")
 
 
 class fa_block_mask(ctypes.Structure):
@@ -76,6 +78,9 @@ def _load():
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_num_sms.argtypes = []
     lib.fa_num_sms.restype = i32
+    lib.fa_flex_attention_fwd_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                                  i32, i32, vp, i32, f32, f32, vp, vp, vp, vp]
+    lib.fa_flex_attention_fwd_noalloc.restype = i32
     return lib
 
 
@@ -89,6 +94,7 @@ fa_flex_attention_fwd = _lib.fa_flex_attention_fwd
 fa_get_last_device_error = _lib.fa_get_last_device_error
 fa_status_string = _lib.fa_status_string
 fa_num_sms = _lib.fa_num_sms
+fa_flex_attention_fwd_noalloc = _lib.fa_flex_attention_fwd_noalloc
 
 
 class FAError(RuntimeError):
@@ -210,6 +216,34 @@ def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask
                                  _stream_handle(stream)),
            "fa_flex_attention_fwd")
     return (out, lse) if return_lse else out
+
+
+def flex_attention_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, mask_kind: int,
+                           window: int = 0, doc_id: Optional[torch.Tensor] = None,
+                           score_mod: int = FA_SCORE_NONE, softcap: float = 0.0,
+                           scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                           lse: Optional[torch.Tensor] = None,
+                           device_error: Optional[torch.Tensor] = None,
+                           stream: Optional[torch.cuda.Stream] = None):
+    """fa_flex_attention_fwd_noalloc: mask build + forward with the library's static
+    scratch (no block tables or workspace from the caller).  `out`, `lse` and
+    `device_error` (int32[1], device) are the caller's; they are created here only
+    if not given.  Returns (out, lse)."""
+    if q.dtype not in _DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share dtype bf16 or fp16")
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("q, k, v must be contiguous 4-D CUDA tensors")
+    B, H, L, D = q.shape
+    S = k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    _check(fa_flex_attention_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], B, H, L, S,
+                                         D, mask_kind, window, _ptr(doc_id), score_mod,
+                                         float(softcap), float(scale), _ptr(out), _ptr(lse),
+                                         _ptr(device_error), _stream_handle(stream)),
+           "fa_flex_attention_fwd_noalloc")
+    return out, lse
 
 
 def last_device_error(device=None, stream: Optional[torch.cuda.Stream] = None) -> int:

@@ -32,6 +32,7 @@ extern "C" const char* fa_status_string(int32_t status) {
     case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
     case FA_ERR_CUDA: return "FA_ERR_CUDA";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_SCRATCH_TOO_SMALL: return "FA_ERR_SCRATCH_TOO_SMALL";
     default: return "FA_ERR_UNKNOWN";
   }
 }

@@ -54,8 +54,10 @@ typedef enum {
   FA_ERR_INVALID_ARG = 1,  /* bad pointer, size, enum value or mismatched shapes */
   FA_ERR_UNSUPPORTED = 2,  /* valid request outside what this build implements (e.g. D=96) */
   FA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (no device, launch error ...) */
-  FA_ERR_TIMEOUT = 4       /* a bounded device-side wait gave up (reported by
+  FA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (reported by
                               fa_get_last_device_error) */
+  FA_ERR_SCRATCH_TOO_SMALL = 5  /* fa_flex_attention_fwd_noalloc: the problem's block
+                                   tables need more than FA_NOALLOC_SCRATCH_BYTES */
 } fa_status;
 
 typedef enum {
@@ -169,6 +171,42 @@ FA_API fa_status fa_flex_attention_fwd(const void* q, const void* k, const void*
                                 const fa_block_mask* bm, int32_t score_kind, float softcap,
                                 float scale, void* out, float* lse, void* workspace,
                                 void* stream);
+
+/*
+ * Allocation-free variant of fa_create_block_mask + fa_flex_attention_fwd.
+ * The pages have no counterpart: this entry point exists for callers that cannot
+ * allocate device memory where they call attention -- an operator or plugin host
+ * that passes only the input and output tensors (no allocator for the block
+ * tables and the workspace the two calls above take from their caller), or a
+ * serving loop that reserved its device memory up front, where cudaMalloc could
+ * fail and would synchronise the whole device.
+ *
+ * Arguments are those of fa_create_block_mask (mask_kind, window, doc_id, with
+ * block 128 and q_len = L, kv_len = S) and of fa_flex_attention_fwd, without `bm`
+ * and `workspace`.  The block tables and the device error word live in one
+ * file-scope device array of FA_NOALLOC_SCRATCH_BYTES (4 MiB) per device: the
+ * tables take about 8 * nQ * nKV bytes, so square problems fit up to
+ * L = S = 723 * 128 = 92544 (L = S = 32768 takes 0.5 MiB).  The call allocates
+ * nothing and calls no allocating routine.  Each call clears the error word, builds the tables, runs
+ * the forward, and, if `device_error` is not NULL (device or pinned host int32),
+ * copies the error word there in stream order: 0 = success, nonzero = a bounded
+ * device wait gave up and the outputs are invalid.  B*H == 0 or L == 0 is a no-op
+ * returning FA_OK (nothing launched, *device_error untouched).
+ *
+ * Every call on a device shares that one array: calls whose GPU work may overlap
+ * (different streams, or several host threads) race on it and must be ordered by
+ * the caller.  Returns FA_ERR_SCRATCH_TOO_SMALL (nothing launched) when the tables
+ * of an (L, S) problem do not fit, the argument errors of the two calls above
+ * (nothing launched), or FA_ERR_CUDA.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+FA_API fa_status fa_flex_attention_fwd_noalloc(const void* q, const void* k, const void* v,
+                                        int32_t dtype, int32_t B, int32_t H, int32_t L,
+                                        int32_t S, int32_t D, int32_t mask_kind,
+                                        int32_t window, const int32_t* doc_id,
+                                        int32_t score_kind, float softcap, float scale,
+                                        void* out, float* lse, int32_t* device_error,
+                                        void* stream);
 
 /* Synchronises `stream`, then reads and clears the error word that the forward
  * kernel keeps in `workspace`.  Returns FA_ERR_TIMEOUT if a bounded device wait gave

@@ -65,7 +65,7 @@ def test_struct_layout_matches_c(fa):
 def test_enum_values_match_header(fa):
     text = open(HEADER).read()
     for name in ("FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
-                 "FA_ERR_TIMEOUT", "FA_MASK_CAUSAL", "FA_MASK_SLIDING_WINDOW_CAUSAL",
+                 "FA_ERR_TIMEOUT", "FA_ERR_SCRATCH_TOO_SMALL", "FA_MASK_CAUSAL", "FA_MASK_SLIDING_WINDOW_CAUSAL",
                  "FA_MASK_DOCUMENT_CAUSAL", "FA_SCORE_NONE", "FA_SCORE_TANH_SOFTCAP",
                  "FA_BF16", "FA_FP16"):
         m = re.search(rf"\b{name}\s*=\s*(\d+)", text)
