@@ -51,11 +51,9 @@ constexpr int kSoftmaxWarps = 4 * kNumSlots;
 constexpr int kProducerWarp = kSoftmaxWarps;      // + slot: one TMA producer warp per slot
 constexpr int kMmaWarp = kSoftmaxWarps + kNumSlots;
 constexpr int kThreads = (kSoftmaxWarps + 4) * 32;  // + one warpgroup: 2 producers, MMA, 1 spare
-// Register split (per thread) after launch: 384 threads x 168 = 64512 registers at
-// launch; softmax warpgroups take 208, the control warpgroup 88:
-// 256 x 208 + 128 x 88 = 64512, and per SM sub-partition 208 + 208 + 88 <= 512.
-constexpr int kRegsSoftmax = 208;
-constexpr int kRegsControl = 88;
+// Every warp keeps the launch count of 168 registers (384 threads x 168 = 64512).
+// No setmaxnreg split: the softmax code fits in 168 without spills, and with a
+// split ptxas spilled in the narrowed control region.
 constexpr int kBlockN = 128;                 // rows of a Q tile / K,V tile
 constexpr int kChunkBytes = 128 * 128;       // one TMA box: 128 rows x 64 elems x 2 B
 constexpr float kLog2e = 1.4426950408889634f;
@@ -622,31 +620,79 @@ __device__ __forceinline__ void load_s_half(uint32_t taddr, float (&x)[64]) {
   for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(xr[i]);
 }
 
+// v if a <= I <= b (and, with bit I % 32 of `same` required, the key's document
+// matches), else -inf: predicated selects, so rows with different bounds in one
+// warp do not diverge.
+template <int I>
+__device__ __forceinline__ float keep_if_in(float v, int a, int b) {
+  float r;
+  asm("{\n\t.reg .pred p;\n\t"
+      "setp.le.s32 p, %2, %3;\n\t"
+      "setp.ge.and.s32 p, %4, %3, p;\n\t"
+      "selp.f32 %0, %1, 0fFF800000, p;\n\t}"
+      : "=f"(r) : "f"(v), "r"(a), "n"(I), "r"(b));
+  return r;
+}
+template <int I>
+__device__ __forceinline__ float keep_if_in_doc(float v, int a, int b, uint32_t same) {
+  float r;
+  asm("{\n\t.reg .pred p;\n\t.reg .b32 t;\n\t"
+      "setp.le.s32 p, %2, %3;\n\t"
+      "setp.ge.and.s32 p, %4, %3, p;\n\t"
+      "and.b32 t, %5, %6;\n\t"
+      "setp.ne.and.u32 p, t, 0, p;\n\t"
+      "selp.f32 %0, %1, 0fFF800000, p;\n\t}"
+      : "=f"(r) : "f"(v), "r"(a), "n"(I), "r"(b), "r"(same), "n"(1u << (I & 31)));
+  return r;
+}
+
+template <int I>
+struct MaskCols {
+  static __device__ __forceinline__ void range(float (&x)[64], int a, int b) {
+    x[I] = keep_if_in<I>(x[I], a, b);
+    MaskCols<I + 1>::range(x, a, b);
+  }
+  static __device__ __forceinline__ void doc(float (&x)[64], int a, int b, uint32_t same) {
+    x[I] = keep_if_in_doc<I>(x[I], a, b, same);
+    if constexpr (I % 32 != 31) MaskCols<I + 1>::doc(x, a, b, same);
+  }
+};
+template <>
+struct MaskCols<64> {
+  static __device__ __forceinline__ void range(float (&)[64], int, int) {}
+};
+
 // Mask rule on 64 columns of a PARTIAL block: column i (key kv0 + i) is live iff
 // a <= i <= b (causal / window interval, clipped to the keys that exist) and, for
 // documents, doc_id[kv0 + i] == dq.  Dead entries become -inf.
 __device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int a, int b, int kv0,
-                                           int dq) {
+                                           int dq, bool dq_uniform) {
   if (p.mask_kind == FA_MASK_DOCUMENT_CAUSAL) {
+    // bit i of `same`: the document of key kv0 + c*32 + i equals the row's; keys past
+    // S read the last id (in bounds) and are excluded by the range anyway
+    uint32_t same[2];
+    if (dq_uniform) {
+      // every row of the warp is in one document: lane i fetches key i's id and a
+      // ballot gives all rows the same bits
+      const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      uint32_t same = 0;
+      for (int c = 0; c < 2; ++c)
+        same[c] = __ballot_sync(0xffffffffu,
+                                ldg_nc(p.doc_id + min(kv0 + c * 32 + lane, p.S - 1)) == dq);
+    } else {
+      same[0] = same[1] = 0u;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int kv = kv0 + c * 32 + i;
-        const int d = kv < p.S ? __ldg(p.doc_id + kv) : dq + 1;
-        same |= (d == dq ? 1u : 0u) << i;
-      }
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int ii = c * 32 + i;
-        if (ii < a || ii > b || !((same >> i) & 1u)) x[ii] = -INFINITY;
-      }
+        for (int i = 0; i < 32; ++i) {
+          const int kv = min(kv0 + c * 32 + i, p.S - 1);
+          same[c] |= (ldg_nc(p.doc_id + kv) == dq ? 1u : 0u) << i;
+        }
     }
+    MaskCols<0>::doc(x, a, b, same[0]);
+    MaskCols<32>::doc(x, a, b, same[1]);
   } else {
-#pragma unroll
-    for (int i = 0; i < 64; ++i)
-      if (i < a || i > b) x[i] = -INFINITY;
+    MaskCols<0>::range(x, a, b);
   }
 }
 
@@ -745,7 +791,14 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
       }
       continue;
     }
-    const int dq = (p.mask_kind == FA_MASK_DOCUMENT_CAUSAL && valid) ? __ldg(p.doc_id + row) : 0;
+    const int dq_own = (p.mask_kind == FA_MASK_DOCUMENT_CAUSAL && valid) ? __ldg(p.doc_id + row) : 0;
+    // all valid rows of this warp in lane 0's document (rows past L do not matter);
+    // the shuffle is taken by every lane, outside any short-circuited expression.
+    // Then every lane, rows past L included, takes lane 0's id: in the ballot of
+    // apply_mask a lane compares the key it fetched for the whole warp.
+    const int dq0 = __shfl_sync(0xffffffffu, dq_own, 0);
+    const bool dq_uniform = __all_sync(0xffffffffu, !valid || dq_own == dq0);
+    const int dq = dq_uniform ? dq0 : dq_own;
     // live keys of this row: kv in [lo, hi] (and, for documents, doc_id[kv] == dq)
     const int hi = min(row, p.S - 1);
     const int lo = p.mask_kind == FA_MASK_SLIDING_WINDOW_CAUSAL ? max(row - p.window + 1, 0) : 0;
@@ -770,8 +823,9 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         if (!full) {
           const int a = lo - kvb * kBlockN;
           const int b = hi - kvb * kBlockN;
-          apply_mask(p, *reinterpret_cast<float(*)[64]>(x), a, b, kvb * kBlockN, dq);
-          apply_mask(p, *reinterpret_cast<float(*)[64]>(x + 64), a - 64, b - 64, kvb * kBlockN + 64, dq);
+          apply_mask(p, *reinterpret_cast<float(*)[64]>(x), a, b, kvb * kBlockN, dq, dq_uniform);
+          apply_mask(p, *reinterpret_cast<float(*)[64]>(x + 64), a - 64, b - 64, kvb * kBlockN + 64, dq,
+                     dq_uniform);
         }
         const float mb = fmaxf(row_max64(*reinterpret_cast<float(*)[64]>(x)),
                                row_max64(*reinterpret_cast<float(*)[64]>(x + 64))) * xs;
@@ -811,7 +865,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         for (int h = 0; h < 2; ++h) {
           float x[64];
           load_s_half(t_s + h * 64, x);
-          if (!full) apply_mask(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq);
+          if (!full) apply_mask(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, dq_uniform);
           rmax = fmaxf(rmax, row_max64(x));
         }
         float mb = rmax;
@@ -877,7 +931,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
               x[i + 1] = v.y;
             }
           }
-          if (!full) apply_mask(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq);
+          if (!full) apply_mask(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, dq_uniform);
           // P = exp2(x * xs - m) as 16-bit pairs; with the split, P_hi = p truncated to
           // bf16 and P_lo = round(p - P_hi), so P_hi + P_lo carries ~16 significant bits.
           float2 sums[4];
@@ -995,16 +1049,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  // Role dispatch.  Each register configuration has its own code path to the end
-  // of the kernel; the final rendezvous is a named barrier over all threads.
+  // Role dispatch; the final rendezvous is a named barrier over all threads.
   if (warp < kSoftmaxWarps) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     softmax_role<D>(sm, p, tmem, warp / 4);
     tc_fence_before();
     named_barrier_sync(1, kThreads);
     return;
   }
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == kProducerWarp) {
     producer_role<D, 0>(sm, p, &tmap_q, &tmap_k, &tmap_v);
   } else if (warp == kProducerWarp + 1) {
