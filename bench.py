@@ -49,8 +49,8 @@ KERNEL_SOURCES = ("block_sparse_attention_create_b200/csrc/fwd_sm100.cu",
                   "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
 NCU_TRAFFIC = {
     "swa256_L32768_B1_H8_D64_bf16": {
-        "bytes": 101163264 + 6274048,
-        "sources_sha256": "29fc015b38e3672630f87c6944e33c9db5c9cfbfc7b5a530dd6e83a440efc772",
+        "bytes": 101042176 + 5957120,
+        "sources_sha256": "1411234e80f93e8412db89f9dddd3bd044cb57fdbfd07929cd7d02476e3e09c9",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_full.md"},
 }
 
