@@ -36,7 +36,7 @@ def _as_f64(x):
 
 
 def attention_head(q, k, v, kind, window=None, doc_id=None, score_kind=NONE, softcap=0.0,
-                   scale=None, rows=None, chunk=256):
+                   scale=None, rows=None, chunk=256, bitmap=None):
     """One (batch, head): q (L,D), k (S,D), v (S,Dv) -> out (R,Dv), lse (R,).
 
     ``rows`` selects the query rows to evaluate (default: all L); each row's
@@ -58,7 +58,7 @@ def attention_head(q, k, v, kind, window=None, doc_id=None, score_kind=NONE, sof
         s = (q[r] @ k.T) * scale                       # (R, S) scaled scores
         if score_kind == TANH_SOFTCAP:
             s = softcap * np.tanh(s / softcap)
-        allowed = masks.mask_rows(kind, r, S, window, doc)
+        allowed = masks.mask_rows(kind, r, S, window, doc, bitmap)
         s = np.where(allowed, s, -np.inf)
         m = s.max(axis=1) if S > 0 else np.full((len(r),), -np.inf)
         live = np.isfinite(m)
@@ -75,7 +75,7 @@ def attention_head(q, k, v, kind, window=None, doc_id=None, score_kind=NONE, sof
 
 
 def attention(q, k, v, kind, window=None, doc_id=None, score_kind=NONE, softcap=0.0, scale=None,
-              rows=None, heads=None, chunk=256):
+              rows=None, heads=None, chunk=256, bitmap=None):
     """Batched oracle on (B,H,L,D) inputs.
 
     ``heads``: optional list of (b, h) pairs to evaluate (default: all).
@@ -86,5 +86,5 @@ def attention(q, k, v, kind, window=None, doc_id=None, score_kind=NONE, softcap=
     res = {}
     for (b, h) in heads:
         res[(b, h)] = attention_head(q[b, h], k[b, h], v[b, h], kind, window, doc_id, score_kind,
-                                     softcap, scale, rows, chunk)
+                                     softcap, scale, rows, chunk, bitmap)
     return res

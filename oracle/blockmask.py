@@ -29,7 +29,7 @@ from . import masks
 BLOCK = 128
 
 
-def classify(kind, q_len, kv_len, window=None, doc_id=None, block=BLOCK):
+def classify(kind, q_len, kv_len, window=None, doc_id=None, block=BLOCK, bitmap=None):
     """Return (live, full) bool arrays of shape (nQ, nKV) and allowed-pair count."""
     nq = -(-q_len // block)
     nkv = -(-kv_len // block)
@@ -42,7 +42,7 @@ def classify(kind, q_len, kv_len, window=None, doc_id=None, block=BLOCK):
         rows = np.arange(i * block, min((i + 1) * block, q_len))
         padded[:] = False
         if kv_len > 0:
-            m = masks.mask_rows(kind, rows, kv_len, window, doc)
+            m = masks.mask_rows(kind, rows, kv_len, window, doc, bitmap)
             padded[: len(rows), :kv_len] = m
             allowed_pairs += int(m.sum())
         blk = padded.reshape(block, nkv, block)
@@ -51,9 +51,9 @@ def classify(kind, q_len, kv_len, window=None, doc_id=None, block=BLOCK):
     return live, full, allowed_pairs
 
 
-def block_tables(kind, q_len, kv_len, window=None, doc_id=None, block=BLOCK):
+def block_tables(kind, q_len, kv_len, window=None, doc_id=None, block=BLOCK, bitmap=None):
     """Integer tables as int32 numpy arrays (partial and full lists kept apart)."""
-    live, full, pairs = classify(kind, q_len, kv_len, window, doc_id, block)
+    live, full, pairs = classify(kind, q_len, kv_len, window, doc_id, block, bitmap)
     partial = live & ~full
     nq, nkv = live.shape
     kv_num = partial.sum(axis=1).astype(np.int32)
@@ -70,7 +70,31 @@ def block_tables(kind, q_len, kv_len, window=None, doc_id=None, block=BLOCK):
             "allowed_pairs": pairs, "n_q_blocks": nq, "n_kv_blocks": nkv}
 
 
-def densities(kind, q_len, kv_len, window=None, doc_id=None, block=BLOCK):
+def densities(kind, q_len, kv_len, window=None, doc_id=None, block=BLOCK, bitmap=None):
     """(token density, block density): allowed pairs / all pairs, live blocks / all blocks."""
-    live, _, pairs = classify(kind, q_len, kv_len, window, doc_id, block)
+    live, _, pairs = classify(kind, q_len, kv_len, window, doc_id, block, bitmap)
     return pairs / float(q_len * kv_len), live.sum() / float(live.size)
+
+
+def transpose(tables):
+    """Column view of the tables (FlexAttention's BlockMask also carries it, for
+    the backward pass): per kv block j, the q blocks i whose block (i, j) is
+    PARTIAL, ascending (``q_num_blocks[j]``, ``q_indices[j, :]``), and those whose
+    block is FULL (``full_q_num_blocks``, ``full_q_indices``); unused entries 0."""
+    nq, nkv = tables["n_q_blocks"], tables["n_kv_blocks"]
+    partial = np.zeros((nq, nkv), dtype=bool)
+    full = np.zeros((nq, nkv), dtype=bool)
+    for i in range(nq):
+        partial[i, tables["kv_indices"][i, : tables["kv_num_blocks"][i]]] = True
+        full[i, tables["full_kv_indices"][i, : tables["full_kv_num_blocks"][i]]] = True
+    q_num = partial.sum(axis=0).astype(np.int32)
+    full_q_num = full.sum(axis=0).astype(np.int32)
+    q_idx = np.zeros((nkv, nq), dtype=np.int32)
+    full_q_idx = np.zeros((nkv, nq), dtype=np.int32)
+    for j in range(nkv):
+        pi = np.nonzero(partial[:, j])[0]
+        fi = np.nonzero(full[:, j])[0]
+        q_idx[j, : len(pi)] = pi
+        full_q_idx[j, : len(fi)] = fi
+    return {"q_num_blocks": q_num, "q_indices": q_idx,
+            "full_q_num_blocks": full_q_num, "full_q_indices": full_q_idx}

@@ -11,7 +11,9 @@ from __future__ import annotations
 import math
 
 
-def allowed(kind, q, kv, window=None, doc=None):
+def allowed(kind, q, kv, window=None, doc=None, bitmap=None):
+    if kind == 3:  # tabulated mask_mod: bit kv % 32 of word kv // 32 of row q
+        return (int(bitmap[q][kv // 32]) >> (kv % 32)) & 1 == 1
     if kind == 0:
         return q >= kv
     if kind == 1:
@@ -21,7 +23,8 @@ def allowed(kind, q, kv, window=None, doc=None):
     raise ValueError(kind)
 
 
-def attention_head(q, k, v, kind, window=None, doc=None, score_kind=0, softcap=0.0, scale=None):
+def attention_head(q, k, v, kind, window=None, doc=None, score_kind=0, softcap=0.0, scale=None,
+                   bitmap=None):
     """q, k, v: lists of lists of floats. Returns (out rows, lse list)."""
     L, D = len(q), len(q[0])
     S = len(k)
@@ -32,7 +35,7 @@ def attention_head(q, k, v, kind, window=None, doc=None, score_kind=0, softcap=0
     for i in range(L):
         scores = []
         for j in range(S):
-            if not allowed(kind, i, j, window, doc):
+            if not allowed(kind, i, j, window, doc, bitmap):
                 continue
             s = 0.0
             for d in range(D):
@@ -58,12 +61,12 @@ def attention_head(q, k, v, kind, window=None, doc=None, score_kind=0, softcap=0
     return outs, lses
 
 
-def classify_block(kind, i, j, q_len, kv_len, window=None, doc=None, block=128):
+def classify_block(kind, i, j, q_len, kv_len, window=None, doc=None, block=128, bitmap=None):
     """'empty' / 'full' / 'partial' for block (i, j) by visiting each pair."""
     n_live = 0
     for q in range(i * block, (i + 1) * block):
         for kv in range(j * block, (j + 1) * block):
-            if q < q_len and kv < kv_len and allowed(kind, q, kv, window, doc):
+            if q < q_len and kv < kv_len and allowed(kind, q, kv, window, doc, bitmap):
                 n_live += 1
     if n_live == 0:
         return "empty"

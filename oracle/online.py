@@ -22,7 +22,7 @@ from .attention import TANH_SOFTCAP, _as_f64
 
 
 def attention_head_tiled(q, k, v, kind, window=None, doc_id=None, score_kind=0, softcap=0.0,
-                         scale=None, rows=None, tile=128):
+                         scale=None, rows=None, tile=128, bitmap=None):
     q = _as_f64(q)
     k = _as_f64(k)
     v = _as_f64(v)
@@ -42,7 +42,7 @@ def attention_head_tiled(q, k, v, kind, window=None, doc_id=None, score_kind=0, 
         s = (qr @ k[t0:t1].T) * scale
         if score_kind == TANH_SOFTCAP:
             s = softcap * np.tanh(s / softcap)
-        allowed = masks.mask_rows(kind, rows, S, window, doc)[:, t0:t1]
+        allowed = masks.mask_rows(kind, rows, S, window, doc, bitmap)[:, t0:t1]
         s = np.where(allowed, s, -np.inf)
         m_new = np.maximum(m, s.max(axis=1))
         # rows with no live entry so far keep m = -inf and contribute nothing

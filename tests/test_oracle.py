@@ -319,3 +319,84 @@ def test_workload_generators_are_seeded():
     assert torch.all(d[1:] >= d[:-1])
     f = W.make_doc_id(W.C4_DOC_FIXED)
     assert int(f[2047]) == 0 and int(f[2048]) == 1 and int(f[4999]) == 1 and int(f[5000]) == 2
+
+
+# ---------------------------------------------------------------- tabulated mask_mod
+
+def test_bitmap_layout_hand_example():
+    """Causal 3 x 3 tabulated by hand: row q keeps keys 0..q, bit kv of word 0."""
+    words = OM.to_bitmap(OM.CAUSAL, 3, 3)
+    assert words.tolist() == [[0b1], [0b11], [0b111]]
+    # key 33 of row 0 lives in word 1, bit 1
+    w = np.zeros((1, 2), dtype=np.uint32)
+    w[0, 1] = 2
+    assert OM.mask_rows(OM.BITMAP, [0], 64, bitmap=w).nonzero()[1].tolist() == [33]
+
+
+@pytest.mark.parametrize("kind,L,S,w", [
+    (OM.CAUSAL, 300, 300, None), (OM.CAUSAL, 1000, 300, None), (OM.CAUSAL, 200, 700, None),
+    (OM.SLIDING_WINDOW_CAUSAL, 385, 385, 70), (OM.DOCUMENT_CAUSAL, 384, 384, None)])
+def test_bitmap_of_a_rule_reduces_to_the_rule(kind, L, S, w):
+    """A bitmap tabulating a mask rule gives that rule's block tables and outputs."""
+    doc = None
+    if kind == OM.DOCUMENT_CAUSAL:
+        doc = np.random.default_rng(7).integers(0, 3, size=max(L, S))
+    words = OM.to_bitmap(kind, L, S, w, doc, words_per_row=4 * (-(-S // 128)))
+    a = OB.block_tables(kind, L, S, w, doc)
+    b = OB.block_tables(OM.BITMAP, L, S, bitmap=words)
+    for key in ("kv_num_blocks", "kv_indices", "full_kv_num_blocks", "full_kv_indices"):
+        assert np.array_equal(a[key], b[key]), key
+    q, k, v = (_rand((n, 32), s) for n, s in ((L, 1), (S, 2), (S, 3)))
+    oa, la = OA.attention_head(q, k, v, kind, window=w, doc_id=doc)
+    ob, lb = OA.attention_head(q, k, v, OM.BITMAP, bitmap=words)
+    assert np.array_equal(oa, ob) and np.array_equal(la, lb)
+
+
+@pytest.mark.parametrize("L,S", [(7, 9), (130, 70), (64, 200)])
+def test_bitmap_bruteforce_tiny(L, S):
+    """Vectorised oracle on a random bitmap equals pure-Python loops."""
+    words = W.random_bitmap(L, S, seed=L + S)
+    q, k, v = (_rand((n, 16), s) for n, s in ((L, 4), (S, 5), (S, 6)))
+    out, lse = OA.attention_head(q, k, v, OM.BITMAP, bitmap=words)
+    bo, bl = BF.attention_head(q.tolist(), k.tolist(), v.tolist(), OM.BITMAP, bitmap=words)
+    assert np.allclose(out, np.array(bo), atol=1e-12, rtol=0)
+    assert np.allclose(lse, np.array(bl), atol=1e-12, rtol=0, equal_nan=False)
+    live, full, _ = OB.classify(OM.BITMAP, L, S, bitmap=words)
+    for i in range(live.shape[0]):
+        for j in range(live.shape[1]):
+            c = BF.classify_block(OM.BITMAP, i, j, L, S, bitmap=words)
+            assert (c != "empty") == live[i, j] and (c == "full") == full[i, j], (i, j, c)
+
+
+def test_bitmap_matches_torch_sdpa_fp64():
+    """torch's CPU SDPA in fp64 given the bitmap as a boolean mask built by
+    per-pair bit extraction."""
+    L = S = 300
+    words = W.random_bitmap(L, S, seed=9)
+    mask = torch.tensor([[(int(words[qq][kk // 32]) >> (kk % 32)) & 1 == 1 for kk in range(S)]
+                         for qq in range(L)])
+    live_rows = mask.any(dim=1)
+    q, k, v = (torch.from_numpy(_rand((1, 1, n, 32), s)) for n, s in ((L, 1), (S, 2), (S, 3)))
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask)[0, 0].numpy()
+    out, lse = OA.attention_head(q[0, 0], k[0, 0], v[0, 0], OM.BITMAP, bitmap=words)
+    assert np.abs(out[live_rows.numpy()] - ref[live_rows.numpy()]).max() < 1e-12
+    assert np.all(out[~live_rows.numpy()] == 0) and np.all(np.isneginf(lse[~live_rows.numpy()]))
+
+
+@pytest.mark.parametrize("kind,L,S,w", [
+    (OM.CAUSAL, 300, 300, None), (OM.SLIDING_WINDOW_CAUSAL, 700, 500, 200),
+    (OM.DOCUMENT_CAUSAL, 384, 384, None), (OM.BITMAP, 400, 300, None)])
+def test_transpose_matches_bruteforce(kind, L, S, w):
+    """Column lists (q blocks per kv block, ascending) from per-pair classification."""
+    doc = np.random.default_rng(3).integers(0, 3, size=max(L, S)) if kind == OM.DOCUMENT_CAUSAL \
+        else None
+    words = W.random_bitmap(L, S, seed=11) if kind == OM.BITMAP else None
+    t = OB.transpose(OB.block_tables(kind, L, S, w, doc, bitmap=words))
+    nq, nkv = -(-L // 128), -(-S // 128)
+    for j in range(nkv):
+        cls = [BF.classify_block(kind, i, j, L, S, w, doc, bitmap=words) for i in range(nq)]
+        part = [i for i in range(nq) if cls[i] == "partial"]
+        full = [i for i in range(nq) if cls[i] == "full"]
+        assert t["q_num_blocks"][j] == len(part) and t["full_q_num_blocks"][j] == len(full)
+        assert t["q_indices"][j].tolist() == part + [0] * (nq - len(part))
+        assert t["full_q_indices"][j].tolist() == full + [0] * (nq - len(full))

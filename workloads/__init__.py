@@ -23,6 +23,7 @@ import dataclasses
 import math
 from typing import Optional, Tuple
 
+import numpy as np
 import torch
 
 MASK_CAUSAL = 0
@@ -142,3 +143,28 @@ def random_qkv(B, H, L, S, D, dtype, seed, scale=1.0, device="cpu"):
     w = Workload(name="adhoc", B=B, H=H, L=L, S=S, D=D, dtype=dtype, mask_kind=MASK_CAUSAL,
                  input_scale=scale, seed=seed)
     return make_qkv(w, device)
+
+
+def random_bitmap(L: int, S: int, seed: int, p_empty: float = 0.35, p_full: float = 0.3,
+                  density: float = 0.5) -> np.ndarray:
+    """Seeded bitmap mask input: uint32 words (L, 4 * ceil(S / 128)), bit kv % 32 of word
+    kv // 32 of row q set when the pair is kept; bits past S are 0.  Each 128 x 128
+    block is drawn empty, all-set, or random bits of the given density, so that every
+    block class occurs."""
+    g = np.random.default_rng(seed)
+    nq, nkv = -(-L // 128), -(-S // 128)
+    bits = np.zeros((nq * 128, nkv * 128), dtype=bool)
+    for i in range(nq):
+        for j in range(nkv):
+            u = g.random()
+            blk = bits[i * 128:(i + 1) * 128, j * 128:(j + 1) * 128]
+            if u < p_empty:
+                continue
+            if u < p_empty + p_full:
+                blk[:] = True
+            else:
+                blk[:] = g.random((128, 128)) < density
+    bits = bits[:L]
+    bits[:, S:] = False
+    words = np.packbits(bits.reshape(L, -1, 32)[:, :, ::-1], axis=2, bitorder="big")
+    return words.view(">u4").reshape(L, nkv * 4).astype(np.uint32)
