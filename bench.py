@@ -88,6 +88,17 @@ def live_blocks_per_row(w: W.Workload):
     out = np.zeros(nq, dtype=np.int64)
     doc = W.make_doc_id(w)
     doc = doc.numpy() if doc is not None else None
+    words = W.make_bitmap(w)
+    if words is not None:  # a block is live if any of its words has a bit set
+        tail = np.uint32((1 << (w.S % 32)) - 1) if w.S % 32 else np.uint32(0xFFFFFFFF)
+        words = words.copy()
+        if w.S % 32:
+            words[:, w.S // 32] &= tail
+        words[:, -(-w.S // 32):] = 0
+        blk = np.zeros((nq * 128, nkv * 4), dtype=np.uint32)
+        blk[: w.L] = words
+        any_bit = blk.reshape(nq, 128, nkv, 4).any(axis=(1, 3))
+        return any_bit.sum(axis=1).astype(np.int64)
     for i in range(nq):
         q0, q1 = i * 128, min(w.L, i * 128 + 128) - 1
         for j in range(nkv):
@@ -178,8 +189,11 @@ def run_ours(args, w: W.Workload, rank, world, device):
     torch.cuda.set_device(device)
     q, k, v = W.make_qkv(w)
     doc = W.make_doc_id(w)
+    words = W.make_bitmap(w)
+    bits = torch.from_numpy(words.view(np.int32)) if words is not None else None
     qd, kd, vd = q.to(device), k.to(device), v.to(device)
     dd = doc.to(device) if doc is not None else None
+    bd = bits.to(device) if bits is not None else None
     out = torch.empty_like(qd)
     lse = torch.empty(w.B, w.H, w.L, dtype=torch.float32, device=device)
     bm = fa.BlockMask(w.L, w.S, device)
@@ -189,7 +203,7 @@ def run_ours(args, w: W.Workload, rank, world, device):
 
     def step():
         fa.create_block_mask(w.mask_kind, w.L, w.S, window=w.window, doc_id=dd, out=bm,
-                             stream=stream)
+                             stream=stream, bitmap=bd)
         fa.flex_attention(qd, kd, vd, bm, score_mod=w.score_kind, softcap=w.softcap, out=out,
                           lse=lse, ws=ws, stream=stream)
 
@@ -217,7 +231,7 @@ def run_ours(args, w: W.Workload, rank, world, device):
             flush.zero_()
             starts[i].record(stream)
             fa.create_block_mask(w.mask_kind, w.L, w.S, window=w.window, doc_id=dd, out=bm,
-                                 stream=stream)
+                                 stream=stream, bitmap=bd)
             mids[i].record(stream)
             fa.flex_attention(qd, kd, vd, bm, score_mod=w.score_kind, softcap=w.softcap,
                               out=out, lse=lse, ws=ws, stream=stream)
@@ -237,14 +251,16 @@ def run_ours(args, w: W.Workload, rank, world, device):
 
     # end to end through the public API: pinned host inputs in, results out
     e2e = ({"ms": float("nan"), "h2d": 0, "d2h": 0} if args.profile
-           else run_e2e(args, w, fa, q, k, v, doc, device, world))
+           else run_e2e(args, w, fa, q, k, v, doc, bits, device, world))
     return {"fig": fig, "total_ms": total_ms, "step_ms": step_ms, "fwd_ms": fwd_ms,
             "mask_ms": mask_ms, "clocks": clk.summary(), "e2e": e2e}
 
 
-def run_e2e(args, w, fa, q, k, v, doc, device, world):
+def run_e2e(args, w, fa, q, k, v, doc, bits, device, world):
     hq, hk, hv = (t.pin_memory() for t in (q, k, v))
     hdoc = doc.pin_memory() if doc is not None else None
+    hbits = bits.pin_memory() if bits is not None else None
+    bd = torch.empty(bits.shape, dtype=bits.dtype, device=device) if bits is not None else None
     hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
     hlse = torch.empty(w.B, w.H, w.L, dtype=torch.float32).pin_memory()
     qd, kd, vd = (torch.empty(t.shape, dtype=t.dtype, device=device) for t in (q, k, v))
@@ -260,8 +276,10 @@ def run_e2e(args, w, fa, q, k, v, doc, device, world):
         vd.copy_(hv, non_blocking=True)
         if dd is not None:
             dd.copy_(hdoc, non_blocking=True)
+        if bd is not None:
+            bd.copy_(hbits, non_blocking=True)
         fa.create_block_mask(w.mask_kind, w.L, w.S, window=w.window, doc_id=dd, out=bm,
-                             stream=stream)
+                             stream=stream, bitmap=bd)
         fa.flex_attention(qd, kd, vd, bm, score_mod=w.score_kind, softcap=w.softcap, out=out,
                           lse=lse, stream=stream)
         hout.copy_(out, non_blocking=True)
@@ -284,7 +302,7 @@ def run_e2e(args, w, fa, q, k, v, doc, device, world):
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         ms = float(t.item())
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + (
-        hdoc.numel() * 4 if hdoc is not None else 0)
+        hdoc.numel() * 4 if hdoc is not None else 0) + (hbits.numel() * 4 if hbits is not None else 0)
     d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
     return {"ms": ms, "h2d": h2d, "d2h": d2h}
 
@@ -294,10 +312,11 @@ def oracle_sample(w: W.Workload, rows, fig):
     from oracle import attention as OA
     q, k, v = W.make_qkv(w)
     doc = W.make_doc_id(w)
+    words = W.make_bitmap(w)
     t0 = time.perf_counter()
     OA.attention_head(q[0, 0], k[0, 0], v[0, 0], w.mask_kind, window=w.window or None,
                       doc_id=None if doc is None else doc.numpy(), score_kind=w.score_kind,
-                      softcap=w.softcap, rows=rows)
+                      softcap=w.softcap, rows=rows, bitmap=words)
     dt = time.perf_counter() - t0
     credited = sum(4.0 * w.D * 128 * int(fig["per_row"][r // 128]) for r in rows)
     return dt, credited

@@ -25,7 +25,7 @@ LIB_PATH = os.path.join(_HERE, "libfa.so")
 
 (FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT,
  FA_ERR_SCRATCH_TOO_SMALL) = range(6)
-FA_MASK_CAUSAL, FA_MASK_SLIDING_WINDOW_CAUSAL, FA_MASK_DOCUMENT_CAUSAL = range(3)
+FA_MASK_CAUSAL, FA_MASK_SLIDING_WINDOW_CAUSAL, FA_MASK_DOCUMENT_CAUSAL, FA_MASK_BITMAP = range(4)
 FA_SCORE_NONE, FA_SCORE_TANH_SOFTCAP = range(2)
 FA_BF16, FA_FP16 = range(2)
 FA_BLOCK = 128
@@ -35,7 +35,8 @@ FA_NOALLOC_SCRATCH_BYTES = 4 << 20
 # Every symbol include/fa.h declares.
 EXPORTED = ("fa_block_mask_dims", "fa_create_block_mask", "fa_fwd_workspace_bytes",
             "fa_flex_attention_fwd", "fa_get_last_device_error", "fa_status_string",
-            "fa_num_sms", "fa_flex_attention_fwd_noalloc")
+            "fa_num_sms", "fa_flex_attention_fwd_noalloc", "fa_create_block_mask_bitmap",
+            "fa_block_mask_transpose")
 
 
 class fa_block_mask(ctypes.Structure):
@@ -54,6 +55,7 @@ class fa_block_mask(ctypes.Structure):
         ("kind", ctypes.c_int32),
         ("window", ctypes.c_int32),
         ("doc_id", ctypes.c_void_p),
+        ("bitmap", ctypes.c_void_p),
     ]
 
 
@@ -81,6 +83,10 @@ def _load():
     lib.fa_flex_attention_fwd_noalloc.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                                   i32, i32, vp, i32, f32, f32, vp, vp, vp, vp]
     lib.fa_flex_attention_fwd_noalloc.restype = i32
+    lib.fa_create_block_mask_bitmap.argtypes = [vp, i32, i32, i32, ctypes.POINTER(fa_block_mask), vp]
+    lib.fa_create_block_mask_bitmap.restype = i32
+    lib.fa_block_mask_transpose.argtypes = [ctypes.POINTER(fa_block_mask), vp, vp, vp, vp, vp]
+    lib.fa_block_mask_transpose.restype = i32
     return lib
 
 
@@ -95,6 +101,8 @@ fa_get_last_device_error = _lib.fa_get_last_device_error
 fa_status_string = _lib.fa_status_string
 fa_num_sms = _lib.fa_num_sms
 fa_flex_attention_fwd_noalloc = _lib.fa_flex_attention_fwd_noalloc
+fa_create_block_mask_bitmap = _lib.fa_create_block_mask_bitmap
+fa_block_mask_transpose = _lib.fa_block_mask_transpose
 
 
 class FAError(RuntimeError):
@@ -140,6 +148,7 @@ class BlockMask:
         self.full_kv_indices = torch.zeros(nq, nkv, **i32)
         self.q_order = torch.zeros(2 * nq, **i32)   # schedule: (row, partial | full << 16)
         self.doc_id: Optional[torch.Tensor] = None
+        self.bitmap: Optional[torch.Tensor] = None
         self.struct = fa_block_mask()
         self.struct.kv_num_blocks = self.kv_num_blocks.data_ptr()
         self.struct.kv_indices = self.kv_indices.data_ptr()
@@ -153,13 +162,39 @@ class BlockMask:
         return {k: getattr(self, k).cpu().numpy() for k in
                 ("kv_num_blocks", "kv_indices", "full_kv_num_blocks", "full_kv_indices", "q_order")}
 
+    def transpose(self, stream: Optional[torch.cuda.Stream] = None):
+        """fa_block_mask_transpose: per kv block, its partial / full q blocks (device
+        tensors q_num_blocks [nKV], q_indices [nKV, nQ], full_q_num_blocks,
+        full_q_indices)."""
+        nq, nkv = self.n_q_blocks, self.n_kv_blocks
+        i32 = dict(dtype=torch.int32, device=self.kv_num_blocks.device)
+        t = {"q_num_blocks": torch.zeros(nkv, **i32), "q_indices": torch.zeros(nkv, nq, **i32),
+             "full_q_num_blocks": torch.zeros(nkv, **i32),
+             "full_q_indices": torch.zeros(nkv, nq, **i32)}
+        _check(fa_block_mask_transpose(ctypes.byref(self.struct), _ptr(t["q_num_blocks"]),
+                                       _ptr(t["q_indices"]), _ptr(t["full_q_num_blocks"]),
+                                       _ptr(t["full_q_indices"]), _stream_handle(stream)),
+               "fa_block_mask_transpose")
+        return t
+
 
 def create_block_mask(kind: int, q_len: int, kv_len: int, window: int = 0,
                       doc_id: Optional[torch.Tensor] = None, device="cuda",
-                      stream: Optional[torch.cuda.Stream] = None, out: Optional[BlockMask] = None
-                      ) -> BlockMask:
-    """fa_create_block_mask on fresh (or the given) device tables."""
+                      stream: Optional[torch.cuda.Stream] = None, out: Optional[BlockMask] = None,
+                      bitmap: Optional[torch.Tensor] = None) -> BlockMask:
+    """fa_create_block_mask (or, for FA_MASK_BITMAP, fa_create_block_mask_bitmap with
+    `bitmap`: an int32 CUDA tensor (q_len, 4 * nKV) holding the 32-bit words) on fresh
+    (or the given) device tables."""
     bm = out if out is not None else BlockMask(q_len, kv_len, device)
+    if kind == FA_MASK_BITMAP:
+        if (bitmap is None or bitmap.dtype != torch.int32 or not bitmap.is_cuda
+                or not bitmap.is_contiguous() or bitmap.shape != (q_len, 4 * bm.n_kv_blocks)):
+            raise ValueError("bitmap must be a contiguous int32 CUDA tensor (q_len, 4 * nKV)")
+        bm.bitmap = bitmap
+        _check(fa_create_block_mask_bitmap(_ptr(bitmap), q_len, kv_len, FA_BLOCK,
+                                           ctypes.byref(bm.struct), _stream_handle(stream)),
+               "fa_create_block_mask_bitmap")
+        return bm
     if doc_id is not None:
         if doc_id.dtype != torch.int32 or not doc_id.is_cuda or not doc_id.is_contiguous():
             raise ValueError("doc_id must be a contiguous int32 CUDA tensor")

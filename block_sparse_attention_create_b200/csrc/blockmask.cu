@@ -10,7 +10,8 @@
 // allowed, PARTIAL otherwise.  Causal and sliding-window blocks are classified in
 // closed form (the allowed keys of row q are the interval (q - W, q]); document
 // blocks are classified exactly for arbitrary ids: a value-range test settles the
-// common cases and a warp visits every pair otherwise.
+// common cases and a warp visits every pair otherwise.  A tabulated mask (one bit
+// per pair) is classified by OR / AND over the block's 128 x 4 words.
 #include <cstdint>
 
 #include "fa_internal.h"
@@ -32,8 +33,9 @@ __device__ __forceinline__ void warp_minmax(int& mn, int& mx) {
 
 // One CTA per q-block row i.  cls[j]: 0 empty, 1 partial, 2 full.
 __global__ void __launch_bounds__(kClassifyThreads)
-classify_rows_kernel(int kind, int window, const int32_t* __restrict__ doc, int q_len, int kv_len,
-                     int n_kv, int32_t* __restrict__ kv_num, int32_t* __restrict__ kv_idx,
+classify_rows_kernel(int kind, int window, const int32_t* __restrict__ doc,
+                     const uint32_t* __restrict__ bitmap, int q_len, int kv_len, int n_kv,
+                     int32_t* __restrict__ kv_num, int32_t* __restrict__ kv_idx,
                      int32_t* __restrict__ full_num, int32_t* __restrict__ full_idx) {
   extern __shared__ uint8_t cls[];
   __shared__ int q_doc_min, q_doc_max;
@@ -43,7 +45,37 @@ classify_rows_kernel(int kind, int window, const int32_t* __restrict__ doc, int 
   const int64_t q1 = min(static_cast<int64_t>(q_len), q0 + kBlock) - 1;
   const bool q_whole = q0 + kBlock <= q_len;
 
-  if (kind != FA_MASK_DOCUMENT_CAUSAL) {
+  if (kind == FA_MASK_BITMAP) {
+    // a warp per kv block: lane l reads rows q0 + l + 32 r (r < 4), all four words;
+    // bits past kv_len do not count, rows past q_len neither
+    const int nwarps = blockDim.x >> 5;
+    const size_t wpr = static_cast<size_t>(n_kv) * 4;  // words per bitmap row
+    for (int j = warp; j < n_kv; j += nwarps) {
+      const int64_t k0 = static_cast<int64_t>(j) * kBlock;
+      uint32_t valid[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int64_t nk = kv_len - (k0 + 32 * w);  // keys of word w that exist
+        valid[w] = nk >= 32 ? 0xFFFFFFFFu : (nk <= 0 ? 0u : ((1u << nk) - 1u));
+      }
+      bool any = false, all = q_whole && k0 + kBlock <= kv_len;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int64_t q = q0 + lane + 32 * r;
+        if (q >= q_len) continue;
+        const uint4 v4 = __ldg(reinterpret_cast<const uint4*>(bitmap + q * wpr + 4 * j));
+        const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          any |= (wv[w] & valid[w]) != 0u;
+          all &= (wv[w] & valid[w]) == valid[w];
+        }
+      }
+      any = __any_sync(0xffffffffu, any);
+      all = __all_sync(0xffffffffu, all);
+      if (lane == 0) cls[j] = any ? (all ? 2 : 1) : 0;
+    }
+  } else if (kind != FA_MASK_DOCUMENT_CAUSAL) {
     for (int j = threadIdx.x; j < n_kv; j += blockDim.x) {
       const int64_t k0 = static_cast<int64_t>(j) * kBlock;
       const int64_t k1 = min(static_cast<int64_t>(kv_len), k0 + kBlock) - 1;
@@ -199,6 +231,57 @@ order_rows_kernel(int n_q, int n_kv, int n_pow2, const int32_t* __restrict__ kv_
   }
 }
 
+// Column lists: one CTA per kv block j.  Every warp classifies q-block rows
+// (i, j) by binary search in row i's ascending partial and full lists; warp 0 then
+// compacts the classes in ascending i.
+__global__ void __launch_bounds__(kClassifyThreads)
+transpose_kernel(int n_q, int n_kv, const int32_t* __restrict__ kv_num,
+                 const int32_t* __restrict__ kv_idx, const int32_t* __restrict__ full_num,
+                 const int32_t* __restrict__ full_idx, int32_t* __restrict__ q_num,
+                 int32_t* __restrict__ q_idx, int32_t* __restrict__ full_q_num,
+                 int32_t* __restrict__ full_q_idx) {
+  extern __shared__ uint8_t cls[];
+  const int j = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  auto contains = [j](const int32_t* list, int n) {
+    int lo = 0, hi = n;  // first position with list[pos] >= j
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(list + mid) < j) lo = mid + 1; else hi = mid;
+    }
+    return lo < n && __ldg(list + lo) == j;
+  };
+  for (int i = threadIdx.x; i < n_q; i += blockDim.x) {
+    const size_t row = static_cast<size_t>(i) * n_kv;
+    uint8_t c = 0;
+    if (contains(full_idx + row, __ldg(full_num + i))) c = 2;
+    else if (contains(kv_idx + row, __ldg(kv_num + i))) c = 1;
+    cls[i] = c;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const size_t base_col = static_cast<size_t>(j) * n_q;
+    int np = 0, nf = 0;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = 0; base < n_q; base += 32) {
+      const int i = base + lane;
+      const uint8_t c = i < n_q ? cls[i] : 0;
+      const unsigned pm = __ballot_sync(0xffffffffu, c == 1);
+      const unsigned fm = __ballot_sync(0xffffffffu, c == 2);
+      if (c == 1) q_idx[base_col + np + __popc(pm & lt)] = i;
+      if (c == 2) full_q_idx[base_col + nf + __popc(fm & lt)] = i;
+      np += __popc(pm);
+      nf += __popc(fm);
+    }
+    for (int t = np + lane; t < n_q; t += 32) q_idx[base_col + t] = 0;
+    for (int t = nf + lane; t < n_q; t += 32) full_q_idx[base_col + t] = 0;
+    if (lane == 0) {
+      q_num[j] = np;
+      full_q_num[j] = nf;
+    }
+  }
+}
+
 }  // namespace
 }  // namespace fa
 
@@ -212,6 +295,50 @@ extern "C" fa_status fa_block_mask_dims(int32_t q_len, int32_t kv_len, int32_t b
   return FA_OK;
 }
 
+namespace fa {
+namespace {
+
+// Shared tail of the two builders: fill the scalar fields, classify, order.
+fa_status build_tables(int32_t kind, int32_t window, const int32_t* doc_id, const uint32_t* bitmap,
+                       int32_t q_len, int32_t kv_len, int32_t block, int32_t nq, int32_t nkv,
+                       fa_block_mask* bm, void* stream) {
+  bm->q_len = q_len;
+  bm->kv_len = kv_len;
+  bm->block = block;
+  bm->n_q_blocks = nq;
+  bm->n_kv_blocks = nkv;
+  bm->kind = kind;
+  bm->window = kind == FA_MASK_SLIDING_WINDOW_CAUSAL ? window : 0;
+  bm->doc_id = kind == FA_MASK_DOCUMENT_CAUSAL ? doc_id : nullptr;
+  bm->bitmap = kind == FA_MASK_BITMAP ? bitmap : nullptr;
+  if (nq == 0) return FA_OK;
+
+  cudaStream_t s = as_stream(stream);
+  classify_rows_kernel<<<nq, kClassifyThreads, nkv > 0 ? nkv : 1, s>>>(
+      kind, bm->window, bm->doc_id, bm->bitmap, q_len, kv_len, nkv, bm->kv_num_blocks,
+      bm->kv_indices, bm->full_kv_num_blocks, bm->full_kv_indices);
+  FA_CUDA_CHECK(cudaGetLastError());
+  int n_pow2 = 1;
+  while (n_pow2 < nq) n_pow2 <<= 1;
+  const size_t order_smem = (nq <= 2048 ? nq : n_pow2) * sizeof(uint32_t);
+  order_rows_kernel<<<1, kOrderThreads, order_smem, s>>>(
+      nq, nkv, n_pow2, bm->kv_num_blocks, bm->full_kv_num_blocks, bm->q_order);
+  FA_CUDA_CHECK(cudaGetLastError());
+  return FA_OK;
+}
+
+bool tables_present(const fa_block_mask* bm, int32_t nq, int32_t nkv) {
+  if (nq > 0 && (bm->kv_num_blocks == nullptr || bm->full_kv_num_blocks == nullptr ||
+                 bm->q_order == nullptr))
+    return false;
+  if (nq > 0 && nkv > 0 && (bm->kv_indices == nullptr || bm->full_kv_indices == nullptr))
+    return false;
+  return true;
+}
+
+}  // namespace
+}  // namespace fa
+
 extern "C" fa_status fa_create_block_mask(int32_t kind, int32_t window, const int32_t* doc_id,
                                           int32_t q_len, int32_t kv_len, int32_t block,
                                           fa_block_mask* bm, void* stream) {
@@ -224,32 +351,40 @@ extern "C" fa_status fa_create_block_mask(int32_t kind, int32_t window, const in
   if (kind == FA_MASK_SLIDING_WINDOW_CAUSAL && window < 1) return FA_ERR_INVALID_ARG;
   if (kind == FA_MASK_DOCUMENT_CAUSAL && doc_id == nullptr && (q_len > 0 || kv_len > 0))
     return FA_ERR_INVALID_ARG;
-  if (nq > 0 && (bm->kv_num_blocks == nullptr || bm->full_kv_num_blocks == nullptr ||
-                 bm->q_order == nullptr))
-    return FA_ERR_INVALID_ARG;
-  if (nq > 0 && nkv > 0 && (bm->kv_indices == nullptr || bm->full_kv_indices == nullptr))
-    return FA_ERR_INVALID_ARG;
+  if (!tables_present(bm, nq, nkv)) return FA_ERR_INVALID_ARG;
+  return build_tables(kind, window, doc_id, nullptr, q_len, kv_len, block, nq, nkv, bm, stream);
+}
 
-  bm->q_len = q_len;
-  bm->kv_len = kv_len;
-  bm->block = block;
-  bm->n_q_blocks = nq;
-  bm->n_kv_blocks = nkv;
-  bm->kind = kind;
-  bm->window = kind == FA_MASK_SLIDING_WINDOW_CAUSAL ? window : 0;
-  bm->doc_id = kind == FA_MASK_DOCUMENT_CAUSAL ? doc_id : nullptr;
-  if (nq == 0) return FA_OK;
+extern "C" fa_status fa_create_block_mask_bitmap(const uint32_t* bitmap, int32_t q_len,
+                                                 int32_t kv_len, int32_t block, fa_block_mask* bm,
+                                                 void* stream) {
+  using namespace fa;
+  if (bm == nullptr) return FA_ERR_INVALID_ARG;
+  int32_t nq = 0, nkv = 0;
+  const fa_status st = fa_block_mask_dims(q_len, kv_len, block, &nq, &nkv);
+  if (st != FA_OK) return st;
+  if (q_len > 0 && kv_len > 0 &&
+      (bitmap == nullptr || (reinterpret_cast<uintptr_t>(bitmap) & 15u) != 0))
+    return FA_ERR_INVALID_ARG;
+  if (!tables_present(bm, nq, nkv)) return FA_ERR_INVALID_ARG;
+  return build_tables(FA_MASK_BITMAP, 0, nullptr, bitmap, q_len, kv_len, block, nq, nkv, bm,
+                      stream);
+}
 
-  cudaStream_t s = as_stream(stream);
-  classify_rows_kernel<<<nq, kClassifyThreads, nkv > 0 ? nkv : 1, s>>>(
-      kind, bm->window, bm->doc_id, q_len, kv_len, nkv, bm->kv_num_blocks, bm->kv_indices,
-      bm->full_kv_num_blocks, bm->full_kv_indices);
-  FA_CUDA_CHECK(cudaGetLastError());
-  int n_pow2 = 1;
-  while (n_pow2 < nq) n_pow2 <<= 1;
-  const size_t order_smem = (nq <= 2048 ? nq : n_pow2) * sizeof(uint32_t);
-  order_rows_kernel<<<1, kOrderThreads, order_smem, s>>>(
-      nq, nkv, n_pow2, bm->kv_num_blocks, bm->full_kv_num_blocks, bm->q_order);
+extern "C" fa_status fa_block_mask_transpose(const fa_block_mask* bm, int32_t* q_num_blocks,
+                                             int32_t* q_indices, int32_t* full_q_num_blocks,
+                                             int32_t* full_q_indices, void* stream) {
+  using namespace fa;
+  if (bm == nullptr || bm->block != FA_BLOCK || bm->n_q_blocks < 0 || bm->n_kv_blocks < 0)
+    return FA_ERR_INVALID_ARG;
+  const int32_t nq = bm->n_q_blocks, nkv = bm->n_kv_blocks;
+  if (nq == 0 || nkv == 0) return FA_OK;
+  if (!tables_present(bm, nq, nkv) || q_num_blocks == nullptr || q_indices == nullptr ||
+      full_q_num_blocks == nullptr || full_q_indices == nullptr)
+    return FA_ERR_INVALID_ARG;
+  transpose_kernel<<<nkv, kClassifyThreads, nq, as_stream(stream)>>>(
+      nq, nkv, bm->kv_num_blocks, bm->kv_indices, bm->full_kv_num_blocks, bm->full_kv_indices,
+      q_num_blocks, q_indices, full_q_num_blocks, full_q_indices);
   FA_CUDA_CHECK(cudaGetLastError());
   return FA_OK;
 }

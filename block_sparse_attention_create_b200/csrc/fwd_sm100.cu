@@ -58,6 +58,14 @@ constexpr int kBlockN = 128;                 // rows of a Q tile / K,V tile
 constexpr int kChunkBytes = 128 * 128;       // one TMA box: 128 rows x 64 elems x 2 B
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+// Mask families, one kernel instantiation each (only its mask code is compiled in):
+// causal and sliding-window (an interval of keys per row), document, tabulated.
+constexpr int kMaskRange = 0;
+constexpr int kMaskDoc = 1;
+constexpr int kMaskBitmap = 2;
+__host__ __device__ constexpr int mask_family(int kind) {
+  return kind == FA_MASK_DOCUMENT_CAUSAL ? kMaskDoc : (kind == FA_MASK_BITMAP ? kMaskBitmap : kMaskRange);
+}
 constexpr float kRescaleThreshold = 8.0f;    // log2 units: O is rescaled only when max grows > 2^8
 
 // TMEM layouts (512 columns, lanes = the 128 rows of a tile):
@@ -114,10 +122,11 @@ struct Params {
   const int32_t* full_idx;
   const int32_t* sched;  // per rank k: [2k] = q-block row, [2k+1] = partial | full << 16
   const int32_t* doc_id;
+  const uint32_t* bitmap;  // tabulated mask: row q's words at bitmap + q * bitmap_words
   void* out;
   float* lse;
   int32_t* err;
-  int BH, L, S, n_kv, num_units;
+  int BH, L, S, n_kv, num_units, bitmap_words;
   int mask_kind, window, softcap_on, is_bf16;
   int split_p;       // P fed to the PV product as two 16-bit terms (hi + lo)
   float scale_log2;  // scale * log2(e)
@@ -664,10 +673,17 @@ struct MaskCols<64> {
 
 // Mask rule on 64 columns of a PARTIAL block: column i (key kv0 + i) is live iff
 // a <= i <= b (causal / window interval, clipped to the keys that exist) and, for
-// documents, doc_id[kv0 + i] == dq.  Dead entries become -inf.
+// documents, doc_id[kv0 + i] == dq; for a tabulated mask, iff its bit in the row's
+// words `brow` is set (and the key exists).  Dead entries become -inf.
+template <int MK>
 __device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int a, int b, int kv0,
-                                           int dq, bool dq_uniform) {
-  if (p.mask_kind == FA_MASK_DOCUMENT_CAUSAL) {
+                                           int dq, bool dq_uniform, const uint32_t* brow) {
+  if constexpr (MK == kMaskBitmap) {
+    // the row's two words of keys kv0 .. kv0 + 63 (kv0 is a multiple of 64)
+    const int2 w = ldg_nc_v2(reinterpret_cast<const int32_t*>(brow + (kv0 >> 5)));
+    MaskCols<0>::doc(x, a, b, static_cast<uint32_t>(w.x));
+    MaskCols<32>::doc(x, a, b, static_cast<uint32_t>(w.y));
+  } else if constexpr (MK == kMaskDoc) {
     // bit i of `same`: the document of key kv0 + c*32 + i equals the row's; keys past
     // S read the last id (in bounds) and are excluded by the range anyway
     uint32_t same[2];
@@ -759,7 +775,7 @@ __device__ __forceinline__ float exp_pack64(const float (&x)[64], float xs, floa
 
 // Softmax warpgroup of one slot: thread t owns row t of the slot's 128-row tile
 // (TMEM lane t), so row max and row sum need no shuffles.
-template <int D>
+template <int D, int MK>
 __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int slot) {
   using C = Cfg<D>;
   const int t = threadIdx.x - slot * 128;   // row of the tile this thread owns
@@ -791,7 +807,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
       }
       continue;
     }
-    const int dq_own = (p.mask_kind == FA_MASK_DOCUMENT_CAUSAL && valid) ? __ldg(p.doc_id + row) : 0;
+    const int dq_own = (MK == kMaskDoc && valid) ? __ldg(p.doc_id + row) : 0;
     // all valid rows of this warp in lane 0's document (rows past L do not matter);
     // the shuffle is taken by every lane, outside any short-circuited expression.
     // Then every lane, rows past L included, takes lane 0's id: in the ballot of
@@ -799,8 +815,13 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
     const int dq0 = __shfl_sync(0xffffffffu, dq_own, 0);
     const bool dq_uniform = __all_sync(0xffffffffu, !valid || dq_own == dq0);
     const int dq = dq_uniform ? dq0 : dq_own;
-    // live keys of this row: kv in [lo, hi] (and, for documents, doc_id[kv] == dq)
-    const int hi = min(row, p.S - 1);
+    // tabulated mask: this row's words (rows past L read the last row, unused)
+    const uint32_t* brow = MK == kMaskBitmap
+                               ? p.bitmap + static_cast<size_t>(min(row, p.L - 1)) * p.bitmap_words
+                               : nullptr;
+    // live keys of this row: kv in [lo, hi] (and, for documents, doc_id[kv] == dq;
+    // for a tabulated mask, its bit); only the causal rules bound hi by the row
+    const int hi = MK == kMaskBitmap ? p.S - 1 : min(row, p.S - 1);
     const int lo = p.mask_kind == FA_MASK_SLIDING_WINDOW_CAUSAL ? max(row - p.window + 1, 0) : 0;
     float m = -INFINITY, l = 0.f;  // running max (log2 units) and running sum
     int kvb = block_index(p, un, 0);
@@ -823,9 +844,10 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         if (!full) {
           const int a = lo - kvb * kBlockN;
           const int b = hi - kvb * kBlockN;
-          apply_mask(p, *reinterpret_cast<float(*)[64]>(x), a, b, kvb * kBlockN, dq, dq_uniform);
-          apply_mask(p, *reinterpret_cast<float(*)[64]>(x + 64), a - 64, b - 64, kvb * kBlockN + 64, dq,
-                     dq_uniform);
+          apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x), a, b, kvb * kBlockN, dq, dq_uniform,
+                     brow);
+          apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x + 64), a - 64, b - 64, kvb * kBlockN + 64, dq,
+                     dq_uniform, brow);
         }
         const float mb = fmaxf(row_max64(*reinterpret_cast<float(*)[64]>(x)),
                                row_max64(*reinterpret_cast<float(*)[64]>(x + 64))) * xs;
@@ -865,7 +887,8 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         for (int h = 0; h < 2; ++h) {
           float x[64];
           load_s_half(t_s + h * 64, x);
-          if (!full) apply_mask(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, dq_uniform);
+          if (!full)
+            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, dq_uniform, brow);
           rmax = fmaxf(rmax, row_max64(x));
         }
         float mb = rmax;
@@ -931,7 +954,8 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
               x[i + 1] = v.y;
             }
           }
-          if (!full) apply_mask(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, dq_uniform);
+          if (!full)
+            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, dq_uniform, brow);
           // P = exp2(x * xs - m) as 16-bit pairs; with the split, P_hi = p truncated to
           // bf16 and P_lo = round(p - P_hi), so P_hi + P_lo carries ~16 significant bits.
           float2 sums[4];
@@ -1001,7 +1025,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
   }
 }
 
-template <int D>
+template <int D, int MK>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
            const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ Params p) {
@@ -1051,7 +1075,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
 
   // Role dispatch; the final rendezvous is a named barrier over all threads.
   if (warp < kSoftmaxWarps) {
-    softmax_role<D>(sm, p, tmem, warp / 4);
+    softmax_role<D, MK>(sm, p, tmem, warp / 4);
     tc_fence_before();
     named_barrier_sync(1, kThreads);
     return;
@@ -1109,7 +1133,7 @@ bool make_map(CUtensorMap* map, const void* ptr, bool bf16, int D, int rows, int
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, int MK>
 fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH, int L, int S,
                  const Params& prm, cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
@@ -1126,7 +1150,7 @@ fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH,
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
     if (!done[dev]) {
-      FA_CUDA_CHECK(cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      FA_CUDA_CHECK(cudaFuncSetAttribute(fwd_kernel<D, MK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem)));
       done[dev] = true;
     }
@@ -1135,7 +1159,7 @@ fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH,
   if (sms <= 0) return FA_ERR_CUDA;
   const int want = (prm.num_units + kNumSlots - 1) / kNumSlots;
   const int grid = want < sms ? want : sms;
-  fwd_kernel<D><<<grid, kThreads, smem, stream>>>(tq, tk, tv, prm);
+  fwd_kernel<D, MK><<<grid, kThreads, smem, stream>>>(tq, tk, tv, prm);
   FA_CUDA_CHECK(cudaGetLastError());
   return FA_OK;
 }
@@ -1172,6 +1196,7 @@ extern "C" fa_status fa_flex_attention_fwd(const void* q, const void* k, const v
   if (bm->kv_num_blocks == nullptr || bm->full_kv_num_blocks == nullptr || bm->q_order == nullptr)
     return FA_ERR_INVALID_ARG;
   if (bm->kind == FA_MASK_DOCUMENT_CAUSAL && bm->doc_id == nullptr) return FA_ERR_INVALID_ARG;
+  if (bm->kind == FA_MASK_BITMAP && S > 0 && bm->bitmap == nullptr) return FA_ERR_INVALID_ARG;
 
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
   Params prm{};
@@ -1179,6 +1204,8 @@ extern "C" fa_status fa_flex_attention_fwd(const void* q, const void* k, const v
   prm.full_idx = bm->full_kv_indices;
   prm.sched = bm->q_order;
   prm.doc_id = bm->doc_id;
+  prm.bitmap = bm->bitmap;
+  prm.bitmap_words = 4 * bm->n_kv_blocks;
   prm.out = out;
   prm.lse = lse;
   prm.err = static_cast<int32_t*>(workspace);
@@ -1197,6 +1224,13 @@ extern "C" fa_status fa_flex_attention_fwd(const void* q, const void* k, const v
   prm.split_p = 1;
   prm.timeout_ns = 2000000000ull;
   const cudaStream_t s = as_stream(stream);
-  if (D == 64) return launch<64>(q, k, v, dtype == FA_BF16, prm.BH, L, S, prm, s);
-  return launch<128>(q, k, v, dtype == FA_BF16, prm.BH, L, S, prm, s);
+  const bool b16 = dtype == FA_BF16;
+  switch (mask_family(bm->kind) * 2 + (D == 64 ? 0 : 1)) {
+    case kMaskRange * 2: return launch<64, kMaskRange>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskRange * 2 + 1: return launch<128, kMaskRange>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskDoc * 2: return launch<64, kMaskDoc>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskDoc * 2 + 1: return launch<128, kMaskDoc>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskBitmap * 2: return launch<64, kMaskBitmap>(q, k, v, b16, prm.BH, L, S, prm, s);
+    default: return launch<128, kMaskBitmap>(q, k, v, b16, prm.BH, L, S, prm, s);
+  }
 }

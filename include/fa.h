@@ -63,7 +63,9 @@ typedef enum {
 typedef enum {
   FA_MASK_CAUSAL = 0,                /* q_idx >= kv_idx                                   */
   FA_MASK_SLIDING_WINDOW_CAUSAL = 1, /* q_idx >= kv_idx && q_idx - kv_idx < window        */
-  FA_MASK_DOCUMENT_CAUSAL = 2        /* q_idx >= kv_idx && doc_id[q_idx] == doc_id[kv_idx] */
+  FA_MASK_DOCUMENT_CAUSAL = 2,       /* q_idx >= kv_idx && doc_id[q_idx] == doc_id[kv_idx] */
+  FA_MASK_BITMAP = 3                 /* bit kv_idx of row q_idx of a caller's bitmap
+                                        (fa_create_block_mask_bitmap)                    */
 } fa_mask_kind;
 
 typedef enum {
@@ -115,6 +117,7 @@ typedef struct fa_block_mask {
   int32_t kind;           /* fa_mask_kind */
   int32_t window;         /* sliding window W (kind 1), else 0 */
   const int32_t* doc_id;  /* device int32[max(q_len, kv_len)] (kind 2), else NULL */
+  const uint32_t* bitmap; /* device bitmap (kind 3, see fa_create_block_mask_bitmap), else NULL */
 } fa_block_mask;
 
 /* nQ and nKV of a (q_len, kv_len) mask with the given block size.
@@ -141,6 +144,39 @@ FA_API fa_status fa_block_mask_dims(int32_t q_len, int32_t kv_len, int32_t block
 FA_API fa_status fa_create_block_mask(int32_t kind, int32_t window, const int32_t* doc_id,
                                int32_t q_len, int32_t kv_len, int32_t block,
                                fa_block_mask* bm, void* stream);
+
+/*
+ * Block tables of a tabulated mask_mod (the FlexAttention how-to's
+ * create_block_mask takes any boolean function of (b, h, q_idx, kv_idx), "Mask 1:
+ * causal"; here it is given as one bit per pair, broadcast over batch and heads).
+ *   bitmap  device uint32 words, row-major (q_len, 4 * nKV), 16-byte aligned: pair
+ *           (q, kv) is kept iff bit kv % 32 (least significant first) of word
+ *           kv / 32 of row q is set.  Rows are padded to whole 128-key blocks; bits
+ *           at kv >= kv_len are ignored.  Kept (not copied): it must stay valid while
+ *           the mask is used, since the forward kernel reads it in PARTIAL blocks.
+ *   q_len, kv_len, block, bm, stream   as for fa_create_block_mask.
+ * Launches two kernels on `stream`.  Returns FA_ERR_INVALID_ARG (nothing launched)
+ * on bad arguments, FA_ERR_CUDA if a launch fails.
+ */
+FA_API fa_status fa_create_block_mask_bitmap(const uint32_t* bitmap, int32_t q_len, int32_t kv_len,
+                                      int32_t block, fa_block_mask* bm, void* stream);
+
+/*
+ * Column view of built tables (FlexAttention's BlockMask carries it for the
+ * backward pass): for each kv block j, the q blocks i whose block (i, j) is
+ * PARTIAL, ascending, and those whose block is FULL.
+ *   bm                   tables from fa_create_block_mask / _bitmap (read only).
+ *   q_num_blocks[nKV]            number of PARTIAL blocks in column j
+ *   q_indices[nKV * nQ]          column j: their q-block indices, ascending, then 0s
+ *   full_q_num_blocks[nKV]       number of FULL blocks in column j
+ *   full_q_indices[nKV * nQ]     column j: their q-block indices, ascending, then 0s
+ * Device arrays owned by the caller.  One kernel on `stream`, ordered after the
+ * build on the same stream.  Returns FA_ERR_INVALID_ARG (nothing launched) on NULL
+ * arguments, FA_ERR_CUDA if the launch fails; nKV == 0 or nQ == 0 launches nothing.
+ */
+FA_API fa_status fa_block_mask_transpose(const fa_block_mask* bm, int32_t* q_num_blocks,
+                                  int32_t* q_indices, int32_t* full_q_num_blocks,
+                                  int32_t* full_q_indices, void* stream);
 
 /* Bytes of the device workspace fa_flex_attention_fwd needs (a small constant).
  * The caller allocates it, ZEROES IT ONCE, and may then reuse it for every call on

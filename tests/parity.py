@@ -24,13 +24,22 @@ MEAN_ERR = 2e-3
 LSE_ERR = 1e-3
 
 
-def run_gpu(q, k, v, kind, window=0, doc_id=None, score_kind=0, softcap=0.0, scale=0.0):
-    """q, k, v CPU tensors -> (out, lse) CPU tensors from the CUDA path."""
+def bitmap_to_device(words):
+    """uint32 numpy words -> int32 CUDA tensor with the same bits."""
+    return torch.from_numpy(np.ascontiguousarray(words).view(np.int32)).to("cuda")
+
+
+def run_gpu(q, k, v, kind, window=0, doc_id=None, score_kind=0, softcap=0.0, scale=0.0,
+            bitmap=None):
+    """q, k, v CPU tensors -> (out, lse) CPU tensors from the CUDA path (`bitmap`:
+    uint32 numpy words for the tabulated mask kind)."""
     import block_sparse_attention_create_b200 as fa
     dev = "cuda"
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     dd = doc_id.to(dev) if doc_id is not None else None
-    bm = fa.create_block_mask(kind, q.shape[2], k.shape[2], window=window, doc_id=dd, device=dev)
+    bd = bitmap_to_device(bitmap) if bitmap is not None else None
+    bm = fa.create_block_mask(kind, q.shape[2], k.shape[2], window=window, doc_id=dd, device=dev,
+                              bitmap=bd)
     out, lse = fa.flex_attention(qd, kd, vd, bm, score_mod=score_kind, softcap=softcap,
                                  scale=scale, return_lse=True)
     torch.cuda.synchronize()
@@ -39,11 +48,11 @@ def run_gpu(q, k, v, kind, window=0, doc_id=None, score_kind=0, softcap=0.0, sca
 
 
 def oracle_rows(q, k, v, b, h, rows, kind, window=0, doc_id=None, score_kind=0, softcap=0.0,
-                scale=0.0):
+                scale=0.0, bitmap=None):
     return OA.attention_head(q[b, h], k[b, h], v[b, h], kind, window=window or None,
                              doc_id=None if doc_id is None else doc_id.numpy(),
                              score_kind=score_kind, softcap=softcap,
-                             scale=scale if scale > 0 else None, rows=rows)
+                             scale=scale if scale > 0 else None, rows=rows, bitmap=bitmap)
 
 
 def out_ulp(ref, dtype):

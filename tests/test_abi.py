@@ -66,7 +66,7 @@ def test_enum_values_match_header(fa):
     text = open(HEADER).read()
     for name in ("FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
                  "FA_ERR_TIMEOUT", "FA_ERR_SCRATCH_TOO_SMALL", "FA_MASK_CAUSAL", "FA_MASK_SLIDING_WINDOW_CAUSAL",
-                 "FA_MASK_DOCUMENT_CAUSAL", "FA_SCORE_NONE", "FA_SCORE_TANH_SOFTCAP",
+                 "FA_MASK_DOCUMENT_CAUSAL", "FA_MASK_BITMAP", "FA_SCORE_NONE", "FA_SCORE_TANH_SOFTCAP",
                  "FA_BF16", "FA_FP16"):
         m = re.search(rf"\b{name}\s*=\s*(\d+)", text)
         assert m and int(m.group(1)) == getattr(fa, name), name
@@ -102,6 +102,30 @@ def test_create_block_mask_rejects_bad_arguments(fa):
     # an empty mask is valid and launches nothing
     assert fa.fa_create_block_mask(0, 0, null, 0, 0, 128, ctypes.byref(bm), null) == fa.FA_OK
     assert (bm.q_len, bm.n_q_blocks, bm.block) == (0, 0, 128)
+
+
+def test_bitmap_builder_and_transpose_reject_bad_arguments(fa):
+    bm = fa.fa_block_mask()
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(1 << 20)            # never dereferenced: rejected first
+    # NULL or misaligned bitmap, NULL struct, NULL tables, bad block
+    assert fa.fa_create_block_mask_bitmap(null, 256, 256, 128, ctypes.byref(bm), null) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_create_block_mask_bitmap(ctypes.c_void_p((1 << 20) + 4), 256, 256, 128,
+                                          ctypes.byref(bm), null) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_create_block_mask_bitmap(fake, 256, 256, 128, None, null) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_create_block_mask_bitmap(fake, 256, 256, 128, ctypes.byref(bm), null) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_create_block_mask_bitmap(fake, 256, 256, 64, ctypes.byref(bm), null) == fa.FA_ERR_INVALID_ARG
+    # the create_block_mask entry point itself does not take the bitmap kind
+    assert fa.fa_create_block_mask(3, 0, null, 256, 256, 128, ctypes.byref(bm), null) == fa.FA_ERR_INVALID_ARG
+    # empty: valid, nothing launched
+    assert fa.fa_create_block_mask_bitmap(null, 0, 0, 128, ctypes.byref(bm), null) == fa.FA_OK
+    assert bm.kind == fa.FA_MASK_BITMAP
+    # transpose: NULL struct / outputs; an empty mask launches nothing
+    assert fa.fa_block_mask_transpose(None, fake, fake, fake, fake, null) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_block_mask_transpose(ctypes.byref(bm), null, null, null, null, null) == fa.FA_OK
+    bm2 = fa.fa_block_mask()
+    bm2.block, bm2.n_q_blocks, bm2.n_kv_blocks = 128, 2, 2
+    assert fa.fa_block_mask_transpose(ctypes.byref(bm2), fake, fake, fake, fake, null) == fa.FA_ERR_INVALID_ARG
 
 
 def _fwd(fa, bm, **kw):

@@ -29,12 +29,13 @@ import torch
 MASK_CAUSAL = 0
 MASK_SLIDING_WINDOW_CAUSAL = 1
 MASK_DOCUMENT_CAUSAL = 2
+MASK_BITMAP = 3
 
 SCORE_NONE = 0
 SCORE_TANH_SOFTCAP = 1
 
 MASK_NAMES = {MASK_CAUSAL: "causal", MASK_SLIDING_WINDOW_CAUSAL: "sliding_window_causal",
-              MASK_DOCUMENT_CAUSAL: "document_causal"}
+              MASK_DOCUMENT_CAUSAL: "document_causal", MASK_BITMAP: "bitmap"}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -71,6 +72,8 @@ class Workload:
             d["window"] = self.window
         if self.mask_kind == MASK_DOCUMENT_CAUSAL:
             d["documents"] = "seeded 4..16" if self.doc_seeded else list(self.doc_boundaries or ())
+        if self.mask_kind == MASK_BITMAP:
+            d["bitmap"] = "seeded random block classes (empty / all-set / bits at density 0.5)"
         if self.score_kind == SCORE_TANH_SOFTCAP:
             d["score_mod"] = f"tanh_softcap({self.softcap:g})"
         if self.input_scale != 1.0:
@@ -101,7 +104,10 @@ C5_SWA1024_SOFTCAP = _w("swa1024_softcap30_L16384_B2_H16_D128_bf16x2", 2, 16, 16
 
 ALL = (C1_CAUSAL_256, C2_CAUSAL_8192) + C2_WINDOWS + (C3_SWA256_32K, C4_DOC_FIXED, C4_DOC_SEEDED,
                                                       C5_SWA1024_SOFTCAP)
-BY_NAME = {w.name: w for w in ALL}
+# A tabulated mask (one bit per pair) at the causal workload's shape.
+BITMAP_8192 = _w("bitmap_L8192_B1_H8_D64_bf16", 1, 8, 8192, 64, torch.bfloat16, MASK_BITMAP, seed=12)
+
+BY_NAME = {w.name: w for w in ALL + (BITMAP_8192,)}
 
 
 def make_qkv(w: Workload, device="cpu"):
@@ -168,3 +174,10 @@ def random_bitmap(L: int, S: int, seed: int, p_empty: float = 0.35, p_full: floa
     bits[:, S:] = False
     words = np.packbits(bits.reshape(L, -1, 32)[:, :, ::-1], axis=2, bitorder="big")
     return words.view(">u4").reshape(L, nkv * 4).astype(np.uint32)
+
+
+def make_bitmap(w: Workload) -> Optional[np.ndarray]:
+    """The bitmap input of a tabulated-mask workload (uint32 words), else None."""
+    if w.mask_kind != MASK_BITMAP:
+        return None
+    return random_bitmap(w.L, w.S, w.seed)
