@@ -74,17 +74,28 @@ def attention_head(q, k, v, kind, window=None, doc_id=None, score_kind=NONE, sof
     return out, lse
 
 
+def kv_head(h, n_head, n_kv_head):
+    """K/V head shared by query head h when n_head query heads share n_kv_head K/V
+    heads (grouped-query attention, SDPA tutorial section 5: consecutive query
+    heads share one K/V head -- 32 clerks sharing 8 shelves, 4 each -- which is
+    what enable_gqa does)."""
+    if n_head % n_kv_head:
+        raise ValueError("the query heads must divide evenly among the K/V heads")
+    return h // (n_head // n_kv_head)
+
+
 def attention(q, k, v, kind, window=None, doc_id=None, score_kind=NONE, softcap=0.0, scale=None,
               rows=None, heads=None, chunk=256, bitmap=None):
-    """Batched oracle on (B,H,L,D) inputs.
+    """Batched oracle on q (B,H,L,D), k and v (B,Hkv,S,D), Hkv dividing H.
 
     ``heads``: optional list of (b, h) pairs to evaluate (default: all).
     Returns dict {(b, h): (out (R,D) fp64, lse (R,) fp64)}.
     """
-    B, H = q.shape[0], q.shape[1]
+    B, H, Hkv = q.shape[0], q.shape[1], k.shape[1]
     heads = [(b, h) for b in range(B) for h in range(H)] if heads is None else heads
     res = {}
     for (b, h) in heads:
-        res[(b, h)] = attention_head(q[b, h], k[b, h], v[b, h], kind, window, doc_id, score_kind,
+        g = kv_head(h, H, Hkv)
+        res[(b, h)] = attention_head(q[b, h], k[b, g], v[b, g], kind, window, doc_id, score_kind,
                                      softcap, scale, rows, chunk, bitmap)
     return res

@@ -400,3 +400,30 @@ def test_transpose_matches_bruteforce(kind, L, S, w):
         assert t["q_num_blocks"][j] == len(part) and t["full_q_num_blocks"][j] == len(full)
         assert t["q_indices"][j].tolist() == part + [0] * (nq - len(part))
         assert t["full_q_indices"][j].tolist() == full + [0] * (nq - len(full))
+
+
+# ---------------------------------------------------------------- grouped-query attention
+
+@pytest.mark.parametrize("H,Hkv", [(8, 2), (4, 1), (6, 6)])
+def test_gqa_matches_torch_sdpa_enable_gqa(H, Hkv):
+    """Batched oracle with H query heads over Hkv K/V heads equals torch's CPU SDPA
+    in fp64 with enable_gqa=True (its own head grouping), causal and window."""
+    B, L = 2, 200
+    q = torch.from_numpy(_rand((B, H, L, 32), 1))
+    k = torch.from_numpy(_rand((B, Hkv, L, 32), 2))
+    v = torch.from_numpy(_rand((B, Hkv, L, 32), 3))
+    for kind, w in ((OM.CAUSAL, None), (OM.SLIDING_WINDOW_CAUSAL, 50)):
+        mask = torch.from_numpy(OM.mask_rows(kind, np.arange(L), L, w))
+        ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask,
+                                                               enable_gqa=True).numpy()
+        res = OA.attention(q, k, v, kind, window=w)
+        for (b, h), (out, _) in res.items():
+            assert np.abs(out - ref[b, h]).max() < 1e-12, (b, h)
+
+
+def test_gqa_head_map_hand_example():
+    """32 query heads over 8 K/V heads: heads 0-3 -> 0, 4-7 -> 1, ..., 28-31 -> 7."""
+    assert [OA.kv_head(h, 32, 8) for h in range(32)] == [h // 4 for h in range(32)]
+    assert [OA.kv_head(h, 5, 1) for h in range(5)] == [0] * 5
+    with pytest.raises(ValueError):
+        OA.kv_head(0, 6, 4)

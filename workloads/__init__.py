@@ -55,6 +55,11 @@ class Workload:
     softcap: float = 0.0
     input_scale: float = 1.0
     seed: int = 0
+    Hkv: Optional[int] = None   # K/V heads (grouped-query attention); None: H
+
+    @property
+    def n_kv_heads(self) -> int:
+        return self.Hkv if self.Hkv is not None else self.H
 
     @property
     def scale(self) -> float:
@@ -78,6 +83,8 @@ class Workload:
             d["score_mod"] = f"tanh_softcap({self.softcap:g})"
         if self.input_scale != 1.0:
             d["input_scale"] = self.input_scale
+        if self.n_kv_heads != self.H:
+            d["Hkv"] = self.n_kv_heads
         return d
 
 
@@ -106,15 +113,20 @@ ALL = (C1_CAUSAL_256, C2_CAUSAL_8192) + C2_WINDOWS + (C3_SWA256_32K, C4_DOC_FIXE
                                                       C5_SWA1024_SOFTCAP)
 # A tabulated mask (one bit per pair) at the causal workload's shape.
 BITMAP_8192 = _w("bitmap_L8192_B1_H8_D64_bf16", 1, 8, 8192, 64, torch.bfloat16, MASK_BITMAP, seed=12)
+# Grouped-query attention: 32 query heads sharing 8 K/V heads (SDPA tutorial, section 5).
+GQA_CAUSAL_8192 = _w("gqa_causal_L8192_B1_H32_Hkv8_D64_bf16", 1, 32, 8192, 64, torch.bfloat16,
+                     MASK_CAUSAL, seed=13, Hkv=8)
 
-BY_NAME = {w.name: w for w in ALL + (BITMAP_8192,)}
+EXTRA = (BITMAP_8192, GQA_CAUSAL_8192)
+BY_NAME = {w.name: w for w in ALL + EXTRA}
 
 
 def make_qkv(w: Workload, device="cpu"):
-    """Seeded Q (B,H,L,D), K, V (B,H,S,D) in the workload dtype, contiguous."""
+    """Seeded Q (B,H,L,D), K, V (B,Hkv,S,D) in the workload dtype, contiguous."""
     g = torch.Generator(device="cpu").manual_seed(w.seed)
     out = []
-    for shape in ((w.B, w.H, w.L, w.D), (w.B, w.H, w.S, w.D), (w.B, w.H, w.S, w.D)):
+    hk = w.n_kv_heads
+    for shape in ((w.B, w.H, w.L, w.D), (w.B, hk, w.S, w.D), (w.B, hk, w.S, w.D)):
         t = torch.randn(shape, generator=g, dtype=torch.float32)
         if w.input_scale != 1.0:
             t.mul_(w.input_scale)
@@ -144,10 +156,10 @@ def doc_id_from_starts(n: int, starts, device="cpu") -> torch.Tensor:
     return doc.to(device)
 
 
-def random_qkv(B, H, L, S, D, dtype, seed, scale=1.0, device="cpu"):
+def random_qkv(B, H, L, S, D, dtype, seed, scale=1.0, device="cpu", Hkv=None):
     """Seeded inputs for an arbitrary (test) shape, same recipe as make_qkv."""
     w = Workload(name="adhoc", B=B, H=H, L=L, S=S, D=D, dtype=dtype, mask_kind=MASK_CAUSAL,
-                 input_scale=scale, seed=seed)
+                 input_scale=scale, seed=seed, Hkv=Hkv)
     return make_qkv(w, device)
 
 
