@@ -36,7 +36,7 @@ FA_NOALLOC_SCRATCH_BYTES = 4 << 20
 EXPORTED = ("fa_block_mask_dims", "fa_create_block_mask", "fa_fwd_workspace_bytes",
             "fa_flex_attention_fwd", "fa_get_last_device_error", "fa_status_string",
             "fa_num_sms", "fa_flex_attention_fwd_noalloc", "fa_create_block_mask_bitmap",
-            "fa_block_mask_transpose")
+            "fa_block_mask_transpose", "fa_flex_attention_fwd_gqa")
 
 
 class fa_block_mask(ctypes.Structure):
@@ -87,6 +87,10 @@ def _load():
     lib.fa_create_block_mask_bitmap.restype = i32
     lib.fa_block_mask_transpose.argtypes = [ctypes.POINTER(fa_block_mask), vp, vp, vp, vp, vp]
     lib.fa_block_mask_transpose.restype = i32
+    lib.fa_flex_attention_fwd_gqa.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                              ctypes.POINTER(fa_block_mask), i32, f32, f32, vp, vp,
+                                              vp, vp]
+    lib.fa_flex_attention_fwd_gqa.restype = i32
     return lib
 
 
@@ -103,6 +107,7 @@ fa_num_sms = _lib.fa_num_sms
 fa_flex_attention_fwd_noalloc = _lib.fa_flex_attention_fwd_noalloc
 fa_create_block_mask_bitmap = _lib.fa_create_block_mask_bitmap
 fa_block_mask_transpose = _lib.fa_block_mask_transpose
+fa_flex_attention_fwd_gqa = _lib.fa_flex_attention_fwd_gqa
 
 
 class FAError(RuntimeError):
@@ -229,27 +234,35 @@ def flex_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, block_mask
                    out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                    return_lse: bool = False, ws: Optional[torch.Tensor] = None,
                    stream: Optional[torch.cuda.Stream] = None):
-    """fa_flex_attention_fwd on torch tensors q (B,H,L,D), k/v (B,H,S,D)."""
+    """fa_flex_attention_fwd on torch tensors q (B,H,L,D), k/v (B,H,S,D); with k/v
+    (B,Hkv,S,D), Hkv < H dividing H, fa_flex_attention_fwd_gqa."""
     if q.dtype not in _DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("q, k, v must share dtype bf16 or fp16")
     for t in (q, k, v):
         if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
             raise ValueError("q, k, v must be contiguous 4-D CUDA tensors")
     B, H, L, D = q.shape
-    S = k.shape[2]
-    if k.shape != (B, H, S, D) or v.shape != (B, H, S, D):
-        raise ValueError("k and v must be (B, H, S, D) with the q's B, H, D")
+    Hkv, S = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, S, D) or v.shape != (B, Hkv, S, D) or Hkv < 1 or H % Hkv:
+        raise ValueError("k and v must be (B, Hkv, S, D) with the q's B and D, Hkv dividing H")
     if out is None:
         out = torch.empty_like(q)
     if lse is None and return_lse:
         lse = torch.empty(B, H, L, dtype=torch.float32, device=q.device)
     if ws is None:
         ws = workspace(q.device)
-    _check(fa_flex_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], B, H, L, S, D,
-                                 ctypes.byref(block_mask.struct), score_mod, float(softcap),
-                                 float(scale), _ptr(out), _ptr(lse), _ptr(ws),
-                                 _stream_handle(stream)),
-           "fa_flex_attention_fwd")
+    if Hkv == H:
+        _check(fa_flex_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], B, H, L, S, D,
+                                     ctypes.byref(block_mask.struct), score_mod, float(softcap),
+                                     float(scale), _ptr(out), _ptr(lse), _ptr(ws),
+                                     _stream_handle(stream)),
+               "fa_flex_attention_fwd")
+    else:
+        _check(fa_flex_attention_fwd_gqa(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], B, H, Hkv, L,
+                                         S, D, ctypes.byref(block_mask.struct), score_mod,
+                                         float(softcap), float(scale), _ptr(out), _ptr(lse),
+                                         _ptr(ws), _stream_handle(stream)),
+               "fa_flex_attention_fwd_gqa")
     return (out, lse) if return_lse else out
 
 

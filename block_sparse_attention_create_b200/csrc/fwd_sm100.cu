@@ -127,6 +127,7 @@ struct Params {
   float* lse;
   int32_t* err;
   int BH, L, S, n_kv, num_units, bitmap_words;
+  int H, Hkv, kv_group;  // query heads, K/V heads, H / Hkv
   int mask_kind, window, softcap_on, is_bf16;
   int split_p;       // P fed to the PV product as two 16-bit terms (hi + lo)
   float scale_log2;  // scale * log2(e)
@@ -142,6 +143,7 @@ struct Params {
 // workers.  Every role of a CTA walks the same sequence.
 struct Unit {
   int bh, qblk, np, n;
+  int kvbh;  // batch * Hkv + K/V head of this unit's query head
 };
 
 __device__ __forceinline__ int2 ldg_nc_v2(const int32_t* ptr) {
@@ -179,6 +181,8 @@ struct UnitIter {
     if (nu < 0) return false;
     const int k = nu / p.BH;
     x.bh = nu - k * p.BH;
+    // grouped-query attention: query head h reads K/V head h / kv_group
+    x.kvbh = p.kv_group == 1 ? x.bh : (x.bh / p.H) * p.Hkv + (x.bh % p.H) / p.kv_group;
     x.qblk = nx.x;
     x.np = nx.y & 0xFFFF;
     x.n = x.np + (nx.y >> 16);
@@ -334,7 +338,7 @@ __device__ __forceinline__ bool produce_k(Smem<D>& sm, const Params& p, const CU
       return false;
   }
   const int st = n.k % C::kKRing;
-  if (!produce<D>(sm, p, tk, kvb * kBlockN, c.cur.bh, sm.k[SLOT][st], &sm.k_full[SLOT][st],
+  if (!produce<D>(sm, p, tk, kvb * kBlockN, c.cur.kvbh, sm.k[SLOT][st], &sm.k_full[SLOT][st],
                   &sm.k_empty[SLOT][st], n.k / C::kKRing, pol_kv))
     return false;
   ++n.k;
@@ -372,7 +376,7 @@ __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* t
     bool pend = false;
     if (c.has_cur) {
       pend_kvb = pc_block(c, p, lane);
-      pend_bh = c.cur.bh;
+      pend_bh = c.cur.kvbh;
       pend = true;
       ok = produce_k<D, SLOT>(sm, p, tq, tk, c, n, pend_kvb, pol_q, pol_kv);
     }
@@ -382,7 +386,7 @@ __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* t
       const bool next = c.has_cur;
       if (next) {
         next_kvb = pc_block(c, p, lane);
-        next_bh = c.cur.bh;
+        next_bh = c.cur.kvbh;
         ok = produce_k<D, SLOT>(sm, p, tq, tk, c, n, next_kvb, pol_q, pol_kv);
       }
       if (ok) ok = produce_v<D, SLOT>(sm, p, tv, n, pend_kvb, pend_bh, pol_kv);
@@ -394,7 +398,7 @@ __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* t
     while (ok && c.has_cur) {
       const int kvb = pc_block(c, p, lane);
       ok = produce_k<D, SLOT>(sm, p, tq, tk, c, n, kvb, pol_q, pol_kv);
-      if (ok) ok = produce_v<D, SLOT>(sm, p, tv, n, kvb, c.cur.bh, pol_kv);
+      if (ok) ok = produce_v<D, SLOT>(sm, p, tv, n, kvb, c.cur.kvbh, pol_kv);
       pc_step(c, p, lane);
     }
   }
@@ -1139,8 +1143,9 @@ fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH,
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, bf16, D, L, BH)) return FA_ERR_CUDA;
   // With S == 0 no K/V tile is ever loaded; the maps only need to be well formed.
-  if (!make_map(&tk, S > 0 ? k : q, bf16, D, S > 0 ? S : L, BH)) return FA_ERR_CUDA;
-  if (!make_map(&tv, S > 0 ? v : q, bf16, D, S > 0 ? S : L, BH)) return FA_ERR_CUDA;
+  const int BHkv = BH / prm.kv_group;
+  if (!make_map(&tk, S > 0 ? k : q, bf16, D, S > 0 ? S : L, S > 0 ? BHkv : BH)) return FA_ERR_CUDA;
+  if (!make_map(&tv, S > 0 ? v : q, bf16, D, S > 0 ? S : L, S > 0 ? BHkv : BH)) return FA_ERR_CUDA;
   const size_t smem = sizeof(Smem<D>) + 1024;
   int dev = 0;
   FA_CUDA_CHECK(cudaGetDevice(&dev));
@@ -1169,16 +1174,17 @@ fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH,
 
 extern "C" size_t fa_fwd_workspace_bytes(void) { return 256; }
 
-extern "C" fa_status fa_flex_attention_fwd(const void* q, const void* k, const void* v,
-                                           int32_t dtype, int32_t B, int32_t H, int32_t L,
-                                           int32_t S, int32_t D, const fa_block_mask* bm,
-                                           int32_t score_kind, float softcap, float scale,
-                                           void* out, float* lse, void* workspace,
-                                           void* stream) {
-  using namespace fa;
+namespace fa {
+namespace {
+
+fa_status fwd_impl(const void* q, const void* k, const void* v, int32_t dtype, int32_t B, int32_t H,
+                   int32_t Hkv, int32_t L, int32_t S, int32_t D, const fa_block_mask* bm,
+                   int32_t score_kind, float softcap, float scale, void* out, float* lse,
+                   void* workspace, void* stream) {
   if (bm == nullptr || workspace == nullptr) return FA_ERR_INVALID_ARG;
   if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
   if (B < 0 || H < 0 || L < 0 || S < 0) return FA_ERR_INVALID_ARG;
+  if (Hkv < 1 || (H > 0 && H % Hkv != 0) || (H == 0 && Hkv != 1)) return FA_ERR_INVALID_ARG;
   if (score_kind != FA_SCORE_NONE && score_kind != FA_SCORE_TANH_SOFTCAP) return FA_ERR_INVALID_ARG;
   if (score_kind == FA_SCORE_TANH_SOFTCAP && !(softcap > 0.f && std::isfinite(softcap)))
     return FA_ERR_INVALID_ARG;
@@ -1210,6 +1216,9 @@ extern "C" fa_status fa_flex_attention_fwd(const void* q, const void* k, const v
   prm.lse = lse;
   prm.err = static_cast<int32_t*>(workspace);
   prm.BH = static_cast<int>(BH64);
+  prm.H = H;
+  prm.Hkv = Hkv;
+  prm.kv_group = H > 0 ? H / Hkv : 1;
   prm.L = L;
   prm.S = S;
   prm.n_kv = bm->n_kv_blocks;
@@ -1233,4 +1242,27 @@ extern "C" fa_status fa_flex_attention_fwd(const void* q, const void* k, const v
     case kMaskBitmap * 2: return launch<64, kMaskBitmap>(q, k, v, b16, prm.BH, L, S, prm, s);
     default: return launch<128, kMaskBitmap>(q, k, v, b16, prm.BH, L, S, prm, s);
   }
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" fa_status fa_flex_attention_fwd(const void* q, const void* k, const void* v,
+                                           int32_t dtype, int32_t B, int32_t H, int32_t L,
+                                           int32_t S, int32_t D, const fa_block_mask* bm,
+                                           int32_t score_kind, float softcap, float scale,
+                                           void* out, float* lse, void* workspace,
+                                           void* stream) {
+  return fa::fwd_impl(q, k, v, dtype, B, H, H > 0 ? H : 1, L, S, D, bm, score_kind, softcap, scale,
+                      out, lse, workspace, stream);
+}
+
+extern "C" fa_status fa_flex_attention_fwd_gqa(const void* q, const void* k, const void* v,
+                                               int32_t dtype, int32_t B, int32_t H, int32_t H_kv,
+                                               int32_t L, int32_t S, int32_t D,
+                                               const fa_block_mask* bm, int32_t score_kind,
+                                               float softcap, float scale, void* out, float* lse,
+                                               void* workspace, void* stream) {
+  return fa::fwd_impl(q, k, v, dtype, B, H, H_kv, L, S, D, bm, score_kind, softcap, scale, out,
+                      lse, workspace, stream);
 }

@@ -244,6 +244,21 @@ FA_API fa_status fa_flex_attention_fwd_noalloc(const void* q, const void* k, con
                                         void* out, float* lse, int32_t* device_error,
                                         void* stream);
 
+/*
+ * Grouped-query attention forward (NEXT-2; SDPA tutorial section 5: several query
+ * heads share one K/V head, SDPA's enable_gqa).  As fa_flex_attention_fwd, except
+ *   k, v      device (B, H_kv, S, D);
+ *   H_kv      >= 1 and dividing H: query head h reads K/V head h / (H / H_kv)
+ *             (consecutive query heads share a K/V head).
+ * H_kv == H is fa_flex_attention_fwd.  Returns FA_ERR_INVALID_ARG (nothing
+ * launched) if H_kv does not divide H, else as fa_flex_attention_fwd.
+ */
+FA_API fa_status fa_flex_attention_fwd_gqa(const void* q, const void* k, const void* v,
+                                    int32_t dtype, int32_t B, int32_t H, int32_t H_kv, int32_t L,
+                                    int32_t S, int32_t D, const fa_block_mask* bm,
+                                    int32_t score_kind, float softcap, float scale, void* out,
+                                    float* lse, void* workspace, void* stream);
+
 /* Synchronises `stream`, then reads and clears the error word that the forward
  * kernel keeps in `workspace`.  Returns FA_ERR_TIMEOUT if a bounded device wait gave
  * up since the last query (the outputs of that call are then invalid), FA_ERR_CUDA

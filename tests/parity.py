@@ -49,7 +49,8 @@ def run_gpu(q, k, v, kind, window=0, doc_id=None, score_kind=0, softcap=0.0, sca
 
 def oracle_rows(q, k, v, b, h, rows, kind, window=0, doc_id=None, score_kind=0, softcap=0.0,
                 scale=0.0, bitmap=None):
-    return OA.attention_head(q[b, h], k[b, h], v[b, h], kind, window=window or None,
+    g = OA.kv_head(h, q.shape[1], k.shape[1])  # K/V head (grouped-query attention)
+    return OA.attention_head(q[b, h], k[b, g], v[b, g], kind, window=window or None,
                              doc_id=None if doc_id is None else doc_id.numpy(),
                              score_kind=score_kind, softcap=softcap,
                              scale=scale if scale > 0 else None, rows=rows, bitmap=bitmap)

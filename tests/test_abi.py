@@ -128,6 +128,16 @@ def test_bitmap_builder_and_transpose_reject_bad_arguments(fa):
     assert fa.fa_block_mask_transpose(ctypes.byref(bm2), fake, fake, fake, fake, null) == fa.FA_ERR_INVALID_ARG
 
 
+def test_gqa_rejects_uneven_head_groups(fa):
+    bm = fa.fa_block_mask()
+    bm.block, bm.q_len, bm.kv_len = 128, 256, 256
+    p = ctypes.c_void_p(1 << 20)   # never dereferenced: rejected before any use
+    null = ctypes.c_void_p(0)
+    for h, hkv in ((6, 4), (4, 0), (4, -1), (2, 4)):
+        assert fa.fa_flex_attention_fwd_gqa(p, p, p, 0, 1, h, hkv, 256, 256, 64, ctypes.byref(bm), 0,
+                                            0.0, 0.0, p, null, p, null) == fa.FA_ERR_INVALID_ARG
+
+
 def _fwd(fa, bm, **kw):
     args = dict(q=1024, k=1024, v=1024, dtype=0, B=1, H=1, L=256, S=256, D=64, sk=0, cap=0.0,
                 scale=0.0, out=1024, lse=0, ws=1024)
