@@ -49,8 +49,8 @@ KERNEL_SOURCES = ("block_sparse_attention_create_b200/csrc/fwd_sm100.cu",
                   "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
 NCU_TRAFFIC = {
     "swa256_L32768_B1_H8_D64_bf16": {
-        "bytes": 101042176 + 5957120,
-        "sources_sha256": "1411234e80f93e8412db89f9dddd3bd044cb57fdbfd07929cd7d02476e3e09c9",
+        "bytes": 101083136 + 6039040,
+        "sources_sha256": "98b7510f590ce52b385c193912c44c1fbe7920793a0b3ce3f054e467890ec4c3",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_full.md"},
 }
 
