@@ -58,7 +58,7 @@ def attention_head(q, k, v, kind, window=None, doc_id=None, score_kind=NONE, sof
         s = (q[r] @ k.T) * scale                       # (R, S) scaled scores
         if score_kind == TANH_SOFTCAP:
             s = softcap * np.tanh(s / softcap)
-        allowed = masks.mask_rows(kind, r, S, window, doc, bitmap)
+        allowed = masks.mask_rows(kind, r, S, window, doc, bitmap, q_len=L)
         s = np.where(allowed, s, -np.inf)
         m = s.max(axis=1) if S > 0 else np.full((len(r),), -np.inf)
         live = np.isfinite(m)

@@ -11,9 +11,12 @@ from __future__ import annotations
 import math
 
 
-def allowed(kind, q, kv, window=None, doc=None, bitmap=None):
+def allowed(kind, q, kv, window=None, doc=None, bitmap=None, q_len=None, kv_len=None):
     if kind == 3:  # tabulated mask_mod: bit kv % 32 of word kv // 32 of row q
         return (int(bitmap[q][kv // 32]) >> (kv % 32)) & 1 == 1
+    if kind in (4, 5, 6):  # decode: query q sits at position q + kv_len - q_len
+        pos = q + kv_len - q_len
+        return kind == 4 or (pos >= kv and (kind == 5 or pos - kv < window))
     if kind == 0:
         return q >= kv
     if kind == 1:
@@ -35,7 +38,7 @@ def attention_head(q, k, v, kind, window=None, doc=None, score_kind=0, softcap=0
     for i in range(L):
         scores = []
         for j in range(S):
-            if not allowed(kind, i, j, window, doc, bitmap):
+            if not allowed(kind, i, j, window, doc, bitmap, L, S):
                 continue
             s = 0.0
             for d in range(D):

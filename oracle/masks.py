@@ -7,6 +7,10 @@ Source: "FlexAttention on Apple Silicon: block mask how-to"
   * "Mask 3: document-packed"       -- causal AND document_id[q] == document_id[kv].
   * a tabulated mask_mod (the how-to's create_block_mask takes any function of
     (b, h, q_idx, kv_idx); "Mask 1: causal" shows the form) -- one bit per pair.
+  * decode against a KV cache (SDPA tutorial, section 4, pitfall 3): L new
+    queries after S - L cached keys see causally aligned to the lower right,
+    q_idx + S - L >= kv_idx (torch's causal_lower_right), optionally within a
+    window of W keys; or no mask at all.
 True means "this pair is used" (the SDPA boolean-mask convention, qiita
 GeneLab_999 SDPA tutorial, section 4, pitfall 1).  Indices are absolute
 positions, so for L != S the causal diagonal is upper-left aligned (SDPA
@@ -20,6 +24,10 @@ CAUSAL = 0
 SLIDING_WINDOW_CAUSAL = 1
 DOCUMENT_CAUSAL = 2
 BITMAP = 3
+# decode against a KV cache (lower-right alignment; need the query length L)
+DECODE_FULL = 4
+DECODE_CAUSAL = 5
+DECODE_SLIDING_WINDOW = 6
 
 
 def causal(q_idx, kv_idx):
@@ -56,8 +64,18 @@ def to_bitmap(kind, q_len, kv_len, window=None, doc_id=None, words_per_row=None)
     return words
 
 
-def mask_rows(kind, q_rows, kv_len, window=None, doc_id=None, bitmap=None):
-    """Dense boolean mask for the given query rows against keys 0..kv_len-1.
+def causal_lower_right(q_idx, kv_idx, q_len, kv_len):
+    return q_idx + (kv_len - q_len) >= kv_idx
+
+
+def sliding_window_lower_right(q_idx, kv_idx, q_len, kv_len, window):
+    pos = q_idx + (kv_len - q_len)   # the query's position in the key sequence
+    return (pos >= kv_idx) & (pos - kv_idx < window)
+
+
+def mask_rows(kind, q_rows, kv_len, window=None, doc_id=None, bitmap=None, q_len=None):
+    """Dense boolean mask for the given query rows against keys 0..kv_len-1
+    (``q_len``: the number of queries, needed by the decode kinds).
 
     Returns a bool array of shape (len(q_rows), kv_len).
     """
@@ -78,4 +96,14 @@ def mask_rows(kind, q_rows, kv_len, window=None, doc_id=None, bitmap=None):
         if bitmap is None:
             raise ValueError("bitmap mask needs the bitmap")
         return bitmap_bits(bitmap, q, kv)
+    if kind in (DECODE_FULL, DECODE_CAUSAL, DECODE_SLIDING_WINDOW):
+        if q_len is None:
+            raise ValueError("decode masks need the query length")
+        if kind == DECODE_FULL:
+            return np.ones((q.shape[0], kv_len), dtype=bool)
+        if kind == DECODE_CAUSAL:
+            return causal_lower_right(q, kv, q_len, kv_len)
+        if window is None:
+            raise ValueError("sliding-window mask needs a window")
+        return sliding_window_lower_right(q, kv, q_len, kv_len, int(window))
     raise ValueError(f"unknown mask kind {kind}")

@@ -427,3 +427,47 @@ def test_gqa_head_map_hand_example():
     assert [OA.kv_head(h, 5, 1) for h in range(5)] == [0] * 5
     with pytest.raises(ValueError):
         OA.kv_head(0, 6, 4)
+
+
+# ---------------------------------------------------------------- decode (KV cache)
+
+@pytest.mark.parametrize("L,S", [(1, 6), (1, 300), (5, 300), (64, 1000)])
+def test_decode_rows_equal_last_rows_of_full_causal(L, S):
+    """SDPA tutorial, section 4, pitfall 3: decoding the last L queries against the
+    whole cache with the lower-right causal mask equals the last L rows of causal
+    attention over all S queries (L = S, where both alignments agree)."""
+    q_all, k, v = _rand((S, 32), 1), _rand((S, 32), 2), _rand((S, 32), 3)
+    full, lfull = OA.attention_head(q_all, k, v, OM.CAUSAL, rows=np.arange(S - L, S))
+    dec, ldec = OA.attention_head(q_all[S - L:], k, v, OM.DECODE_CAUSAL)
+    assert np.array_equal(full, dec) and np.array_equal(lfull, ldec)
+    fw, lw = OA.attention_head(q_all, k, v, OM.SLIDING_WINDOW_CAUSAL, window=40,
+                               rows=np.arange(S - L, S))
+    dw, ldw = OA.attention_head(q_all[S - L:], k, v, OM.DECODE_SLIDING_WINDOW, window=40)
+    assert np.array_equal(fw, dw) and np.array_equal(lw, ldw)
+
+
+def test_decode_matches_torch_causal_lower_right():
+    """torch's CPU SDPA in fp64 with its causal_lower_right bias."""
+    from torch.nn.attention.bias import causal_lower_right
+    L, S = 7, 200
+    q = torch.from_numpy(_rand((1, 2, L, 32), 4))
+    k = torch.from_numpy(_rand((1, 2, S, 32), 5))
+    v = torch.from_numpy(_rand((1, 2, S, 32), 6))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q, k, v, attn_mask=causal_lower_right(L, S)).numpy()
+    nomask = torch.nn.functional.scaled_dot_product_attention(q, k, v).numpy()
+    for h in range(2):
+        out, _ = OA.attention_head(q[0, h], k[0, h], v[0, h], OM.DECODE_CAUSAL)
+        assert np.abs(out - ref[0, h]).max() < 1e-12
+        full, _ = OA.attention_head(q[0, h], k[0, h], v[0, h], OM.DECODE_FULL)
+        assert np.abs(full - nomask[0, h]).max() < 1e-12
+
+
+@pytest.mark.parametrize("kind", [OM.DECODE_FULL, OM.DECODE_CAUSAL, OM.DECODE_SLIDING_WINDOW])
+def test_decode_bruteforce_tiny(kind):
+    L, S = 3, 11
+    q, k, v = (_rand((n, 8), s) for n, s in ((L, 7), (S, 8), (S, 9)))
+    out, lse = OA.attention_head(q, k, v, kind, window=4)
+    bo, bl = BF.attention_head(q.tolist(), k.tolist(), v.tolist(), kind, 4)
+    assert np.allclose(out, np.array(bo), atol=1e-13, rtol=0)
+    assert np.allclose(lse, np.array(bl), atol=1e-13, rtol=0)
