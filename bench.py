@@ -115,7 +115,28 @@ def live_blocks_per_row(w: W.Workload):
     return out
 
 
+def decode_pairs_per_row(w: W.Workload):
+    """Keys each of the L new queries sees (decode, lower-right alignment)."""
+    pos = w.S - w.L + np.arange(w.L)          # key position of each query
+    if w.mask_kind == W.MASK_DECODE_FULL:
+        return np.full(w.L, w.S, dtype=np.int64)
+    hi = np.clip(pos + 1, 0, w.S)              # keys 0 .. pos
+    if w.mask_kind == W.MASK_DECODE_CAUSAL:
+        return hi.astype(np.int64)
+    return np.clip(hi - np.clip(pos - w.window + 1, 0, None), 0, None).astype(np.int64)
+
+
+def is_decode(w: W.Workload) -> bool:
+    return w.mask_kind >= W.MASK_DECODE_FULL
+
+
 def work_figures(w: W.Workload):
+    if is_decode(w):
+        pairs = decode_pairs_per_row(w)
+        flops = 4.0 * w.D * float(pairs.sum()) * w.B * w.H
+        bytes_ = (w.B * w.H * w.L * w.D * 2 * 2 + w.B * w.n_kv_heads * w.S * w.D * 2 * 2
+                  + w.B * w.H * w.L * 4)
+        return {"live_blocks": None, "pairs": pairs, "flops": flops, "bytes": bytes_}
     per_row = live_blocks_per_row(w)
     live = int(per_row.sum())
     flops = 4.0 * w.D * 128 * 128 * live * w.B * w.H
@@ -184,6 +205,31 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples_under_load": busy}
 
 
+def step_calls(fa, w, qd, kd, vd, dd, bd, out, lse, device, stream):
+    """(mask build, forward, device-error query) of one step through the public API.
+    Decode workloads have no mask tables: the build is empty."""
+    if is_decode(w):
+        nbytes = int(fa.fa_decode_workspace_bytes(w.B, w.H, w.n_kv_heads, w.L, w.S, w.D))
+        dws = fa.decode_workspace(device, nbytes)
+
+        def attend():
+            fa.flex_attention_decode(qd, kd, vd, mask=w.mask_kind - W.MASK_DECODE_FULL,
+                                     window=w.window, score_mod=w.score_kind, softcap=w.softcap,
+                                     out=out, lse=lse, ws=dws, stream=stream)
+        return (lambda: None), attend, (lambda: fa.last_decode_error(device))
+    bm = fa.BlockMask(w.L, w.S, device)
+    ws = fa.workspace(device)
+
+    def build():
+        fa.create_block_mask(w.mask_kind, w.L, w.S, window=w.window, doc_id=dd, out=bm,
+                             stream=stream, bitmap=bd)
+
+    def attend():
+        fa.flex_attention(qd, kd, vd, bm, score_mod=w.score_kind, softcap=w.softcap, out=out,
+                          lse=lse, ws=ws, stream=stream)
+    return build, attend, (lambda: fa.last_device_error(device))
+
+
 def run_ours(args, w: W.Workload, rank, world, device):
     import block_sparse_attention_create_b200 as fa
     torch.cuda.set_device(device)
@@ -196,22 +242,19 @@ def run_ours(args, w: W.Workload, rank, world, device):
     bd = bits.to(device) if bits is not None else None
     out = torch.empty_like(qd)
     lse = torch.empty(w.B, w.H, w.L, dtype=torch.float32, device=device)
-    bm = fa.BlockMask(w.L, w.S, device)
-    ws = fa.workspace(device)
     stream = torch.cuda.current_stream()
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+    build, attend, dev_error = step_calls(fa, w, qd, kd, vd, dd, bd, out, lse, device, stream)
 
     def step():
-        fa.create_block_mask(w.mask_kind, w.L, w.S, window=w.window, doc_id=dd, out=bm,
-                             stream=stream, bitmap=bd)
-        fa.flex_attention(qd, kd, vd, bm, score_mod=w.score_kind, softcap=w.softcap, out=out,
-                          lse=lse, ws=ws, stream=stream)
+        build()
+        attend()
 
     fig = work_figures(w)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    assert fa.last_device_error(device) == fa.FA_OK
+    assert dev_error() == fa.FA_OK
 
     # keep the GPU at load clocks for ~1 s inside the sampling window, untimed
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -230,16 +273,14 @@ def run_ours(args, w: W.Workload, rank, world, device):
         for i in range(args.steps):
             flush.zero_()
             starts[i].record(stream)
-            fa.create_block_mask(w.mask_kind, w.L, w.S, window=w.window, doc_id=dd, out=bm,
-                                 stream=stream, bitmap=bd)
+            build()
             mids[i].record(stream)
-            fa.flex_attention(qd, kd, vd, bm, score_mod=w.score_kind, softcap=w.softcap,
-                              out=out, lse=lse, ws=ws, stream=stream)
+            attend()
             ends[i].record(stream)
         torch.cuda.synchronize()
         if world > 1:
             torch.distributed.barrier()
-    assert fa.last_device_error(device) == fa.FA_OK
+    assert dev_error() == fa.FA_OK
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     fwd_ms = [m.elapsed_time(e) for m, e in zip(mids, ends)]
     mask_ms = [s.elapsed_time(m) for s, m in zip(starts, mids)]
@@ -267,8 +308,8 @@ def run_e2e(args, w, fa, q, k, v, doc, bits, device, world):
     dd = torch.empty(doc.shape, dtype=doc.dtype, device=device) if doc is not None else None
     out = torch.empty_like(qd)
     lse = torch.empty(w.B, w.H, w.L, dtype=torch.float32, device=device)
-    bm = fa.BlockMask(w.L, w.S, device)
     stream = torch.cuda.current_stream()
+    build, attend, _ = step_calls(fa, w, qd, kd, vd, dd, bd, out, lse, device, stream)
 
     def step():
         qd.copy_(hq, non_blocking=True)
@@ -278,10 +319,8 @@ def run_e2e(args, w, fa, q, k, v, doc, bits, device, world):
             dd.copy_(hdoc, non_blocking=True)
         if bd is not None:
             bd.copy_(hbits, non_blocking=True)
-        fa.create_block_mask(w.mask_kind, w.L, w.S, window=w.window, doc_id=dd, out=bm,
-                             stream=stream, bitmap=bd)
-        fa.flex_attention(qd, kd, vd, bm, score_mod=w.score_kind, softcap=w.softcap, out=out,
-                          lse=lse, stream=stream)
+        build()
+        attend()
         hout.copy_(out, non_blocking=True)
         hlse.copy_(lse, non_blocking=True)
 
@@ -313,6 +352,14 @@ def oracle_sample(w: W.Workload, rows, fig):
     q, k, v = W.make_qkv(w)
     doc = W.make_doc_id(w)
     words = W.make_bitmap(w)
+    if is_decode(w):  # every new query of the first `rows` heads
+        t0 = time.perf_counter()
+        for h in range(len(rows)):
+            g = OA.kv_head(h, w.H, w.n_kv_heads)
+            OA.attention_head(q[0, h], k[0, g], v[0, g], w.mask_kind, window=w.window or None,
+                              score_kind=w.score_kind, softcap=w.softcap)
+        dt = time.perf_counter() - t0
+        return dt, 4.0 * w.D * float(fig["pairs"].sum()) * len(rows)
     t0 = time.perf_counter()
     OA.attention_head(q[0, 0], k[0, 0], v[0, 0], w.mask_kind, window=w.window or None,
                       doc_id=None if doc is None else doc.numpy(), score_kind=w.score_kind,
@@ -414,26 +461,35 @@ def main():
             "dtype": w.dtype_name, "data": "synthetic",
             "config": {**w.describe(), "parallelism": f"replicas x{world}" if world > 1 else "none",
                        "l2": "flushed between timed steps (512 MiB write, untimed)",
-                       "step": "fa_create_block_mask + fa_flex_attention_fwd"},
+                       "step": ("fa_flex_attention_decode" if is_decode(w)
+                                else "fa_create_block_mask + fa_flex_attention_fwd")},
             "fwd_ms": fwd_avg, "fwd_ms_median": fwd_med, "fwd_tflops": fwd_tflops,
             "fwd_tensor_frac": tensor_frac, "fwd_hbm_gbs": fwd_gbs, "fwd_hbm_frac": hbm_frac,
             "mask_build_ms": statistics.mean(r["mask_ms"]),
             "live_blocks_per_head": fig["live_blocks"], "live_gflop": fig["flops"] / 1e9,
+            **({"step_kind": "decode (split-KV forward + merge; no mask tables)"}
+               if is_decode(w) else {}),
             "algorithmic_mb": fig["bytes"] / 1e6,
             "roofline": roof,
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": (2 if is_decode(w) else 3) * args.steps,
             "clocks": r["clocks"],
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": r["e2e"]["h2d"],
                     "d2h_bytes_per_step": r["e2e"]["d2h"],
                     "ms_per_step": r["e2e"]["ms"] / args.steps}}
     if rank == 0 and world == 1 and not args.profile:
-        rows = np.sort(np.random.default_rng(1).choice(w.L, size=min(args.cpu_rows, w.L),
-                                                       replace=False))
+        if is_decode(w):  # the oracle on all new queries of every head of batch 0
+            rows = np.arange(w.H)
+        else:
+            rows = np.sort(np.random.default_rng(1).choice(w.L, size=min(args.cpu_rows, w.L),
+                                                           replace=False))
         dt, credited = oracle_sample(w, rows, fig)
         line["cpu_baseline"] = {"value": credited / dt / 1e12, "unit": UNIT, "cores": cpu_threads(),
                                 "kind": "oracle",
-                                "sample": f"{len(rows)} random query rows of head (0,0), "
-                                          f"{dt:.1f} s; live-block FLOPs of those rows credited"}
+                                "sample": (f"all {w.L} new queries of the {len(rows)} heads of "
+                                           f"batch 0, {dt:.1f} s; visible-pair FLOPs credited"
+                                           if is_decode(w) else
+                                           f"{len(rows)} random query rows of head (0,0), "
+                                           f"{dt:.1f} s; live-block FLOPs of those rows credited")}
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:

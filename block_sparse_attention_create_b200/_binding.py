@@ -28,6 +28,8 @@ LIB_PATH = os.path.join(_HERE, "libfa.so")
 FA_MASK_CAUSAL, FA_MASK_SLIDING_WINDOW_CAUSAL, FA_MASK_DOCUMENT_CAUSAL, FA_MASK_BITMAP = range(4)
 FA_SCORE_NONE, FA_SCORE_TANH_SOFTCAP = range(2)
 FA_BF16, FA_FP16 = range(2)
+FA_DECODE_FULL, FA_DECODE_CAUSAL, FA_DECODE_SLIDING_WINDOW = range(3)
+FA_DECODE_MAX_ROWS = 32
 FA_BLOCK = 128
 FA_MAX_LEN = 8192 * 128
 FA_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -36,7 +38,8 @@ FA_NOALLOC_SCRATCH_BYTES = 4 << 20
 EXPORTED = ("fa_block_mask_dims", "fa_create_block_mask", "fa_fwd_workspace_bytes",
             "fa_flex_attention_fwd", "fa_get_last_device_error", "fa_status_string",
             "fa_num_sms", "fa_flex_attention_fwd_noalloc", "fa_create_block_mask_bitmap",
-            "fa_block_mask_transpose", "fa_flex_attention_fwd_gqa")
+            "fa_block_mask_transpose", "fa_flex_attention_fwd_gqa", "fa_decode_workspace_bytes",
+            "fa_flex_attention_decode")
 
 
 class fa_block_mask(ctypes.Structure):
@@ -91,6 +94,11 @@ def _load():
                                               ctypes.POINTER(fa_block_mask), i32, f32, f32, vp, vp,
                                               vp, vp]
     lib.fa_flex_attention_fwd_gqa.restype = i32
+    lib.fa_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
+    lib.fa_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa_flex_attention_decode.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
+                                             i32, i32, f32, f32, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.fa_flex_attention_decode.restype = i32
     return lib
 
 
@@ -108,6 +116,8 @@ fa_flex_attention_fwd_noalloc = _lib.fa_flex_attention_fwd_noalloc
 fa_create_block_mask_bitmap = _lib.fa_create_block_mask_bitmap
 fa_block_mask_transpose = _lib.fa_block_mask_transpose
 fa_flex_attention_fwd_gqa = _lib.fa_flex_attention_fwd_gqa
+fa_decode_workspace_bytes = _lib.fa_decode_workspace_bytes
+fa_flex_attention_decode = _lib.fa_flex_attention_decode
 
 
 class FAError(RuntimeError):
@@ -292,6 +302,58 @@ def flex_attention_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ma
                                          _ptr(device_error), _stream_handle(stream)),
            "fa_flex_attention_fwd_noalloc")
     return out, lse
+
+
+_decode_workspaces = {}
+
+
+def decode_workspace(device, nbytes: int) -> torch.Tensor:
+    """A zeroed decode workspace of at least `nbytes` per device (grown on demand)."""
+    dev = torch.device(device)
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    ws = _decode_workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=f"cuda:{key}")
+        _decode_workspaces[key] = ws
+    return ws
+
+
+def flex_attention_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                          mask: int = FA_DECODE_CAUSAL, window: int = 0,
+                          score_mod: int = FA_SCORE_NONE, softcap: float = 0.0, scale: float = 0.0,
+                          out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                          return_lse: bool = False, ws: Optional[torch.Tensor] = None,
+                          stream: Optional[torch.cuda.Stream] = None):
+    """fa_flex_attention_decode: q (B,H,L,D) new queries against the cache k/v
+    (B,Hkv,S,D), lower-right aligned."""
+    if q.dtype not in _DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share dtype bf16 or fp16")
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError("q, k, v must be contiguous 4-D CUDA tensors")
+    B, H, L, D = q.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, S, D) or v.shape != (B, Hkv, S, D) or Hkv < 1 or H % Hkv:
+        raise ValueError("k and v must be (B, Hkv, S, D) with the q's B and D, Hkv dividing H")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty(B, H, L, dtype=torch.float32, device=q.device)
+    need = int(fa_decode_workspace_bytes(B, H, Hkv, L, S, D))
+    if ws is None:
+        ws = decode_workspace(q.device, need)
+    _check(fa_flex_attention_decode(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], B, H, Hkv, L, S, D,
+                                    mask, window, score_mod, float(softcap), float(scale),
+                                    _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                    _stream_handle(stream)),
+           "fa_flex_attention_decode")
+    return (out, lse) if return_lse else out
+
+
+def last_decode_error(device=None, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """fa_get_last_device_error on the per-device decode workspace."""
+    dev = device if device is not None else torch.cuda.current_device()
+    return fa_get_last_device_error(_ptr(decode_workspace(dev, 256)), _stream_handle(stream))
 
 
 def last_device_error(device=None, stream: Optional[torch.cuda.Stream] = None) -> int:

@@ -1,0 +1,439 @@
+// Decode against a KV cache (SDPA tutorial, section 4, pitfall 3): L new queries
+// after S - L cached keys, the causal mask aligned to the lower right (query i sits
+// at key position S - L + i), optionally within a window of W keys, or no mask.
+// L is small (a token or a short chunk), S long, so the work is reading K and V
+// once: the path is bound by HBM, not by the tensor cores, and runs on the CUDA
+// cores.
+//
+// Split-KV: CTA (split, b * Hkv + kvh) takes every query row that reads K/V head
+// kvh -- the H / Hkv query heads of the group times the L queries, R <= 32 rows --
+// against one contiguous chunk of keys, streamed through shared memory in 64-key
+// tiles by TMA (128-byte swizzle, double-buffered, bounded mbarrier waits).  It
+// leaves the chunk's running max, sum and unnormalised output per row in the
+// workspace; a second kernel merges the chunks of each row (rescaling each by
+// 2^(m_chunk - m)) into out and LSE.  Chunks no row can see (sliding window) load
+// nothing.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "fa_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace fa {
+namespace {
+
+constexpr int kTile = 64;            // keys per K/V tile
+constexpr int kDecThreads = 128;
+constexpr int kMaxRows = FA_DECODE_MAX_ROWS;
+constexpr int kTargetCtas = 2 * 148;  // two waves of B200's SMs
+constexpr int kBoxBytes = kTile * 128;  // one TMA box: 64 keys x 64 elements
+constexpr int kDecWorkspaceHeader = 256;  // word 0: device error flags
+constexpr float kDecLog2e = 1.4426950408889634f;
+constexpr float kDecLn2 = 0.6931471805599453f;
+
+struct DecParams {
+  const uint16_t* q;  // (B, H, L, D)
+  void* out;          // (B, H, L, D)
+  float* lse;         // (B, H, L) or null
+  float* part;        // per (b, h, i, split): m, l, O[D]
+  int32_t* err;
+  int H, Hkv, G, L, S, nsplit, chunk, mask, window, softcap_on, is_bf16;
+  float q_scale;  // folded into Q: scale * log2(e), or scale alone under the softcap
+  float cap_c;    // softcap c
+  float cap_a;    // c * log2(e)
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct __align__(1024) DecSmem {
+  uint8_t k[2][D / 64][kBoxBytes];
+  uint8_t v[2][D / 64][kBoxBytes];
+  float qs[kMaxRows][D];
+  float sc[kMaxRows][kTile];
+  float m[kMaxRows], l[kMaxRows], alpha[kMaxRows];
+  uint64_t full[2];
+  volatile int abort_flag;
+};
+
+__device__ __forceinline__ float load16(const uint16_t* ptr, bool bf16) {
+  const uint16_t u = __ldg(ptr);
+  return bf16 ? __uint_as_float(static_cast<uint32_t>(u) << 16)
+              : __half2float(__ushort_as_half(u));
+}
+
+// 8 consecutive 16-bit values -> fp32.
+__device__ __forceinline__ void unpack8(const uint4 raw, bool bf16, float (&f)[8]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (bf16) {
+      f[2 * i] = __uint_as_float(w[i] << 16);
+      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    } else {
+      const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+      f[2 * i] = h.x;
+      f[2 * i + 1] = h.y;
+    }
+  }
+}
+
+// 16-byte chunk c (elements 8c .. 8c+7) of key row j of a tile: box c / 8, swizzled
+// position (c % 8) ^ (j % 8) inside the row's 128 bytes.
+template <int NB>
+__device__ __forceinline__ uint4 tile_chunk(const uint8_t (&tile)[NB][kBoxBytes], int j, int c) {
+  return *reinterpret_cast<const uint4*>(&tile[c >> 3][j * 128 + (((c & 7) ^ (j & 7)) << 4)]);
+}
+
+template <int D>
+__device__ __forceinline__ bool dec_wait(DecSmem<D>& sm, uint64_t* bar, uint32_t parity,
+                                         const DecParams& p) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (sm.abort_flag) return false;
+    if (globaltimer_ns() - t0 > p.timeout_ns) {
+      sm.abort_flag = 1;
+      atomicOr(p.err, kDevErrTimeout);
+      return false;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecThreads)
+decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                    const __grid_constant__ DecParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = smem_u32(smem_raw);
+  DecSmem<D>& sm = *reinterpret_cast<DecSmem<D>*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
+  constexpr int kChunks = D / 8;                  // 16-byte chunks of a row
+  constexpr int kGroups = kDecThreads / kChunks;  // row groups of the PV step
+  constexpr int kRowsPer = kMaxRows / kGroups;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int split = blockIdx.x, bkv = blockIdx.y;
+  const int b = bkv / p.Hkv, kvh = bkv - b * p.Hkv;
+  const int R = p.G * p.L;
+  const bool bf16 = p.is_bf16 != 0;
+
+  // keys of this chunk that some row can see: the window's lower edge for row 0
+  int k_start = split * p.chunk;
+  const int c1 = min(p.S, k_start + p.chunk);
+  if (p.mask == FA_DECODE_SLIDING_WINDOW) k_start = max(k_start, p.S - p.L - p.window + 1);
+  const int ntiles = k_start < c1 ? (c1 - k_start + kTile - 1) / kTile : 0;
+
+  if (tid == 0) {
+    mbar_init(&sm.full[0], 1);
+    mbar_init(&sm.full[1], 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  // query rows r = g * L + i (query head kvh * G + g, query i), scaled
+  for (int e = tid; e < R * D; e += kDecThreads) {
+    const int r = e / D, d = e - (e / D) * D;
+    const int g = r / p.L, i = r - g * p.L;
+    const size_t qi = (static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i) * D + d;
+    sm.qs[r][d] = load16(p.q + qi, bf16) * p.q_scale;
+  }
+  for (int r = tid; r < R; r += kDecThreads) {
+    sm.m[r] = -INFINITY;
+    sm.l[r] = 0.f;
+  }
+  __syncthreads();
+
+  const uint64_t pol = policy_evict_first();
+  auto issue = [&](int t) {
+    const int buf = t & 1;
+    const int k0 = k_start + t * kTile;
+    fence_proxy_async_shared();
+    mbar_arrive_expect_tx(&sm.full[buf], 2 * (D / 64) * kBoxBytes);
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      tma_load_3d(sm.k[buf][c], &tk, &sm.full[buf], c * 64, k0, bkv, pol);
+      tma_load_3d(sm.v[buf][c], &tv, &sm.full[buf], c * 64, k0, bkv, pol);
+    }
+  };
+  if (tid == 0 && ntiles > 0) issue(0);
+
+  const int oc = tid % kChunks, og = tid / kChunks;  // PV: 16-byte chunk, row group
+  float o[kRowsPer][8];
+#pragma unroll
+  for (int k = 0; k < kRowsPer; ++k)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[k][e] = 0.f;
+
+  int t = 0;
+  for (; t < ntiles; ++t) {
+    const int buf = t & 1;
+    const int k0 = k_start + t * kTile;
+    if (tid == 0 && t + 1 < ntiles) issue(t + 1);  // its buffer was released after tile t - 1
+    const bool ok = dec_wait(sm, &sm.full[buf], (t >> 1) & 1, p);
+    if (!__syncthreads_and(ok)) break;
+
+    // scores: thread = (key j, row parity); rows r = rg, rg + 2, ...
+    {
+      const int j = tid & (kTile - 1), rg = tid >> 6;
+      float acc[kMaxRows / 2];
+#pragma unroll
+      for (int k = 0; k < kMaxRows / 2; ++k) acc[k] = 0.f;
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
+        float kf[8];
+        unpack8(tile_chunk(sm.k[buf], j, c), bf16, kf);
+#pragma unroll
+        for (int k = 0; k < kMaxRows / 2; ++k) {
+          const int r = rg + 2 * k;
+          if (r < R) {
+            const float4 qa = *reinterpret_cast<const float4*>(&sm.qs[r][c * 8]);
+            const float4 qb = *reinterpret_cast<const float4*>(&sm.qs[r][c * 8 + 4]);
+            acc[k] += qa.x * kf[0] + qa.y * kf[1] + qa.z * kf[2] + qa.w * kf[3] +
+                      qb.x * kf[4] + qb.y * kf[5] + qb.z * kf[6] + qb.w * kf[7];
+          }
+        }
+      }
+      const int kv = k0 + j;
+#pragma unroll
+      for (int k = 0; k < kMaxRows / 2; ++k) {
+        const int r = rg + 2 * k;
+        if (r < R) {
+          const int pos = p.S - p.L + (r % p.L);  // the query's key position
+          bool keep = kv < c1;
+          if (p.mask != FA_DECODE_FULL) keep = keep && kv <= pos;
+          if (p.mask == FA_DECODE_SLIDING_WINDOW) keep = keep && pos - kv < p.window;
+          float s = acc[k];
+          if (p.softcap_on) s = p.cap_a * tanhf(s / p.cap_c);
+          sm.sc[r][j] = keep ? s : -INFINITY;
+        }
+      }
+    }
+    __syncthreads();
+
+    // online softmax: warp w takes rows w, w + 4, ...; lane holds keys lane, lane + 32
+    for (int r = warp; r < R; r += 4) {
+      const float s0 = sm.sc[r][lane], s1 = sm.sc[r][lane + 32];
+      float mx = fmaxf(s0, s1);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float m_old = sm.m[r];
+      const float m_new = fmaxf(m_old, mx);
+      const float mu = m_new == -INFINITY ? 0.f : m_new;  // a row with no key yet: p = 0
+      const float p0 = ex2_approx(s0 - mu), p1 = ex2_approx(s1 - mu);
+      float sum = p0 + p1;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      sm.sc[r][lane] = p0;
+      sm.sc[r][lane + 32] = p1;
+      __syncwarp();
+      if (lane == 0) {
+        const float a = ex2_approx(m_old - mu);  // 0 while the row had no key
+        sm.alpha[r] = a;
+        sm.l[r] = sm.l[r] * a + sum;
+        sm.m[r] = m_new;
+      }
+    }
+    __syncthreads();
+
+    // O += P V: thread = (16-byte chunk oc of a V row, row group og)
+    {
+      float al[kRowsPer];
+#pragma unroll
+      for (int k = 0; k < kRowsPer; ++k) {
+        const int r = og + kGroups * k;
+        al[k] = r < R ? sm.alpha[r] : 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[k][e] *= al[k];
+      }
+      const int nk = min(kTile, c1 - k0);
+      for (int j = 0; j < nk; ++j) {
+        float vf[8];
+        unpack8(tile_chunk(sm.v[buf], j, oc), bf16, vf);
+#pragma unroll
+        for (int k = 0; k < kRowsPer; ++k) {
+          const int r = og + kGroups * k;
+          if (r < R) {
+            const float pj = sm.sc[r][j];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) o[k][e] = fmaf(pj, vf[e], o[k][e]);
+          }
+        }
+      }
+    }
+    __syncthreads();  // tile buffer and scores free
+  }
+
+  if (t < ntiles) {
+    // aborted: let the copies still in flight land (bounded) before the CTA exits
+    if (tid == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      for (int u = t; u < min(ntiles, t + 2); ++u)
+        while (!mbar_try_wait(&sm.full[u & 1], (u >> 1) & 1) &&
+               globaltimer_ns() - t0 < p.timeout_ns) {
+        }
+    }
+    return;
+  }
+
+  // this chunk's partial result per row
+#pragma unroll
+  for (int k = 0; k < kRowsPer; ++k) {
+    const int r = og + kGroups * k;
+    if (r < R) {
+      const int g = r / p.L, i = r - g * p.L;
+      const size_t row = static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i;
+      float* rec = p.part + (row * p.nsplit + split) * (D + 2);
+      if (oc == 0) {
+        rec[0] = sm.m[r];
+        rec[1] = sm.l[r];
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) rec[2 + oc * 8 + e] = o[k][e];
+    }
+  }
+}
+
+// One CTA per query row, one thread per output column: merge the chunks.
+template <int D>
+__global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant__ DecParams p) {
+  const size_t row = blockIdx.x;
+  const int d = threadIdx.x;
+  const float* rec0 = p.part + row * p.nsplit * (D + 2);
+  float mx = -INFINITY;
+  for (int s = 0; s < p.nsplit; ++s) mx = fmaxf(mx, rec0[static_cast<size_t>(s) * (D + 2)]);
+  float l = 0.f, acc = 0.f;
+  if (mx != -INFINITY) {
+    for (int s = 0; s < p.nsplit; ++s) {
+      const float* rec = rec0 + static_cast<size_t>(s) * (D + 2);
+      const float w = ex2_approx(rec[0] - mx);  // 0 for a chunk that saw no key
+      l = fmaf(w, rec[1], l);
+      acc = fmaf(w, rec[2 + d], acc);
+    }
+  }
+  const float o = l > 0.f ? acc / l : 0.f;
+  uint16_t* dst = static_cast<uint16_t*>(p.out) + row * D + d;
+  if (p.is_bf16) {
+    *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(o);
+  } else {
+    *reinterpret_cast<__half*>(dst) = __float2half_rn(o);
+  }
+  if (d == 0 && p.lse) p.lse[row] = l > 0.f ? (mx + log2f(l)) * kDecLn2 : -INFINITY;
+}
+
+// Chunking of the keys: about kTargetCtas CTAs over (B * Hkv) groups, whole tiles.
+void decode_plan(int B, int Hkv, int S, int* nsplit, int* chunk) {
+  const int groups = B * Hkv > 0 ? B * Hkv : 1;
+  const int tiles = S > 0 ? (S + kTile - 1) / kTile : 1;
+  int n = (kTargetCtas + groups - 1) / groups;
+  n = n < tiles ? n : tiles;
+  const int tiles_per = (tiles + n - 1) / n;
+  *chunk = tiles_per * kTile;
+  *nsplit = S > 0 ? (S + *chunk - 1) / *chunk : 1;
+}
+
+template <int D>
+fa_status decode_launch(const void* k, const void* v, bool bf16, int B, int S, const DecParams& prm,
+                        cudaStream_t stream) {
+  CUtensorMap tk, tv;
+  // With S == 0 no tile is loaded; the maps only need to be well formed.
+  const void* kp = S > 0 ? k : prm.q;
+  const void* vp = S > 0 ? v : prm.q;
+  const int rows = S > 0 ? S : 1, bh = S > 0 ? B * prm.Hkv : 1;
+  if (!make_tile_map(&tk, kp, bf16, D, rows, bh, kTile)) return FA_ERR_CUDA;
+  if (!make_tile_map(&tv, vp, bf16, D, rows, bh, kTile)) return FA_ERR_CUDA;
+  const size_t smem = sizeof(DecSmem<D>) + 1024;
+  int dev = 0;
+  FA_CUDA_CHECK(cudaGetDevice(&dev));
+  {
+    static std::mutex mu;
+    static bool done[kMaxDevices] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    if (!done[dev]) {
+      FA_CUDA_CHECK(cudaFuncSetAttribute(decode_split_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem)));
+      done[dev] = true;
+    }
+  }
+  const dim3 grid(prm.nsplit, B * prm.Hkv);
+  decode_split_kernel<D><<<grid, kDecThreads, smem, stream>>>(tk, tv, prm);
+  FA_CUDA_CHECK(cudaGetLastError());
+  decode_combine_kernel<D><<<B * prm.H * prm.L, D, 0, stream>>>(prm);
+  FA_CUDA_CHECK(cudaGetLastError());
+  return FA_OK;
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" size_t fa_decode_workspace_bytes(int32_t B, int32_t H, int32_t H_kv, int32_t L,
+                                            int32_t S, int32_t D) {
+  if (B < 0 || H < 0 || H_kv < 1 || L < 0 || S < 0 || D < 0) return 0;
+  int nsplit = 0, chunk = 0;
+  fa::decode_plan(B, H_kv, S, &nsplit, &chunk);
+  return fa::kDecWorkspaceHeader + static_cast<size_t>(B) * H * L * nsplit * (D + 2) * sizeof(float);
+}
+
+extern "C" fa_status fa_flex_attention_decode(const void* q, const void* k, const void* v,
+                                              int32_t dtype, int32_t B, int32_t H, int32_t H_kv,
+                                              int32_t L, int32_t S, int32_t D, int32_t mask,
+                                              int32_t window, int32_t score_kind, float softcap,
+                                              float scale, void* out, float* lse, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  using namespace fa;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (B < 0 || H < 0 || L < 0 || S < 0 || H_kv < 1 || (H > 0 && H % H_kv != 0))
+    return FA_ERR_INVALID_ARG;
+  if (S > FA_MAX_LEN) return FA_ERR_INVALID_ARG;
+  if (mask < FA_DECODE_FULL || mask > FA_DECODE_SLIDING_WINDOW) return FA_ERR_INVALID_ARG;
+  if (mask == FA_DECODE_SLIDING_WINDOW && window < 1) return FA_ERR_INVALID_ARG;
+  if (score_kind != FA_SCORE_NONE && score_kind != FA_SCORE_TANH_SOFTCAP) return FA_ERR_INVALID_ARG;
+  if (score_kind == FA_SCORE_TANH_SOFTCAP && !(softcap > 0.f && std::isfinite(softcap)))
+    return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  const int G = H > 0 ? H / H_kv : 1;
+  if (static_cast<int64_t>(G) * L > kMaxRows) return FA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H * L == 0) return FA_OK;
+  if (static_cast<int64_t>(B) * H * L > INT32_MAX || static_cast<int64_t>(B) * H_kv > 65535)
+    return FA_ERR_UNSUPPORTED;
+  if (workspace == nullptr || workspace_bytes < fa_decode_workspace_bytes(B, H, H_kv, L, S, D))
+    return FA_ERR_INVALID_ARG;
+  if (q == nullptr || out == nullptr || (S > 0 && (k == nullptr || v == nullptr)))
+    return FA_ERR_INVALID_ARG;
+  auto misaligned = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
+  if (misaligned(q) || misaligned(out) || misaligned(workspace) ||
+      (S > 0 && (misaligned(k) || misaligned(v))))
+    return FA_ERR_INVALID_ARG;
+
+  DecParams prm{};
+  prm.q = static_cast<const uint16_t*>(q);
+  prm.out = out;
+  prm.lse = lse;
+  prm.err = static_cast<int32_t*>(workspace);
+  prm.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kDecWorkspaceHeader);
+  prm.H = H;
+  prm.Hkv = H_kv;
+  prm.G = G;
+  prm.L = L;
+  prm.S = S;
+  decode_plan(B, H_kv, S, &prm.nsplit, &prm.chunk);
+  prm.mask = mask;
+  prm.window = mask == FA_DECODE_SLIDING_WINDOW ? window : 0;
+  prm.softcap_on = score_kind == FA_SCORE_TANH_SOFTCAP ? 1 : 0;
+  prm.is_bf16 = dtype == FA_BF16 ? 1 : 0;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  prm.q_scale = prm.softcap_on ? sc : sc * kDecLog2e;
+  prm.cap_c = prm.softcap_on ? softcap : 1.f;
+  prm.cap_a = prm.softcap_on ? softcap * kDecLog2e : 0.f;
+  prm.timeout_ns = 2000000000ull;
+  const cudaStream_t s = as_stream(stream);
+  if (D == 64) return decode_launch<64>(k, v, dtype == FA_BF16, B, S, prm, s);
+  return decode_launch<128>(k, v, dtype == FA_BF16, B, S, prm, s);
+}

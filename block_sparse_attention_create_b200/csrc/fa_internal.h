@@ -1,6 +1,7 @@
 // Host-side helpers shared by the library's translation units (not part of the ABI).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "fa.h"
@@ -17,6 +18,12 @@ constexpr int kDevErrTimeout = 1;
 
 // Per-device state (kernel attributes, SM counts) is kept for this many devices.
 constexpr int kMaxDevices = 64;
+
+// 3-D TMA map over a contiguous (bh, rows, D) 16-bit tensor: box = 64 elements x
+// box_rows rows x 1, 128-byte swizzle; rows past `rows` read as zeros.  False if the
+// driver's encoder is unavailable or rejects the arguments.
+bool make_tile_map(CUtensorMap* map, const void* ptr, bool bf16, int D, int rows, int bh,
+                   int box_rows);
 
 }  // namespace fa
 

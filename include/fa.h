@@ -259,6 +259,41 @@ FA_API fa_status fa_flex_attention_fwd_gqa(const void* q, const void* k, const v
                                     int32_t score_kind, float softcap, float scale, void* out,
                                     float* lse, void* workspace, void* stream);
 
+/*
+ * Decode against a KV cache (NEXT-4; SDPA tutorial, section 4, pitfall 3): L new
+ * queries after S - L cached keys.  Query i sits at key position S - L + i, so the
+ * causal mask is aligned to the lower right (torch's causal_lower_right).
+ *   q         device (B, H, L, D);   k, v  device (B, H_kv, S, D);  16-byte aligned.
+ *   H_kv      >= 1 dividing H (grouped-query attention as in fa_flex_attention_fwd_gqa);
+ *             (H / H_kv) * L <= FA_DECODE_MAX_ROWS (the query rows sharing one K/V
+ *             head are processed together, reading K and V once).
+ *   mask      fa_decode_mask; window W >= 1 for FA_DECODE_SLIDING_WINDOW
+ *             (query i sees keys in (S - L + i - W, S - L + i]).
+ *   score_kind, softcap, scale, dtype, D as for fa_flex_attention_fwd.
+ *   out, lse  device (B, H, L, D) in dtype / (B, H, L) fp32 (lse may be NULL).
+ *   workspace device, at least fa_decode_workspace_bytes(B, H, H_kv, L, S, D) bytes,
+ *             16-byte aligned; its first word is the device error word (zero it once;
+ *             fa_get_last_device_error reads and clears it).  Calls that run
+ *             concurrently need distinct workspaces.
+ * Split-KV: the keys are cut into chunks processed by different CTAs, then merged.
+ * Two kernels on `stream`.  B*H*L == 0 is a no-op.  Returns FA_ERR_INVALID_ARG /
+ * FA_ERR_UNSUPPORTED (nothing launched) or FA_ERR_CUDA.
+ */
+typedef enum {
+  FA_DECODE_FULL = 0,            /* every cached key */
+  FA_DECODE_CAUSAL = 1,          /* kv_idx <= S - L + q_idx */
+  FA_DECODE_SLIDING_WINDOW = 2   /* and S - L + q_idx - kv_idx < window */
+} fa_decode_mask;
+#define FA_DECODE_MAX_ROWS 32
+FA_API size_t fa_decode_workspace_bytes(int32_t B, int32_t H, int32_t H_kv, int32_t L, int32_t S,
+                                 int32_t D);
+FA_API fa_status fa_flex_attention_decode(const void* q, const void* k, const void* v,
+                                   int32_t dtype, int32_t B, int32_t H, int32_t H_kv, int32_t L,
+                                   int32_t S, int32_t D, int32_t mask, int32_t window,
+                                   int32_t score_kind, float softcap, float scale, void* out,
+                                   float* lse, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
 /* Synchronises `stream`, then reads and clears the error word that the forward
  * kernel keeps in `workspace`.  Returns FA_ERR_TIMEOUT if a bounded device wait gave
  * up since the last query (the outputs of that call are then invalid), FA_ERR_CUDA

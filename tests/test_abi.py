@@ -138,6 +138,27 @@ def test_gqa_rejects_uneven_head_groups(fa):
                                             0.0, 0.0, p, null, p, null) == fa.FA_ERR_INVALID_ARG
 
 
+def test_decode_rejects_bad_arguments(fa):
+    p = ctypes.c_void_p(1 << 20)   # never dereferenced: rejected before any use
+    null = ctypes.c_void_p(0)
+    need = fa.fa_decode_workspace_bytes(1, 8, 2, 1, 1000, 64)
+    assert need > 256
+
+    def call(**kw):
+        a = dict(B=1, H=8, Hkv=2, L=1, S=1000, D=64, mask=1, window=0, ws=need)
+        a.update(kw)
+        return fa.fa_flex_attention_decode(p, p, p, 0, a["B"], a["H"], a["Hkv"], a["L"], a["S"],
+                                           a["D"], a["mask"], a["window"], 0, 0.0, 0.0, p, null, p,
+                                           a["ws"], null)
+    assert call(Hkv=3) == fa.FA_ERR_INVALID_ARG            # H not a multiple of Hkv
+    assert call(mask=7) == fa.FA_ERR_INVALID_ARG
+    assert call(mask=2, window=0) == fa.FA_ERR_INVALID_ARG
+    assert call(D=96) == fa.FA_ERR_UNSUPPORTED
+    assert call(H=8, Hkv=1, L=5) == fa.FA_ERR_UNSUPPORTED  # 40 rows share one K/V head
+    assert call(ws=need - 4) == fa.FA_ERR_INVALID_ARG
+    assert call(B=0) == fa.FA_OK                            # empty: nothing launched
+
+
 def _fwd(fa, bm, **kw):
     args = dict(q=1024, k=1024, v=1024, dtype=0, B=1, H=1, L=256, S=256, D=64, sk=0, cap=0.0,
                 scale=0.0, out=1024, lse=0, ws=1024)

@@ -30,12 +30,18 @@ MASK_CAUSAL = 0
 MASK_SLIDING_WINDOW_CAUSAL = 1
 MASK_DOCUMENT_CAUSAL = 2
 MASK_BITMAP = 3
+# decode against a KV cache (lower-right aligned): full, causal, sliding window
+MASK_DECODE_FULL = 4
+MASK_DECODE_CAUSAL = 5
+MASK_DECODE_SLIDING_WINDOW = 6
 
 SCORE_NONE = 0
 SCORE_TANH_SOFTCAP = 1
 
 MASK_NAMES = {MASK_CAUSAL: "causal", MASK_SLIDING_WINDOW_CAUSAL: "sliding_window_causal",
-              MASK_DOCUMENT_CAUSAL: "document_causal", MASK_BITMAP: "bitmap"}
+              MASK_DOCUMENT_CAUSAL: "document_causal", MASK_BITMAP: "bitmap",
+              MASK_DECODE_FULL: "decode_full", MASK_DECODE_CAUSAL: "decode_causal_lower_right",
+              MASK_DECODE_SLIDING_WINDOW: "decode_sliding_window_lower_right"}
 
 
 @dataclasses.dataclass(frozen=True)
@@ -73,7 +79,7 @@ class Workload:
         d = {"workload": self.name, "B": self.B, "H": self.H, "L": self.L, "S": self.S,
              "D": self.D, "dtype": self.dtype_name, "mask": MASK_NAMES[self.mask_kind],
              "block": 128, "seed": self.seed}
-        if self.mask_kind == MASK_SLIDING_WINDOW_CAUSAL:
+        if self.mask_kind in (MASK_SLIDING_WINDOW_CAUSAL, MASK_DECODE_SLIDING_WINDOW):
             d["window"] = self.window
         if self.mask_kind == MASK_DOCUMENT_CAUSAL:
             d["documents"] = "seeded 4..16" if self.doc_seeded else list(self.doc_boundaries or ())
@@ -117,7 +123,12 @@ BITMAP_8192 = _w("bitmap_L8192_B1_H8_D64_bf16", 1, 8, 8192, 64, torch.bfloat16, 
 GQA_CAUSAL_8192 = _w("gqa_causal_L8192_B1_H32_Hkv8_D64_bf16", 1, 32, 8192, 64, torch.bfloat16,
                      MASK_CAUSAL, seed=13, Hkv=8)
 
-EXTRA = (BITMAP_8192, GQA_CAUSAL_8192)
+# Decode: one new token per sequence against a 32768-token KV cache, 32 query heads
+# over 8 K/V heads, batch 8 (SDPA tutorial, section 4, pitfall 3: L = 1, S = cache).
+DECODE_32K = Workload(name="decode_L1_S32768_B8_H32_Hkv8_D128_bf16", B=8, H=32, L=1, S=32768,
+                      D=128, dtype=torch.bfloat16, mask_kind=MASK_DECODE_CAUSAL, seed=14, Hkv=8)
+
+EXTRA = (BITMAP_8192, GQA_CAUSAL_8192, DECODE_32K)
 BY_NAME = {w.name: w for w in ALL + EXTRA}
 
 
