@@ -31,7 +31,7 @@ namespace {
 constexpr int kTile = 64;            // keys per K/V tile
 constexpr int kDecThreads = 128;
 constexpr int kMaxRows = FA_DECODE_MAX_ROWS;
-constexpr int kTargetCtas = 2 * 148;  // two waves of B200's SMs
+constexpr int kTargetCtas = 3 * 148;  // about three CTAs on each of B200's SMs
 constexpr int kBoxBytes = kTile * 128;  // one TMA box: 64 keys x 64 elements
 constexpr int kDecWorkspaceHeader = 256;  // word 0: device error flags
 constexpr float kDecLog2e = 1.4426950408889634f;
@@ -50,13 +50,13 @@ struct DecParams {
   unsigned long long timeout_ns;
 };
 
-template <int D>
+template <int D, int RM>
 struct __align__(1024) DecSmem {
   uint8_t k[2][D / 64][kBoxBytes];
   uint8_t v[2][D / 64][kBoxBytes];
-  float qs[kMaxRows][D];
-  float sc[kMaxRows][kTile];
-  float m[kMaxRows], l[kMaxRows], alpha[kMaxRows];
+  float qs[RM][D];
+  float sc[RM][kTile];
+  float m[RM], l[RM], alpha[RM];
   uint64_t full[2];
   volatile int abort_flag;
 };
@@ -90,8 +90,8 @@ __device__ __forceinline__ uint4 tile_chunk(const uint8_t (&tile)[NB][kBoxBytes]
   return *reinterpret_cast<const uint4*>(&tile[c >> 3][j * 128 + (((c & 7) ^ (j & 7)) << 4)]);
 }
 
-template <int D>
-__device__ __forceinline__ bool dec_wait(DecSmem<D>& sm, uint64_t* bar, uint32_t parity,
+template <class Sm>
+__device__ __forceinline__ bool dec_wait(Sm& sm, uint64_t* bar, uint32_t parity,
                                          const DecParams& p) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -107,16 +107,22 @@ __device__ __forceinline__ bool dec_wait(DecSmem<D>& sm, uint64_t* bar, uint32_t
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(kDecThreads)
+// RM: bound on the rows R, 4, 8 or 32.  With RM <= 8 every PV thread keeps all rows
+// for one 16-byte column chunk over a subset of the tile's keys (key group), and
+// the key groups are summed once per CTA at the end; with RM = 32 a thread keeps
+// a few rows over all keys.
+template <int D, int RM>
+__global__ void __launch_bounds__(kDecThreads, 3)
 decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                     const __grid_constant__ DecParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
-  DecSmem<D>& sm = *reinterpret_cast<DecSmem<D>*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
+  using Sm = DecSmem<D, RM>;
+  Sm& sm = *reinterpret_cast<Sm*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
   constexpr int kChunks = D / 8;                  // 16-byte chunks of a row
-  constexpr int kGroups = kDecThreads / kChunks;  // row groups of the PV step
-  constexpr int kRowsPer = kMaxRows / kGroups;
+  constexpr int kGroups = kDecThreads / kChunks;  // PV thread groups (rows or keys)
+  constexpr bool kKeyGroups = RM <= 8;
+  constexpr int kRowsPer = kKeyGroups ? RM : RM / kGroups;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int split = blockIdx.x, bkv = blockIdx.y;
   const int b = bkv / p.Hkv, kvh = bkv - b * p.Hkv;
@@ -180,34 +186,39 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
     // scores: thread = (key j, row parity); rows r = rg, rg + 2, ...
     {
       const int j = tid & (kTile - 1), rg = tid >> 6;
-      float acc[kMaxRows / 2];
+      // four independent partial sums per row keep the FMA chains short
+      float acc[RM / 2][4];
 #pragma unroll
-      for (int k = 0; k < kMaxRows / 2; ++k) acc[k] = 0.f;
+      for (int k = 0; k < RM / 2; ++k)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[k][u] = 0.f;
 #pragma unroll
       for (int c = 0; c < kChunks; ++c) {
         float kf[8];
         unpack8(tile_chunk(sm.k[buf], j, c), bf16, kf);
 #pragma unroll
-        for (int k = 0; k < kMaxRows / 2; ++k) {
+        for (int k = 0; k < RM / 2; ++k) {
           const int r = rg + 2 * k;
           if (r < R) {
             const float4 qa = *reinterpret_cast<const float4*>(&sm.qs[r][c * 8]);
             const float4 qb = *reinterpret_cast<const float4*>(&sm.qs[r][c * 8 + 4]);
-            acc[k] += qa.x * kf[0] + qa.y * kf[1] + qa.z * kf[2] + qa.w * kf[3] +
-                      qb.x * kf[4] + qb.y * kf[5] + qb.z * kf[6] + qb.w * kf[7];
+            acc[k][0] = fmaf(qa.x, kf[0], fmaf(qb.x, kf[4], acc[k][0]));
+            acc[k][1] = fmaf(qa.y, kf[1], fmaf(qb.y, kf[5], acc[k][1]));
+            acc[k][2] = fmaf(qa.z, kf[2], fmaf(qb.z, kf[6], acc[k][2]));
+            acc[k][3] = fmaf(qa.w, kf[3], fmaf(qb.w, kf[7], acc[k][3]));
           }
         }
       }
       const int kv = k0 + j;
 #pragma unroll
-      for (int k = 0; k < kMaxRows / 2; ++k) {
+      for (int k = 0; k < RM / 2; ++k) {
         const int r = rg + 2 * k;
         if (r < R) {
           const int pos = p.S - p.L + (r % p.L);  // the query's key position
           bool keep = kv < c1;
           if (p.mask != FA_DECODE_FULL) keep = keep && kv <= pos;
           if (p.mask == FA_DECODE_SLIDING_WINDOW) keep = keep && pos - kv < p.window;
-          float s = acc[k];
+          float s = (acc[k][0] + acc[k][1]) + (acc[k][2] + acc[k][3]);
           if (p.softcap_on) s = p.cap_a * tanhf(s / p.cap_c);
           sm.sc[r][j] = keep ? s : -INFINITY;
         }
@@ -240,8 +251,26 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
     }
     __syncthreads();
 
-    // O += P V: thread = (16-byte chunk oc of a V row, row group og)
-    {
+    // O += P V: thread = (16-byte chunk oc of a V row, group og: rows or keys)
+    if constexpr (kKeyGroups) {
+#pragma unroll
+      for (int r = 0; r < RM; ++r) {
+        const float a = r < R ? sm.alpha[r] : 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[r][e] *= a;
+      }
+      const int nk = min(kTile, c1 - k0);
+      for (int j = og; j < nk; j += kGroups) {
+        float vf[8];
+        unpack8(tile_chunk(sm.v[buf], j, oc), bf16, vf);
+#pragma unroll
+        for (int r = 0; r < RM; ++r) {
+          const float pj = r < R ? sm.sc[r][j] : 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[r][e] = fmaf(pj, vf[e], o[r][e]);
+        }
+      }
+    } else {
       float al[kRowsPer];
 #pragma unroll
       for (int k = 0; k < kRowsPer; ++k) {
@@ -281,19 +310,46 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
   }
 
   // this chunk's partial result per row
+  if constexpr (kKeyGroups) {
+    // sum the key groups through shared memory: the K and V tile buffers (adjacent,
+    // free now) hold [kGroups][RM][D] floats
+    float* red = reinterpret_cast<float*>(&sm.k[0][0][0]);
+    static_assert(sizeof(Sm::k) + sizeof(Sm::v) >= sizeof(float) * kGroups * RM * D,
+                  "reduction space");
 #pragma unroll
-  for (int k = 0; k < kRowsPer; ++k) {
-    const int r = og + kGroups * k;
-    if (r < R) {
+    for (int r = 0; r < RM; ++r)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red[(og * RM + r) * D + oc * 8 + e] = o[r][e];
+    __syncthreads();
+    for (int x = tid; x < R * D; x += kDecThreads) {
+      const int r = x / D, d = x - (x / D) * D;
+      float sum = 0.f;
+#pragma unroll
+      for (int gk = 0; gk < kGroups; ++gk) sum += red[(gk * RM + r) * D + d];
       const int g = r / p.L, i = r - g * p.L;
       const size_t row = static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i;
       float* rec = p.part + (row * p.nsplit + split) * (D + 2);
-      if (oc == 0) {
+      if (d == 0) {
         rec[0] = sm.m[r];
         rec[1] = sm.l[r];
       }
+      rec[2 + d] = sum;
+    }
+  } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) rec[2 + oc * 8 + e] = o[k][e];
+    for (int k = 0; k < kRowsPer; ++k) {
+      const int r = og + kGroups * k;
+      if (r < R) {
+        const int g = r / p.L, i = r - g * p.L;
+        const size_t row = static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i;
+        float* rec = p.part + (row * p.nsplit + split) * (D + 2);
+        if (oc == 0) {
+          rec[0] = sm.m[r];
+          rec[1] = sm.l[r];
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) rec[2 + oc * 8 + e] = o[k][e];
+      }
     }
   }
 }
@@ -336,7 +392,7 @@ void decode_plan(int B, int Hkv, int S, int* nsplit, int* chunk) {
   *nsplit = S > 0 ? (S + *chunk - 1) / *chunk : 1;
 }
 
-template <int D>
+template <int D, int RM>
 fa_status decode_launch(const void* k, const void* v, bool bf16, int B, int S, const DecParams& prm,
                         cudaStream_t stream) {
   CUtensorMap tk, tv;
@@ -346,7 +402,7 @@ fa_status decode_launch(const void* k, const void* v, bool bf16, int B, int S, c
   const int rows = S > 0 ? S : 1, bh = S > 0 ? B * prm.Hkv : 1;
   if (!make_tile_map(&tk, kp, bf16, D, rows, bh, kTile)) return FA_ERR_CUDA;
   if (!make_tile_map(&tv, vp, bf16, D, rows, bh, kTile)) return FA_ERR_CUDA;
-  const size_t smem = sizeof(DecSmem<D>) + 1024;
+  const size_t smem = sizeof(DecSmem<D, RM>) + 1024;
   int dev = 0;
   FA_CUDA_CHECK(cudaGetDevice(&dev));
   {
@@ -355,14 +411,14 @@ fa_status decode_launch(const void* k, const void* v, bool bf16, int B, int S, c
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
     if (!done[dev]) {
-      FA_CUDA_CHECK(cudaFuncSetAttribute(decode_split_kernel<D>,
+      FA_CUDA_CHECK(cudaFuncSetAttribute(decode_split_kernel<D, RM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem)));
       done[dev] = true;
     }
   }
   const dim3 grid(prm.nsplit, B * prm.Hkv);
-  decode_split_kernel<D><<<grid, kDecThreads, smem, stream>>>(tk, tv, prm);
+  decode_split_kernel<D, RM><<<grid, kDecThreads, smem, stream>>>(tk, tv, prm);
   FA_CUDA_CHECK(cudaGetLastError());
   decode_combine_kernel<D><<<B * prm.H * prm.L, D, 0, stream>>>(prm);
   FA_CUDA_CHECK(cudaGetLastError());
@@ -434,6 +490,14 @@ extern "C" fa_status fa_flex_attention_decode(const void* q, const void* k, cons
   prm.cap_a = prm.softcap_on ? softcap * kDecLog2e : 0.f;
   prm.timeout_ns = 2000000000ull;
   const cudaStream_t s = as_stream(stream);
-  if (D == 64) return decode_launch<64>(k, v, dtype == FA_BF16, B, S, prm, s);
-  return decode_launch<128>(k, v, dtype == FA_BF16, B, S, prm, s);
+  const bool b16 = dtype == FA_BF16;
+  const int rows = G * L;
+  if (D == 64) {
+    if (rows <= 4) return decode_launch<64, 4>(k, v, b16, B, S, prm, s);
+    if (rows <= 8) return decode_launch<64, 8>(k, v, b16, B, S, prm, s);
+    return decode_launch<64, 32>(k, v, b16, B, S, prm, s);
+  }
+  if (rows <= 4) return decode_launch<128, 4>(k, v, b16, B, S, prm, s);
+  if (rows <= 8) return decode_launch<128, 8>(k, v, b16, B, S, prm, s);
+  return decode_launch<128, 32>(k, v, b16, B, S, prm, s);
 }
