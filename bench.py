@@ -42,23 +42,30 @@ PAGE_FWD_MS = {"swa256_L32768_B1_H8_D64_bf16": 75.27, "causal_L8192_B1_H8_D64_bf
                "swa64_L8192_B1_H8_D64_bf16": 11.75, "swa256_L8192_B1_H8_D64_bf16": 19.14,
                "swa1024_L8192_B1_H8_D64_bf16": 56.24, "swa4096_L8192_B1_H8_D64_bf16": 169.24}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) of one forward launch from an ncu capture, per workload,
-# with the hash of the kernel sources it was taken on: reported as roofline.traffic
-# only while the sources still hash to that value (null once the kernel changed).
-KERNEL_SOURCES = ("block_sparse_attention_create_b200/csrc/fwd_sm100.cu",
+# DRAM bytes (read + write) of one launch of the dominant kernel from an ncu capture,
+# per workload, with the hash of the kernel sources it was taken on: reported as
+# roofline.traffic only while the sources still hash to that value (null once the
+# kernel changed).
+FWD_SOURCES = ("block_sparse_attention_create_b200/csrc/fwd_sm100.cu",
+               "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
+DECODE_SOURCES = ("block_sparse_attention_create_b200/csrc/decode.cu",
                   "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
 NCU_TRAFFIC = {
     "swa256_L32768_B1_H8_D64_bf16": {
-        "bytes": 101083136 + 6039040,
+        "bytes": 101083136 + 6039040, "sources": FWD_SOURCES,
         "sources_sha256": "98b7510f590ce52b385c193912c44c1fbe7920793a0b3ce3f054e467890ec4c3",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_full.md"},
+    "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
+        "bytes": 1073855232 + 3912192, "sources": DECODE_SOURCES,
+        "sources_sha256": "4561db7fb9acecdf26fc79a0105816905b05dfa63132417a3fff9544728ad9c4",
+        "summary": "profiles/decode_split_kernel_L1_S32768_B8_H32_Hkv8_D128_full.md"},
 }
 
 
-def kernel_sources_hash():
+def kernel_sources_hash(sources):
     import hashlib
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -66,7 +73,7 @@ def kernel_sources_hash():
 
 def ncu_traffic(w: W.Workload):
     rec = NCU_TRAFFIC.get(w.name)
-    if rec is None or rec["sources_sha256"] != kernel_sources_hash():
+    if rec is None or rec["sources_sha256"] != kernel_sources_hash(rec["sources"]):
         return None
     return rec["bytes"]
 
@@ -452,7 +459,8 @@ def main():
         roof = {"bound": "tensor", "achieved": fwd_tflops, "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": tensor_frac, "traffic": ncu_traffic(w)}
     roof["peak_source"] = f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"
-    roof["kernel"] = "fwd_kernel (fa_flex_attention_fwd)"
+    roof["kernel"] = ("decode_split_kernel (fa_flex_attention_decode)" if is_decode(w)
+                      else "fwd_kernel (fa_flex_attention_fwd)")
     page_ms = PAGE_FWD_MS.get(w.name)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": r["total_ms"] / args.steps,
