@@ -39,7 +39,7 @@ EXPORTED = ("fa_block_mask_dims", "fa_create_block_mask", "fa_fwd_workspace_byte
             "fa_flex_attention_fwd", "fa_get_last_device_error", "fa_status_string",
             "fa_num_sms", "fa_flex_attention_fwd_noalloc", "fa_create_block_mask_bitmap",
             "fa_block_mask_transpose", "fa_flex_attention_fwd_gqa", "fa_decode_workspace_bytes",
-            "fa_flex_attention_decode")
+            "fa_flex_attention_decode", "fa_debug_set_mma_stall")
 
 
 class fa_block_mask(ctypes.Structure):
@@ -99,6 +99,8 @@ def _load():
     lib.fa_flex_attention_decode.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, i32,
                                              i32, i32, f32, f32, vp, vp, vp, ctypes.c_size_t, vp]
     lib.fa_flex_attention_decode.restype = i32
+    lib.fa_debug_set_mma_stall.argtypes = [i32, ctypes.c_uint64]
+    lib.fa_debug_set_mma_stall.restype = None
     return lib
 
 
@@ -118,6 +120,7 @@ fa_block_mask_transpose = _lib.fa_block_mask_transpose
 fa_flex_attention_fwd_gqa = _lib.fa_flex_attention_fwd_gqa
 fa_decode_workspace_bytes = _lib.fa_decode_workspace_bytes
 fa_flex_attention_decode = _lib.fa_flex_attention_decode
+fa_debug_set_mma_stall = _lib.fa_debug_set_mma_stall
 
 
 class FAError(RuntimeError):

@@ -36,6 +36,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -134,6 +135,7 @@ struct Params {
   float cap_k;       // 2 * scale * log2(e) / c : exp2(s * cap_k) = e^(2 s scale / c)
   float cap_a;       // c * log2(e)
   unsigned long long timeout_ns;
+  int stall_mma;  // testing hook: the MMA warp issues nothing (see fa_debug_set_mma_stall)
 };
 
 // ---------------------------------------------------------------- scheduling
@@ -567,8 +569,11 @@ __device__ void mma_role(Smem<D>& sm, const Params& p, uint32_t tmem) {
   uint64_t last_progress = 0;  // 0: progress since the last idle check
   int idle = 0;
   while (p0.active || p1.active) {
-    bool progress = mma_slot<D, 0>(sm, p, s0, p0, ms);
-    progress |= mma_slot<D, 1>(sm, p, s1, p1, ms);
+    bool progress = false;
+    if (!p.stall_mma) {
+      progress = mma_slot<D, 0>(sm, p, s0, p0, ms);
+      progress |= mma_slot<D, 1>(sm, p, s1, p1, ms);
+    }
     if (progress) {
       idle = 0;
       last_progress = 0;
@@ -1145,6 +1150,10 @@ extern "C" size_t fa_fwd_workspace_bytes(void) { return 256; }
 namespace fa {
 namespace {
 
+// Testing hook for the bounded-wait failure path (fa_debug_set_mma_stall).
+std::atomic<int> g_stall_mma{0};
+std::atomic<unsigned long long> g_stall_wait_limit_ns{2000000000ull};
+
 fa_status fwd_impl(const void* q, const void* k, const void* v, int32_t dtype, int32_t B, int32_t H,
                    int32_t Hkv, int32_t L, int32_t S, int32_t D, const fa_block_mask* bm,
                    int32_t score_kind, float softcap, float scale, void* out, float* lse,
@@ -1200,6 +1209,10 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, int32_t dtype, i
   prm.cap_a = prm.softcap_on ? softcap * kLog2e : 0.f;
   prm.split_p = 1;
   prm.timeout_ns = 2000000000ull;
+  if (g_stall_mma.load()) {
+    prm.stall_mma = 1;
+    prm.timeout_ns = g_stall_wait_limit_ns.load();
+  }
   const cudaStream_t s = as_stream(stream);
   const bool b16 = dtype == FA_BF16;
   switch (mask_family(bm->kind) * 2 + (D == 64 ? 0 : 1)) {
@@ -1233,4 +1246,9 @@ extern "C" fa_status fa_flex_attention_fwd_gqa(const void* q, const void* k, con
                                                void* workspace, void* stream) {
   return fa::fwd_impl(q, k, v, dtype, B, H, H_kv, L, S, D, bm, score_kind, softcap, scale, out,
                       lse, workspace, stream);
+}
+
+extern "C" void fa_debug_set_mma_stall(int32_t on, uint64_t wait_limit_ns) {
+  fa::g_stall_wait_limit_ns.store(wait_limit_ns > 0 ? wait_limit_ns : 2000000000ull);
+  fa::g_stall_mma.store(on ? 1 : 0);
 }

@@ -294,6 +294,16 @@ FA_API fa_status fa_flex_attention_decode(const void* q, const void* k, const vo
                                    float* lse, void* workspace, size_t workspace_bytes,
                                    void* stream);
 
+/*
+ * Testing hook for failure detection (no counterpart on the pages).  While `on`,
+ * the forward kernel's MMA warp issues nothing, so the kernel's bounded waits run
+ * out after `wait_limit_ns` (0: the default 2 s), the kernel stops every role,
+ * drains its copies, frees TMEM and returns, and fa_get_last_device_error then
+ * reports FA_ERR_TIMEOUT (the outputs of that call are invalid).  Nothing faults,
+ * traps or hangs.  Process-wide; off by default.
+ */
+FA_API void fa_debug_set_mma_stall(int32_t on, uint64_t wait_limit_ns);
+
 /* Synchronises `stream`, then reads and clears the error word that the forward
  * kernel keeps in `workspace`.  Returns FA_ERR_TIMEOUT if a bounded device wait gave
  * up since the last query (the outputs of that call are then invalid), FA_ERR_CUDA

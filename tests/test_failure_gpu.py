@@ -1,0 +1,42 @@
+"""Failure detection on the GPU without a fault: with the testing hook that makes
+the forward kernel's MMA warp issue nothing, every bounded wait of the kernel runs
+out, the kernel stops all roles and returns, the host reads FA_ERR_TIMEOUT from the
+workspace error word, and the context stays usable for the next, correct call."""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import masks as OM
+from parity import compare, oracle_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_waits_report_timeout_and_context_survives():
+    import block_sparse_attention_create_b200 as fa
+    q, k, v = W.random_qkv(1, 2, 1000, 1000, 64, torch.bfloat16, seed=61)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    bm = fa.create_block_mask(OM.SLIDING_WINDOW_CAUSAL, 1000, 1000, window=300, device="cuda")
+    torch.cuda.synchronize()
+    assert fa.last_device_error() == fa.FA_OK          # start from a clear error word
+    fa.fa_debug_set_mma_stall(1, 50_000_000)           # 50 ms wait limit
+    try:
+        t0 = time.perf_counter()
+        fa.flex_attention(qd, kd, vd, bm)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        fa.fa_debug_set_mma_stall(0, 0)
+    assert fa.last_device_error() == fa.FA_ERR_TIMEOUT
+    assert elapsed < 10.0
+    assert fa.last_device_error() == fa.FA_OK          # reading cleared it
+    out, lse = fa.flex_attention(qd, kd, vd, bm, return_lse=True)
+    torch.cuda.synchronize()
+    assert fa.last_device_error() == fa.FA_OK
+    rows = np.arange(0, 1000, 7)
+    for h in range(2):
+        o_ref, l_ref = oracle_rows(q, k, v, 0, h, rows, OM.SLIDING_WINDOW_CAUSAL, 300)
+        compare(out[0, h].cpu()[rows], lse[0, h].cpu()[rows], o_ref, l_ref, f"h{h}")
