@@ -52,8 +52,8 @@ DECODE_SOURCES = ("block_sparse_attention_create_b200/csrc/decode.cu",
                   "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
 NCU_TRAFFIC = {
     "swa256_L32768_B1_H8_D64_bf16": {
-        "bytes": 101083136 + 6039040, "sources": FWD_SOURCES,
-        "sources_sha256": "98b7510f590ce52b385c193912c44c1fbe7920793a0b3ce3f054e467890ec4c3",
+        "bytes": 101092608 + 5255168, "sources": FWD_SOURCES,
+        "sources_sha256": "e21f669bf3e4a1be55d6b208ca89057859e15ac3f3ee9a8b6196896b1ed67f1c",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_full.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
         "bytes": 1073855232 + 3912192, "sources": DECODE_SOURCES,
