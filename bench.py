@@ -412,11 +412,16 @@ def main():
             return
         rows_per_step = 64
         g = np.random.default_rng(0)
+
+        def sample():  # decode: the new queries of the first few heads
+            if is_decode(w):
+                return np.arange(min(w.H, 8))
+            return np.sort(g.integers(0, w.L, rows_per_step))
         for _ in range(args.warmup):
-            oracle_sample(w, np.sort(g.integers(0, w.L, rows_per_step)), fig)
+            oracle_sample(w, sample(), fig)
         tot_s, tot_f = 0.0, 0.0
         for _ in range(args.steps):
-            dt, fl = oracle_sample(w, np.sort(g.integers(0, w.L, rows_per_step)), fig)
+            dt, fl = oracle_sample(w, sample(), fig)
             tot_s += dt
             tot_f += fl
         value = tot_f / tot_s / 1e12
@@ -428,8 +433,11 @@ def main():
                 "config": {**w.describe(), "parallelism": "none (host cores)"},
                 "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(),
                                  "kind": "oracle",
-                                 "sample": f"{rows_per_step} random query rows of head (0,0) per "
-                                           "step; ms_per_step extrapolates to the whole workload"},
+                                 "sample": (f"all new queries of {min(w.H, 8)} heads of batch 0 per step"
+                                            if is_decode(w) else
+                                            f"{rows_per_step} random query rows of head (0,0) per "
+                                            "step") + "; ms_per_step extrapolates to the whole "
+                                                      "workload"},
                 "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
