@@ -56,8 +56,8 @@ NCU_TRAFFIC = {
         "sources_sha256": "e21f669bf3e4a1be55d6b208ca89057859e15ac3f3ee9a8b6196896b1ed67f1c",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_full.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
-        "bytes": 1073855232 + 3912192, "sources": DECODE_SOURCES,
-        "sources_sha256": "4561db7fb9acecdf26fc79a0105816905b05dfa63132417a3fff9544728ad9c4",
+        "bytes": 1073943296 + 7651328, "sources": DECODE_SOURCES,
+        "sources_sha256": "7d84849a563dc019493219a78d36bc25086dc5688cd4c99eb537030c4bcbf4f0",
         "summary": "profiles/decode_split_kernel_L1_S32768_B8_H32_Hkv8_D128_full.md"},
 }
 

@@ -29,9 +29,14 @@ namespace fa {
 namespace {
 
 constexpr int kTile = 64;            // keys per K/V tile
-constexpr int kDecThreads = 128;
 constexpr int kMaxRows = FA_DECODE_MAX_ROWS;
-constexpr int kTargetCtas = 3 * 148;  // about three CTAs on each of B200's SMs
+// Threads per CTA and CTAs per SM by head dim: D = 128 runs 8 warps, two CTAs per
+// SM; D = 64 runs 4 warps, three per SM.  The grid is sized for that many CTAs.
+template <int D>
+struct DecCfg {
+  static constexpr int kThreads = D == 128 ? 256 : 128;
+  static constexpr int kCtasPerSm = D == 128 ? 2 : 3;
+};
 constexpr int kBoxBytes = kTile * 128;  // one TMA box: 64 keys x 64 elements
 constexpr int kDecWorkspaceHeader = 256;  // word 0: device error flags
 constexpr float kDecLog2e = 1.4426950408889634f;
@@ -112,15 +117,18 @@ __device__ __forceinline__ bool dec_wait(Sm& sm, uint64_t* bar, uint32_t parity,
 // the key groups are summed once per CTA at the end; with RM = 32 a thread keeps
 // a few rows over all keys.
 template <int D, int RM>
-__global__ void __launch_bounds__(kDecThreads, 3)
+__global__ void __launch_bounds__(DecCfg<D>::kThreads, DecCfg<D>::kCtasPerSm)
 decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                     const __grid_constant__ DecParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
   using Sm = DecSmem<D, RM>;
   Sm& sm = *reinterpret_cast<Sm*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
+  constexpr int kThr = DecCfg<D>::kThreads;
+  constexpr int kWarps = kThr / 32;
+  constexpr int kRowGroups = kThr / kTile;        // score threads per key
   constexpr int kChunks = D / 8;                  // 16-byte chunks of a row
-  constexpr int kGroups = kDecThreads / kChunks;  // PV thread groups (rows or keys)
+  constexpr int kGroups = kThr / kChunks;         // PV thread groups (rows or keys)
   constexpr bool kKeyGroups = RM <= 8;
   constexpr int kRowsPer = kKeyGroups ? RM : RM / kGroups;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -142,13 +150,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
     fence_barrier_init();
   }
   // query rows r = g * L + i (query head kvh * G + g, query i), scaled
-  for (int e = tid; e < R * D; e += kDecThreads) {
+  for (int e = tid; e < R * D; e += kThr) {
     const int r = e / D, d = e - (e / D) * D;
     const int g = r / p.L, i = r - g * p.L;
     const size_t qi = (static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i) * D + d;
     sm.qs[r][d] = load16(p.q + qi, bf16) * p.q_scale;
   }
-  for (int r = tid; r < R; r += kDecThreads) {
+  for (int r = tid; r < R; r += kThr) {
     sm.m[r] = -INFINITY;
     sm.l[r] = 0.f;
   }
@@ -183,42 +191,41 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
     const bool ok = dec_wait(sm, &sm.full[buf], (t >> 1) & 1, p);
     if (!__syncthreads_and(ok)) break;
 
-    // scores: thread = (key j, row parity); rows r = rg, rg + 2, ...
+    // scores: thread = (key j, row group rg); rows r = rg, rg + kRowGroups, ...
     {
-      const int j = tid & (kTile - 1), rg = tid >> 6;
-      // four independent partial sums per row keep the FMA chains short
-      float acc[RM / 2][4];
+      constexpr int kRowsS = RM / kRowGroups > 0 ? RM / kRowGroups : 1;
+      const int j = tid & (kTile - 1), rg = tid / kTile;
+      // two independent packed partial sums per row keep the FMA chains short
+      float2 acc[kRowsS][2];
 #pragma unroll
-      for (int k = 0; k < RM / 2; ++k)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) acc[k][u] = 0.f;
+      for (int k = 0; k < kRowsS; ++k) acc[k][0] = acc[k][1] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < kChunks; ++c) {
         float kf[8];
         unpack8(tile_chunk(sm.k[buf], j, c), bf16, kf);
 #pragma unroll
-        for (int k = 0; k < RM / 2; ++k) {
-          const int r = rg + 2 * k;
+        for (int k = 0; k < kRowsS; ++k) {
+          const int r = rg + kRowGroups * k;
           if (r < R) {
             const float4 qa = *reinterpret_cast<const float4*>(&sm.qs[r][c * 8]);
             const float4 qb = *reinterpret_cast<const float4*>(&sm.qs[r][c * 8 + 4]);
-            acc[k][0] = fmaf(qa.x, kf[0], fmaf(qb.x, kf[4], acc[k][0]));
-            acc[k][1] = fmaf(qa.y, kf[1], fmaf(qb.y, kf[5], acc[k][1]));
-            acc[k][2] = fmaf(qa.z, kf[2], fmaf(qb.z, kf[6], acc[k][2]));
-            acc[k][3] = fmaf(qa.w, kf[3], fmaf(qb.w, kf[7], acc[k][3]));
+            acc[k][0] = fma2(make_float2(qa.x, qa.y), make_float2(kf[0], kf[1]), acc[k][0]);
+            acc[k][1] = fma2(make_float2(qa.z, qa.w), make_float2(kf[2], kf[3]), acc[k][1]);
+            acc[k][0] = fma2(make_float2(qb.x, qb.y), make_float2(kf[4], kf[5]), acc[k][0]);
+            acc[k][1] = fma2(make_float2(qb.z, qb.w), make_float2(kf[6], kf[7]), acc[k][1]);
           }
         }
       }
       const int kv = k0 + j;
 #pragma unroll
-      for (int k = 0; k < RM / 2; ++k) {
-        const int r = rg + 2 * k;
+      for (int k = 0; k < kRowsS; ++k) {
+        const int r = rg + kRowGroups * k;
         if (r < R) {
           const int pos = p.S - p.L + (r % p.L);  // the query's key position
           bool keep = kv < c1;
           if (p.mask != FA_DECODE_FULL) keep = keep && kv <= pos;
           if (p.mask == FA_DECODE_SLIDING_WINDOW) keep = keep && pos - kv < p.window;
-          float s = (acc[k][0] + acc[k][1]) + (acc[k][2] + acc[k][3]);
+          float s = (acc[k][0].x + acc[k][0].y) + (acc[k][1].x + acc[k][1].y);
           if (p.softcap_on) s = p.cap_a * tanhf(s / p.cap_c);
           sm.sc[r][j] = keep ? s : -INFINITY;
         }
@@ -227,7 +234,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
     __syncthreads();
 
     // online softmax: warp w takes rows w, w + 4, ...; lane holds keys lane, lane + 32
-    for (int r = warp; r < R; r += 4) {
+    for (int r = warp; r < R; r += kWarps) {
       const float s0 = sm.sc[r][lane], s1 = sm.sc[r][lane + 32];
       float mx = fmaxf(s0, s1);
 #pragma unroll
@@ -266,8 +273,13 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
 #pragma unroll
         for (int r = 0; r < RM; ++r) {
           const float pj = r < R ? sm.sc[r][j] : 0.f;
+          const float2 p2 = make_float2(pj, pj);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) o[r][e] = fmaf(pj, vf[e], o[r][e]);
+          for (int e = 0; e < 8; e += 2) {
+            const float2 acc2 = fma2(p2, make_float2(vf[e], vf[e + 1]), make_float2(o[r][e], o[r][e + 1]));
+            o[r][e] = acc2.x;
+            o[r][e + 1] = acc2.y;
+          }
         }
       }
     } else {
@@ -321,7 +333,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
 #pragma unroll
       for (int e = 0; e < 8; ++e) red[(og * RM + r) * D + oc * 8 + e] = o[r][e];
     __syncthreads();
-    for (int x = tid; x < R * D; x += kDecThreads) {
+    for (int x = tid; x < R * D; x += kThr) {
       const int r = x / D, d = x - (x / D) * D;
       float sum = 0.f;
 #pragma unroll
@@ -381,11 +393,13 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
   if (d == 0 && p.lse) p.lse[row] = l > 0.f ? (mx + log2f(l)) * kDecLn2 : -INFINITY;
 }
 
-// Chunking of the keys: about kTargetCtas CTAs over (B * Hkv) groups, whole tiles.
-void decode_plan(int B, int Hkv, int S, int* nsplit, int* chunk) {
+// Chunking of the keys: about DecCfg::kCtasPerSm CTAs per SM over the (B * Hkv)
+// groups, whole tiles.
+void decode_plan(int B, int Hkv, int S, int D, int* nsplit, int* chunk) {
   const int groups = B * Hkv > 0 ? B * Hkv : 1;
   const int tiles = S > 0 ? (S + kTile - 1) / kTile : 1;
-  int n = (kTargetCtas + groups - 1) / groups;
+  const int target = 148 * (D == 128 ? DecCfg<128>::kCtasPerSm : DecCfg<64>::kCtasPerSm);
+  int n = (target + groups - 1) / groups;
   n = n < tiles ? n : tiles;
   const int tiles_per = (tiles + n - 1) / n;
   *chunk = tiles_per * kTile;
@@ -418,7 +432,7 @@ fa_status decode_launch(const void* k, const void* v, bool bf16, int B, int S, c
     }
   }
   const dim3 grid(prm.nsplit, B * prm.Hkv);
-  decode_split_kernel<D, RM><<<grid, kDecThreads, smem, stream>>>(tk, tv, prm);
+  decode_split_kernel<D, RM><<<grid, DecCfg<D>::kThreads, smem, stream>>>(tk, tv, prm);
   FA_CUDA_CHECK(cudaGetLastError());
   decode_combine_kernel<D><<<B * prm.H * prm.L, D, 0, stream>>>(prm);
   FA_CUDA_CHECK(cudaGetLastError());
@@ -432,7 +446,7 @@ extern "C" size_t fa_decode_workspace_bytes(int32_t B, int32_t H, int32_t H_kv, 
                                             int32_t S, int32_t D) {
   if (B < 0 || H < 0 || H_kv < 1 || L < 0 || S < 0 || D < 0) return 0;
   int nsplit = 0, chunk = 0;
-  fa::decode_plan(B, H_kv, S, &nsplit, &chunk);
+  fa::decode_plan(B, H_kv, S, D, &nsplit, &chunk);
   return fa::kDecWorkspaceHeader + static_cast<size_t>(B) * H * L * nsplit * (D + 2) * sizeof(float);
 }
 
@@ -479,7 +493,7 @@ extern "C" fa_status fa_flex_attention_decode(const void* q, const void* k, cons
   prm.G = G;
   prm.L = L;
   prm.S = S;
-  decode_plan(B, H_kv, S, &prm.nsplit, &prm.chunk);
+  decode_plan(B, H_kv, S, D, &prm.nsplit, &prm.chunk);
   prm.mask = mask;
   prm.window = mask == FA_DECODE_SLIDING_WINDOW ? window : 0;
   prm.softcap_on = score_kind == FA_SCORE_TANH_SOFTCAP ? 1 : 0;
