@@ -52,8 +52,8 @@ DECODE_SOURCES = ("block_sparse_attention_create_b200/csrc/decode.cu",
                   "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
 NCU_TRAFFIC = {
     "swa256_L32768_B1_H8_D64_bf16": {
-        "bytes": 101092608 + 5255168, "sources": FWD_SOURCES,
-        "sources_sha256": "e21f669bf3e4a1be55d6b208ca89057859e15ac3f3ee9a8b6196896b1ed67f1c",
+        "bytes": 101135616 + 7600128, "sources": FWD_SOURCES,
+        "sources_sha256": "8101f3984bd4516552eae4457515a92c585ab66a302819add03a1499c6d960aa",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_full.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
         "bytes": 1073943296 + 7651328, "sources": DECODE_SOURCES,

@@ -39,7 +39,7 @@ EXPORTED = ("fa_block_mask_dims", "fa_create_block_mask", "fa_fwd_workspace_byte
             "fa_flex_attention_fwd", "fa_get_last_device_error", "fa_status_string",
             "fa_num_sms", "fa_flex_attention_fwd_noalloc", "fa_create_block_mask_bitmap",
             "fa_block_mask_transpose", "fa_flex_attention_fwd_gqa", "fa_decode_workspace_bytes",
-            "fa_flex_attention_decode", "fa_debug_set_mma_stall")
+            "fa_flex_attention_decode", "fa_debug_set_mma_stall", "fa_create_block_mask_bh")
 
 
 class fa_block_mask(ctypes.Structure):
@@ -59,6 +59,8 @@ class fa_block_mask(ctypes.Structure):
         ("window", ctypes.c_int32),
         ("doc_id", ctypes.c_void_p),
         ("bitmap", ctypes.c_void_p),
+        ("mask_batch", ctypes.c_int32),
+        ("mask_heads", ctypes.c_int32),
     ]
 
 
@@ -101,6 +103,9 @@ def _load():
     lib.fa_flex_attention_decode.restype = i32
     lib.fa_debug_set_mma_stall.argtypes = [i32, ctypes.c_uint64]
     lib.fa_debug_set_mma_stall.restype = None
+    lib.fa_create_block_mask_bh.argtypes = [i32, i32, vp, vp, i32, i32, i32, i32, i32,
+                                            ctypes.POINTER(fa_block_mask), vp]
+    lib.fa_create_block_mask_bh.restype = i32
     return lib
 
 
@@ -121,6 +126,7 @@ fa_flex_attention_fwd_gqa = _lib.fa_flex_attention_fwd_gqa
 fa_decode_workspace_bytes = _lib.fa_decode_workspace_bytes
 fa_flex_attention_decode = _lib.fa_flex_attention_decode
 fa_debug_set_mma_stall = _lib.fa_debug_set_mma_stall
+fa_create_block_mask_bh = _lib.fa_create_block_mask_bh
 
 
 class FAError(RuntimeError):
@@ -157,14 +163,17 @@ class BlockMask:
     at them; reuse one BlockMask across forwards, as the how-to recommends.
     """
 
-    def __init__(self, q_len: int, kv_len: int, device, block: int = FA_BLOCK):
+    def __init__(self, q_len: int, kv_len: int, device, block: int = FA_BLOCK,
+                 mask_batch: int = 1, mask_heads: int = 1):
         nq, nkv = block_mask_dims(q_len, kv_len, block)
+        inst = mask_batch * mask_heads   # per-(batch, head) instances, instance-major
         i32 = dict(dtype=torch.int32, device=device)
-        self.kv_num_blocks = torch.zeros(nq, **i32)
-        self.kv_indices = torch.zeros(nq, nkv, **i32)
-        self.full_kv_num_blocks = torch.zeros(nq, **i32)
-        self.full_kv_indices = torch.zeros(nq, nkv, **i32)
-        self.q_order = torch.zeros(2 * nq, **i32)   # schedule: (row, partial | full << 16)
+        self.kv_num_blocks = torch.zeros(inst * nq, **i32)
+        self.kv_indices = torch.zeros(inst * nq, nkv, **i32)
+        self.full_kv_num_blocks = torch.zeros(inst * nq, **i32)
+        self.full_kv_indices = torch.zeros(inst * nq, nkv, **i32)
+        self.q_order = torch.zeros(inst * 2 * nq, **i32)   # schedule: (row, partial | full << 16)
+        self.mask_batch, self.mask_heads = mask_batch, mask_heads
         self.doc_id: Optional[torch.Tensor] = None
         self.bitmap: Optional[torch.Tensor] = None
         self.struct = fa_block_mask()
@@ -185,10 +194,12 @@ class BlockMask:
         tensors q_num_blocks [nKV], q_indices [nKV, nQ], full_q_num_blocks,
         full_q_indices)."""
         nq, nkv = self.n_q_blocks, self.n_kv_blocks
+        inst = self.mask_batch * self.mask_heads
         i32 = dict(dtype=torch.int32, device=self.kv_num_blocks.device)
-        t = {"q_num_blocks": torch.zeros(nkv, **i32), "q_indices": torch.zeros(nkv, nq, **i32),
-             "full_q_num_blocks": torch.zeros(nkv, **i32),
-             "full_q_indices": torch.zeros(nkv, nq, **i32)}
+        t = {"q_num_blocks": torch.zeros(inst * nkv, **i32),
+             "q_indices": torch.zeros(inst * nkv, nq, **i32),
+             "full_q_num_blocks": torch.zeros(inst * nkv, **i32),
+             "full_q_indices": torch.zeros(inst * nkv, nq, **i32)}
         _check(fa_block_mask_transpose(ctypes.byref(self.struct), _ptr(t["q_num_blocks"]),
                                        _ptr(t["q_indices"]), _ptr(t["full_q_num_blocks"]),
                                        _ptr(t["full_q_indices"]), _stream_handle(stream)),
@@ -199,10 +210,34 @@ class BlockMask:
 def create_block_mask(kind: int, q_len: int, kv_len: int, window: int = 0,
                       doc_id: Optional[torch.Tensor] = None, device="cuda",
                       stream: Optional[torch.cuda.Stream] = None, out: Optional[BlockMask] = None,
-                      bitmap: Optional[torch.Tensor] = None) -> BlockMask:
+                      bitmap: Optional[torch.Tensor] = None, B: Optional[int] = None,
+                      H: Optional[int] = None) -> BlockMask:
     """fa_create_block_mask (or, for FA_MASK_BITMAP, fa_create_block_mask_bitmap with
     `bitmap`: an int32 CUDA tensor (q_len, 4 * nKV) holding the 32-bit words) on fresh
-    (or the given) device tables."""
+    (or the given) device tables.  With B and / or H (the how-to's create_block_mask
+    arguments), one mask per batch element / head: fa_create_block_mask_bh, with
+    doc_id (instances, max(q_len, kv_len)) or bitmap (instances, q_len, 4 * nKV)."""
+    mb, mh = (B or 1), (H or 1)
+    if mb > 1 or mh > 1:
+        bm = out if out is not None else BlockMask(q_len, kv_len, device, mask_batch=mb,
+                                                   mask_heads=mh)
+        n = max(q_len, kv_len)
+        if doc_id is not None:
+            if (doc_id.dtype != torch.int32 or not doc_id.is_cuda or not doc_id.is_contiguous()
+                    or doc_id.numel() < mb * mh * n):
+                raise ValueError("doc_id must be a contiguous int32 CUDA tensor (B*H, max(L, S))")
+            bm.doc_id = doc_id
+        if bitmap is not None:
+            if (bitmap.dtype != torch.int32 or not bitmap.is_cuda or not bitmap.is_contiguous()
+                    or bitmap.numel() != mb * mh * q_len * 4 * bm.n_kv_blocks):
+                raise ValueError("bitmap must be a contiguous int32 CUDA tensor "
+                                 "(B*H, q_len, 4 * nKV)")
+            bm.bitmap = bitmap
+        _check(fa_create_block_mask_bh(kind, window, _ptr(doc_id), _ptr(bitmap), mb, mh, q_len,
+                                       kv_len, FA_BLOCK, ctypes.byref(bm.struct),
+                                       _stream_handle(stream)),
+               "fa_create_block_mask_bh")
+        return bm
     bm = out if out is not None else BlockMask(q_len, kv_len, device)
     if kind == FA_MASK_BITMAP:
         if (bitmap is None or bitmap.dtype != torch.int32 or not bitmap.is_cuda

@@ -31,15 +31,26 @@ __device__ __forceinline__ void warp_minmax(int& mn, int& mx) {
   }
 }
 
-// One CTA per q-block row i.  cls[j]: 0 empty, 1 partial, 2 full.
+// One CTA per q-block row i (blockIdx.x) of mask instance blockIdx.y.  cls[j]: 0
+// empty, 1 partial, 2 full.
 __global__ void __launch_bounds__(kClassifyThreads)
-classify_rows_kernel(int kind, int window, const int32_t* __restrict__ doc,
-                     const uint32_t* __restrict__ bitmap, int q_len, int kv_len, int n_kv,
+classify_rows_kernel(int kind, int window, const int32_t* __restrict__ doc_all,
+                     const uint32_t* __restrict__ bitmap_all, int q_len, int kv_len, int n_kv,
                      int32_t* __restrict__ kv_num, int32_t* __restrict__ kv_idx,
                      int32_t* __restrict__ full_num, int32_t* __restrict__ full_idx) {
   extern __shared__ uint8_t cls[];
   __shared__ int q_doc_min, q_doc_max;
   const int i = blockIdx.x;
+  const int64_t inst = blockIdx.y;
+  const int n_q = gridDim.x;
+  // this instance's mask data and tables
+  const int32_t* doc = doc_all ? doc_all + inst * max(q_len, kv_len) : nullptr;
+  const uint32_t* bitmap =
+      bitmap_all ? bitmap_all + inst * static_cast<int64_t>(q_len) * n_kv * 4 : nullptr;
+  kv_num += inst * n_q;
+  full_num += inst * n_q;
+  kv_idx += inst * n_q * static_cast<int64_t>(n_kv);
+  full_idx += inst * n_q * static_cast<int64_t>(n_kv);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t q0 = static_cast<int64_t>(i) * kBlock;
   const int64_t q1 = min(static_cast<int64_t>(q_len), q0 + kBlock) - 1;
@@ -187,6 +198,10 @@ __global__ void __launch_bounds__(kOrderThreads)
 order_rows_kernel(int n_q, int n_kv, int n_pow2, const int32_t* __restrict__ kv_num,
                   const int32_t* __restrict__ full_num, int32_t* __restrict__ sched) {
   extern __shared__ uint32_t keys[];
+  // one CTA per mask instance
+  kv_num += static_cast<int64_t>(blockIdx.x) * n_q;
+  full_num += static_cast<int64_t>(blockIdx.x) * n_q;
+  sched += static_cast<int64_t>(blockIdx.x) * 2 * n_q;
   const bool rank_sort = n_q <= 2048;
   const int n_keys = rank_sort ? n_q : n_pow2;
   for (int t = threadIdx.x; t < n_keys; t += blockDim.x) {
@@ -243,6 +258,17 @@ transpose_kernel(int n_q, int n_kv, const int32_t* __restrict__ kv_num,
   extern __shared__ uint8_t cls[];
   const int j = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  {  // this instance's tables and column lists
+    const int64_t inst = blockIdx.y;
+    kv_num += inst * n_q;
+    full_num += inst * n_q;
+    kv_idx += inst * n_q * static_cast<int64_t>(n_kv);
+    full_idx += inst * n_q * static_cast<int64_t>(n_kv);
+    q_num += inst * n_kv;
+    full_q_num += inst * n_kv;
+    q_idx += inst * n_kv * static_cast<int64_t>(n_q);
+    full_q_idx += inst * n_kv * static_cast<int64_t>(n_q);
+  }
   auto contains = [j](const int32_t* list, int n) {
     int lo = 0, hi = n;  // first position with list[pos] >= j
     while (lo < hi) {
@@ -300,8 +326,8 @@ namespace {
 
 // Shared tail of the two builders: fill the scalar fields, classify, order.
 fa_status build_tables(int32_t kind, int32_t window, const int32_t* doc_id, const uint32_t* bitmap,
-                       int32_t q_len, int32_t kv_len, int32_t block, int32_t nq, int32_t nkv,
-                       fa_block_mask* bm, void* stream) {
+                       int32_t mask_batch, int32_t mask_heads, int32_t q_len, int32_t kv_len,
+                       int32_t block, int32_t nq, int32_t nkv, fa_block_mask* bm, void* stream) {
   bm->q_len = q_len;
   bm->kv_len = kv_len;
   bm->block = block;
@@ -311,17 +337,20 @@ fa_status build_tables(int32_t kind, int32_t window, const int32_t* doc_id, cons
   bm->window = kind == FA_MASK_SLIDING_WINDOW_CAUSAL ? window : 0;
   bm->doc_id = kind == FA_MASK_DOCUMENT_CAUSAL ? doc_id : nullptr;
   bm->bitmap = kind == FA_MASK_BITMAP ? bitmap : nullptr;
+  bm->mask_batch = mask_batch;
+  bm->mask_heads = mask_heads;
   if (nq == 0) return FA_OK;
 
+  const int inst = mask_batch * mask_heads;
   cudaStream_t s = as_stream(stream);
-  classify_rows_kernel<<<nq, kClassifyThreads, nkv > 0 ? nkv : 1, s>>>(
+  classify_rows_kernel<<<dim3(nq, inst), kClassifyThreads, nkv > 0 ? nkv : 1, s>>>(
       kind, bm->window, bm->doc_id, bm->bitmap, q_len, kv_len, nkv, bm->kv_num_blocks,
       bm->kv_indices, bm->full_kv_num_blocks, bm->full_kv_indices);
   FA_CUDA_CHECK(cudaGetLastError());
   int n_pow2 = 1;
   while (n_pow2 < nq) n_pow2 <<= 1;
   const size_t order_smem = (nq <= 2048 ? nq : n_pow2) * sizeof(uint32_t);
-  order_rows_kernel<<<1, kOrderThreads, order_smem, s>>>(
+  order_rows_kernel<<<inst, kOrderThreads, order_smem, s>>>(
       nq, nkv, n_pow2, bm->kv_num_blocks, bm->full_kv_num_blocks, bm->q_order);
   FA_CUDA_CHECK(cudaGetLastError());
   return FA_OK;
@@ -352,7 +381,8 @@ extern "C" fa_status fa_create_block_mask(int32_t kind, int32_t window, const in
   if (kind == FA_MASK_DOCUMENT_CAUSAL && doc_id == nullptr && (q_len > 0 || kv_len > 0))
     return FA_ERR_INVALID_ARG;
   if (!tables_present(bm, nq, nkv)) return FA_ERR_INVALID_ARG;
-  return build_tables(kind, window, doc_id, nullptr, q_len, kv_len, block, nq, nkv, bm, stream);
+  return build_tables(kind, window, doc_id, nullptr, 1, 1, q_len, kv_len, block, nq, nkv, bm,
+                      stream);
 }
 
 extern "C" fa_status fa_create_block_mask_bitmap(const uint32_t* bitmap, int32_t q_len,
@@ -367,8 +397,31 @@ extern "C" fa_status fa_create_block_mask_bitmap(const uint32_t* bitmap, int32_t
       (bitmap == nullptr || (reinterpret_cast<uintptr_t>(bitmap) & 15u) != 0))
     return FA_ERR_INVALID_ARG;
   if (!tables_present(bm, nq, nkv)) return FA_ERR_INVALID_ARG;
-  return build_tables(FA_MASK_BITMAP, 0, nullptr, bitmap, q_len, kv_len, block, nq, nkv, bm,
+  return build_tables(FA_MASK_BITMAP, 0, nullptr, bitmap, 1, 1, q_len, kv_len, block, nq, nkv, bm,
                       stream);
+}
+
+extern "C" fa_status fa_create_block_mask_bh(int32_t kind, int32_t window, const int32_t* doc_id,
+                                             const uint32_t* bitmap, int32_t mask_batch,
+                                             int32_t mask_heads, int32_t q_len, int32_t kv_len,
+                                             int32_t block, fa_block_mask* bm, void* stream) {
+  using namespace fa;
+  if (bm == nullptr) return FA_ERR_INVALID_ARG;
+  if (kind < FA_MASK_CAUSAL || kind > FA_MASK_BITMAP) return FA_ERR_INVALID_ARG;
+  if (mask_batch < 1 || mask_heads < 1 || static_cast<int64_t>(mask_batch) * mask_heads > 65535)
+    return FA_ERR_INVALID_ARG;
+  int32_t nq = 0, nkv = 0;
+  const fa_status st = fa_block_mask_dims(q_len, kv_len, block, &nq, &nkv);
+  if (st != FA_OK) return st;
+  if (kind == FA_MASK_SLIDING_WINDOW_CAUSAL && window < 1) return FA_ERR_INVALID_ARG;
+  if (kind == FA_MASK_DOCUMENT_CAUSAL && doc_id == nullptr && (q_len > 0 || kv_len > 0))
+    return FA_ERR_INVALID_ARG;
+  if (kind == FA_MASK_BITMAP && q_len > 0 && kv_len > 0 &&
+      (bitmap == nullptr || (reinterpret_cast<uintptr_t>(bitmap) & 15u) != 0))
+    return FA_ERR_INVALID_ARG;
+  if (!tables_present(bm, nq, nkv)) return FA_ERR_INVALID_ARG;
+  return build_tables(kind, window, doc_id, bitmap, mask_batch, mask_heads, q_len, kv_len, block,
+                      nq, nkv, bm, stream);
 }
 
 extern "C" fa_status fa_block_mask_transpose(const fa_block_mask* bm, int32_t* q_num_blocks,
@@ -382,7 +435,8 @@ extern "C" fa_status fa_block_mask_transpose(const fa_block_mask* bm, int32_t* q
   if (!tables_present(bm, nq, nkv) || q_num_blocks == nullptr || q_indices == nullptr ||
       full_q_num_blocks == nullptr || full_q_indices == nullptr)
     return FA_ERR_INVALID_ARG;
-  transpose_kernel<<<nkv, kClassifyThreads, nq, as_stream(stream)>>>(
+  const int inst = (bm->mask_batch > 1 ? bm->mask_batch : 1) * (bm->mask_heads > 1 ? bm->mask_heads : 1);
+  transpose_kernel<<<dim3(nkv, inst), kClassifyThreads, nq, as_stream(stream)>>>(
       nq, nkv, bm->kv_num_blocks, bm->kv_indices, bm->full_kv_num_blocks, bm->full_kv_indices,
       q_num_blocks, q_indices, full_q_num_blocks, full_q_indices);
   FA_CUDA_CHECK(cudaGetLastError());

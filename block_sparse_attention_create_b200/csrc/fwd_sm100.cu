@@ -129,6 +129,9 @@ struct Params {
   int32_t* err;
   int BH, L, S, n_kv, num_units, bitmap_words;
   int H, Hkv, kv_group;  // query heads, K/V heads, H / Hkv
+  // per-(batch, head) masks: instance of (b, h) = (mask_b ? b : 0) * mask_heads +
+  // (mask_h ? h : 0); each instance has its tables, schedule and mask data
+  int n_q, mask_b, mask_h, mask_heads, doc_len;
   int mask_kind, window, softcap_on, is_bf16;
   int split_p;       // P fed to the PV product as two 16-bit terms (hi + lo)
   float scale_log2;  // scale * log2(e)
@@ -146,7 +149,14 @@ struct Params {
 struct Unit {
   int bh, qblk, np, n;
   int kvbh;  // batch * Hkv + K/V head of this unit's query head
+  int inst;  // mask instance of (b, h)
 };
+
+__device__ __forceinline__ int mask_instance(const Params& p, int bh) {
+  if (!(p.mask_b | p.mask_h)) return 0;
+  const int b = bh / p.H;
+  return (p.mask_b ? b : 0) * p.mask_heads + (p.mask_h ? bh - b * p.H : 0);
+}
 
 __device__ __forceinline__ int2 ldg_nc_v2(const int32_t* ptr) {
   int2 v;
@@ -177,7 +187,10 @@ struct UnitIter {
     const int u = round * workers + ((round & 1) ? (workers - 1 - worker) : worker);
     ++round;
     nu = u < p.num_units ? u : -1;
-    if (nu >= 0) nx = ldg_nc_v2(p.sched + 2 * (nu / p.BH));
+    if (nu >= 0) {
+      const int k = nu / p.BH;
+      nx = ldg_nc_v2(p.sched + 2 * (static_cast<size_t>(mask_instance(p, nu - k * p.BH)) * p.n_q + k));
+    }
   }
   __device__ __forceinline__ bool pop(const Params& p, Unit& x) {
     if (nu < 0) return false;
@@ -185,6 +198,7 @@ struct UnitIter {
     x.bh = nu - k * p.BH;
     // grouped-query attention: query head h reads K/V head h / kv_group
     x.kvbh = p.kv_group == 1 ? x.bh : (x.bh / p.H) * p.Hkv + (x.bh % p.H) / p.kv_group;
+    x.inst = mask_instance(p, x.bh);
     x.qblk = nx.x;
     x.np = nx.y & 0xFFFF;
     x.n = x.np + (nx.y >> 16);
@@ -200,7 +214,7 @@ struct UnitIter {
 
 // kv-block index of the j-th block of the unit: partial blocks first, then full ones.
 __device__ __forceinline__ int block_index(const Params& p, const Unit& x, int j) {
-  const size_t row = static_cast<size_t>(x.qblk) * p.n_kv;
+  const size_t row = (static_cast<size_t>(x.inst) * p.n_q + x.qblk) * p.n_kv;
   return j < x.np ? ldg_nc(p.kv_idx + row + j) : ldg_nc(p.full_idx + row + (j - x.np));
 }
 
@@ -686,7 +700,8 @@ struct MaskCols<64> {
 // words `brow` is set (and the key exists).  Dead entries become -inf.
 template <int MK>
 __device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int a, int b, int kv0,
-                                           int dq, bool dq_uniform, const uint32_t* brow) {
+                                           int dq, bool dq_uniform, const int32_t* docs,
+                                           const uint32_t* brow) {
   if constexpr (MK == kMaskBitmap) {
     // the row's two words of keys kv0 .. kv0 + 63 (kv0 is a multiple of 64)
     const int2 w = ldg_nc_v2(reinterpret_cast<const int32_t*>(brow + (kv0 >> 5)));
@@ -703,7 +718,7 @@ __device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int 
 #pragma unroll
       for (int c = 0; c < 2; ++c)
         same[c] = __ballot_sync(0xffffffffu,
-                                ldg_nc(p.doc_id + min(kv0 + c * 32 + lane, p.S - 1)) == dq);
+                                ldg_nc(docs + min(kv0 + c * 32 + lane, p.S - 1)) == dq);
     } else {
       same[0] = same[1] = 0u;
 #pragma unroll
@@ -711,7 +726,7 @@ __device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int 
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int kv = min(kv0 + c * 32 + i, p.S - 1);
-          same[c] |= (ldg_nc(p.doc_id + kv) == dq ? 1u : 0u) << i;
+          same[c] |= (ldg_nc(docs + kv) == dq ? 1u : 0u) << i;
         }
     }
     MaskCols<0>::doc(x, a, b, same[0]);
@@ -816,7 +831,9 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
       }
       continue;
     }
-    const int dq_own = (MK == kMaskDoc && valid) ? __ldg(p.doc_id + row) : 0;
+    // this unit's mask instance: its document ids / bitmap rows
+    const int32_t* docs = MK == kMaskDoc ? p.doc_id + static_cast<size_t>(un.inst) * p.doc_len : nullptr;
+    const int dq_own = (MK == kMaskDoc && valid) ? __ldg(docs + row) : 0;
     // all valid rows of this warp in lane 0's document (rows past L do not matter);
     // the shuffle is taken by every lane, outside any short-circuited expression.
     // Then every lane, rows past L included, takes lane 0's id: in the ballot of
@@ -826,7 +843,8 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
     const int dq = dq_uniform ? dq0 : dq_own;
     // tabulated mask: this row's words (rows past L read the last row, unused)
     const uint32_t* brow = MK == kMaskBitmap
-                               ? p.bitmap + static_cast<size_t>(min(row, p.L - 1)) * p.bitmap_words
+                               ? p.bitmap + (static_cast<size_t>(un.inst) * p.L + min(row, p.L - 1)) *
+                                                p.bitmap_words
                                : nullptr;
     // live keys of this row: kv in [lo, hi] (and, for documents, doc_id[kv] == dq;
     // for a tabulated mask, its bit); only the causal rules bound hi by the row
@@ -854,9 +872,9 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
           const int a = lo - kvb * kBlockN;
           const int b = hi - kvb * kBlockN;
           apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x), a, b, kvb * kBlockN, dq, dq_uniform,
-                     brow);
+                     docs, brow);
           apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x + 64), a - 64, b - 64, kvb * kBlockN + 64, dq,
-                     dq_uniform, brow);
+                     dq_uniform, docs, brow);
         }
         const float mb = fmaxf(row_max64(*reinterpret_cast<float(*)[64]>(x)),
                                row_max64(*reinterpret_cast<float(*)[64]>(x + 64))) * xs;
@@ -897,7 +915,8 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
           float x[64];
           load_s_half(t_s + h * 64, x);
           if (!full)
-            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, dq_uniform, brow);
+            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, dq_uniform, docs,
+                           brow);
           rmax = fmaxf(rmax, row_max64(x));
         }
         float mb = rmax;
@@ -964,7 +983,8 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
             }
           }
           if (!full)
-            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, dq_uniform, brow);
+            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, dq_uniform, docs,
+                           brow);
           // P = exp2(x * xs - m) as 16-bit pairs; with the split, P_hi = p truncated to
           // bf16 and P_lo = round(p - P_hi), so P_hi + P_lo carries ~16 significant bits.
           float2 sums[4];
@@ -1180,6 +1200,10 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, int32_t dtype, i
     return FA_ERR_INVALID_ARG;
   if (bm->kind == FA_MASK_DOCUMENT_CAUSAL && bm->doc_id == nullptr) return FA_ERR_INVALID_ARG;
   if (bm->kind == FA_MASK_BITMAP && S > 0 && bm->bitmap == nullptr) return FA_ERR_INVALID_ARG;
+  // per-(batch, head) masks: one instance per batch element and / or head (0 reads as 1)
+  const int mb = bm->mask_batch > 1 ? bm->mask_batch : 1;
+  const int mh = bm->mask_heads > 1 ? bm->mask_heads : 1;
+  if ((mb != 1 && mb != B) || (mh != 1 && mh != H)) return FA_ERR_INVALID_ARG;
 
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
   Params prm{};
@@ -1189,6 +1213,11 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, int32_t dtype, i
   prm.doc_id = bm->doc_id;
   prm.bitmap = bm->bitmap;
   prm.bitmap_words = 4 * bm->n_kv_blocks;
+  prm.n_q = bm->n_q_blocks;
+  prm.mask_b = mb > 1 ? 1 : 0;
+  prm.mask_h = mh > 1 ? 1 : 0;
+  prm.mask_heads = mh;
+  prm.doc_len = L > S ? L : S;
   prm.out = out;
   prm.lse = lse;
   prm.err = static_cast<int32_t*>(workspace);

@@ -118,6 +118,8 @@ typedef struct fa_block_mask {
   int32_t window;         /* sliding window W (kind 1), else 0 */
   const int32_t* doc_id;  /* device int32[max(q_len, kv_len)] (kind 2), else NULL */
   const uint32_t* bitmap; /* device bitmap (kind 3, see fa_create_block_mask_bitmap), else NULL */
+  int32_t mask_batch;     /* 1: one mask for every batch element; B: one per element */
+  int32_t mask_heads;     /* 1: one mask for every head; H: one per head */
 } fa_block_mask;
 
 /* nQ and nKV of a (q_len, kv_len) mask with the given block size.
@@ -146,6 +148,28 @@ FA_API fa_status fa_create_block_mask(int32_t kind, int32_t window, const int32_
                                fa_block_mask* bm, void* stream);
 
 /*
+ * Block tables of per-(batch, head) masks (the how-to's create_block_mask(mask_mod,
+ * B, H, Q_LEN, KV_LEN) with B and H given instead of None, "Mask 1: causal": the
+ * mask may depend on b and h).  mask_batch is 1 (broadcast over the batch) or the
+ * batch size B; mask_heads is 1 or the head count H; instance
+ * n = (b or 0) * mask_heads + (h or 0) holds the tables of (b, h).
+ *   kind      as fa_create_block_mask, or FA_MASK_BITMAP.
+ *   doc_id    kind 2: device int32[instances][max(q_len, kv_len)], instance-major.
+ *   bitmap    kind 3: device words [instances][q_len][4 * nKV], 16-byte aligned.
+ *   bm        the five arrays sized for all instances: kv_num_blocks[inst * nQ],
+ *             kv_indices[inst * nQ * nKV], full_* likewise, q_order[inst * 2 * nQ]
+ *             (instance-major; each instance as fa_create_block_mask writes it).
+ * The forward kernel reads instance n of a (b, h) unit; fa_block_mask_transpose
+ * writes instance-major column lists.  Launches two kernels on `stream`.  Returns
+ * FA_ERR_INVALID_ARG (nothing launched) on bad arguments, FA_ERR_CUDA if a launch
+ * fails.  fa_create_block_mask and fa_create_block_mask_bitmap build one instance.
+ */
+FA_API fa_status fa_create_block_mask_bh(int32_t kind, int32_t window, const int32_t* doc_id,
+                                  const uint32_t* bitmap, int32_t mask_batch,
+                                  int32_t mask_heads, int32_t q_len, int32_t kv_len,
+                                  int32_t block, fa_block_mask* bm, void* stream);
+
+/*
  * Block tables of a tabulated mask_mod (the FlexAttention how-to's
  * create_block_mask takes any boolean function of (b, h, q_idx, kv_idx), "Mask 1:
  * causal"; here it is given as one bit per pair, broadcast over batch and heads).
@@ -170,6 +194,7 @@ FA_API fa_status fa_create_block_mask_bitmap(const uint32_t* bitmap, int32_t q_l
  *   q_indices[nKV * nQ]          column j: their q-block indices, ascending, then 0s
  *   full_q_num_blocks[nKV]       number of FULL blocks in column j
  *   full_q_indices[nKV * nQ]     column j: their q-block indices, ascending, then 0s
+ *   (per-(batch, head) tables: every array times mask_batch * mask_heads, instance-major)
  * Device arrays owned by the caller.  One kernel on `stream`, ordered after the
  * build on the same stream.  Returns FA_ERR_INVALID_ARG (nothing launched) on NULL
  * arguments, FA_ERR_CUDA if the launch fails; nKV == 0 or nQ == 0 launches nothing.

@@ -159,6 +159,23 @@ def test_decode_rejects_bad_arguments(fa):
     assert call(B=0) == fa.FA_OK                            # empty: nothing launched
 
 
+def test_bh_builder_rejects_bad_arguments(fa):
+    bm = fa.fa_block_mask()
+    null = ctypes.c_void_p(0)
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: rejected first
+    for kind, mb, mh, doc, bits in ((0, 0, 1, null, null), (0, 1, -2, null, null),
+                                    (2, 2, 1, null, null), (3, 1, 2, null, null), (9, 1, 1, null, null)):
+        assert fa.fa_create_block_mask_bh(kind, 0, doc, bits, mb, mh, 256, 256, 128,
+                                          ctypes.byref(bm), null) == fa.FA_ERR_INVALID_ARG
+    # NULL tables for a non-empty mask
+    assert fa.fa_create_block_mask_bh(0, 0, null, null, 2, 2, 256, 256, 128, ctypes.byref(bm),
+                                      null) == fa.FA_ERR_INVALID_ARG
+    # empty: valid, nothing launched, instance counts recorded
+    assert fa.fa_create_block_mask_bh(3, 0, null, fake, 2, 3, 0, 0, 128, ctypes.byref(bm),
+                                      null) == fa.FA_OK
+    assert (bm.mask_batch, bm.mask_heads) == (2, 3)
+
+
 def _fwd(fa, bm, **kw):
     args = dict(q=1024, k=1024, v=1024, dtype=0, B=1, H=1, L=256, S=256, D=64, sk=0, cap=0.0,
                 scale=0.0, out=1024, lse=0, ws=1024)
