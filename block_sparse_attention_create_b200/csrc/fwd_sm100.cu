@@ -152,8 +152,11 @@ struct Unit {
   int inst;  // mask instance of (b, h)
 };
 
+// BHM: the kernel serves per-(batch, head) masks; without it every unit reads
+// instance 0 and the instance arithmetic is compiled out.
+template <bool BHM>
 __device__ __forceinline__ int mask_instance(const Params& p, int bh) {
-  if (!(p.mask_b | p.mask_h)) return 0;
+  if constexpr (!BHM) return 0;
   const int b = bh / p.H;
   return (p.mask_b ? b : 0) * p.mask_heads + (p.mask_h ? bh - b * p.H : 0);
 }
@@ -172,6 +175,7 @@ __device__ __forceinline__ int ldg_nc(const int32_t* ptr) {
 // Unit sequence of one worker with a one-unit lookahead: the schedule entry of
 // the next unit is requested when the current one is handed out, so its global
 // load latency overlaps a whole unit of work.
+template <bool BHM>
 struct UnitIter {
   int worker, round;
   int nu;   // next unit id, -1 when exhausted
@@ -189,7 +193,7 @@ struct UnitIter {
     nu = u < p.num_units ? u : -1;
     if (nu >= 0) {
       const int k = nu / p.BH;
-      nx = ldg_nc_v2(p.sched + 2 * (static_cast<size_t>(mask_instance(p, nu - k * p.BH)) * p.n_q + k));
+      nx = ldg_nc_v2(p.sched + 2 * (static_cast<size_t>(mask_instance<BHM>(p, nu - k * p.BH)) * p.n_q + k));
     }
   }
   __device__ __forceinline__ bool pop(const Params& p, Unit& x) {
@@ -198,7 +202,7 @@ struct UnitIter {
     x.bh = nu - k * p.BH;
     // grouped-query attention: query head h reads K/V head h / kv_group
     x.kvbh = p.kv_group == 1 ? x.bh : (x.bh / p.H) * p.Hkv + (x.bh % p.H) / p.kv_group;
-    x.inst = mask_instance(p, x.bh);
+    x.inst = mask_instance<BHM>(p, x.bh);
     x.qblk = nx.x;
     x.np = nx.y & 0xFFFF;
     x.n = x.np + (nx.y >> 16);
@@ -268,8 +272,9 @@ __device__ __forceinline__ bool wait_lane0(Smem<D>& sm, uint64_t* bar, uint32_t 
 
 // Producer-side position in a slot's block stream, with block indices fetched 32
 // at a time (one per lane) and the next unit's first chunk requested early.
+template <bool BHM>
 struct ProdCursor {
-  UnitIter it;
+  UnitIter<BHM> it;
   Unit cur, nxt;
   bool has_cur, has_nxt;
   int j;      // block of `cur`
@@ -283,7 +288,8 @@ __device__ __forceinline__ int chunk_index(const Params& p, const Unit& x, int c
   return jj < x.n ? block_index(p, x, jj) : 0;
 }
 
-__device__ __forceinline__ void pc_enter_next(ProdCursor& c, const Params& p, int lane) {
+template <bool BHM>
+__device__ __forceinline__ void pc_enter_next(ProdCursor<BHM>& c, const Params& p, int lane) {
   c.has_cur = c.has_nxt;
   c.cur = c.nxt;
   c.idx = c.nxt_idx;
@@ -294,7 +300,8 @@ __device__ __forceinline__ void pc_enter_next(ProdCursor& c, const Params& p, in
   if (c.has_nxt) c.nxt_idx = chunk_index(p, c.nxt, 0, lane);
 }
 
-__device__ __forceinline__ void pc_init(ProdCursor& c, const Params& p, int slot, int lane) {
+template <bool BHM>
+__device__ __forceinline__ void pc_init(ProdCursor<BHM>& c, const Params& p, int slot, int lane) {
   c.it.init(p, slot);
   c.units = 0;
   c.has_nxt = c.it.pop_nonempty(p, c.nxt);
@@ -302,11 +309,13 @@ __device__ __forceinline__ void pc_init(ProdCursor& c, const Params& p, int slot
   pc_enter_next(c, p, lane);
 }
 
-__device__ __forceinline__ void pc_step(ProdCursor& c, const Params& p, int lane) {
+template <bool BHM>
+__device__ __forceinline__ void pc_step(ProdCursor<BHM>& c, const Params& p, int lane) {
   if (++c.j >= c.cur.n) pc_enter_next(c, p, lane);
 }
 
-__device__ __forceinline__ int pc_block(ProdCursor& c, const Params& p, int lane) {
+template <bool BHM>
+__device__ __forceinline__ int pc_block(ProdCursor<BHM>& c, const Params& p, int lane) {
   const int chunk = c.j >> 5;
   if (chunk != c.chunk) {
     c.idx = chunk_index(p, c.cur, chunk, lane);
@@ -341,9 +350,9 @@ struct ProdCounts {
   int k, v;  // K / V tiles issued on this slot
 };
 
-template <int D, int SLOT>
+template <int D, int SLOT, bool BHM>
 __device__ __forceinline__ bool produce_k(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
-                                          const CUtensorMap* tk, ProdCursor& c, ProdCounts& n,
+                                          const CUtensorMap* tk, ProdCursor<BHM>& c, ProdCounts& n,
                                           int kvb, uint64_t pol_q, uint64_t pol_kv) {
   using C = Cfg<D>;
   if (c.j == 0) {  // the unit's Q tile first
@@ -376,14 +385,14 @@ __device__ __forceinline__ bool produce_v(Smem<D>& sm, const Params& p, const CU
 // One producer warp per slot.  Separate-P layout: K runs one block ahead of V
 // (K_0, K_1, V_0, K_2, V_1, ...), matching S_{i+1} being issued during softmax i.
 // Aliased layout: K_i, V_i, K_{i+1}, ...
-template <int D, int SLOT>
+template <int D, int SLOT, bool BHM>
 __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
                               const CUtensorMap* tk, const CUtensorMap* tv) {
   using C = Cfg<D>;
   const int lane = threadIdx.x & 31;
   const uint64_t pol_kv = policy_evict_last();
   const uint64_t pol_q = policy_evict_first();
-  ProdCursor c;
+  ProdCursor<BHM> c;
   ProdCounts n{0, 0};
   pc_init(c, p, SLOT, lane);
   bool ok = true;
@@ -445,8 +454,9 @@ __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* t
 }
 
 // MMA-side position in a slot's block stream (no block indices needed).
+template <bool BHM>
 struct MmaStream {
-  UnitIter it;
+  UnitIter<BHM> it;
   Unit cur;
   bool active;
   int j;      // block of `cur`
@@ -454,18 +464,21 @@ struct MmaStream {
   int i;      // position in the slot's block stream
 };
 
-__device__ __forceinline__ void ms_enter_next(MmaStream& c, const Params& p) {
+template <bool BHM>
+__device__ __forceinline__ void ms_enter_next(MmaStream<BHM>& c, const Params& p) {
   c.active = c.it.pop_nonempty(p, c.cur);
   c.j = 0;
   if (c.active) ++c.units;
 }
-__device__ __forceinline__ void ms_init(MmaStream& c, const Params& p, int slot) {
+template <bool BHM>
+__device__ __forceinline__ void ms_init(MmaStream<BHM>& c, const Params& p, int slot) {
   c.it.init(p, slot);
   c.units = 0;
   c.i = 0;
   ms_enter_next(c, p);
 }
-__device__ __forceinline__ void ms_step(MmaStream& c, const Params& p) {
+template <bool BHM>
+__device__ __forceinline__ void ms_step(MmaStream<BHM>& c, const Params& p) {
   ++c.i;
   if (++c.j >= c.cur.n) ms_enter_next(c, p);
 }
@@ -485,8 +498,9 @@ __device__ __forceinline__ bool probe(uint64_t* bar, uint32_t parity) {
 // S_i = Q K_i^T for the slot's stream position `c`, if its inputs are ready.
 // `prev_done`: the S buffer may be overwritten (aliased layout: PV_{i-1} issued;
 // separate-P layout: the softmax has read S_{i-1}).
-template <int D, int SLOT>
-__device__ __forceinline__ bool try_s(Smem<D>& sm, const Params& p, MmaStream& c, MmaShared& ms) {
+template <int D, int SLOT, bool BHM>
+__device__ __forceinline__ bool try_s(Smem<D>& sm, const Params& p, MmaStream<BHM>& c,
+                                      MmaShared& ms) {
   using C = Cfg<D>;
   const int u = c.units - 1;
   const int b = u % C::kQBuf;
@@ -520,8 +534,9 @@ __device__ __forceinline__ bool try_s(Smem<D>& sm, const Params& p, MmaStream& c
 }
 
 // O += P_i V_i for the slot's stream position `c`, if its inputs are ready.
-template <int D, int SLOT>
-__device__ __forceinline__ bool try_pv(Smem<D>& sm, const Params& p, MmaStream& c, MmaShared& ms) {
+template <int D, int SLOT, bool BHM>
+__device__ __forceinline__ bool try_pv(Smem<D>& sm, const Params& p, MmaStream<BHM>& c,
+                                       MmaShared& ms) {
   using C = Cfg<D>;
   const int st = c.i % C::kVRing;
   if (!probe(&sm.p_full[SLOT], c.i & 1)) return false;
@@ -557,16 +572,16 @@ __device__ __forceinline__ bool try_pv(Smem<D>& sm, const Params& p, MmaStream& 
 // Per slot: its S stream and its PV stream (the PV stream trails).  In the aliased
 // layout S_{i+1} may only follow PV_i (the MMAs of one thread run in issue order,
 // so PV_i has read P before S_{i+1} overwrites it).
-template <int D, int SLOT>
-__device__ __forceinline__ bool mma_slot(Smem<D>& sm, const Params& p, MmaStream& cs,
-                                         MmaStream& cp, MmaShared& ms) {
+template <int D, int SLOT, bool BHM>
+__device__ __forceinline__ bool mma_slot(Smem<D>& sm, const Params& p, MmaStream<BHM>& cs,
+                                         MmaStream<BHM>& cp, MmaShared& ms) {
   bool progress = false;
   if (cs.active && (Cfg<D>::kSepP || cs.i == cp.i)) progress |= try_s<D, SLOT>(sm, p, cs, ms);
   if (cp.active && (!cs.active || cp.i < cs.i)) progress |= try_pv<D, SLOT>(sm, p, cp, ms);
   return progress;
 }
 
-template <int D>
+template <int D, bool BHM>
 __device__ void mma_role(Smem<D>& sm, const Params& p, uint32_t tmem) {
   static_assert(kNumSlots == 2, "the MMA loop serves two slots");
   MmaShared ms;
@@ -574,7 +589,7 @@ __device__ void mma_role(Smem<D>& sm, const Params& p, uint32_t tmem) {
   ms.idesc_s = idesc_f16_f32(p.is_bf16 != 0, 128, 128, false);
   ms.idesc_pv = idesc_f16_f32(p.is_bf16 != 0, 128, D, true);
   ms.split = p.split_p != 0 && !Cfg<D>::kSepP;
-  MmaStream s0, p0, s1, p1;
+  MmaStream<BHM> s0, p0, s1, p1;
   ms_init(s0, p, 0);
   ms_init(p0, p, 0);
   ms_init(s1, p, 1);
@@ -799,7 +814,7 @@ __device__ __forceinline__ float exp_pack64(const float (&x)[64], float xs, floa
 
 // Softmax warpgroup of one slot: thread t owns row t of the slot's 128-row tile
 // (TMEM lane t), so row max and row sum need no shuffles.
-template <int D, int MK>
+template <int D, int MK, bool BHM>
 __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int slot) {
   using C = Cfg<D>;
   const int t = threadIdx.x - slot * 128;   // row of the tile this thread owns
@@ -813,7 +828,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
   // kept (and scaled inside the exponent's FFMA) unless a score_mod rewrote it.
   const float xs = p.softcap_on ? 1.f : p.scale_log2;
   const bool split = p.split_p != 0 && !C::kSepP;
-  UnitIter it;
+  UnitIter<BHM> it;
   it.init(p, slot);
   int blk = 0, units = 0;
   Unit un;
@@ -1054,7 +1069,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
   }
 }
 
-template <int D, int MK>
+template <int D, int MK, bool BHM>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
            const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ Params p) {
@@ -1104,17 +1119,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
 
   // Role dispatch; the final rendezvous is a named barrier over all threads.
   if (warp < kSoftmaxWarps) {
-    softmax_role<D, MK>(sm, p, tmem, warp / 4);
+    softmax_role<D, MK, BHM>(sm, p, tmem, warp / 4);
     tc_fence_before();
     named_barrier_sync(1, kThreads);
     return;
   }
   if (warp == kProducerWarp) {
-    producer_role<D, 0>(sm, p, &tmap_q, &tmap_k, &tmap_v);
+    producer_role<D, 0, BHM>(sm, p, &tmap_q, &tmap_k, &tmap_v);
   } else if (warp == kProducerWarp + 1) {
-    producer_role<D, 1>(sm, p, &tmap_q, &tmap_k, &tmap_v);
+    producer_role<D, 1, BHM>(sm, p, &tmap_q, &tmap_k, &tmap_v);
   } else if (warp == kMmaWarp) {
-    mma_role<D>(sm, p, tmem);
+    mma_role<D, BHM>(sm, p, tmem);
   }
   tc_fence_before();
   named_barrier_sync(1, kThreads);
@@ -1130,7 +1145,7 @@ bool make_map(CUtensorMap* map, const void* ptr, bool bf16, int D, int rows, int
   return make_tile_map(map, ptr, bf16, D, rows, bh, kBlockN);
 }
 
-template <int D, int MK>
+template <int D, int MK, bool BHM>
 fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH, int L, int S,
                  const Params& prm, cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
@@ -1148,7 +1163,7 @@ fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH,
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
     if (!done[dev]) {
-      FA_CUDA_CHECK(cudaFuncSetAttribute(fwd_kernel<D, MK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      FA_CUDA_CHECK(cudaFuncSetAttribute(fwd_kernel<D, MK, BHM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem)));
       done[dev] = true;
     }
@@ -1157,7 +1172,7 @@ fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH,
   if (sms <= 0) return FA_ERR_CUDA;
   const int want = (prm.num_units + kNumSlots - 1) / kNumSlots;
   const int grid = want < sms ? want : sms;
-  fwd_kernel<D, MK><<<grid, kThreads, smem, stream>>>(tq, tk, tv, prm);
+  fwd_kernel<D, MK, BHM><<<grid, kThreads, smem, stream>>>(tq, tk, tv, prm);
   FA_CUDA_CHECK(cudaGetLastError());
   return FA_OK;
 }
@@ -1169,6 +1184,20 @@ extern "C" size_t fa_fwd_workspace_bytes(void) { return 256; }
 
 namespace fa {
 namespace {
+
+// The instantiation for a head dim, mask family and (broadcast or per-instance) mask.
+template <bool BHM>
+fa_status launch_family(int kind, int D, const void* q, const void* k, const void* v, bool b16,
+                        int L, int S, const Params& prm, cudaStream_t s) {
+  switch (mask_family(kind) * 2 + (D == 64 ? 0 : 1)) {
+    case kMaskRange * 2: return launch<64, kMaskRange, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskRange * 2 + 1: return launch<128, kMaskRange, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskDoc * 2: return launch<64, kMaskDoc, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskDoc * 2 + 1: return launch<128, kMaskDoc, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskBitmap * 2: return launch<64, kMaskBitmap, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
+    default: return launch<128, kMaskBitmap, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
+  }
+}
 
 // Testing hook for the bounded-wait failure path (fa_debug_set_mma_stall).
 std::atomic<int> g_stall_mma{0};
@@ -1244,14 +1273,8 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, int32_t dtype, i
   }
   const cudaStream_t s = as_stream(stream);
   const bool b16 = dtype == FA_BF16;
-  switch (mask_family(bm->kind) * 2 + (D == 64 ? 0 : 1)) {
-    case kMaskRange * 2: return launch<64, kMaskRange>(q, k, v, b16, prm.BH, L, S, prm, s);
-    case kMaskRange * 2 + 1: return launch<128, kMaskRange>(q, k, v, b16, prm.BH, L, S, prm, s);
-    case kMaskDoc * 2: return launch<64, kMaskDoc>(q, k, v, b16, prm.BH, L, S, prm, s);
-    case kMaskDoc * 2 + 1: return launch<128, kMaskDoc>(q, k, v, b16, prm.BH, L, S, prm, s);
-    case kMaskBitmap * 2: return launch<64, kMaskBitmap>(q, k, v, b16, prm.BH, L, S, prm, s);
-    default: return launch<128, kMaskBitmap>(q, k, v, b16, prm.BH, L, S, prm, s);
-  }
+  if (prm.mask_b | prm.mask_h) return launch_family<true>(bm->kind, D, q, k, v, b16, L, S, prm, s);
+  return launch_family<false>(bm->kind, D, q, k, v, b16, L, S, prm, s);
 }
 
 }  // namespace
