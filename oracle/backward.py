@@ -1,0 +1,55 @@
+"""Gradients of the attention forward (fp64, dense), for the backward pass.
+
+Test infrastructure only, like the rest of oracle/.
+
+The FlashAttention-2 article (media.tcdigital.jp, "あえて再計算して転送を減らす")
+describes the backward pass as recomputing the attention matrix on chip from the
+saved inputs instead of storing it; what it computes is the derivative of the
+forward, written out here from the definition (SDPA tutorial, section 1):
+
+    s = q k^T * scale  (then c * tanh(s / c) under the softcap), masked -> -inf
+    P = softmax(s) row by row,  O = P V
+    dV = P^T dO
+    dP = dO V^T
+    dS = P * (dP - rowsum(dO * O))            (softmax backward)
+    dS_raw = dS * (1 - tanh(s_scaled / c)^2)  (softcap backward, else dS)
+    dQ = dS_raw K * scale,  dK = dS_raw^T Q * scale
+
+A row with no live key has P = 0 and contributes nothing.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import masks
+from .attention import TANH_SOFTCAP, _as_f64
+
+
+def attention_head_backward(q, k, v, dout, kind, window=None, doc_id=None, score_kind=0,
+                            softcap=0.0, scale=None, bitmap=None):
+    """One (batch, head): q (L,D), k (S,D), v (S,Dv), dout (L,Dv) -> dq, dk, dv (fp64)."""
+    q, k, v, dout = (_as_f64(t) for t in (q, k, v, dout))
+    L, D = q.shape
+    S = k.shape[0]
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(D)
+    doc = None if doc_id is None else _as_f64(doc_id).astype(np.int64)
+    allowed = masks.mask_rows(kind, np.arange(L), S, window, doc, bitmap, q_len=L)
+    t = (q @ k.T) * scale                                  # scaled scores
+    s = softcap * np.tanh(t / softcap) if score_kind == TANH_SOFTCAP else t
+    s = np.where(allowed, s, -np.inf)
+    m = s.max(axis=1, initial=-np.inf) if S > 0 else np.full(L, -np.inf)
+    live = np.isfinite(m)
+    p = np.zeros_like(s)
+    p[live] = np.exp(s[live] - m[live, None])
+    p[live] /= p[live].sum(axis=1, keepdims=True)
+    out = p @ v
+    dv = p.T @ dout
+    dp = dout @ v.T
+    delta = (dout * out).sum(axis=1, keepdims=True)
+    ds = p * (dp - delta)
+    if score_kind == TANH_SOFTCAP:
+        ds = ds * (1.0 - np.tanh(t / softcap) ** 2)
+    dq = ds @ k * scale
+    dk = ds.T @ q * scale
+    return dq, dk, dv

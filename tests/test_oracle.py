@@ -471,3 +471,58 @@ def test_decode_bruteforce_tiny(kind):
     bo, bl = BF.attention_head(q.tolist(), k.tolist(), v.tolist(), kind, 4)
     assert np.allclose(out, np.array(bo), atol=1e-13, rtol=0)
     assert np.allclose(lse, np.array(bl), atol=1e-13, rtol=0)
+
+
+# ---------------------------------------------------------------- backward
+
+from oracle import backward as OBW  # noqa: E402
+
+
+@pytest.mark.parametrize("kind,w", [(OM.CAUSAL, None), (OM.SLIDING_WINDOW_CAUSAL, 40),
+                                    (OM.DOCUMENT_CAUSAL, None), (OM.BITMAP, None)])
+def test_backward_matches_torch_autograd_fp64(kind, w):
+    """Gradients equal torch autograd through its CPU SDPA in fp64 with the same
+    boolean mask (rows with no live key excluded from SDPA's comparison)."""
+    L, S, D = 150, 130, 16
+    doc = np.random.default_rng(2).integers(0, 3, size=max(L, S)) if kind == OM.DOCUMENT_CAUSAL \
+        else None
+    words = W.random_bitmap(L, S, seed=3) if kind == OM.BITMAP else None
+    mask = OM.mask_rows(kind, np.arange(L), S, w, doc, words, q_len=L)
+    live = mask.any(axis=1)
+    q, k, v, do = (_rand(shape, s) for shape, s in (((L, D), 1), ((S, D), 2), ((S, D), 3),
+                                                    ((L, D), 4)))
+    do[~live] = 0.0   # SDPA gives dead rows a zero output; give them no gradient either
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(tq[None, None], tk[None, None],
+                                                           tv[None, None],
+                                                           attn_mask=torch.from_numpy(mask))
+    out[0, 0].backward(torch.from_numpy(do))
+    dq, dk, dv = OBW.attention_head_backward(q, k, v, do, kind, window=w, doc_id=doc, bitmap=words)
+    assert np.abs(dq - tq.grad.numpy()).max() < 1e-10
+    assert np.abs(dk - tk.grad.numpy()).max() < 1e-10
+    assert np.abs(dv - tv.grad.numpy()).max() < 1e-10
+
+
+def test_backward_softcap_finite_differences():
+    """Central differences of sum(out * dO) reproduce every gradient under the softcap."""
+    L, S, D = 5, 7, 4
+    q, k, v, do = (_rand(shape, s, 2.0) for shape, s in (((L, D), 5), ((S, D), 6), ((S, D), 7),
+                                                         ((L, D), 8)))
+    args = dict(score_kind=1, softcap=1.5)
+
+    def f(qq, kk, vv):
+        out, _ = OA.attention_head(qq, kk, vv, OM.SLIDING_WINDOW_CAUSAL, window=4, **args)
+        return float((out * do).sum())
+    dq, dk, dv = OBW.attention_head_backward(q, k, v, do, OM.SLIDING_WINDOW_CAUSAL, window=4, **args)
+    h = 1e-6
+    for x, g, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            a = [q, k, v]
+            a[which] = xp
+            fp = f(*a)
+            a[which] = xm
+            fm = f(*a)
+            assert abs((fp - fm) / (2 * h) - g[idx]) < 1e-7, (which, idx)
