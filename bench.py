@@ -304,6 +304,63 @@ def run_ours(args, w: W.Workload, rank, world, device):
             "mask_ms": mask_ms, "clocks": clk.summary(), "e2e": e2e}
 
 
+def run_backward(args, w: W.Workload, world, device, fig):
+    """Backward step timed like the forward: the mask's column lists and
+    fa_flex_attention_bwd, L2 flushed between steps, CUDA events, max over ranks.
+    FLOPs credited: 2.5 x the forward's live-block FLOPs (five block products:
+    S, dP, dV, dQ, dK against the forward's two)."""
+    import block_sparse_attention_create_b200 as fa
+    torch.cuda.set_device(device)
+    q, k, v = (t.to(device) for t in W.make_qkv(w))
+    doc = W.make_doc_id(w)
+    dd = doc.to(device) if doc is not None else None
+    words = W.make_bitmap(w)
+    bd = torch.from_numpy(words.view(np.int32)).to(device) if words is not None else None
+    g = torch.Generator().manual_seed(w.seed + 1)
+    dout = torch.randn(q.shape, generator=g).to(q.dtype).to(device)
+    bm = fa.create_block_mask(w.mask_kind, w.L, w.S, window=w.window, doc_id=dd, device=device,
+                              bitmap=bd)
+    out, lse = fa.flex_attention(q, k, v, bm, score_mod=w.score_kind, softcap=w.softcap,
+                                 return_lse=True)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    def step():
+        cols = bm.transpose()
+        return fa.flex_attention_backward(q, k, v, out, dout, lse, bm, score_mod=w.score_kind,
+                                          softcap=w.softcap, columns=cols)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    total = sum(ms)
+    if world > 1:
+        t = torch.tensor([total], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total = float(t.item())
+    flops = 2.5 * fig["flops"]
+    peaks, _ = load_peaks()
+    tflops = flops * args.steps * world / (total * 1e-3) / 1e12
+    line = {"metric": "backward live-block TFLOP/s (2.5 x forward FLOPs)", "value": tflops,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype_name, "data": "synthetic",
+            "config": {**w.describe(), "step": "fa_block_mask_transpose + fa_flex_attention_bwd",
+                       "l2": "flushed between timed steps (512 MiB write, untimed)"},
+            "roofline": {"bound": "tensor", "achieved": tflops / world, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": tflops / world / peaks["bf16_tflops"],
+                         "traffic": None},
+            "gpu_launches": 4 * args.steps}
+    print(json.dumps(line))
+
+
 def run_e2e(args, w, fa, q, k, v, doc, bits, device, world):
     hq, hk, hv = (t.pin_memory() for t in (q, k, v))
     hdoc = doc.pin_memory() if doc is not None else None
@@ -396,6 +453,9 @@ def main():
     ap.add_argument("--workload", default=W.C3_SWA256_32K.name, choices=sorted(W.BY_NAME))
     ap.add_argument("--cpu-rows", type=int, default=32768,
                     help="oracle rows timed for cpu_baseline (bounded sample)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (column lists + fa_flex_attention_bwd) of the "
+                         "workload instead of the forward step; prints its own JSON line")
     ap.add_argument("--profile", action="store_true",
                     help="short run for profilers: warm-up and timed steps only (no clock "
                          "window, no end-to-end leg, no CPU baseline); not a bench value")
@@ -446,6 +506,11 @@ def main():
     if world > 1:
         torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
+    if args.backward:
+        run_backward(args, w, world, device, fig)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     r = run_ours(args, w, rank, world, device)
 
     total_flops = fig["flops"] * args.steps * world

@@ -39,7 +39,8 @@ EXPORTED = ("fa_block_mask_dims", "fa_create_block_mask", "fa_fwd_workspace_byte
             "fa_flex_attention_fwd", "fa_get_last_device_error", "fa_status_string",
             "fa_num_sms", "fa_flex_attention_fwd_noalloc", "fa_create_block_mask_bitmap",
             "fa_block_mask_transpose", "fa_flex_attention_fwd_gqa", "fa_decode_workspace_bytes",
-            "fa_flex_attention_decode", "fa_debug_set_mma_stall", "fa_create_block_mask_bh")
+            "fa_flex_attention_decode", "fa_debug_set_mma_stall", "fa_create_block_mask_bh",
+            "fa_bwd_workspace_bytes", "fa_flex_attention_bwd")
 
 
 class fa_block_mask(ctypes.Structure):
@@ -106,6 +107,12 @@ def _load():
     lib.fa_create_block_mask_bh.argtypes = [i32, i32, vp, vp, i32, i32, i32, i32, i32,
                                             ctypes.POINTER(fa_block_mask), vp]
     lib.fa_create_block_mask_bh.restype = i32
+    lib.fa_bwd_workspace_bytes.argtypes = [i32, i32, i32]
+    lib.fa_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.fa_flex_attention_bwd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32,
+                                          ctypes.POINTER(fa_block_mask), vp, vp, vp, vp, i32, f32,
+                                          f32, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.fa_flex_attention_bwd.restype = i32
     return lib
 
 
@@ -127,6 +134,8 @@ fa_decode_workspace_bytes = _lib.fa_decode_workspace_bytes
 fa_flex_attention_decode = _lib.fa_flex_attention_decode
 fa_debug_set_mma_stall = _lib.fa_debug_set_mma_stall
 fa_create_block_mask_bh = _lib.fa_create_block_mask_bh
+fa_bwd_workspace_bytes = _lib.fa_bwd_workspace_bytes
+fa_flex_attention_bwd = _lib.fa_flex_attention_bwd
 
 
 class FAError(RuntimeError):
@@ -386,6 +395,39 @@ def flex_attention_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                                     _stream_handle(stream)),
            "fa_flex_attention_decode")
     return (out, lse) if return_lse else out
+
+
+def flex_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                            dout: torch.Tensor, lse: torch.Tensor, block_mask: BlockMask,
+                            score_mod: int = FA_SCORE_NONE, softcap: float = 0.0,
+                            scale: float = 0.0, columns: Optional[dict] = None,
+                            stream: Optional[torch.cuda.Stream] = None):
+    """fa_flex_attention_bwd: (dq, dk, dv) of the forward that produced out and lse.
+    `columns`: the mask's column lists (block_mask.transpose()); built here if None."""
+    for t in (q, k, v, out, dout):
+        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4 or t.dtype != q.dtype:
+            raise ValueError("q, k, v, out, dout must be contiguous 4-D CUDA tensors of one dtype")
+    if q.dtype not in _DTYPES:
+        raise ValueError("dtype must be bf16 or fp16")
+    B, H, L, D = q.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    if k.shape != (B, Hkv, S, D) or v.shape != k.shape or out.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if lse.dtype != torch.float32 or not lse.is_contiguous() or lse.shape != (B, H, L):
+        raise ValueError("lse must be a contiguous float32 (B, H, L) tensor")
+    cols = columns if columns is not None else block_mask.transpose(stream)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nbytes = int(fa_bwd_workspace_bytes(B, H, L))
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    _check(fa_flex_attention_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                                 _DTYPES[q.dtype], B, H, Hkv, L, S, D,
+                                 ctypes.byref(block_mask.struct), _ptr(cols["q_num_blocks"]),
+                                 _ptr(cols["q_indices"]), _ptr(cols["full_q_num_blocks"]),
+                                 _ptr(cols["full_q_indices"]), score_mod, float(softcap),
+                                 float(scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
+                                 _stream_handle(stream)),
+           "fa_flex_attention_bwd")
+    return dq, dk, dv
 
 
 def last_decode_error(device=None, stream: Optional[torch.cuda.Stream] = None) -> int:

@@ -270,7 +270,7 @@ FA_API fa_status fa_flex_attention_fwd_noalloc(const void* q, const void* k, con
                                         void* stream);
 
 /*
- * Grouped-query attention forward (NEXT-2; SDPA tutorial section 5: several query
+ * Grouped-query attention forward (SDPA tutorial section 5: several query
  * heads share one K/V head, SDPA's enable_gqa).  As fa_flex_attention_fwd, except
  *   k, v      device (B, H_kv, S, D);
  *   H_kv      >= 1 and dividing H: query head h reads K/V head h / (H / H_kv)
@@ -285,7 +285,7 @@ FA_API fa_status fa_flex_attention_fwd_gqa(const void* q, const void* k, const v
                                     float* lse, void* workspace, void* stream);
 
 /*
- * Decode against a KV cache (NEXT-4; SDPA tutorial, section 4, pitfall 3): L new
+ * Decode against a KV cache (SDPA tutorial, section 4, pitfall 3): L new
  * queries after S - L cached keys.  Query i sits at key position S - L + i, so the
  * causal mask is aligned to the lower right (torch's causal_lower_right).
  *   q         device (B, H, L, D);   k, v  device (B, H_kv, S, D);  16-byte aligned.
@@ -318,6 +318,34 @@ FA_API fa_status fa_flex_attention_decode(const void* q, const void* k, const vo
                                    int32_t score_kind, float softcap, float scale, void* out,
                                    float* lse, void* workspace, size_t workspace_bytes,
                                    void* stream);
+
+/*
+ * Backward pass (FlashAttention-2 article, "あえて再計算して転送を減らす":
+ * the attention matrix is recomputed block by block from the inputs and the
+ * forward's LSE rather than stored).  Gradients of the forward with the same
+ * mask, score_mod and scale:
+ *   q, out, dout  device (B, H, L, D);  k, v  device (B, H_kv, S, D);  dtype as forward.
+ *   lse       device (B, H, L) fp32 from the forward (natural log; -inf rows get no gradient).
+ *   bm        the forward's tables (broadcast masks; per-(b, h) tables: FA_ERR_UNSUPPORTED).
+ *   q_num_blocks, q_indices, full_q_num_blocks, full_q_indices
+ *             the column lists of bm from fa_block_mask_transpose.
+ *   dq        device (B, H, L, D);  dk, dv  device (B, H_kv, S, D);  in dtype.
+ *   workspace device, at least fa_bwd_workspace_bytes(B, H, L) bytes (row sums of
+ *             dO * O; no initial contents needed).
+ * Pointers 4-byte aligned; D 64 or 128; B * H * L and B * H_kv * S at most 2^33
+ * (else FA_ERR_UNSUPPORTED).  Three kernels on `stream` (row sums, dQ per query row,
+ * dK and dV per key row over the column lists; no atomics).  Returns
+ * FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED (nothing launched) or FA_ERR_CUDA.
+ */
+FA_API size_t fa_bwd_workspace_bytes(int32_t B, int32_t H, int32_t L);
+FA_API fa_status fa_flex_attention_bwd(const void* q, const void* k, const void* v, const void* out,
+                                const void* dout, const float* lse, int32_t dtype, int32_t B,
+                                int32_t H, int32_t H_kv, int32_t L, int32_t S, int32_t D,
+                                const fa_block_mask* bm, const int32_t* q_num_blocks,
+                                const int32_t* q_indices, const int32_t* full_q_num_blocks,
+                                const int32_t* full_q_indices, int32_t score_kind, float softcap,
+                                float scale, void* dq, void* dk, void* dv, void* workspace,
+                                size_t workspace_bytes, void* stream);
 
 /*
  * Testing hook for failure detection (no counterpart on the pages).  While `on`,

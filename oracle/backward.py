@@ -26,8 +26,9 @@ from .attention import TANH_SOFTCAP, _as_f64
 
 
 def attention_head_backward(q, k, v, dout, kind, window=None, doc_id=None, score_kind=0,
-                            softcap=0.0, scale=None, bitmap=None):
-    """One (batch, head): q (L,D), k (S,D), v (S,Dv), dout (L,Dv) -> dq, dk, dv (fp64)."""
+                            softcap=0.0, scale=None, bitmap=None, return_probs=False):
+    """One (batch, head): q (L,D), k (S,D), v (S,Dv), dout (L,Dv) -> dq, dk, dv (fp64);
+    with ``return_probs`` also P (L,S), for error bounds that need it."""
     q, k, v, dout = (_as_f64(t) for t in (q, k, v, dout))
     L, D = q.shape
     S = k.shape[0]
@@ -52,4 +53,6 @@ def attention_head_backward(q, k, v, dout, kind, window=None, doc_id=None, score
         ds = ds * (1.0 - np.tanh(t / softcap) ** 2)
     dq = ds @ k * scale
     dk = ds.T @ q * scale
+    if return_probs:
+        return dq, dk, dv, p
     return dq, dk, dv
