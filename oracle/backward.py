@@ -28,7 +28,8 @@ from .attention import TANH_SOFTCAP, _as_f64
 def attention_head_backward(q, k, v, dout, kind, window=None, doc_id=None, score_kind=0,
                             softcap=0.0, scale=None, bitmap=None, return_probs=False):
     """One (batch, head): q (L,D), k (S,D), v (S,Dv), dout (L,Dv) -> dq, dk, dv (fp64);
-    with ``return_probs`` also P (L,S), for error bounds that need it."""
+    with ``return_probs`` also P and dS (both (L,S), dS after the softcap factor),
+    for error bounds that need them."""
     q, k, v, dout = (_as_f64(t) for t in (q, k, v, dout))
     L, D = q.shape
     S = k.shape[0]
@@ -54,5 +55,5 @@ def attention_head_backward(q, k, v, dout, kind, window=None, doc_id=None, score
     dq = ds @ k * scale
     dk = ds.T @ q * scale
     if return_probs:
-        return dq, dk, dv, p
+        return dq, dk, dv, p, ds
     return dq, dk, dv
