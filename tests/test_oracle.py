@@ -526,3 +526,47 @@ def test_backward_softcap_finite_differences():
             a[which] = xm
             fm = f(*a)
             assert abs((fp - fm) / (2 * h) - g[idx]) < 1e-7, (which, idx)
+
+
+def test_backward_single_visible_key_closed_form():
+    """Causal row 0 sees key 0 alone: P = 1 there, so dO_0 . v_0 equals the row sum
+    rowsum(dO_0 * O_0) and dS vanishes on the row, giving dq_0 = 0; its only effect on
+    dv is dO_0 added to dv_0, and it adds nothing to dk."""
+    L, S, D = 6, 6, 8
+    q, k, v, do = (_rand((n, D), s) for n, s in ((L, 11), (S, 12), (S, 13), (L, 14)))
+    dq, dk, dv = OBW.attention_head_backward(q, k, v, do, OM.CAUSAL)
+    assert np.abs(dq[0]).max() < 1e-12
+    do_rest = do.copy()
+    do_rest[0] = 0.0
+    _, dk_rest, dv_rest = OBW.attention_head_backward(q, k, v, do_rest, OM.CAUSAL)
+    assert np.abs(dv[0] - dv_rest[0] - do[0]).max() < 1e-12
+    assert np.abs(dv[1:] - dv_rest[1:]).max() < 1e-12
+    assert np.abs(dk - dk_rest).max() < 1e-12
+
+
+def test_backward_grouped_heads_sum_over_the_group():
+    """With two query heads on one K/V head, dk and dv of the shared head are the
+    sums of the per-head gradients: checked against torch autograd through fp64
+    SDPA with enable_gqa."""
+    L, S, D = 40, 40, 8
+    q = np.stack([_rand((L, D), 21), _rand((L, D), 22)])
+    k, v = _rand((S, D), 23), _rand((S, D), 24)
+    do = np.stack([_rand((L, D), 25), _rand((L, D), 26)])
+    mask = OM.mask_rows(OM.SLIDING_WINDOW_CAUSAL, np.arange(L), S, 9, q_len=L)
+    tq = torch.tensor(q[None], requires_grad=True)
+    tk = torch.tensor(k[None, None], requires_grad=True)
+    tv = torch.tensor(v[None, None], requires_grad=True)
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv,
+                                                           attn_mask=torch.from_numpy(mask),
+                                                           enable_gqa=True)
+    out.backward(torch.from_numpy(do[None]))
+    dk = np.zeros((S, D))
+    dv = np.zeros((S, D))
+    for h in range(2):
+        gq, gk, gv = OBW.attention_head_backward(q[h], k, v, do[h], OM.SLIDING_WINDOW_CAUSAL,
+                                                 window=9)
+        assert np.abs(gq - tq.grad.numpy()[0, h]).max() < 1e-10
+        dk += gk
+        dv += gv
+    assert np.abs(dk - tk.grad.numpy()[0, 0]).max() < 1e-10
+    assert np.abs(dv - tv.grad.numpy()[0, 0]).max() < 1e-10
