@@ -215,6 +215,60 @@ def test_fwd_rejects_bad_arguments_on_host(fa):
     assert _fwd(fa, bm0, L=0) == fa.FA_OK
 
 
+def _bwd(fa, bm, **kw):
+    args = dict(q=1024, k=1024, v=1024, out=1024, dout=1024, lse=1024, dtype=0, B=1, H=2, Hkv=1,
+                L=256, S=256, D=64, cols=4096, sk=0, cap=0.0, scale=0.0, dq=1024, dk=1024,
+                dv=1024, ws=1024, ws_bytes=None)
+    args.update(kw)
+    if args["ws_bytes"] is None:
+        args["ws_bytes"] = fa.fa_bwd_workspace_bytes(args["B"], args["H"], args["L"])
+    vp = ctypes.c_void_p
+    c = vp(args["cols"])
+    return fa.fa_flex_attention_bwd(vp(args["q"]), vp(args["k"]), vp(args["v"]), vp(args["out"]),
+                                    vp(args["dout"]), vp(args["lse"]), args["dtype"], args["B"],
+                                    args["H"], args["Hkv"], args["L"], args["S"], args["D"],
+                                    ctypes.byref(bm) if bm is not None else None, c, c, c, c,
+                                    args["sk"], args["cap"], args["scale"], vp(args["dq"]),
+                                    vp(args["dk"]), vp(args["dv"]), vp(args["ws"]),
+                                    args["ws_bytes"], vp(0))
+
+
+def test_bwd_rejects_bad_arguments_on_host(fa):
+    """Every case below is refused before any CUDA call (the pointers are fake)."""
+    bm = fa.fa_block_mask()
+    bm.q_len, bm.kv_len, bm.block, bm.n_q_blocks, bm.n_kv_blocks = 256, 256, 128, 2, 2
+    bm.kv_num_blocks = bm.full_kv_num_blocks = bm.q_order = 4096
+    bm.kv_indices = bm.full_kv_indices = 4096
+    E, U = fa.FA_ERR_INVALID_ARG, fa.FA_ERR_UNSUPPORTED
+    assert fa.fa_bwd_workspace_bytes(1, 2, 256) >= 2 * 256 * 4
+    assert _bwd(fa, None) == E
+    assert _bwd(fa, bm, dtype=5) == E
+    assert _bwd(fa, bm, Hkv=3) == E                 # H not a multiple of H_kv
+    assert _bwd(fa, bm, Hkv=0) == E
+    assert _bwd(fa, bm, L=128) == E                 # L != mask q_len
+    assert _bwd(fa, bm, S=512) == E                 # S != mask kv_len
+    assert _bwd(fa, bm, sk=1, cap=0.0) == E
+    assert _bwd(fa, bm, sk=2) == E
+    assert _bwd(fa, bm, scale=float("inf")) == E
+    assert _bwd(fa, bm, D=32) == U
+    assert _bwd(fa, bm, ws=0) == E
+    assert _bwd(fa, bm, ws_bytes=16) == E           # below fa_bwd_workspace_bytes
+    assert _bwd(fa, bm, dq=0) == E
+    assert _bwd(fa, bm, dv=0) == E
+    assert _bwd(fa, bm, cols=0) == E                # column lists missing
+    assert _bwd(fa, bm, dout=1026) == E             # not 4-byte aligned
+    bm_doc = fa.fa_block_mask()
+    ctypes.pointer(bm_doc)[0] = bm
+    bm_doc.kind = fa.FA_MASK_DOCUMENT_CAUSAL        # document ids missing
+    assert _bwd(fa, bm_doc) == E
+    bm_bh = fa.fa_block_mask()
+    ctypes.pointer(bm_bh)[0] = bm
+    bm_bh.mask_heads = 2                            # per-(b, h) tables
+    assert _bwd(fa, bm_bh) == U
+    # nothing to do: no query rows and no key rows
+    assert _bwd(fa, bm, B=0) == fa.FA_OK
+
+
 def test_workspace_size(fa):
     assert fa.fa_fwd_workspace_bytes() >= 4
 
