@@ -643,9 +643,12 @@ extern "C" fa_status fa_flex_attention_bwd(
     return FA_ERR_INVALID_ARG;
   if (bm->kind == FA_MASK_DOCUMENT_CAUSAL && bm->doc_id == nullptr) return FA_ERR_INVALID_ARG;
   if (bm->kind == FA_MASK_BITMAP && S > 0 && bm->bitmap == nullptr) return FA_ERR_INVALID_ARG;
-  auto misaligned = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) != 0; };
-  if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(out) || misaligned(dout) ||
-      misaligned(dq) || misaligned(dk) || misaligned(dv) || misaligned(workspace))
+  // q, k, v, dout are staged by 16-byte cp.async copies; the rest is accessed in
+  // 4-byte pairs / floats
+  auto off16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
+  auto off4 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) != 0; };
+  if (off16(q) || off16(k) || off16(v) || off16(dout) || off4(out) || off4(dq) || off4(dk) ||
+      off4(dv) || off4(workspace))
     return FA_ERR_INVALID_ARG;
 
   BwdParams prm{};

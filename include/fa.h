@@ -332,9 +332,12 @@ FA_API fa_status fa_flex_attention_decode(const void* q, const void* k, const vo
  *   dq        device (B, H, L, D);  dk, dv  device (B, H_kv, S, D);  in dtype.
  *   workspace device, at least fa_bwd_workspace_bytes(B, H, L) bytes (row sums of
  *             dO * O; no initial contents needed).
- * Pointers 4-byte aligned; D 64 or 128; B * H * L and B * H_kv * S at most 2^33
- * (else FA_ERR_UNSUPPORTED).  Three kernels on `stream` (row sums, dQ per query row,
- * dK and dV per key row over the column lists; no atomics).  Returns
+ * q, k, v, dout 16-byte aligned, the other pointers 4-byte aligned (else
+ * FA_ERR_INVALID_ARG); D 64 or 128; B * H * L and B * H_kv * S at most 2^33
+ * (else FA_ERR_UNSUPPORTED).  Three kernels on `stream`: row sums of dO * O; dQ per
+ * 128-query tile over its row lists; dK and dV per 128-key tile over its column lists
+ * and the query heads sharing its K/V head (each output tile has one owner: no
+ * atomics, deterministic).  Returns
  * FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED (nothing launched) or FA_ERR_CUDA.
  */
 FA_API size_t fa_bwd_workspace_bytes(int32_t B, int32_t H, int32_t L);

@@ -257,6 +257,8 @@ def test_bwd_rejects_bad_arguments_on_host(fa):
     assert _bwd(fa, bm, dv=0) == E
     assert _bwd(fa, bm, cols=0) == E                # column lists missing
     assert _bwd(fa, bm, dout=1026) == E             # not 4-byte aligned
+    assert _bwd(fa, bm, q=1028) == E                # 4- but not 16-byte aligned (cp.async source)
+    assert _bwd(fa, bm, k=1032) == E
     bm_doc = fa.fa_block_mask()
     ctypes.pointer(bm_doc)[0] = bm
     bm_doc.kind = fa.FA_MASK_DOCUMENT_CAUSAL        # document ids missing
