@@ -648,7 +648,11 @@ extern "C" fa_status fa_flex_attention_bwd(
   auto off16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
   auto off4 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) != 0; };
   if (off16(q) || off16(k) || off16(v) || off16(dout) || off4(out) || off4(dq) || off4(dk) ||
-      off4(dv) || off4(workspace))
+      off4(dv) || off4(workspace) || off4(lse))
+    return FA_ERR_INVALID_ARG;
+  if (off4(bm->kv_num_blocks) || off4(bm->full_kv_num_blocks) || off4(bm->kv_indices) ||
+      off4(bm->full_kv_indices) || off4(bm->q_order) || off4(bm->doc_id) || off4(bm->bitmap) ||
+      off4(q_num_blocks) || off4(q_indices) || off4(full_q_num_blocks) || off4(full_q_indices))
     return FA_ERR_INVALID_ARG;
 
   BwdParams prm{};

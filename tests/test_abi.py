@@ -259,6 +259,8 @@ def test_bwd_rejects_bad_arguments_on_host(fa):
     assert _bwd(fa, bm, dout=1026) == E             # not 4-byte aligned
     assert _bwd(fa, bm, q=1028) == E                # 4- but not 16-byte aligned (cp.async source)
     assert _bwd(fa, bm, k=1032) == E
+    assert _bwd(fa, bm, lse=1026) == E
+    assert _bwd(fa, bm, cols=4098) == E             # column lists not 4-byte aligned
     bm_doc = fa.fa_block_mask()
     ctypes.pointer(bm_doc)[0] = bm
     bm_doc.kind = fa.FA_MASK_DOCUMENT_CAUSAL        # document ids missing
