@@ -148,7 +148,8 @@ def work_figures(w: W.Workload):
     live = int(per_row.sum())
     flops = 4.0 * w.D * 128 * 128 * live * w.B * w.H
     esz = 2
-    bytes_ = (w.B * w.H * (w.L * w.D * esz * 2 + w.S * w.D * esz * 2 + w.L * 4)
+    bytes_ = (w.B * w.H * (w.L * w.D * esz * 2 + w.L * 4)           # Q, out, LSE
+              + w.B * w.n_kv_heads * w.S * w.D * esz * 2              # K, V once per K/V head
               + per_row.size * (3 + 2 * (-(-w.S // 128))) * 4)
     return {"live_blocks": live, "per_row": per_row, "flops": flops, "bytes": bytes_}
 
