@@ -57,3 +57,65 @@ def attention_head_backward(q, k, v, dout, kind, window=None, doc_id=None, score
     if return_probs:
         return dq, dk, dv, p, ds
     return dq, dk, dv
+
+
+def attention_head_backward_sampled(q, k, v, dout, kind, q_rows, k_rows, window=None,
+                                    doc_id=None, score_kind=0, softcap=0.0, scale=None,
+                                    bitmap=None, chunk=256):
+    """Exact gradients for a sample of one (batch, head) too large for the dense form:
+    dq of the query rows ``q_rows``, dk and dv of the key rows ``k_rows``.
+
+    Each query row's P, dP and dS depend on that row alone (against all keys), and a
+    key's dk, dv collect only the rows that see it.  So the rows evaluated are
+    q_rows and every query row that sees some key of k_rows, a chunk at a time, by
+    the formulas of attention_head_backward.
+
+    Returns a dict: dq (len(q_rows), D), dk and dv (len(k_rows), D) in the given
+    orders; rows, the evaluated query rows (ascending); p and ds (len(rows), S), P and
+    dS of those rows, for error bounds.
+    """
+    q, k, v, dout = (_as_f64(t) for t in (q, k, v, dout))
+    L, D = q.shape
+    S = k.shape[0]
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(D)
+    q_rows = np.asarray(q_rows, dtype=np.int64)
+    k_rows = np.asarray(k_rows, dtype=np.int64)
+    doc = None if doc_id is None else _as_f64(doc_id).astype(np.int64)
+
+    def allowed_of(r):
+        return masks.mask_rows(kind, r, S, window, doc, bitmap, q_len=L)
+
+    need = np.zeros(L, dtype=bool)
+    need[q_rows] = True
+    for c0 in range(0, L, 512):
+        r = np.arange(c0, min(L, c0 + 512))
+        need[r] |= allowed_of(r)[:, k_rows].any(axis=1)
+    rows = np.flatnonzero(need)
+
+    p_all = np.zeros((len(rows), S))
+    ds_all = np.zeros((len(rows), S))
+    dk = np.zeros((len(k_rows), D))
+    dv = np.zeros((len(k_rows), v.shape[1]))
+    for c0 in range(0, len(rows), chunk):
+        r = rows[c0:c0 + chunk]
+        t = (q[r] @ k.T) * scale
+        s = softcap * np.tanh(t / softcap) if score_kind == TANH_SOFTCAP else t
+        s = np.where(allowed_of(r), s, -np.inf)
+        m = s.max(axis=1, initial=-np.inf)
+        live = np.isfinite(m)
+        p = np.zeros_like(s)
+        p[live] = np.exp(s[live] - m[live, None])
+        p[live] /= p[live].sum(axis=1, keepdims=True)
+        out = p @ v
+        delta = (dout[r] * out).sum(axis=1, keepdims=True)
+        ds = p * (dout[r] @ v.T - delta)
+        if score_kind == TANH_SOFTCAP:
+            ds = ds * (1.0 - np.tanh(t / softcap) ** 2)
+        p_all[c0:c0 + len(r)] = p
+        ds_all[c0:c0 + len(r)] = ds
+        dk += ds[:, k_rows].T @ q[r] * scale
+        dv += p[:, k_rows].T @ dout[r]
+    pos = np.searchsorted(rows, q_rows)
+    dq = ds_all[pos] @ k * scale
+    return {"dq": dq, "dk": dk, "dv": dv, "rows": rows, "p": p_all, "ds": ds_all}

@@ -107,3 +107,46 @@ def test_backward_documents_and_bitmap():
 def test_backward_softcap_and_grouped_heads():
     _run(1, 4, 2, 256, 256, 128, torch.bfloat16, OM.CAUSAL, sk=1, cap=5.0, seed=8)
     _run(1, 4, 1, 300, 300, 64, torch.float16, OM.SLIDING_WINDOW_CAUSAL, window=64, seed=9)
+
+
+@pytest.mark.parametrize("name,heads,q_rows,k_rows", [
+    ("swa256_L32768_B1_H8_D64_bf16", (5,), [*range(0, 64), *range(20000, 20064)],
+     [*range(1000, 1064), *range(32704, 32768)]),
+    ("causal_L8192_B1_H8_D64_bf16", (0, 7), [*range(0, 64), *range(8128, 8192)],
+     [*range(8064, 8192)])])
+def test_backward_full_size_sampled(name, heads, q_rows, k_rows):
+    """The backward workloads bench.py --backward times, at full size and with its
+    inputs: all heads computed on the GPU in one call; sampled rows of dq and of
+    dk / dv against the oracle's sampled gradients, with the tolerance derived above
+    (its terms from the sampled rows of P and dS)."""
+    import block_sparse_attention_create_b200 as fa
+    w = W.BY_NAME[name]
+    q, k, v = W.make_qkv(w)
+    g = torch.Generator().manual_seed(w.seed + 1)
+    dout = torch.randn(q.shape, generator=g).to(q.dtype)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, dout))
+    bm = fa.create_block_mask(w.mask_kind, w.L, w.S, window=w.window)
+    out, lse = fa.flex_attention(qd, kd, vd, bm, return_lse=True)
+    dq, dk, dv = fa.flex_attention_backward(qd, kd, vd, out, dod, lse, bm)
+    torch.cuda.synchronize()
+    assert fa.last_device_error() == fa.FA_OK
+    kind = {W.MASK_CAUSAL: OM.CAUSAL, W.MASK_SLIDING_WINDOW_CAUSAL: OM.SLIDING_WINDOW_CAUSAL}[
+        w.mask_kind]
+    u = 2.0 ** -8 if q.dtype == torch.bfloat16 else 2.0 ** -11
+    scale = 1.0 / np.sqrt(w.D)
+    for h in heads:
+        res = OBW.attention_head_backward_sampled(q[0, h], k[0, h], v[0, h], dout[0, h], kind,
+                                                  q_rows, k_rows, window=w.window or None)
+        rows, p, ds = res["rows"], res["p"], res["ds"]
+        ka, va = (np.abs(t[0, h].double().numpy()) for t in (k, v))
+        qa, ga = (np.abs(t[0, h].double().numpy()[rows]) for t in (q, dout))
+        A = 2 * u * np.sqrt(((ga * (p @ va)) ** 2).sum(axis=1))
+        at = np.searchsorted(rows, q_rows)
+        dq_prop = (scale * A[at, None] * (p[at] @ ka)
+                   + 3 * u * scale * np.sqrt(ds[at] ** 2 @ ka ** 2))
+        pk, dsk = p[:, k_rows], ds[:, k_rows]
+        dk_prop = scale * (pk.T @ (A[:, None] * qa)) + 3 * u * scale * np.sqrt(dsk.T ** 2 @ qa ** 2)
+        dv_prop = 3 * u * np.sqrt(pk.T ** 2 @ ga ** 2)
+        _check_grad(dq[0, h].cpu()[q_rows], res["dq"], dq_prop, f"{name} dq h{h}")
+        _check_grad(dk[0, h].cpu()[k_rows], res["dk"], dk_prop, f"{name} dk h{h}")
+        _check_grad(dv[0, h].cpu()[k_rows], res["dv"], dv_prop, f"{name} dv h{h}")

@@ -570,3 +570,30 @@ def test_backward_grouped_heads_sum_over_the_group():
         dv += gv
     assert np.abs(dk - tk.grad.numpy()[0, 0]).max() < 1e-10
     assert np.abs(dv - tv.grad.numpy()[0, 0]).max() < 1e-10
+
+
+@pytest.mark.parametrize("kind,w,sk", [(OM.CAUSAL, None, 0), (OM.SLIDING_WINDOW_CAUSAL, 37, 0),
+                                       (OM.DOCUMENT_CAUSAL, None, 1), (OM.BITMAP, None, 0)])
+def test_backward_sampled_rows_equal_the_dense_gradients(kind, w, sk):
+    """The sampled form gives the dense form's rows of dq, dk, dv, P and dS, for
+    scattered query and key samples (the dense form is pinned to torch autograd)."""
+    L, S, D = 300, 260, 16
+    doc = np.random.default_rng(5).integers(0, 4, size=max(L, S)) \
+        if kind == OM.DOCUMENT_CAUSAL else None
+    words = W.random_bitmap(L, S, seed=9) if kind == OM.BITMAP else None
+    q, k, v, do = (_rand(shape, s) for shape, s in (((L, D), 31), ((S, D), 32), ((S, D), 33),
+                                                    ((L, D), 34)))
+    args = dict(window=w, doc_id=doc, bitmap=words, score_kind=sk, softcap=4.0 if sk else 0.0)
+    dq, dk, dv, p, ds = OBW.attention_head_backward(q, k, v, do, kind, return_probs=True, **args)
+    g = np.random.default_rng(7)
+    q_rows = np.concatenate([[0, L - 1], g.choice(L, 20, replace=False)])
+    k_rows = np.concatenate([[S - 1, 0], g.choice(S, 20, replace=False)])
+    r = OBW.attention_head_backward_sampled(q, k, v, do, kind, q_rows, k_rows, chunk=64, **args)
+    assert np.abs(r["dq"] - dq[q_rows]).max() < 1e-12
+    assert np.abs(r["dk"] - dk[k_rows]).max() < 1e-12
+    assert np.abs(r["dv"] - dv[k_rows]).max() < 1e-12
+    assert np.abs(r["p"] - p[r["rows"]]).max() < 1e-13
+    assert np.abs(r["ds"] - ds[r["rows"]]).max() < 1e-12
+    # every row with a live pair on a sampled key was evaluated
+    sees = OM.mask_rows(kind, np.arange(L), S, w, doc, words, q_len=L)[:, k_rows].any(axis=1)
+    assert set(np.flatnonzero(sees)) <= set(r["rows"].tolist())
