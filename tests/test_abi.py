@@ -297,3 +297,21 @@ def test_product_never_imports_the_oracle():
         for f in files:
             if f.endswith(".py"):
                 assert not pat.search(open(os.path.join(dirpath, f)).read()), f
+
+
+def test_ops_refuse_host_tensors(fa):
+    """The torch-facing calls take device tensors only: host tensors are refused
+    before the library is called (no host computation path exists)."""
+    import torch
+    q = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 2, 128, dtype=torch.float32)
+    with pytest.raises(ValueError):
+        fa.flex_attention(q, q, q, None)
+    with pytest.raises(ValueError):
+        fa.flex_attention_noalloc(q, q, q, fa.FA_MASK_CAUSAL)
+    with pytest.raises(ValueError):
+        fa.flex_attention_decode(q, q, q)
+    with pytest.raises(ValueError):
+        fa.flex_attention_backward(q, q, q, q, q, lse, None)
+    with pytest.raises(ValueError):
+        fa.flex_attention(q.float(), q.float(), q.float(), None)   # fp32 inputs
