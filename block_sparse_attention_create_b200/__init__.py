@@ -1,8 +1,10 @@
-"""B200 (sm_100a) block-sparse attention: BlockMask builder and fused forward.
+"""B200 (sm_100a) block-sparse attention: BlockMask builders, fused forward,
+decode against a KV cache, and backward.
 
 The package exposes the C-ABI of libfa.so (include/fa.h) under the same names
-(``fa_create_block_mask``, ``fa_flex_attention_fwd``, ...) plus the thin torch
-conveniences ``create_block_mask`` / ``flex_attention``; see ``_binding``.
+(``fa_create_block_mask``, ``fa_flex_attention_fwd``, ``fa_flex_attention_bwd``,
+...) plus thin torch conveniences (``create_block_mask``, ``flex_attention``,
+``flex_attention_decode``, ``flex_attention_backward``, ...); see ``_binding``.
 
 The library is loaded on first use of any of those names.  There is no
 fallback: if libfa.so is missing, that first use raises ImportError.  Build the
