@@ -1,5 +1,6 @@
 """Backward pass on the GPU (dQ, dK, dV recomputed over the BlockMask from the
-forward's LSE) against the fp64 CPU oracle's gradients, element by element.
+forward's LSE) against the fp64 CPU oracle's gradients: element by element on
+small ragged shapes, and on sampled rows of the full-size benchmark workloads.
 
 Tolerance (derived).  Three sources of error:
   - fp32 accumulation and the 16-bit store of dq / dk / dv (unit roundoff u =
