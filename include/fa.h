@@ -329,7 +329,9 @@ FA_API fa_status fa_flex_attention_decode(const void* q, const void* k, const vo
  *   bm        the forward's tables (broadcast masks; per-(b, h) tables: FA_ERR_UNSUPPORTED).
  *   q_num_blocks, q_indices, full_q_num_blocks, full_q_indices
  *             the column lists of bm from fa_block_mask_transpose.
- *   dq        device (B, H, L, D);  dk, dv  device (B, H_kv, S, D);  in dtype.
+ *   dq        device (B, H, L, D);  dk, dv  device (B, H_kv, S, D);  in dtype, fully
+ *             overwritten.  With H_kv < H, dk and dv of a K/V head are the sums over
+ *             the H / H_kv query heads that read it (h / (H / H_kv) == kv head).
  *   workspace device, at least fa_bwd_workspace_bytes(B, H, L) bytes (row sums of
  *             dO * O; no initial contents needed).
  * q, k, v, dout 16-byte aligned, the other pointers 4-byte aligned (else
