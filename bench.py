@@ -292,11 +292,7 @@ def run_ours(args, w: W.Workload, rank, world, device):
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     fwd_ms = [m.elapsed_time(e) for m, e in zip(mids, ends)]
     mask_ms = [s.elapsed_time(m) for s, m in zip(starts, mids)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), device)
 
     # end to end through the public API: pinned host inputs in, results out
     e2e = ({"ms": float("nan"), "h2d": 0, "d2h": 0} if args.profile
@@ -341,11 +337,7 @@ def run_backward(args, w: W.Workload, world, device, fig):
         e1.record()
         torch.cuda.synchronize()
         ms.append(e0.elapsed_time(e1))
-    total = sum(ms)
-    if world > 1:
-        t = torch.tensor([total], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total = float(t.item())
+    total = max_over_ranks(sum(ms), device)
     flops = 2.5 * fig["flops"]
     peaks, _ = load_peaks()
     tflops = flops * args.steps * world / (total * 1e-3) / 1e12
@@ -400,11 +392,7 @@ def run_e2e(args, w, fa, q, k, v, doc, bits, device, world):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), device)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + (
         hdoc.numel() * 4 if hdoc is not None else 0) + (hbits.numel() * 4 if hbits is not None else 0)
     d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
@@ -434,6 +422,61 @@ def oracle_sample(w: W.Workload, rows, fig):
     return dt, credited
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The maximum of a per-rank figure over all ranks (a time: the slowest rank
+    decides the job's time); the figure itself on one rank."""
+    if not torch.distributed.is_available() or not torch.distributed.is_initialized():
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launch_ranks(argv, n: int) -> int:
+    """Start this script as n ranks on this node (one process per GPU) through
+    torch.distributed.run, rendezvous on 127.0.0.1; returns the launcher's exit code."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={free_port()}",
+           os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def init_ranks(backend: str, local: int):
+    from datetime import timedelta
+    kw = {"timeout": timedelta(seconds=120)}
+    if backend == "nccl":
+        kw["device_id"] = torch.device("cuda", local)
+    torch.distributed.init_process_group(backend, **kw)
+
+
+def dry_run(args, rank, world):
+    """Launcher and timing check without a GPU (gloo, CPU): each rank "steps" for a
+    rank-dependent time; the job's time is the maximum over ranks, as in the real
+    bench, and rank 0 prints one JSON line."""
+    per_step = 0.01 * (rank + 1)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time.sleep(per_step)
+    ms = (time.perf_counter() - t0) * 1e3
+    gathered = [None] * world
+    if world > 1:
+        torch.distributed.all_gather_object(gathered, ms)
+    else:
+        gathered = [ms]
+    job_ms = max_over_ranks(ms, "cpu")
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "n_gpus": world, "steps": args.steps,
+                          "ms_per_step": job_ms / args.steps, "rank_ms": gathered,
+                          "value": world * args.steps / (job_ms * 1e-3), "unit": "steps/s"}))
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -460,11 +503,27 @@ def main():
     ap.add_argument("--profile", action="store_true",
                     help="short run for profilers: warm-up and timed steps only (no clock "
                          "window, no end-to-end leg, no CPU baseline); not a bench value")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="launcher and max-over-ranks timing check on CPU (gloo); no GPU")
     args = ap.parse_args()
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start the ranks here (the driver may start them itself)
+        sys.exit(launch_ranks(sys.argv[1:], args.gpus))
     w = W.BY_NAME[args.workload]
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but {world} ranks were launched")
+    if args.dry_run:
+        if world > 1:
+            init_ranks("gloo", local)
+        dry_run(args, rank, world)
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     peaks, peaks_src = load_peaks()
     fig = work_figures(w)
 
@@ -486,10 +545,15 @@ def main():
             tot_s += dt
             tot_f += fl
         value = tot_f / tot_s / 1e12
-        ms_step = fig["flops"] / (value * 1e12) * 1e3
         line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
-                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                # each step is a bounded sample of the workload (see cpu_baseline.sample):
+                # ms_per_step is the time those samples took; the whole workload at this
+                # rate would take ms_per_step_extrapolated
+                "ms_per_step": tot_s * 1e3 / args.steps,
+                "ms_per_step_extrapolated": fig["flops"] / (value * 1e12) * 1e3,
+                "sampled_s": tot_s,
+                "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": {**w.describe(), "parallelism": "none (host cores)"},
                 "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(),
@@ -497,15 +561,16 @@ def main():
                                  "sample": (f"all new queries of {min(w.H, 8)} heads of batch 0 per step"
                                             if is_decode(w) else
                                             f"{rows_per_step} random query rows of head (0,0) per "
-                                            "step") + "; ms_per_step extrapolates to the whole "
-                                                      "workload"},
+                                            "step") + "; ms_per_step is the sample's time, "
+                                                      "ms_per_step_extrapolated the whole "
+                                                      "workload's"},
                 "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
         return
 
     if world > 1:
-        torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local))
+        init_ranks("nccl", local)
     device = torch.device("cuda", local)
     if args.backward:
         run_backward(args, w, world, device, fig)

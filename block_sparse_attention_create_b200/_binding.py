@@ -40,7 +40,7 @@ EXPORTED = ("fa_block_mask_dims", "fa_create_block_mask", "fa_fwd_workspace_byte
             "fa_num_sms", "fa_flex_attention_fwd_noalloc", "fa_create_block_mask_bitmap",
             "fa_block_mask_transpose", "fa_flex_attention_fwd_gqa", "fa_decode_workspace_bytes",
             "fa_flex_attention_decode", "fa_debug_set_mma_stall", "fa_create_block_mask_bh",
-            "fa_bwd_workspace_bytes", "fa_flex_attention_bwd")
+            "fa_bwd_workspace_bytes", "fa_flex_attention_bwd", "fa_block_mask_validate")
 
 
 class fa_block_mask(ctypes.Structure):
@@ -113,6 +113,9 @@ def _load():
                                           ctypes.POINTER(fa_block_mask), vp, vp, vp, vp, i32, f32,
                                           f32, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.fa_flex_attention_bwd.restype = i32
+    lib.fa_block_mask_validate.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32,
+                                           ctypes.POINTER(ctypes.c_int64)]
+    lib.fa_block_mask_validate.restype = i32
     return lib
 
 
@@ -136,6 +139,7 @@ fa_debug_set_mma_stall = _lib.fa_debug_set_mma_stall
 fa_create_block_mask_bh = _lib.fa_create_block_mask_bh
 fa_bwd_workspace_bytes = _lib.fa_bwd_workspace_bytes
 fa_flex_attention_bwd = _lib.fa_flex_attention_bwd
+fa_block_mask_validate = _lib.fa_block_mask_validate
 
 
 class FAError(RuntimeError):
@@ -198,6 +202,12 @@ class BlockMask:
         return {k: getattr(self, k).cpu().numpy() for k in
                 ("kv_num_blocks", "kv_indices", "full_kv_num_blocks", "full_kv_indices", "q_order")}
 
+    def validate(self):
+        """fa_block_mask_validate on host copies of the tables (synchronises).
+        Returns (status, first offending instance * nQ + row or -1)."""
+        return validate_tables(self.tables(), self.n_q_blocks, self.n_kv_blocks,
+                               self.mask_batch * self.mask_heads)
+
     def transpose(self, stream: Optional[torch.cuda.Stream] = None):
         """fa_block_mask_transpose: per kv block, its partial / full q blocks (device
         tensors q_num_blocks [nKV], q_indices [nKV, nQ], full_q_num_blocks,
@@ -214,6 +224,19 @@ class BlockMask:
                                        _ptr(t["full_q_indices"]), _stream_handle(stream)),
                "fa_block_mask_transpose")
         return t
+
+
+def validate_tables(tables: dict, n_q_blocks: int, n_kv_blocks: int, instances: int = 1):
+    """fa_block_mask_validate on host (numpy) tables: keys kv_num_blocks, kv_indices,
+    full_kv_num_blocks, full_kv_indices, q_order (as BlockMask.tables() returns them).
+    Returns (status, first offending instance * nQ + row, or -1)."""
+    import numpy as np
+    arrs = [np.ascontiguousarray(tables[k], dtype=np.int32) for k in
+            ("kv_num_blocks", "kv_indices", "full_kv_num_blocks", "full_kv_indices", "q_order")]
+    bad = ctypes.c_int64(0)
+    st = fa_block_mask_validate(*(ctypes.c_void_p(a.ctypes.data) for a in arrs), n_q_blocks,
+                                n_kv_blocks, instances, ctypes.byref(bad))
+    return st, bad.value
 
 
 def create_block_mask(kind: int, q_len: int, kv_len: int, window: int = 0,
@@ -328,26 +351,58 @@ def flex_attention_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, ma
                            score_mod: int = FA_SCORE_NONE, softcap: float = 0.0,
                            scale: float = 0.0, out: Optional[torch.Tensor] = None,
                            lse: Optional[torch.Tensor] = None,
-                           device_error: Optional[torch.Tensor] = None,
+                           device_error: Optional[torch.Tensor] = None, check: bool = False,
                            stream: Optional[torch.cuda.Stream] = None):
     """fa_flex_attention_fwd_noalloc: mask build + forward with the library's static
-    scratch (no block tables or workspace from the caller).  `out`, `lse` and
-    `device_error` (int32[1], device) are the caller's; they are created here only
-    if not given.  Returns (out, lse)."""
+    scratch (no block tables or workspace from the caller).
+
+    q (B,H,L,D), k / v (B,H,S,D) share dtype and device.  `out` (B,H,L,D, q's dtype),
+    `lse` (B,H,L float32) and `device_error` (int32, at least one element) belong to
+    the caller; any that is not given is created here with torch (so this
+    convenience allocates; the C entry point itself does not).  The device error
+    word is copied into `device_error` in stream order: nonzero means a bounded
+    device wait gave up and the outputs are invalid.  With `check`, the stream is
+    synchronised and a nonzero word raises FAError(FA_ERR_TIMEOUT); without it,
+    the caller reads `device_error` when it likes.  Returns (out, lse)."""
+    # shapes and dtypes first, then devices (so each mistake gets its own message)
     if q.dtype not in _DTYPES or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("q, k, v must share dtype bf16 or fp16")
-    for t in (q, k, v):
-        if not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
-            raise ValueError("q, k, v must be contiguous 4-D CUDA tensors")
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D")
     B, H, L, D = q.shape
     S = k.shape[2]
+    if k.shape != (B, H, S, D) or v.shape != (B, H, S, D):
+        raise ValueError("k and v must be (B, H, S, D) with the q's B, H and D")
+    if mask_kind == FA_MASK_DOCUMENT_CAUSAL and (
+            doc_id is None or doc_id.dtype != torch.int32 or doc_id.numel() < max(L, S)):
+        raise ValueError("doc_id must be an int32 tensor of max(L, S) ids")
+    if out is not None and (out.shape != q.shape or out.dtype != q.dtype):
+        raise ValueError("out must have q's shape and dtype")
+    if lse is not None and (lse.shape != (B, H, L) or lse.dtype != torch.float32):
+        raise ValueError("lse must be a float32 (B, H, L) tensor")
+    if device_error is not None and (device_error.dtype != torch.int32
+                                     or device_error.numel() < 1):
+        raise ValueError("device_error must be an int32 tensor of at least one element")
+    given = [t for t in (q, k, v, doc_id, out, lse, device_error) if t is not None]
+    if any(not t.is_cuda or t.device != q.device or not t.is_contiguous() for t in given):
+        raise ValueError("every tensor must be a contiguous CUDA tensor on q's device")
     if out is None:
         out = torch.empty_like(q)
-    _check(fa_flex_attention_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], B, H, L, S,
-                                         D, mask_kind, window, _ptr(doc_id), score_mod,
-                                         float(softcap), float(scale), _ptr(out), _ptr(lse),
-                                         _ptr(device_error), _stream_handle(stream)),
-           "fa_flex_attention_fwd_noalloc")
+    if lse is None:
+        lse = torch.empty(B, H, L, dtype=torch.float32, device=q.device)
+    if device_error is None:
+        device_error = torch.zeros(1, dtype=torch.int32, device=q.device)
+    # the scratch is the current device's: make q's device current for the call
+    with torch.cuda.device(q.device):
+        _check(fa_flex_attention_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _DTYPES[q.dtype], B, H, L,
+                                             S, D, mask_kind, window, _ptr(doc_id), score_mod,
+                                             float(softcap), float(scale), _ptr(out), _ptr(lse),
+                                             _ptr(device_error), _stream_handle(stream)),
+               "fa_flex_attention_fwd_noalloc")
+        if check:
+            (stream if stream is not None else torch.cuda.current_stream()).synchronize()
+            if int(device_error.reshape(-1)[0].item()) != 0:
+                raise FAError(FA_ERR_TIMEOUT, "fa_flex_attention_fwd_noalloc")
     return out, lse
 
 

@@ -14,7 +14,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libfa.so")
-SOURCES = ["api.cu", "blockmask.cu", "tmap.cu", "fwd_sm100.cu", "fwd_noalloc.cu", "decode.cu", "bwd.cu"]
+SOURCES = ["api.cu", "blockmask.cu", "tmap.cu", "fwd_sm100.cu", "fwd_noalloc.cu", "decode.cu", "bwd.cu", "validate.cu"]
 HEADERS = ["fa_internal.h", "sm100_ptx.cuh"]
 
 NVCC_FLAGS = [

@@ -13,6 +13,7 @@
 // The array is fixed at FA_NOALLOC_SCRATCH_BYTES per device; problems whose tables
 // do not fit are rejected before anything is launched.  Every call on a device
 // uses the same array, so calls whose GPU work overlaps race on it.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -51,19 +52,56 @@ ScratchLayout scratch_layout(int32_t nq, int32_t nkv) {
   return l;
 }
 
-// Device address of the scratch on the current device: looked up once per device,
-// with that device current, and cached.  nullptr if the lookup fails.
+// Identity of the CUDA context current on this thread (0 if none or if the driver
+// entry points are unavailable): a cudaDeviceReset replaces the device's primary
+// context, and the module -- with the scratch array -- is loaded again in the new
+// one, possibly at another address.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+      get_id = reinterpret_cast<CtxGetIdFn>(b);
+    }
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of the scratch on the current device.  The set-up -- the
+// cudaGetSymbolAddress lookup, which on the first call in a context also loads
+// this file's device module and so reserves the array -- runs once per device and
+// context, with that device current; later calls read the cached address.
+// nullptr if the lookup fails.
 unsigned char* scratch_on_current_device() {
   static std::mutex mu;
   static unsigned char* addr[kMaxDevices] = {};
+  static unsigned long long ctx_of[kMaxDevices] = {};
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (addr[dev] == nullptr || ctx == 0 || ctx != ctx_of[dev]) {
     void* ptr = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
     if (e != cudaSuccess || ptr == nullptr) return nullptr;
     addr[dev] = static_cast<unsigned char*>(ptr);
+    ctx_of[dev] = current_context_id();  // the lookup made the context current if none was
   }
   return addr[dev];
 }

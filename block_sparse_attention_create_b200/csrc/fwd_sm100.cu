@@ -9,24 +9,27 @@
 // media.tcdigital.jp, "分割統治法（Tiling）によるSRAM活用"), so the L x S score
 // matrix never reaches HBM, and EMPTY blocks of the BlockMask are never touched.
 //
-// Kernel organisation (one persistent CTA per SM, 320 threads):
+// Kernel organisation (one persistent CTA per SM, 352 threads, 11 warps):
 //   warps 0-3   softmax warpgroup of slot 0     warps 4-7   softmax warpgroup of slot 1
-//   warp 8      TMA producer (one lane)         warp 9      tcgen05.mma issuer + TMEM owner
-// A "slot" owns one 128-row Q tile, an S/P region (128 TMEM columns) and an O
-// accumulator (D TMEM columns).  The two slots work on independent work units
-// (batch*head, q-block) so that the tensor core computes one slot's S = Q K^T and
-// O += P V while the other slot's softmax runs.  K and V tiles stream through a
-// shared ring of shared-memory stages filled by TMA (128-byte swizzle, no multicast).
+//   warp 8      TMA producer of slot 0          warp 9      TMA producer of slot 1
+//   warp 10     tcgen05.mma issuer of both slots and TMEM owner
+// A "slot" owns one 128-row Q tile at a time, an S region and a P region in TMEM and
+// an O accumulator (D TMEM columns).  The two slots work on independent work units
+// (batch*head, q-block) so that the tensor core computes one slot's products while
+// the other slot's softmax runs.  Each slot streams its own K and V tiles through
+// shared-memory rings filled by TMA (128-byte swizzle, no multicast).  The MMA warp
+// polls both slots and issues whichever product is ready.
 //
-// Per block j of a unit, in the order the MMA warp issues them:
+// Per block j of a unit:
 //   S_j  = Q K_j^T        (SS MMA, M=128 N=128 K=D, fp32 in TMEM)    -> s_full
 //   softmax warpgroup: S -> registers, scale (+ softcap), mask on PARTIAL blocks only,
-//   running max with deferred rescaling of O, P = exp2(x - m) as bf16/fp16 written
-//   back into the S columns                                           -> p_full
-//   O   += P V_j          (TS MMA: A = P from TMEM, B = V MN-major)   -> (next S_j+1)
-// Because tcgen05 operations of one thread complete in issue order and S_{j+1} is
-// issued after PV_j, the commit that signals S_{j+1} also guarantees PV_j is done:
-// the softmax may rescale O in TMEM right after it sees S_{j+1}.
+//   running max with rescaling of O, P = exp2(x - m) as 16-bit values   -> p_full
+//   O   += P V_j          (TS MMA: A = P from TMEM, B = V MN-major)
+// D = 64: P has its own TMEM columns, so S_{j+1} is computed during softmax j and the
+// softmax waits for PV_{j-1} (pv_done) only before it overwrites P.  D = 128: P
+// overwrites the S it came from (TMEM holds no more), S_{j+1} is issued after PV_j
+// (tcgen05 operations of one thread run in issue order), and the commit that
+// signals S_{j+1} also means PV_j is done.
 //
 // Every mbarrier wait is bounded: after `timeout_ns` the waiting warp sets an abort
 // flag and the device error word, all roles stop, in-flight copies and MMAs are
@@ -51,10 +54,10 @@ constexpr int kNumSlots = 2;
 constexpr int kSoftmaxWarps = 4 * kNumSlots;
 constexpr int kProducerWarp = kSoftmaxWarps;      // + slot: one TMA producer warp per slot
 constexpr int kMmaWarp = kSoftmaxWarps + kNumSlots;
-constexpr int kThreads = (kSoftmaxWarps + 4) * 32;  // + one warpgroup: 2 producers, MMA, 1 spare
-// Every warp keeps the launch count of 168 registers (384 threads x 168 = 64512).
-// No setmaxnreg split: the softmax code fits in 168 without spills, and with a
-// split ptxas spilled in the narrowed control region.
+constexpr int kThreads = (kSoftmaxWarps + kNumSlots + 1) * 32;  // + 2 producers, MMA
+// Registers: 168 per thread.  Warps are spread over the SM's four sub-partitions,
+// three per sub-partition here, and each sub-partition has a quarter of the
+// register file (16384): 3 x 32 x 168 fits, 3 x 32 x 176 does not.
 constexpr int kBlockN = 128;                 // rows of a Q tile / K,V tile
 constexpr int kChunkBytes = 128 * 128;       // one TMA box: 128 rows x 64 elems x 2 B
 constexpr float kLog2e = 1.4426950408889634f;
@@ -67,7 +70,6 @@ constexpr int kMaskBitmap = 2;
 __host__ __device__ constexpr int mask_family(int kind) {
   return kind == FA_MASK_DOCUMENT_CAUSAL ? kMaskDoc : (kind == FA_MASK_BITMAP ? kMaskBitmap : kMaskRange);
 }
-constexpr float kRescaleThreshold = 8.0f;    // log2 units: O is rescaled only when max grows > 2^8
 
 // TMEM layouts (512 columns, lanes = the 128 rows of a tile):
 //  D = 64  ("separate P"): S0 [0,128) S1 [128,256) P0 [256,320) P1 [320,384)
@@ -134,6 +136,10 @@ struct Params {
   int n_q, mask_b, mask_h, mask_heads, doc_len;
   int mask_kind, window, softcap_on, is_bf16;
   int split_p;       // P fed to the PV product as two 16-bit terms (hi + lo)
+  // Deferred rescale: the running max used for P (and O, l) moves only when the
+  // block max exceeds it by more than this (log2 units).  0: P always uses the
+  // exact running max, so each row's largest weight is exactly 1 in 16 bits.
+  float rescale_thr;
   float scale_log2;  // scale * log2(e)
   float cap_k;       // 2 * scale * log2(e) / c : exp2(s * cap_k) = e^(2 s scale / c)
   float cap_a;       // c * log2(e)
@@ -896,7 +902,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         const float m_new = fmaxf(m, mb);
         float alpha = 1.f;
         bool rescale_o = false;
-        if (m_new > m + kRescaleThreshold) {
+        if (m_new > m + p.rescale_thr) {
           if (m != -INFINITY) {
             alpha = ex2_approx(m - m_new);
             l *= alpha;
@@ -947,7 +953,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         // than 2^8; exact, because l and O always use the same max.
         float alpha = 1.f;
         bool rescale_o = false;
-        if (m_new > m + kRescaleThreshold) {
+        if (m_new > m + p.rescale_thr) {
           if (m != -INFINITY) {
             alpha = ex2_approx(m - m_new);
             l *= alpha;
@@ -1222,13 +1228,27 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, int32_t dtype, i
   if (BH64 * bm->n_q_blocks > INT32_MAX) return FA_ERR_UNSUPPORTED;
   if (q == nullptr || out == nullptr || (S > 0 && (k == nullptr || v == nullptr)))
     return FA_ERR_INVALID_ARG;
-  auto misaligned = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
-  if (misaligned(q) || misaligned(out) || (S > 0 && (misaligned(k) || misaligned(v))))
+  // Alignment of everything the kernel reads or writes, checked here so that a
+  // misaligned pointer is an argument error and never a device fault: Q, K, V, out
+  // (TMA tiles, 16-byte stores) 16 bytes; the schedule table (8-byte loads) and a
+  // tabulated mask (8-byte loads of word pairs) 8 bytes; block lists, document ids,
+  // LSE and the error word 4 bytes.
+  auto misaligned = [](const void* ptr, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0;
+  };
+  if (misaligned(q, 16) || misaligned(out, 16) || (S > 0 && (misaligned(k, 16) || misaligned(v, 16))))
     return FA_ERR_INVALID_ARG;
-  if (bm->kv_num_blocks == nullptr || bm->full_kv_num_blocks == nullptr || bm->q_order == nullptr)
+  if (misaligned(lse, 4) || misaligned(workspace, 4)) return FA_ERR_INVALID_ARG;
+  if (bm->kv_num_blocks == nullptr || bm->full_kv_num_blocks == nullptr || bm->q_order == nullptr ||
+      (bm->n_kv_blocks > 0 && (bm->kv_indices == nullptr || bm->full_kv_indices == nullptr)))
     return FA_ERR_INVALID_ARG;
-  if (bm->kind == FA_MASK_DOCUMENT_CAUSAL && bm->doc_id == nullptr) return FA_ERR_INVALID_ARG;
-  if (bm->kind == FA_MASK_BITMAP && S > 0 && bm->bitmap == nullptr) return FA_ERR_INVALID_ARG;
+  if (misaligned(bm->q_order, 8) || misaligned(bm->kv_indices, 4) ||
+      misaligned(bm->full_kv_indices, 4))
+    return FA_ERR_INVALID_ARG;
+  if (bm->kind == FA_MASK_DOCUMENT_CAUSAL && (bm->doc_id == nullptr || misaligned(bm->doc_id, 4)))
+    return FA_ERR_INVALID_ARG;
+  if (bm->kind == FA_MASK_BITMAP && S > 0 && (bm->bitmap == nullptr || misaligned(bm->bitmap, 8)))
+    return FA_ERR_INVALID_ARG;
   // per-(batch, head) masks: one instance per batch element and / or head (0 reads as 1)
   const int mb = bm->mask_batch > 1 ? bm->mask_batch : 1;
   const int mh = bm->mask_heads > 1 ? bm->mask_heads : 1;
@@ -1265,7 +1285,13 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, int32_t dtype, i
   prm.scale_log2 = sc * kLog2e;
   prm.cap_k = prm.softcap_on ? 2.f * sc * kLog2e / softcap : 0.f;
   prm.cap_a = prm.softcap_on ? softcap * kLog2e : 0.f;
-  prm.split_p = 1;
+  // bf16 P carries 8 significant bits; in a peaked row the largest weights set the
+  // error.  D = 64: P always uses the exact running max (threshold 0), so each
+  // row's largest weight is exactly 1.  D = 128 (P overwrites S, O rescales are
+  // kept rare): P is fed as hi + lo, ~16 bits.  fp16 P (11 significant bits) is fed
+  // as one term, with the deferred rescale.
+  prm.split_p = (dtype == FA_BF16 && D == 128) ? 1 : 0;
+  prm.rescale_thr = (dtype == FA_BF16 && D == 64) ? 0.f : 8.f;
   prm.timeout_ns = 2000000000ull;
   if (g_stall_mma.load()) {
     prm.stall_mma = 1;

@@ -31,7 +31,7 @@
  *    never live.
  *  - A query row with no live key returns out = 0 and lse = -inf (SDPA returns 0
  *    for such rows, SDPA tutorial section 4).
- *  - Device pointers passed to fa_flex_attention_fwd must be 16-byte aligned.
+ *  - Each call states the alignment its pointers need and checks it on the host.
  */
 #ifndef FA_H_
 #define FA_H_
@@ -203,6 +203,28 @@ FA_API fa_status fa_block_mask_transpose(const fa_block_mask* bm, int32_t* q_num
                                   int32_t* q_indices, int32_t* full_q_num_blocks,
                                   int32_t* full_q_indices, void* stream);
 
+/*
+ * Host-side check of block tables (no CUDA call), for tables that did not come
+ * from the builders above: the forward kernel trusts the tables it is given.  The
+ * layout is that of the FlexAttention BlockMask (FlexAttention vs SDPA on M1 Max,
+ * qiita kiarina, "役割とデータの流れ"): per q-block row, the PARTIAL and the FULL kv
+ * blocks.  All pointers are HOST arrays (copies of the device tables), for
+ * `instances` mask instances stored instance-major as fa_create_block_mask_bh
+ * writes them (1 for a broadcast mask).
+ * Checked per row: 0 <= partial, full <= 65535, partial + full <= nKV; each list's
+ * indices in [0, nKV), strictly ascending; no block in both lists; unused entries
+ * 0.  Per instance, q_order lists every row exactly once with its two counts, by
+ * descending live count, ties by ascending row.
+ * Returns FA_OK, or FA_ERR_INVALID_ARG for bad sizes / NULL arrays or tables that
+ * break a rule; then, if first_bad is not NULL, *first_bad = instance * nQ + row of
+ * the first offending row (-1 for a size or pointer error).
+ */
+FA_API fa_status fa_block_mask_validate(const int32_t* kv_num_blocks, const int32_t* kv_indices,
+                                        const int32_t* full_kv_num_blocks,
+                                        const int32_t* full_kv_indices, const int32_t* q_order,
+                                        int32_t n_q_blocks, int32_t n_kv_blocks,
+                                        int32_t instances, int64_t* first_bad);
+
 /* Bytes of the device workspace fa_flex_attention_fwd needs (a small constant).
  * The caller allocates it, ZEROES IT ONCE, and may then reuse it for every call on
  * one stream; calls that run concurrently must use distinct workspaces. */
@@ -222,10 +244,15 @@ FA_API size_t fa_fwd_workspace_bytes(void);
  *   lse       device (B, H, L) float32: natural-log softmax denominator
  *             m + ln(sum exp(s - m)); may be NULL.
  *   workspace device buffer of fa_fwd_workspace_bytes() bytes (see there).
+ * Alignment (checked on the host; a misaligned pointer returns FA_ERR_INVALID_ARG
+ * before any launch): q, k, v, out 16 bytes; bm->q_order and a tabulated mask's
+ * bitmap 8 bytes; bm->kv_indices, bm->full_kv_indices, doc_id, lse and workspace 4
+ * bytes.
  * The kernel is persistent (one CTA per SM) and processes (batch*head, q-block) work
- * units in the order of bm->q_order.  Returns FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED
- * (nothing launched) or FA_ERR_CUDA.  Device-side timeouts are reported by
- * fa_get_last_device_error.
+ * units in the order of bm->q_order.  It trusts the tables' contents: tables that
+ * did not come from the builders can be checked first with fa_block_mask_validate.
+ * Returns FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED (nothing launched) or FA_ERR_CUDA.
+ * Device-side timeouts are reported by fa_get_last_device_error.
  */
 FA_API fa_status fa_flex_attention_fwd(const void* q, const void* k, const void* v, int32_t dtype,
                                 int32_t B, int32_t H, int32_t L, int32_t S, int32_t D,
@@ -256,7 +283,15 @@ FA_API fa_status fa_flex_attention_fwd(const void* q, const void* k, const void*
  *
  * Every call on a device shares that one array: calls whose GPU work may overlap
  * (different streams, or several host threads) race on it and must be ordered by
- * the caller.  Returns FA_ERR_SCRATCH_TOO_SMALL (nothing launched) when the tables
+ * the caller.  The array keeps the last call's contents; each call clears the
+ * error word and rebuilds the tables before the forward reads them.
+ *
+ * Set-up: the first call on a device (and the first after a cudaDeviceReset, which
+ * replaces the device's context) looks up the array's device address with that
+ * device current; in that lookup the CUDA runtime loads the library's device
+ * module, which reserves the array's 4 MiB on the device.  Later calls read the
+ * cached address.  Make that first call before any stream capture and outside
+ * sections that must not wait on the device; after it, calls reserve nothing.  Returns FA_ERR_SCRATCH_TOO_SMALL (nothing launched) when the tables
  * of an (L, S) problem do not fit, the argument errors of the two calls above
  * (nothing launched), or FA_ERR_CUDA.
  */

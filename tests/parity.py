@@ -108,4 +108,7 @@ def check_workload(w: W.Workload, heads=None, rows=None, seed=0):
                                    w.softcap)
         results.append(compare(out[b, h][rows], lse[b, h][rows], o_ref, l_ref,
                                f"{w.name} b{b} h{h}"))
+    # elements above 2e-2 (allowed only where |ref| >= 8, see the module docstring)
+    print(f"{w.name}: max |err| {max(r['max'] for r in results):.3e}, "
+          f"elements over 2e-2: {sum(r['over_2e-2'] for r in results)}")
     return results

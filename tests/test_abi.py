@@ -315,3 +315,33 @@ def test_ops_refuse_host_tensors(fa):
         fa.flex_attention_backward(q, q, q, q, q, lse, None)
     with pytest.raises(ValueError):
         fa.flex_attention(q.float(), q.float(), q.float(), None)   # fp32 inputs
+
+
+def test_noalloc_binding_checks_shapes_before_the_call(fa):
+    """flex_attention_noalloc refuses mismatched K / V, a short or missing document
+    id tensor and wrongly shaped outputs, each with its own error, before anything
+    reaches the library (shape checks come before the device checks, so they run
+    here without a GPU)."""
+    import torch
+    q = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 2, 256, 64, dtype=torch.bfloat16)
+    cases = [
+        ((q, k[:, :1], k[:, :1], fa.FA_MASK_CAUSAL), {}, "k and v"),           # fewer heads
+        ((q, k[..., :32], k[..., :32], fa.FA_MASK_CAUSAL), {}, "k and v"),     # smaller D
+        ((q, k, k[:, :, :128], fa.FA_MASK_CAUSAL), {}, "k and v"),             # v shorter
+        ((q, k, k, fa.FA_MASK_DOCUMENT_CAUSAL), {}, "doc_id"),                  # no ids
+        ((q, k, k, fa.FA_MASK_DOCUMENT_CAUSAL),
+         {"doc_id": torch.zeros(200, dtype=torch.int32)}, "doc_id"),           # short ids
+        ((q, k, k, fa.FA_MASK_DOCUMENT_CAUSAL),
+         {"doc_id": torch.zeros(256, dtype=torch.int64)}, "doc_id"),           # wrong dtype
+        ((q, k, k, fa.FA_MASK_CAUSAL), {"lse": torch.zeros(1, 2, 64)}, "lse"),  # wrong shape
+        ((q, k, k, fa.FA_MASK_CAUSAL), {"lse": torch.zeros(1, 2, 128, dtype=torch.float64)}, "lse"),
+        ((q, k, k, fa.FA_MASK_CAUSAL), {"out": torch.zeros(1, 2, 128, 32, dtype=torch.bfloat16)},
+         "out"),
+        ((q, k, k, fa.FA_MASK_CAUSAL), {"device_error": torch.zeros(1, dtype=torch.int64)},
+         "device_error"),
+        ((q, k, k, fa.FA_MASK_CAUSAL), {}, "CUDA"),                             # host tensors
+    ]
+    for args, kw, what in cases:
+        with pytest.raises(ValueError, match=what):
+            fa.flex_attention_noalloc(*args, **kw)

@@ -55,3 +55,39 @@ def test_decode_pairs_match_lower_right_masks(kind, L, S, window):
                    mask_kind=kind, window=window)
     m = OM.mask_rows(kind, np.arange(L), S, window or None, q_len=L)
     np.testing.assert_array_equal(bench.decode_pairs_per_row(w), m.sum(axis=1))
+
+
+def test_replica_launcher_and_max_over_ranks_on_cpu():
+    """`bench.py --gpus 2` without an outer launcher starts two ranks itself
+    (torch.distributed.run, 127.0.0.1), they rendezvous over gloo, and the job's
+    time is the slowest rank's: rank 1 steps twice as long as rank 0, so the
+    reported time per step is rank 1's and n_gpus is the number of ranks."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                        "--dry-run", "--steps", "5"], capture_output=True, text=True, env=env,
+                       timeout=240)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout   # rank 0 alone prints
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and len(d["rank_ms"]) == 2
+    assert d["rank_ms"][1] > d["rank_ms"][0]
+    assert abs(d["ms_per_step"] * d["steps"] - max(d["rank_ms"])) < 1e-6
+    assert abs(d["value"] - 2 * 5 / (max(d["rank_ms"]) * 1e-3)) < 1e-6
+
+
+def test_ranks_must_match_gpus():
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                        "--dry-run"], capture_output=True, text=True, env=env, timeout=120)
+    assert r.returncode != 0 and "ranks were launched" in r.stderr

@@ -88,20 +88,16 @@ def test_softcap_and_custom_scale():
     _full_compare(q, k, v, 1, window=200, scale=0.3)
 
 
-def test_d64_bf16_p_rounding_bound():
-    """At D=64 P enters the PV product rounded to bf16 (8 significant bits), so each
-    weight carries a relative error up to 2^-8 and the output error is bounded by
-    2^-8 * max|v| plus half an output ulp; check that bound on x2-scaled inputs,
-    where 2e-2 can be exceeded."""
+def test_d64_bf16_peaked_rows_within_tolerance():
+    """x2-scaled bf16 inputs at D=64 with a large scale (|v| up to ~9, softmax rows
+    dominated by one or two keys): a weight near 1 rounded to bf16 alone would be
+    off by up to 2^-9 relative, i.e. ~0.018 at |v| ~ 9 before output rounding, so
+    this case needs the two-term (hi + lo) P of the bf16 path to meet the stated
+    2e-2 / 2e-3 / 1e-3 bar."""
     q, k, v = W.random_qkv(1, 2, 512, 512, 64, torch.bfloat16, seed=11, scale=2.0)
-    out, lse = run_gpu(q, k, v, 1, 200, None, 0, 0.0, 0.3)
-    vmax = float(v.abs().max())
-    for h in range(2):
-        o_ref, l_ref = oracle_rows(q, k, v, 0, h, np.arange(512), 1, 200, None, 0, 0.0, 0.3)
-        err = np.abs(out[0, h].double().numpy() - o_ref)
-        bound = 2.0 ** -8 * vmax + 0.5 * np.abs(o_ref) * 2.0 ** -7
-        assert (err <= bound + 1e-3).all(), float((err - bound).max())
-        assert np.abs(lse[0, h].double().numpy() - l_ref).max() <= 1e-3
+    _, _, res = _full_compare(q, k, v, 1, window=200, scale=0.3)
+    for r in res:
+        assert r["over_2e-2"] == 0, r
 
 
 def test_fully_masked_rows_zero_and_minus_inf():
