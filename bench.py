@@ -52,8 +52,8 @@ DECODE_SOURCES = ("block_sparse_attention_create_b200/csrc/decode.cu",
                   "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
 NCU_TRAFFIC = {
     "swa256_L32768_B1_H8_D64_bf16": {
-        "bytes": 101075200 + 5619968, "sources": FWD_SOURCES,
-        "sources_sha256": "dcce04ca28ee4428d1782a852a5e4ba4882a729f05555ee3ebf06baee1d4ef64",
+        "bytes": 101098240 + 6616320, "sources": FWD_SOURCES,
+        "sources_sha256": "b4d5c8550a2ec34f268b52cc24585e3158f08cd2d48a3e4e9d92c195358fc4ac",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_full.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
         "bytes": 1073943296 + 7651328, "sources": DECODE_SOURCES,

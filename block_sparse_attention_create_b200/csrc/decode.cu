@@ -477,9 +477,14 @@ extern "C" fa_status fa_flex_attention_decode(const void* q, const void* k, cons
     return FA_ERR_INVALID_ARG;
   if (q == nullptr || out == nullptr || (S > 0 && (k == nullptr || v == nullptr)))
     return FA_ERR_INVALID_ARG;
-  auto misaligned = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
-  if (misaligned(q) || misaligned(out) || misaligned(workspace) ||
-      (S > 0 && (misaligned(k) || misaligned(v))))
+  // Q, K, V (TMA tiles and 16-byte loads), out and the workspace: 16 bytes; LSE
+  // (4-byte stores): 4 bytes.  Checked here so that a misaligned pointer is an
+  // argument error, never a device fault.
+  auto misaligned = [](const void* ptr, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) != 0;
+  };
+  if (misaligned(q, 16) || misaligned(out, 16) || misaligned(workspace, 16) ||
+      (S > 0 && (misaligned(k, 16) || misaligned(v, 16))) || misaligned(lse, 4))
     return FA_ERR_INVALID_ARG;
 
   DecParams prm{};

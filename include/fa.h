@@ -330,7 +330,8 @@ FA_API fa_status fa_flex_attention_fwd_gqa(const void* q, const void* k, const v
  *   mask      fa_decode_mask; window W >= 1 for FA_DECODE_SLIDING_WINDOW
  *             (query i sees keys in (S - L + i - W, S - L + i]).
  *   score_kind, softcap, scale, dtype, D as for fa_flex_attention_fwd.
- *   out, lse  device (B, H, L, D) in dtype / (B, H, L) fp32 (lse may be NULL).
+ *   out, lse  device (B, H, L, D) in dtype, 16-byte aligned / (B, H, L) fp32, 4-byte
+ *             aligned (lse may be NULL).
  *   workspace device, at least fa_decode_workspace_bytes(B, H, H_kv, L, S, D) bytes,
  *             16-byte aligned; its first word is the device error word (zero it once;
  *             fa_get_last_device_error reads and clears it).  Calls that run

@@ -345,3 +345,66 @@ def test_noalloc_binding_checks_shapes_before_the_call(fa):
     for args, kw, what in cases:
         with pytest.raises(ValueError, match=what):
             fa.flex_attention_noalloc(*args, **kw)
+
+
+def _fake_mask(fa, nq=2, nkv=2, L=256, S=256, kind=0, base=0x10000000):
+    """A block-mask struct whose device pointers are never dereferenced on the host
+    (the calls below return on their argument checks before any CUDA call)."""
+    bm = fa.fa_block_mask()
+    bm.kv_num_blocks = base
+    bm.kv_indices = base + 0x1000
+    bm.full_kv_num_blocks = base + 0x2000
+    bm.full_kv_indices = base + 0x3000
+    bm.q_order = base + 0x4000
+    bm.q_len, bm.kv_len, bm.block, bm.n_q_blocks, bm.n_kv_blocks = L, S, 128, nq, nkv
+    bm.kind, bm.window = kind, 0
+    bm.doc_id = base + 0x5000 if kind == 2 else None
+    bm.bitmap = base + 0x6000 if kind == 3 else None
+    bm.mask_batch = bm.mask_heads = 1
+    return bm
+
+
+def test_forward_rejects_each_misaligned_pointer_before_any_launch(fa):
+    """Every pointer the forward kernel reads or writes is checked on the host:
+    Q, K, V, out 16 bytes; the schedule and a bitmap 8; block lists, document ids,
+    LSE and the workspace 4.  A misaligned one returns FA_ERR_INVALID_ARG; with
+    every pointer aligned the call gets past the checks (to a CUDA error here,
+    where there is no GPU)."""
+    A = 0x20000000
+    good = dict(q=A, k=A + 0x100000, v=A + 0x200000, out=A + 0x300000, lse=A + 0x400000,
+                ws=A + 0x500000)
+    vp = ctypes.c_void_p
+
+    def call(ptrs, bm):
+        return fa.fa_flex_attention_fwd(vp(ptrs["q"]), vp(ptrs["k"]), vp(ptrs["v"]), fa.FA_BF16,
+                                        1, 2, 256, 256, 64, ctypes.byref(bm), 0, 0.0, 0.0,
+                                        vp(ptrs["out"]), vp(ptrs["lse"]), vp(ptrs["ws"]), None)
+    for kind in (0, 2, 3):
+        assert call(good, _fake_mask(fa, kind=kind)) == fa.FA_ERR_CUDA
+    for name, off in (("q", 8), ("k", 4), ("v", 2), ("out", 8), ("lse", 2), ("ws", 1)):
+        bad = dict(good)
+        bad[name] += off
+        assert call(bad, _fake_mask(fa)) == fa.FA_ERR_INVALID_ARG, name
+    for field, off, kind in (("q_order", 4, 0), ("kv_indices", 2, 0), ("full_kv_indices", 1, 0),
+                             ("doc_id", 2, 2), ("bitmap", 4, 3)):
+        bm = _fake_mask(fa, kind=kind)
+        setattr(bm, field, getattr(bm, field) + off)
+        assert call(good, bm) == fa.FA_ERR_INVALID_ARG, field
+
+
+def test_decode_rejects_misaligned_pointers_before_any_launch(fa):
+    vp = ctypes.c_void_p
+    A = 0x20000000
+    need = int(fa.fa_decode_workspace_bytes(1, 4, 1, 1, 1024, 64))
+    good = dict(q=A, k=A + 0x100000, v=A + 0x200000, out=A + 0x300000, lse=A + 0x400000,
+                ws=A + 0x500000)
+
+    def call(p):
+        return fa.fa_flex_attention_decode(vp(p["q"]), vp(p["k"]), vp(p["v"]), fa.FA_BF16, 1, 4, 1,
+                                           1, 1024, 64, fa.FA_DECODE_CAUSAL, 0, 0, 0.0, 0.0,
+                                           vp(p["out"]), vp(p["lse"]), vp(p["ws"]), need, None)
+    assert call(good) == fa.FA_ERR_CUDA
+    for name, off in (("q", 8), ("k", 4), ("v", 2), ("out", 8), ("lse", 2), ("ws", 8)):
+        bad = dict(good)
+        bad[name] += off
+        assert call(bad) == fa.FA_ERR_INVALID_ARG, name
