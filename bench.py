@@ -43,18 +43,19 @@ PAGE_FWD_MS = {"swa256_L32768_B1_H8_D64_bf16": 75.27, "causal_L8192_B1_H8_D64_bf
                "swa1024_L8192_B1_H8_D64_bf16": 56.24, "swa4096_L8192_B1_H8_D64_bf16": 169.24}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one launch of the dominant kernel from an ncu capture,
-# per workload, with the hash of the kernel sources it was taken on: reported as
-# roofline.traffic only while the sources still hash to that value (null once the
-# kernel changed).
+# per workload, with the hash of the kernel's device code it was taken on (each .cu
+# file up to its "host side" marker, and the PTX helpers): reported as
+# roofline.traffic only while the device code still hashes to that value (null once
+# the kernel changed).
 FWD_SOURCES = ("block_sparse_attention_create_b200/csrc/fwd_sm100.cu",
                "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
 DECODE_SOURCES = ("block_sparse_attention_create_b200/csrc/decode.cu",
                   "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
 NCU_TRAFFIC = {
     "swa256_L32768_B1_H8_D64_bf16": {
-        "bytes": 101098240 + 6616320, "sources": FWD_SOURCES,
-        "sources_sha256": "b4d5c8550a2ec34f268b52cc24585e3158f08cd2d48a3e4e9d92c195358fc4ac",
-        "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_full.md"},
+        "bytes": 101097685 + 2582485, "sources": FWD_SOURCES,
+        "sources_sha256": "24dcbe326e4c71e45960251b4bd663ec11aeabefecacfde0809e516bb7658776",
+        "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_launches.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
         "bytes": 1073943296 + 7651328, "sources": DECODE_SOURCES,
         "sources_sha256": "7d84849a563dc019493219a78d36bc25086dc5688cd4c99eb537030c4bcbf4f0",
@@ -62,12 +63,20 @@ NCU_TRAFFIC = {
 }
 
 
+HOST_MARKER = b"// ---------------------------------------------------------------- host side"
+
+
 def kernel_sources_hash(sources):
+    """sha256 of the device code: each .cu source up to its host-side marker (the
+    whole file if it has none), and every header whole."""
     import hashlib
     h = hashlib.sha256()
     for rel in sources:
         with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+            data = f.read()
+        if rel.endswith(".cu") and HOST_MARKER in data:
+            data = data[:data.index(HOST_MARKER)]
+        h.update(data)
     return h.hexdigest()
 
 

@@ -1,7 +1,9 @@
-// Host-side entry points shared by both operations: status strings, device
-// queries and the device error word of the forward workspace.
+// Host-side entry points shared by the operations: status strings, device
+// queries, the device error word of the workspaces and the testing hook that
+// makes the kernels' bounded waits run out.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 
@@ -23,7 +25,24 @@ int num_sms_current_device() {
   return cache[dev];
 }
 
+namespace {
+// Testing hook for the bounded-wait failure path (fa_debug_set_mma_stall).
+std::atomic<int> g_stall{0};
+std::atomic<unsigned long long> g_stall_wait_limit_ns{2000000000ull};
+}  // namespace
+
+bool debug_stall(unsigned long long* wait_limit_ns) {
+  if (!g_stall.load()) return false;
+  *wait_limit_ns = g_stall_wait_limit_ns.load();
+  return true;
+}
+
 }  // namespace fa
+
+extern "C" void fa_debug_set_mma_stall(int32_t on, uint64_t wait_limit_ns) {
+  fa::g_stall_wait_limit_ns.store(wait_limit_ns > 0 ? wait_limit_ns : 2000000000ull);
+  fa::g_stall.store(on ? 1 : 0);
+}
 
 extern "C" const char* fa_status_string(int32_t status) {
   switch (status) {

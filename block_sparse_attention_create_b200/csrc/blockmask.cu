@@ -40,6 +40,9 @@ classify_rows_kernel(int kind, int window, const int32_t* __restrict__ doc_all,
                      int32_t* __restrict__ full_num, int32_t* __restrict__ full_idx) {
   extern __shared__ uint8_t cls[];
   __shared__ int q_doc_min, q_doc_max;
+  __shared__ int q_ids[kBlock];  // document masks: the ids of this q-block's rows
+  grid_dep_launch_dependents();  // programmatic dependent launch, see interval_tables_kernel
+  grid_dep_wait();
   const int i = blockIdx.x;
   const int64_t inst = blockIdx.y;
   const int n_q = gridDim.x;
@@ -102,7 +105,8 @@ classify_rows_kernel(int kind, int window, const int32_t* __restrict__ doc_all,
       cls[j] = live ? (full ? 2 : 1) : 0;
     }
   } else {
-    // value range of the ids of this q-block
+    // the ids of this q-block, and their value range
+    for (int64_t q = q0 + threadIdx.x; q <= q1; q += blockDim.x) q_ids[q - q0] = __ldg(doc + q);
     if (warp == 0) {
       int mn = INT32_MAX, mx = INT32_MIN;
       for (int64_t q = q0 + lane; q <= q1; q += 32) {
@@ -140,25 +144,23 @@ classify_rows_kernel(int kind, int window, const int32_t* __restrict__ doc_all,
         // below the diagonal, one id on both sides (and they overlap, so equal)
         c = (q_whole && k0 + kBlock <= kv_len) ? 2 : 1;
       } else {
-        // visit every pair: lane owns 4 query rows
-        bool any = false, all = true;
-        for (int r = 0; r < 4; ++r) {
-          const int64_t q = q0 + lane * 4 + r;
-          if (q >= q_len) {
-            all = false;
-            continue;
-          }
-          const int dq = __ldg(doc + q);
-          for (int cc = 0; cc < kBlock; ++cc) {
-            const int64_t kv = k0 + cc;
-            const bool ok = kv < kv_len && kv <= q && __ldg(doc + kv) == dq;
-            any |= ok;
-            all &= ok;
+        // Not FULL: that needs one id on both sides.  Live iff some key k has a query
+        // q >= k of its document: lane l takes keys k0 + l + 32 r and scans the
+        // block's query ids (staged in shared memory) from max(q0, k) up, stopping at
+        // the first match.
+        bool any = false;
+        for (int r = 0; r < 4 && !any; ++r) {
+          const int64_t kv = k0 + lane + 32 * r;
+          if (kv > k1) break;
+          const int dk = __ldg(doc + kv);
+          for (int64_t q = kv > q0 ? kv : q0; q <= q1; ++q) {
+            if (q_ids[q - q0] == dk) {
+              any = true;
+              break;
+            }
           }
         }
-        any = __any_sync(0xffffffffu, any);
-        all = __all_sync(0xffffffffu, all);
-        c = any ? (all ? 2 : 1) : 0;
+        c = __any_sync(0xffffffffu, any) ? 1 : 0;
       }
       if (lane == 0) cls[j] = c;
     }
@@ -198,6 +200,8 @@ __global__ void __launch_bounds__(kOrderThreads)
 order_rows_kernel(int n_q, int n_kv, int n_pow2, const int32_t* __restrict__ kv_num,
                   const int32_t* __restrict__ full_num, int32_t* __restrict__ sched) {
   extern __shared__ uint32_t keys[];
+  grid_dep_launch_dependents();
+  grid_dep_wait();  // the counts come from classify_rows_kernel
   // one CTA per mask instance
   kv_num += static_cast<int64_t>(blockIdx.x) * n_q;
   full_num += static_cast<int64_t>(blockIdx.x) * n_q;
@@ -243,6 +247,106 @@ order_rows_kernel(int n_q, int n_kv, int n_pow2, const int32_t* __restrict__ kv_
     const int row = static_cast<int>(keys[t] & 0x1FFFu);
     sched[2 * t] = row;
     sched[2 * t + 1] = kv_num[row] | (full_num[row] << 16);
+  }
+}
+
+// Causal and sliding-window masks in one launch.  Their live kv blocks of row i form
+// one interval [lo, hi] and the FULL ones a sub-interval [flo, fhi]; so each row's
+// lists, counts and the schedule follow from closed forms with no classification
+// pass.  Row q-block i covers q in [q0, q1], kv block j covers [k0, k1] with
+// k0 = 128 j, k1 = min(128 j + 127, kv_len - 1):
+//   live  iff k0 <= q1 (causal) and k1 >= q0 - W + 1 (window);
+//   full  iff both blocks are whole, k1 <= q0 (all pairs causal) and q1 - k0 < W.
+struct RowRanges {
+  int lo, hi, flo, fhi;  // live [lo, hi], full [flo, fhi]; empty when lo > hi / flo > fhi
+};
+
+__device__ __forceinline__ RowRanges interval_row(int kind, int window, int q_len, int kv_len,
+                                                  int n_kv, int i) {
+  RowRanges r{1, 0, 1, 0};
+  if (n_kv == 0) return r;
+  const int q0 = i * kBlock;
+  const int q1 = min(q_len, q0 + kBlock) - 1;
+  r.hi = min(q1 / kBlock, n_kv - 1);
+  r.lo = 0;
+  if (kind == FA_MASK_SLIDING_WINDOW_CAUSAL) {
+    const int64_t t = static_cast<int64_t>(q0) - window + 1;  // smallest key any row sees
+    if (t > kv_len - 1) return RowRanges{1, 0, 1, 0};
+    r.lo = t <= 0 ? 0 : static_cast<int>(t / kBlock);
+  }
+  if (q0 + kBlock <= q_len && q0 >= kBlock - 1) {
+    r.fhi = min((q0 - (kBlock - 1)) / kBlock, kv_len / kBlock - 1);
+    if (kind == FA_MASK_SLIDING_WINDOW_CAUSAL) {
+      const int64_t d = static_cast<int64_t>(q1) - window;
+      r.flo = d < 0 ? 0 : static_cast<int>(d / kBlock) + 1;
+    } else {
+      r.flo = 0;
+    }
+  }
+  return r;
+}
+
+__device__ __forceinline__ int live_count(const RowRanges& r) { return max(0, r.hi - r.lo + 1); }
+__device__ __forceinline__ int full_count(const RowRanges& r) { return max(0, r.fhi - r.flo + 1); }
+
+// CTA b builds rows b, b + gridDim.x, ...; every CTA first tabulates the live
+// count of all rows in shared memory, from which a row's rank in the schedule
+// (descending live count, ties by ascending row) is a count.  Mask instance
+// blockIdx.y gets its own copy (the rule does not depend on batch or head).
+__global__ void __launch_bounds__(kClassifyThreads)
+interval_tables_kernel(int kind, int window, int q_len, int kv_len, int n_q, int n_kv,
+                       int32_t* __restrict__ kv_num, int32_t* __restrict__ kv_idx,
+                       int32_t* __restrict__ full_num, int32_t* __restrict__ full_idx,
+                       int32_t* __restrict__ sched) {
+  extern __shared__ int32_t live_cnt[];
+  __shared__ int warp_sum[kClassifyThreads / 32];
+  // launched as a programmatic dependent: a kernel still running before this one may
+  // read the tables (a forward of the previous step)
+  grid_dep_launch_dependents();
+  grid_dep_wait();
+  {
+    const int64_t inst = blockIdx.y;
+    kv_num += inst * n_q;
+    full_num += inst * n_q;
+    kv_idx += inst * n_q * static_cast<int64_t>(n_kv);
+    full_idx += inst * n_q * static_cast<int64_t>(n_kv);
+    sched += inst * 2 * n_q;
+  }
+  for (int r = threadIdx.x; r < n_q; r += blockDim.x)
+    live_cnt[r] = live_count(interval_row(kind, window, q_len, kv_len, n_kv, r));
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int i = blockIdx.x; i < n_q; i += gridDim.x) {
+    const RowRanges rr = interval_row(kind, window, q_len, kv_len, n_kv, i);
+    const int nf = full_count(rr);
+    const int np = live_count(rr) - nf;
+    // partial blocks: [lo, flo) then (fhi, hi] around the full ones (or all of [lo, hi])
+    const int part_a = nf > 0 ? rr.flo - rr.lo : np;
+    const size_t row = static_cast<size_t>(i) * n_kv;
+    for (int e = threadIdx.x; e < n_kv; e += blockDim.x) {
+      kv_idx[row + e] = e < np ? (e < part_a ? rr.lo + e : rr.fhi + 1 + (e - part_a)) : 0;
+      full_idx[row + e] = e < nf ? rr.flo + e : 0;
+    }
+    // rank = rows with a larger live count + earlier rows with the same count
+    const int c = live_cnt[i];
+    int rank = 0;
+    for (int r = threadIdx.x; r < n_q; r += blockDim.x) {
+      const int cr = live_cnt[r];
+      rank += (cr > c || (cr == c && r < i)) ? 1 : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+    if (lane == 0) warp_sum[warp] = rank;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int total = 0;
+      for (int w = 0; w < kClassifyThreads / 32; ++w) total += warp_sum[w];
+      kv_num[i] = np;
+      full_num[i] = nf;
+      sched[2 * total] = i;
+      sched[2 * total + 1] = np | (nf << 16);
+    }
+    __syncthreads();
   }
 }
 
@@ -343,16 +447,26 @@ fa_status build_tables(int32_t kind, int32_t window, const int32_t* doc_id, cons
 
   const int inst = mask_batch * mask_heads;
   cudaStream_t s = as_stream(stream);
-  classify_rows_kernel<<<dim3(nq, inst), kClassifyThreads, nkv > 0 ? nkv : 1, s>>>(
-      kind, bm->window, bm->doc_id, bm->bitmap, q_len, kv_len, nkv, bm->kv_num_blocks,
-      bm->kv_indices, bm->full_kv_num_blocks, bm->full_kv_indices);
-  FA_CUDA_CHECK(cudaGetLastError());
+  if (kind == FA_MASK_CAUSAL || kind == FA_MASK_SLIDING_WINDOW_CAUSAL) {
+    // closed forms: lists, counts and schedule in one launch
+    const int sms = num_sms_current_device();
+    if (sms <= 0) return FA_ERR_CUDA;
+    const int grid = nq < 2 * sms ? nq : 2 * sms;
+    FA_CUDA_CHECK(launch_pdl(interval_tables_kernel, dim3(grid, inst), dim3(kClassifyThreads),
+                             nq * sizeof(int32_t), s, kind, bm->window, q_len, kv_len, nq, nkv,
+                             bm->kv_num_blocks, bm->kv_indices, bm->full_kv_num_blocks,
+                             bm->full_kv_indices, bm->q_order));
+    return FA_OK;
+  }
+  FA_CUDA_CHECK(launch_pdl(classify_rows_kernel, dim3(nq, inst), dim3(kClassifyThreads),
+                           static_cast<size_t>(nkv > 0 ? nkv : 1), s, kind, bm->window, bm->doc_id,
+                           bm->bitmap, q_len, kv_len, nkv, bm->kv_num_blocks, bm->kv_indices,
+                           bm->full_kv_num_blocks, bm->full_kv_indices));
   int n_pow2 = 1;
   while (n_pow2 < nq) n_pow2 <<= 1;
   const size_t order_smem = (nq <= 2048 ? nq : n_pow2) * sizeof(uint32_t);
-  order_rows_kernel<<<inst, kOrderThreads, order_smem, s>>>(
-      nq, nkv, n_pow2, bm->kv_num_blocks, bm->full_kv_num_blocks, bm->q_order);
-  FA_CUDA_CHECK(cudaGetLastError());
+  FA_CUDA_CHECK(launch_pdl(order_rows_kernel, dim3(inst), dim3(kOrderThreads), order_smem, s, nq,
+                           nkv, n_pow2, bm->kv_num_blocks, bm->full_kv_num_blocks, bm->q_order));
   return FA_OK;
 }
 

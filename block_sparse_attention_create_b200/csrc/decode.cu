@@ -53,6 +53,7 @@ struct DecParams {
   float cap_c;    // softcap c
   float cap_a;    // c * log2(e)
   unsigned long long timeout_ns;
+  int stall_loads;  // testing hook: no K/V tile is loaded (see fa_debug_set_mma_stall)
 };
 
 template <int D, int RM>
@@ -174,7 +175,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
       tma_load_3d(sm.v[buf][c], &tv, &sm.full[buf], c * 64, k0, bkv, pol);
     }
   };
-  if (tid == 0 && ntiles > 0) issue(0);
+  if (tid == 0 && ntiles > 0 && !p.stall_loads) issue(0);
 
   const int oc = tid % kChunks, og = tid / kChunks;  // PV: 16-byte chunk, row group
   float o[kRowsPer][8];
@@ -187,7 +188,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
   for (; t < ntiles; ++t) {
     const int buf = t & 1;
     const int k0 = k_start + t * kTile;
-    if (tid == 0 && t + 1 < ntiles) issue(t + 1);  // its buffer was released after tile t - 1
+    // its buffer was released after tile t - 1
+    if (tid == 0 && t + 1 < ntiles && !p.stall_loads) issue(t + 1);
     const bool ok = dec_wait(sm, &sm.full[buf], (t >> 1) & 1, p);
     if (!__syncthreads_and(ok)) break;
 
@@ -310,8 +312,9 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
   }
 
   if (t < ntiles) {
-    // aborted: let the copies still in flight land (bounded) before the CTA exits
-    if (tid == 0) {
+    // aborted: let the copies still in flight (tiles t and t + 1) land, bounded,
+    // before the CTA exits
+    if (tid == 0 && !p.stall_loads) {
       const uint64_t t0 = globaltimer_ns();
       for (int u = t; u < min(ntiles, t + 2); ++u)
         while (!mbar_try_wait(&sm.full[u & 1], (u >> 1) & 1) &&
@@ -393,6 +396,7 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
   if (d == 0 && p.lse) p.lse[row] = l > 0.f ? (mx + log2f(l)) * kDecLn2 : -INFINITY;
 }
 
+// ---------------------------------------------------------------- host side
 // Chunking of the keys: about DecCfg::kCtasPerSm CTAs per SM over the (B * Hkv)
 // groups, whole tiles.
 void decode_plan(int B, int Hkv, int S, int D, int* nsplit, int* chunk) {
@@ -508,6 +512,7 @@ extern "C" fa_status fa_flex_attention_decode(const void* q, const void* k, cons
   prm.cap_c = prm.softcap_on ? softcap : 1.f;
   prm.cap_a = prm.softcap_on ? softcap * kDecLog2e : 0.f;
   prm.timeout_ns = 2000000000ull;
+  if (debug_stall(&prm.timeout_ns)) prm.stall_loads = 1;
   const cudaStream_t s = as_stream(stream);
   const bool b16 = dtype == FA_BF16;
   const int rows = G * L;

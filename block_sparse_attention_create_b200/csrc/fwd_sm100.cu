@@ -1122,6 +1122,10 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  // Launched as a programmatic dependent: everything above overlaps the end of the
+  // previous kernel on the stream (typically the block-mask build); nothing in
+  // global memory is read before this wait.
+  grid_dep_wait();
 
   // Role dispatch; the final rendezvous is a named barrier over all threads.
   if (warp < kSoftmaxWarps) {
@@ -1178,8 +1182,8 @@ fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH,
   if (sms <= 0) return FA_ERR_CUDA;
   const int want = (prm.num_units + kNumSlots - 1) / kNumSlots;
   const int grid = want < sms ? want : sms;
-  fwd_kernel<D, MK, BHM><<<grid, kThreads, smem, stream>>>(tq, tk, tv, prm);
-  FA_CUDA_CHECK(cudaGetLastError());
+  FA_CUDA_CHECK(launch_pdl(fwd_kernel<D, MK, BHM>, dim3(grid), dim3(kThreads), smem, stream, tq, tk,
+                           tv, prm));
   return FA_OK;
 }
 
@@ -1204,10 +1208,6 @@ fa_status launch_family(int kind, int D, const void* q, const void* k, const voi
     default: return launch<128, kMaskBitmap, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
   }
 }
-
-// Testing hook for the bounded-wait failure path (fa_debug_set_mma_stall).
-std::atomic<int> g_stall_mma{0};
-std::atomic<unsigned long long> g_stall_wait_limit_ns{2000000000ull};
 
 fa_status fwd_impl(const void* q, const void* k, const void* v, int32_t dtype, int32_t B, int32_t H,
                    int32_t Hkv, int32_t L, int32_t S, int32_t D, const fa_block_mask* bm,
@@ -1293,10 +1293,7 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, int32_t dtype, i
   prm.split_p = (dtype == FA_BF16 && D == 128) ? 1 : 0;
   prm.rescale_thr = (dtype == FA_BF16 && D == 64) ? 0.f : 8.f;
   prm.timeout_ns = 2000000000ull;
-  if (g_stall_mma.load()) {
-    prm.stall_mma = 1;
-    prm.timeout_ns = g_stall_wait_limit_ns.load();
-  }
+  if (debug_stall(&prm.timeout_ns)) prm.stall_mma = 1;
   const cudaStream_t s = as_stream(stream);
   const bool b16 = dtype == FA_BF16;
   if (prm.mask_b | prm.mask_h) return launch_family<true>(bm->kind, D, q, k, v, b16, L, S, prm, s);
@@ -1324,9 +1321,4 @@ extern "C" fa_status fa_flex_attention_fwd_gqa(const void* q, const void* k, con
                                                void* workspace, void* stream) {
   return fa::fwd_impl(q, k, v, dtype, B, H, H_kv, L, S, D, bm, score_kind, softcap, scale, out,
                       lse, workspace, stream);
-}
-
-extern "C" void fa_debug_set_mma_stall(int32_t on, uint64_t wait_limit_ns) {
-  fa::g_stall_wait_limit_ns.store(wait_limit_ns > 0 ? wait_limit_ns : 2000000000ull);
-  fa::g_stall_mma.store(on ? 1 : 0);
 }

@@ -390,11 +390,12 @@ FA_API fa_status fa_flex_attention_bwd(const void* q, const void* k, const void*
 
 /*
  * Testing hook for failure detection (no counterpart on the pages).  While `on`,
- * the forward kernel's MMA warp issues nothing, so the kernel's bounded waits run
- * out after `wait_limit_ns` (0: the default 2 s), the kernel stops every role,
- * drains its copies, frees TMEM and returns, and fa_get_last_device_error then
- * reports FA_ERR_TIMEOUT (the outputs of that call are invalid).  Nothing faults,
- * traps or hangs.  Process-wide; off by default.
+ * the forward kernel's MMA warp issues nothing and the decode kernel loads no K/V
+ * tile, so the kernels' bounded waits run out after `wait_limit_ns` (0: the
+ * default 2 s); each kernel stops, drains what it has in flight, frees TMEM and
+ * returns, and fa_get_last_device_error on that call's workspace then reports
+ * FA_ERR_TIMEOUT (the outputs of that call are invalid).  Nothing faults, traps or
+ * hangs.  Process-wide; off by default.
  */
 FA_API void fa_debug_set_mma_stall(int32_t on, uint64_t wait_limit_ns);
 

@@ -40,3 +40,38 @@ def test_bounded_waits_report_timeout_and_context_survives():
     for h in range(2):
         o_ref, l_ref = oracle_rows(q, k, v, 0, h, rows, OM.SLIDING_WINDOW_CAUSAL, 300)
         compare(out[0, h].cpu()[rows], lse[0, h].cpu()[rows], o_ref, l_ref, f"h{h}")
+
+
+def test_decode_bounded_waits_report_timeout_and_context_survives():
+    """The decode kernel's waits on its K/V tiles are bounded too: with the hook on,
+    no tile is loaded, every CTA's first wait runs out, the CTAs return, the host
+    reads FA_ERR_TIMEOUT from the decode workspace, and the next decode is correct."""
+    import block_sparse_attention_create_b200 as fa
+    B, H, Hkv, L, S, D = 2, 8, 2, 1, 4096, 128
+    g = torch.Generator().manual_seed(63)
+    q = torch.randn(B, H, L, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, Hkv, S, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, S, D, generator=g).to(torch.bfloat16)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    fa.flex_attention_decode(qd, kd, vd, mask=fa.FA_DECODE_CAUSAL)
+    torch.cuda.synchronize()
+    assert fa.last_decode_error() == fa.FA_OK
+    fa.fa_debug_set_mma_stall(1, 50_000_000)
+    try:
+        t0 = time.perf_counter()
+        fa.flex_attention_decode(qd, kd, vd, mask=fa.FA_DECODE_CAUSAL)
+        torch.cuda.synchronize()
+        elapsed = time.perf_counter() - t0
+    finally:
+        fa.fa_debug_set_mma_stall(0, 0)
+    assert fa.last_decode_error() == fa.FA_ERR_TIMEOUT
+    assert elapsed < 10.0
+    assert fa.last_decode_error() == fa.FA_OK
+    out, lse = fa.flex_attention_decode(qd, kd, vd, mask=fa.FA_DECODE_CAUSAL, return_lse=True)
+    torch.cuda.synchronize()
+    assert fa.last_decode_error() == fa.FA_OK
+    from oracle import attention as OA
+    for b, h in ((0, 0), (1, 7)):
+        o_ref, l_ref = OA.attention_head(q[b, h], k[b, h // (H // Hkv)], v[b, h // (H // Hkv)],
+                                         OM.DECODE_CAUSAL)
+        compare(out[b, h].cpu(), lse[b, h].cpu(), o_ref, l_ref, f"b{b} h{h}")

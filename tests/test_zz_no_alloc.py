@@ -86,3 +86,23 @@ def test_noalloc_equals_existing_entry_points_on_two_calls_in_a_row():
     for (o, l), (ro, rl) in zip(got, refs):
         assert torch.equal(o, ro)
         assert torch.equal(l, rl)
+
+
+@pytest.mark.gpu
+def test_noalloc_causal_at_the_scratch_limit():
+    """Causal masks, and a problem whose tables fill the scratch to its last block
+    (L = S = 723 * 128: 723 x 723 blocks), equal the existing entry points bit for
+    bit, twice in a row."""
+    fa = _fa()
+    L = 723 * 128
+    cases = [(*(t.cuda() for t in W.random_qkv(1, 3, 1500, 1500, 64, torch.bfloat16, seed=24)),),
+             (*(t.cuda() for t in W.random_qkv(1, 1, L, L, 64, torch.bfloat16, seed=25)),)]
+    err = torch.full((4,), -1, dtype=torch.int32, device="cuda")
+    for n, (q, k, v) in enumerate(cases):
+        ro, rl = _existing_path(fa, q, k, v, fa.FA_MASK_CAUSAL, 0, None, fa.FA_SCORE_NONE, 0.0)
+        for rep in range(2):
+            o, l = fa.flex_attention_noalloc(q, k, v, fa.FA_MASK_CAUSAL,
+                                             device_error=err[2 * n + rep:2 * n + rep + 1])
+            torch.cuda.synchronize()
+            assert torch.equal(o, ro) and torch.equal(l, rl), (n, rep)
+    assert err.tolist() == [0, 0, 0, 0]
