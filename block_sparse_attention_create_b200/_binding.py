@@ -456,9 +456,11 @@ def flex_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
                             dout: torch.Tensor, lse: torch.Tensor, block_mask: BlockMask,
                             score_mod: int = FA_SCORE_NONE, softcap: float = 0.0,
                             scale: float = 0.0, columns: Optional[dict] = None,
-                            stream: Optional[torch.cuda.Stream] = None):
+                            check: bool = False, stream: Optional[torch.cuda.Stream] = None):
     """fa_flex_attention_bwd: (dq, dk, dv) of the forward that produced out and lse.
-    `columns`: the mask's column lists (block_mask.transpose()); built here if None."""
+    `columns`: the mask's column lists (block_mask.transpose()); built here if None.
+    With `check`, the stream is synchronised and a bounded device wait that gave up
+    raises FAError(FA_ERR_TIMEOUT)."""
     for t in (q, k, v, out, dout):
         if not t.is_cuda or not t.is_contiguous() or t.dim() != 4 or t.dtype != q.dtype:
             raise ValueError("q, k, v, out, dout must be contiguous 4-D CUDA tensors of one dtype")
@@ -474,6 +476,7 @@ def flex_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     nbytes = int(fa_bwd_workspace_bytes(B, H, L))
     ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    ws[:256].zero_()  # the device error word
     _check(fa_flex_attention_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
                                  _DTYPES[q.dtype], B, H, Hkv, L, S, D,
                                  ctypes.byref(block_mask.struct), _ptr(cols["q_num_blocks"]),
@@ -482,6 +485,8 @@ def flex_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o
                                  float(scale), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws), ws.numel(),
                                  _stream_handle(stream)),
            "fa_flex_attention_bwd")
+    if check:
+        _check(fa_get_last_device_error(_ptr(ws), _stream_handle(stream)), "fa_flex_attention_bwd")
     return dq, dk, dv
 
 

@@ -9,33 +9,63 @@
 //   dK_j   = scale * sum_i dS_ij q_i,  dV_j = sum_i P_ij dO_i
 //                                            (kv-block columns: the column lists)
 //
-// Three kernels: delta (a warp per row); dQ, one CTA per 128-query tile in the
-// forward's schedule order; dK and dV, one CTA per 128-key tile over its column
-// lists and the query heads that share its K/V head.  Every output tile is owned by
-// one CTA (no atomics; dQ recomputes S and dP instead of accumulating into global
-// memory).  The products run on the tensor cores as warp-level mma.sync
-// m16n8k16 tiles (16-bit operands, fp32 accumulation) fed from shared memory by
-// cp.async double buffering; P and dS enter the second products rounded to the
-// input dtype, as in FlashAttention-2.
+// Three kernels: delta (a warp per row); dK and dV, one CTA per 128-key tile over
+// its column lists and the query heads that share its K/V head; dQ, one CTA per
+// 128-query tile over its row lists, in the forward's schedule order.  Every
+// output tile is owned by one CTA (no atomics, deterministic; dQ recomputes S and
+// dP instead of accumulating into global memory).
+//
+// Both gradient kernels have one shape: a stationary 128-row tile pair (dK/dV: K
+// and V; dQ: Q and dO) and 64-row sub-tiles of the other pair streamed through a
+// two-stage shared-memory ring by TMA.  Per sub-tile the products run on the 5th-
+// generation tensor cores with fp32 accumulators in Tensor Memory:
+//   X = A0 B0^T, Y = A1 B1^T     (SS MMAs, M = 128, N = 64, K = D)
+//     dK/dV: X = S^T = K Q^T, Y = dP^T = V dO^T;   dQ: X = S = Q K^T, Y = dP = dO V^T
+//   thread t of the compute warpgroup owns TMEM lane t (row t of the stationary
+//   tile): it turns its row of X and Y into P and dS, rounded to 16 bits and
+//   written back over X and Y, as the A operands of
+//   dK/dV: dV += P^T dO, dK += dS^T Q;   dQ: dQ += dS K
+//     (TS MMAs: A from TMEM, B the streamed tile read MN-major, accumulators in TMEM).
+// Warps 0-3 compute, warp 4 loads (TMA, and the row statistics the sub-tile needs),
+// warp 5 issues the MMAs and owns TMEM.  The next sub-tile's X and Y are issued
+// right after the current one's accumulating products by the same thread, so they
+// overwrite P and dS only after those products have read them (tcgen05 operations
+// of one thread run in issue order).  At D = 64 a CTA takes 256 TMEM columns and two
+// CTAs share an SM, so one CTA's MMAs overlap the other's elementwise work.
+//
+// Every mbarrier wait is bounded (2 s): on expiry the kernel sets the error word
+// (word 0 of the workspace), stops every role, drains its copies and MMAs, frees
+// TMEM and returns; fa_get_last_device_error reports FA_ERR_TIMEOUT.
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "fa_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace fa {
 namespace {
 
-constexpr int kBwdWarps = 8;
+constexpr int kBwdWarps = 8;  // delta kernel
 constexpr float kBwdLog2e = 1.4426950408889634f;
+constexpr int kSub = 64;                    // rows of a streamed sub-tile
+constexpr int kTcThreads = 192;             // warps 0-3 compute, 4 loads, 5 MMA
+constexpr int kLoadWarp = 4;
+constexpr int kIssueWarp = 5;
+constexpr int kModeDkdv = 0;
+constexpr int kModeDq = 1;
+constexpr int kBwdWorkspaceHeader = 256;  // word 0: device error flags, then delta
 
 struct BwdParams {
   const uint16_t *q, *k, *v, *out, *dout;
   const float* lse;
   float* delta;
+  int32_t* err;
   uint16_t *dq, *dk, *dv;
   const int32_t *kv_num, *kv_idx, *full_num, *full_idx;      // row lists
   const int32_t *q_num, *q_idx, *full_q_num, *full_q_idx;   // column lists
@@ -43,7 +73,12 @@ struct BwdParams {
   const int32_t* doc_id;
   const uint32_t* bitmap;
   int B, H, Hkv, G, L, S, n_q, n_kv, kind, window, softcap_on, is_bf16;
-  float scale, cap_c;
+  // per-(batch, head) masks: instance of (b, h) = (mask_b ? b : 0) * mask_heads +
+  // (mask_h ? h : 0), with its own lists, schedule, ids or bitmap rows
+  int mask_b, mask_h, mask_heads, doc_len;
+  float scale, scale_log2, cap_c, cap_k;
+  unsigned long long timeout_ns;
+  int stall;  // testing hook: nothing is loaded, the waits run out
 };
 
 __device__ __forceinline__ float2 load_pair(const uint16_t* ptr, bool bf16) {
@@ -52,45 +87,10 @@ __device__ __forceinline__ float2 load_pair(const uint16_t* ptr, bool bf16) {
   return __half22float2(*reinterpret_cast<const __half2*>(&u));
 }
 
-__device__ __forceinline__ void store_pair(uint16_t* ptr, float2 x, bool bf16) {
-  if (bf16) {
-    *reinterpret_cast<__nv_bfloat162*>(ptr) = __floats2bfloat162_rn(x.x, x.y);
-  } else {
-    *reinterpret_cast<__half2*>(ptr) = __floats2half2_rn(x.x, x.y);
-  }
-}
-
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
-}
-
-// The mask rule for (query i, key j) inside a PARTIAL block (FULL blocks skip it).
-__device__ __forceinline__ bool pair_live(const BwdParams& p, int i, int j) {
-  switch (p.kind) {
-    case FA_MASK_CAUSAL: return j <= i;
-    case FA_MASK_SLIDING_WINDOW_CAUSAL: return j <= i && i - j < p.window;
-    case FA_MASK_DOCUMENT_CAUSAL: return j <= i && __ldg(p.doc_id + i) == __ldg(p.doc_id + j);
-    default: {
-      const uint32_t w = __ldg(p.bitmap + static_cast<size_t>(i) * 4 * p.n_kv + (j >> 5));
-      return ((w >> (j & 31)) & 1u) != 0u;
-    }
-  }
-}
-
-// P and dS of one pair from the two dot products (natural-log LSE of the row).
-__device__ __forceinline__ void pair_grads(const BwdParams& p, float qk, float dov, float lse2,
-                                           float delta, float& pij, float& dsij) {
-  const float t = qk * p.scale;
-  float s = t, dcap = 1.f;
-  if (p.softcap_on) {
-    const float th = tanhf(t / p.cap_c);
-    s = p.cap_c * th;
-    dcap = 1.f - th * th;
-  }
-  pij = exp2f(s * kBwdLog2e - lse2);
-  dsij = pij * (dov - delta) * dcap;
 }
 
 // delta_i = rowsum(dO_i * O_i): one warp per row of (B * H * L).
@@ -111,488 +111,651 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_delta_kernel(const BwdPara
   if (lane == 0) p.delta[row] = acc;
 }
 
-// ---- tensor-core tiles (mma.sync m16n8k16, fp32 accumulate) ---------------------
-//
-// Fragment layouts (PTX ISA, "Matrix fragments for mma.m16n8k16"): lane = 4 g + t.
-// A 16x16 (row): {(g, 2t..2t+1), (g+8, 2t..), (g, 2t+8..), (g+8, 2t+8..)}.
-// B 16x8 (col):  {(k = 2t..2t+1, n = g), (k = 2t+8.., n = g)}.
-// C 16x8 fp32:   {(g, 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1)}.
-// Two adjacent C tiles of a 16-row product, rounded to 16 bits, are the A operand
-// of a 16-deep k step: how P and dS feed the second product without shared memory.
-// Shared-memory tiles are row-major with rows padded to D + 8 elements, so the
-// eight 16-byte rows of one ldmatrix land in eight different bank groups.
+// ---------------------------------------------------------------- tcgen05 kernels
+template <int D>
+struct TcCfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kStatBytes = 128 * D * 2;    // a stationary 128-row tile
+  static constexpr int kSubBytes = kSub * D * 2;    // a streamed 64-row tile
+  static constexpr int kStatChunk = 128 * 128;      // one 64-column box of 128 rows
+  static constexpr int kSubChunk = kSub * 128;      // one 64-column box of 64 rows
+  // TMEM: X [0, 64), Y [64, 128), accumulators from 128 (D columns each)
+  __host__ __device__ static constexpr uint32_t tmem_cols(int mode) {
+    return (128 + (mode == kModeDkdv ? 2 : 1) * D) <= 256 ? 256u : 512u;
+  }
+  static constexpr int kCtasPerSm = D == 64 ? 2 : 1;
+};
 
-__device__ __forceinline__ uint32_t smem_addr(const void* ptr) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
+template <int D>
+struct __align__(1024) TcSmem {
+  uint8_t stat[2][TcCfg<D>::kStatBytes];            // dK/dV: K, V;  dQ: Q, dO
+  uint8_t sub[2][2][TcCfg<D>::kSubBytes];           // [stage][operand] dK/dV: Q, dO; dQ: K, V
+  float lse2[2][kSub];                              // dK/dV: per streamed query row
+  float delta[2][kSub];
+  int32_t aux[2][kSub * 4];                         // partial blocks: ids or bitmap words
+  uint64_t stat_full;
+  uint64_t full[2], empty[2];
+  uint64_t x_full, comp_done, acc_full, drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+};
+
+// Mask instance of (batch, head).
+__device__ __forceinline__ int bwd_instance(const BwdParams& p, int64_t bh) {
+  const int64_t b = bh / p.H, h = bh - b * p.H;
+  return static_cast<int>((p.mask_b ? b : 0) * p.mask_heads + (p.mask_h ? h : 0));
 }
 
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
+// The sequence of 64-row sub-tiles one CTA streams.  dK/dV (CTA = key tile jb of K/V
+// head kvbh): for each query head of the group, each block of column jb's lists,
+// both halves of the q block.  dQ (CTA = query tile qb of head bh): each block of
+// row qb's lists, both halves of the kv block.  Every role walks the same sequence.
+template <int MODE>
+struct StepIter {
+  // fixed per CTA
+  int64_t tile_bh;  // dK/dV: kvbh; dQ: bh
+  int tile_blk;     // dK/dV: jb; dQ: qb
+  // current list
+  int g, np, nf, t, half;
+  int64_t list_base;
+  int inst;
+  // current step
+  int64_t bh;     // query head of the step (dK/dV) / of the tile (dQ)
+  int blk;        // dK/dV: q block; dQ: kv block
+  bool full;
+
+  __device__ __forceinline__ void open_list(const BwdParams& p) {
+    if constexpr (MODE == kModeDkdv) {
+      const int64_t b = tile_bh / p.Hkv, kvh = tile_bh - b * p.Hkv;
+      bh = b * p.H + kvh * p.G + g;
+      inst = bwd_instance(p, bh);
+      const int64_t col = static_cast<int64_t>(inst) * p.n_kv + tile_blk;
+      np = p.n_q > 0 ? __ldg(p.q_num + col) : 0;
+      nf = p.n_q > 0 ? __ldg(p.full_q_num + col) : 0;
+      list_base = col * p.n_q;
+    } else {
+      bh = tile_bh;
+      inst = bwd_instance(p, bh);
+      const int64_t row = static_cast<int64_t>(inst) * p.n_q + tile_blk;
+      np = p.n_kv > 0 ? __ldg(p.kv_num + row) : 0;
+      nf = p.n_kv > 0 ? __ldg(p.full_num + row) : 0;
+      list_base = row * p.n_kv;
+    }
+    t = 0;
+    half = 0;
+  }
+  __device__ __forceinline__ void init(const BwdParams& p, int64_t tbh, int tblk) {
+    tile_bh = tbh;
+    tile_blk = tblk;
+    g = 0;
+    open_list(p);
+  }
+  // Advance to the next step; false when the sequence is exhausted.
+  __device__ __forceinline__ bool next(const BwdParams& p) {
+    while (t >= np + nf) {
+      if (MODE == kModeDq || ++g >= p.G) return false;
+      open_list(p);
+    }
+    full = t >= np;
+    const int32_t* idx = MODE == kModeDkdv ? (full ? p.full_q_idx : p.q_idx)
+                                           : (full ? p.full_idx : p.kv_idx);
+    blk = __ldg(idx + list_base + (full ? t - np : t));
+    return true;
+  }
+  __device__ __forceinline__ int row0() const { return blk * 128 + half * kSub; }
+  __device__ __forceinline__ void step() {
+    if (++half == 2) {
+      half = 0;
+      ++t;
+    }
+  }
+};
+
+template <int D>
+__device__ __noinline__ bool tc_wait_slow(TcSmem<D>& sm, uint64_t* bar, uint32_t parity,
+                                          const BwdParams& p) {
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (sm.abort_flag) return false;
+    if (globaltimer_ns() - t0 > p.timeout_ns) {
+      sm.abort_flag = 1;
+      atomicOr(p.err, kDevErrTimeout);
+      return false;
+    }
+  }
+}
+template <int D>
+__device__ __forceinline__ bool tc_wait(TcSmem<D>& sm, uint64_t* bar, uint32_t parity,
+                                        const BwdParams& p) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return tc_wait_slow(sm, bar, parity, p);
+}
+// whole warp waits; the warp agrees on the outcome
+template <int D>
+__device__ __forceinline__ bool tc_wait_warp(TcSmem<D>& sm, uint64_t* bar, uint32_t parity,
+                                             const BwdParams& p) {
+  return __all_sync(0xffffffffu, tc_wait(sm, bar, parity, p));
+}
+// lane 0 waits, the warp gets the outcome
+template <int D>
+__device__ __forceinline__ bool tc_wait_lane0(TcSmem<D>& sm, uint64_t* bar, uint32_t parity,
+                                              const BwdParams& p) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = tc_wait(sm, bar, parity, p);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
+template <int D>
+__device__ __forceinline__ void tma_tile(const CUtensorMap* map, int row0, int64_t z, uint8_t* dst,
+                                         int chunk_bytes, uint64_t* bar, uint64_t pol) {
+#pragma unroll
+  for (int c = 0; c < TcCfg<D>::kChunks; ++c)
+    tma_load_3d(dst + c * chunk_bytes, map, bar, c * 64, row0, static_cast<int32_t>(z), pol);
 }
 
-template <bool BF>
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  if constexpr (BF) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-  } else {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
-        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+// Warp 4: the stationary tiles once, then per step the two streamed sub-tiles (TMA)
+// and what the compute warps need per streamed row: dK/dV the query rows' log2-scale
+// LSE and delta; PARTIAL blocks of document / tabulated masks the ids / words.
+template <int MODE, int D>
+__device__ void tc_load_role(TcSmem<D>& sm, const BwdParams& p, const CUtensorMap* ts0,
+                             const CUtensorMap* ts1, const CUtensorMap* tb0, const CUtensorMap* tb1,
+                             int64_t tile_bh, int tile_blk, int64_t stat_z) {
+  using C = TcCfg<D>;
+  const int lane = threadIdx.x & 31;
+  const uint64_t pol = policy_evict_last();
+  if (p.stall) return;  // testing hook: nothing is loaded
+  if (lane == 0) {
+    mbar_arrive_expect_tx(&sm.stat_full, 2 * C::kStatBytes);
+    tma_tile<D>(ts0, tile_blk * 128, stat_z, sm.stat[0], C::kStatChunk, &sm.stat_full, pol);
+    tma_tile<D>(ts1, tile_blk * 128, stat_z, sm.stat[1], C::kStatChunk, &sm.stat_full, pol);
+  }
+  StepIter<MODE> it;
+  it.init(p, tile_bh, tile_blk);
+  int s = 0;
+  bool ok = true;
+  for (; it.next(p); it.step(), ++s) {
+    const int st = s & 1;
+    if (!tc_wait_lane0(sm, &sm.empty[st], ((s >> 1) & 1) ^ 1, p)) {
+      ok = false;
+      break;
+    }
+    const int r0 = it.row0();
+    // the streamed rows: dK/dV query rows of head it.bh; dQ key rows of its K/V head
+    const int64_t kvbh = MODE == kModeDkdv ? tile_bh
+                                           : (it.bh / p.H) * p.Hkv + (it.bh % p.H) / p.G;
+    if constexpr (MODE == kModeDkdv) {
+      for (int r = lane; r < kSub; r += 32) {
+        const int i = r0 + r;
+        float l2 = INFINITY, dl = 0.f;  // rows past L, or with no live key: P = 0
+        if (i < p.L) {
+          const float l = __ldg(p.lse + it.bh * p.L + i);
+          if (l != -INFINITY) {
+            l2 = l * kBwdLog2e;
+            dl = p.delta[it.bh * p.L + i];
+          }
+        }
+        sm.lse2[st][r] = l2;
+        sm.delta[st][r] = dl;
+      }
+    }
+    if (!it.full && p.kind == FA_MASK_DOCUMENT_CAUSAL) {
+      // ids of the streamed rows (queries for dK/dV, keys for dQ) of this instance
+      const int32_t* docs = p.doc_id + static_cast<int64_t>(it.inst) * p.doc_len;
+      const int n = MODE == kModeDkdv ? p.L : p.S;
+      for (int r = lane; r < kSub; r += 32) sm.aux[st][r] = __ldg(docs + min(r0 + r, n - 1));
+    } else if (MODE == kModeDkdv && !it.full && p.kind == FA_MASK_BITMAP) {
+      // the 4 words of key tile tile_blk in each of the 64 query rows
+      const uint32_t* rows = p.bitmap + static_cast<int64_t>(it.inst) * p.L * 4 * p.n_kv;
+      for (int e = lane; e < kSub * 4; e += 32) {
+        const int i = min(r0 + e / 4, p.L - 1);
+        sm.aux[st][e] = static_cast<int32_t>(
+            __ldg(rows + static_cast<int64_t>(i) * 4 * p.n_kv + 4 * tile_blk + (e & 3)));
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sm.full[st], 2 * C::kSubBytes);
+      const int64_t z = MODE == kModeDkdv ? it.bh : kvbh;
+      tma_tile<D>(tb0, r0, z, sm.sub[st][0], C::kSubChunk, &sm.full[st], pol);
+      tma_tile<D>(tb1, r0, z, sm.sub[st][1], C::kSubChunk, &sm.full[st], pol);
+    }
+    __syncwarp();
+  }
+  if (!ok && lane == 0) {
+    // let the copies in flight land (bounded) before the CTA exits
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&sm.stat_full, 0) && globaltimer_ns() - t0 < p.timeout_ns) {
+    }
+    for (int u = s - 2; u < s; ++u) {
+      if (u < 0) continue;
+      while (!mbar_try_wait(&sm.full[u & 1], (u >> 1) & 1) && globaltimer_ns() - t0 < p.timeout_ns) {
+      }
+    }
   }
 }
 
-// Two floats as one 16-bit pair, the first in the low half.
-template <bool BF>
-__device__ __forceinline__ uint32_t pack16(float lo, float hi) {
-  if constexpr (BF) {
+// Warp 5: per step s, the accumulating products of step s - 1 (once its P / dS are
+// written), then X and Y of step s.
+template <int MODE, int D>
+__device__ void tc_issue_role(TcSmem<D>& sm, const BwdParams& p, uint32_t tmem, int64_t tile_bh,
+                              int tile_blk) {
+  using C = TcCfg<D>;
+  const bool bf16 = p.is_bf16 != 0;
+  const uint32_t id_x = idesc_f16_f32(bf16, 128, kSub, false);
+  const uint32_t id_acc = idesc_f16_f32(bf16, 128, D, true);
+  const uint32_t t_x = tmem, t_y = tmem + 64, t_acc0 = tmem + 128, t_acc1 = tmem + 128 + D;
+  StepIter<MODE> it;
+  it.init(p, tile_bh, tile_blk);
+  bool ok = tc_wait_lane0(sm, &sm.stat_full, 0, p);
+  int s = 0;
+  bool acc_started = false;
+  // the accumulating products of the step whose operands sit in stage st
+  auto issue_acc = [&](int st) {
+    if (elect_one_sync()) {
+#pragma unroll
+      for (int kk = 0; kk < kSub / 16; ++kk) {
+        const uint32_t acc = (acc_started || kk > 0) ? 1u : 0u;
+        if constexpr (MODE == kModeDkdv) {
+          // dV += P^T dO (B = dO sub-tile, MN-major), dK += dS^T Q (B = Q sub-tile)
+          const uint64_t bdo = sdesc_sw128(smem_u32(sm.sub[st][1]), C::kSubChunk, 1024);
+          const uint64_t bq = sdesc_sw128(smem_u32(sm.sub[st][0]), C::kSubChunk, 1024);
+          umma_ts(t_acc0, t_x + kk * 8, bdo + static_cast<uint64_t>(kk * 128), id_acc, acc);
+          umma_ts(t_acc1, t_y + kk * 8, bq + static_cast<uint64_t>(kk * 128), id_acc, acc);
+        } else {
+          // dQ += dS K (B = K sub-tile, MN-major)
+          const uint64_t bk = sdesc_sw128(smem_u32(sm.sub[st][0]), C::kSubChunk, 1024);
+          umma_ts(t_acc0, t_y + kk * 8, bk + static_cast<uint64_t>(kk * 128), id_acc, acc);
+        }
+      }
+      umma_commit(&sm.empty[st]);
+    }
+    __syncwarp();
+    acc_started = true;
+  };
+  for (; ok && it.next(p); it.step(), ++s) {
+    const int st = s & 1;
+    if (s > 0) {
+      ok = tc_wait_lane0(sm, &sm.comp_done, (s - 1) & 1, p);
+      if (!ok) break;
+      tc_fence_after();
+      issue_acc(st ^ 1);
+    }
+    ok = tc_wait_lane0(sm, &sm.full[st], (s >> 1) & 1, p);
+    if (!ok) break;
+    tc_fence_after();
+    if (elect_one_sync()) {
+      const uint64_t a0 = sdesc_sw128(smem_u32(sm.stat[0]), 16, 1024);
+      const uint64_t a1 = sdesc_sw128(smem_u32(sm.stat[1]), 16, 1024);
+      const uint64_t b0 = sdesc_sw128(smem_u32(sm.sub[st][0]), 16, 1024);
+      const uint64_t b1 = sdesc_sw128(smem_u32(sm.sub[st][1]), 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        // K step kk: 32 bytes into the 128-byte swizzled rows, 64-column box kk / 4
+        const uint64_t oa = static_cast<uint64_t>(((kk >> 2) * C::kStatChunk + (kk & 3) * 32) >> 4);
+        const uint64_t ob = static_cast<uint64_t>(((kk >> 2) * C::kSubChunk + (kk & 3) * 32) >> 4);
+        umma_ss(t_x, a0 + oa, b0 + ob, id_x, kk > 0 ? 1u : 0u);
+        umma_ss(t_y, a1 + oa, b1 + ob, id_x, kk > 0 ? 1u : 0u);
+      }
+      umma_commit(&sm.x_full);
+    }
+    __syncwarp();
+  }
+  if (ok && s > 0) {
+    ok = tc_wait_lane0(sm, &sm.comp_done, (s - 1) & 1, p);
+    if (ok) {
+      tc_fence_after();
+      issue_acc((s - 1) & 1);
+    }
+  }
+  if (ok) {
+    if (elect_one_sync()) umma_commit(&sm.acc_full);  // with no step: arrives at once
+    __syncwarp();
+  } else {
+    // drain every MMA this warp issued before TMEM is released
+    if (elect_one_sync()) umma_commit(&sm.drain);
+    __syncwarp();
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&sm.drain, 0) && globaltimer_ns() - t0 < p.timeout_ns) {
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack16(float lo, float hi, bool bf16) {
+  if (bf16) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&h);
-  } else {
-    const __half2 h = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&h);
   }
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// 16-byte global -> shared copy; with valid == false the 16 bytes are zero-filled
-// and nothing is read.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  const int n = valid ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
-}
-
-// Rows [r0, r0 + R) of a (rows x D) 16-bit tensor into a padded shared tile; rows at
-// or past n_rows are zero.  All threads of the CTA take part.
-template <int D, int R>
-__device__ __forceinline__ void load_tile(uint16_t* tile, const uint16_t* src, int64_t r0,
-                                          int64_t n_rows) {
-  constexpr int kChunks = D / 8, LD = D + 8;
-  for (int c = threadIdx.x; c < R * kChunks; c += kBwdWarps * 32) {
-    const int r = c / kChunks, col = (c - r * kChunks) * 8;
-    const bool ok = r0 + r < n_rows;
-    const uint16_t* g = src + (ok ? (r0 + r) * D + col : 0);
-    cp_async16(smem_addr(tile + r * LD + col), g, ok);
-  }
-}
-
-// Per row of a query tile: lse * log2(e), or +inf for rows past L and rows with no
-// live key (P = exp2(s - inf) = 0 there), and delta.
-__device__ __forceinline__ void row_stats(const BwdParams& p, int64_t bh, int64_t i, float& l2,
-                                          float& dl) {
-  l2 = INFINITY;
-  dl = 0.f;
-  if (i < p.L) {
-    const float l = p.lse[bh * p.L + i];
-    if (l != -INFINITY) {
-      l2 = l * kBwdLog2e;
-      dl = p.delta[bh * p.L + i];
-    }
-  }
-}
-
-// Entry t of a block list: the t-th PARTIAL block, then the FULL ones after np.
-__device__ __forceinline__ int list_entry(const int32_t* idx, const int32_t* fidx, int np,
-                                          int64_t base, int t, bool& full) {
-  full = t >= np;
-  return full ? __ldg(fidx + base + (t - np)) : __ldg(idx + base + t);
-}
-
-// dK, dV of one 128-key tile (b, kv head, kv block), over the query heads of its
-// group and the q blocks of its column lists, BR query rows at a time.  Warp w owns
-// keys 16 w .. 16 w + 15 and computes the transposed products:
-//   S^T = K Q^T,  dP^T = V dO^T  (16 x BR),  then  dV += P^T dO,  dK += dS^T Q.
-template <int D>
-struct DkdvTile {
-  static constexpr int BR = D == 64 ? 64 : 32;
-  static constexpr int LD = D + 8;
-  static constexpr size_t kSmem =
-      (2 * 128 + 4 * BR) * LD * sizeof(uint16_t) + 4 * BR * sizeof(float);
+// What one 32-column group of a step needs besides X and Y.
+struct GroupArgs {
+  const float* lse2;   // dK/dV: the columns' log2-scale LSE and delta (shared memory)
+  const float* delta;
+  const int32_t* aux;  // PARTIAL blocks: the columns' document ids / tabulated words
+  float my_l2, my_dl;  // dQ: this row's
+  int my, r0, c0;      // this thread's row index; first streamed row; first column
+  int my_id;           // documents: this row's id
+  uint32_t word;       // dQ tabulated masks: this row's word for the group's 32 keys
 };
 
-template <int D, bool BF>
-__global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_dkdv_mma_kernel(const BwdParams p) {
-  using T = DkdvTile<D>;
-  constexpr int BR = T::BR, LD = T::LD, KT = D / 16, NQ = BR / 8, ND = D / 8, SUBS = 128 / BR;
-  extern __shared__ __align__(16) uint16_t smem[];
-  uint16_t* Ks = smem;                  // [128][LD]
-  uint16_t* Vs = Ks + 128 * LD;         // [128][LD]
-  uint16_t* Qs = Vs + 128 * LD;         // [2][BR][LD]
-  uint16_t* Gs = Qs + 2 * BR * LD;      // [2][BR][LD]  dO
-  float* Ls = reinterpret_cast<float*>(Gs + 2 * BR * LD);  // [2][BR]
-  float* Dl = Ls + 2 * BR;                                 // [2][BR]
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-  const int64_t n_kvbh = static_cast<int64_t>(p.B) * p.Hkv;
-  const int jb = static_cast<int>(blockIdx.x / n_kvbh);   // column-major: longest columns first
-  const int64_t kvbh = blockIdx.x - static_cast<int64_t>(jb) * n_kvbh;
-  const int64_t b = kvbh / p.Hkv, kvh = kvbh - b * p.Hkv;
-  const int j0 = jb * 128;
-
-  load_tile<D, 128>(Ks, p.k, kvbh * p.S + j0, kvbh * p.S + p.S);
-  load_tile<D, 128>(Vs, p.v, kvbh * p.S + j0, kvbh * p.S + p.S);
-  cp_async_commit();
-
-  const int np = p.n_q > 0 ? __ldg(p.q_num + jb) : 0;
-  const int nf = p.n_q > 0 ? __ldg(p.full_q_num + jb) : 0;
-  const int nblk = np + nf;
-  const int n_it = p.G * nblk * SUBS;
-  const int64_t list_base = static_cast<int64_t>(jb) * p.n_q;
-
-  // iteration it -> (query head in the group, list entry, BR-row slice)
-  auto decode = [&](int it, int64_t& bh, int& i0, bool& full) {
-    const int sub = it % SUBS, rest = it / SUBS;
-    const int t = rest % nblk, gg = rest / nblk;
-    const int ib = list_entry(p.q_idx, p.full_q_idx, np, list_base, t, full);
-    i0 = ib * 128 + sub * BR;
-    bh = b * p.H + kvh * p.G + gg;
-  };
-  auto prefetch = [&](int it, int st) {
-    int64_t bh;
-    int i0;
-    bool full;
-    decode(it, bh, i0, full);
-    load_tile<D, BR>(Qs + st * BR * LD, p.q, bh * p.L + i0, bh * p.L + p.L);
-    load_tile<D, BR>(Gs + st * BR * LD, p.dout, bh * p.L + i0, bh * p.L + p.L);
-    for (int r = threadIdx.x; r < BR; r += kBwdWarps * 32)
-      row_stats(p, bh, static_cast<int64_t>(i0) + r, Ls[st * BR + r], Dl[st * BR + r]);
-  };
-
-  if (n_it > 0) prefetch(0, 0);
-  cp_async_commit();
-  cp_async_wait<1>();  // the K / V tile
-  __syncthreads();
-
-  // K and V rows of this warp as A operands: held in registers for the whole
-  // column at D = 64, re-read from shared memory per use at D = 128 (registers)
-  constexpr bool kHold = D == 64;
-  constexpr int KH = kHold ? KT : 1;
-  const int a_row = 16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1);
-  const int a_col = 8 * (lane >> 4);
-  uint32_t kf[KH][4], vf[KH][4];
-  if constexpr (kHold) {
+// P and dS for 32 columns of this thread's row, packed to 16-bit pairs.  FULL,
+// SOFTCAP and the mask KIND are compile-time, so a step runs one short variant.
+template <int MODE, bool FULL, bool SOFTCAP, int KIND>
+__device__ __forceinline__ void group_grads(const BwdParams& p, const uint32_t (&xr)[32],
+                                            const uint32_t (&yr)[32], const GroupArgs& a,
+                                            bool bf16, uint32_t (&pk_p)[16], uint32_t (&pk_d)[16]) {
 #pragma unroll
-    for (int kk = 0; kk < KT; ++kk) {
-      ldsm_x4(kf[kk], smem_addr(Ks + a_row * LD + kk * 16 + a_col));
-      ldsm_x4(vf[kk], smem_addr(Vs + a_row * LD + kk * 16 + a_col));
-    }
-  }
-  const int kr0 = j0 + 16 * warp + g;  // key of C rows g; kr0 + 8 for rows g + 8
-
-  float dk[ND][4], dv[ND][4];
+  for (int c2 = 0; c2 < 16; ++c2) {
+    float pv[2], dv[2];
 #pragma unroll
-  for (int n = 0; n < ND; ++n)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) dk[n][c] = dv[n][c] = 0.f;
-
-  for (int it = 0; it < n_it; ++it) {
-    const int st = it & 1;
-    if (it + 1 < n_it) prefetch(it + 1, st ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    int64_t bh;
-    int i0;
-    bool full;
-    decode(it, bh, i0, full);
-    const uint16_t* Qt = Qs + st * BR * LD;
-    const uint16_t* Gt = Gs + st * BR * LD;
-    const float* Lt = Ls + st * BR;
-    const float* Dt = Dl + st * BR;
-
-    float s[NQ][4], dp[NQ][4];
-#pragma unroll
-    for (int n = 0; n < NQ; ++n)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) s[n][c] = dp[n][c] = 0.f;
-    {
-      // B operands: Q / dO rows (n = query, k = d), two 8-query tiles per ldmatrix
-      const int row = (lane & 7) + 8 * (lane >> 4);
-      const int col = 8 * ((lane >> 3) & 1);
-#pragma unroll
-      for (int kk = 0; kk < KT; ++kk) {
-        uint32_t ka[4], va[4];
-        if constexpr (kHold) {
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            ka[r] = kf[kk][r];
-            va[r] = vf[kk][r];
-          }
+    for (int e = 0; e < 2; ++e) {
+      const int cc = 2 * c2 + e;  // column a.c0 + cc: streamed row a.r0 + a.c0 + cc
+      const float x = __uint_as_float(xr[cc]);
+      const float y = __uint_as_float(yr[cc]);
+      const float l2 = MODE == kModeDkdv ? a.lse2[a.c0 + cc] : a.my_l2;
+      const float dl = MODE == kModeDkdv ? a.delta[a.c0 + cc] : a.my_dl;
+      // s (log2 units) and the softcap's derivative, tanh y = 1 - 2 / (e^{2y} + 1)
+      float sl2, dcap = 1.f;
+      if constexpr (SOFTCAP) {
+        const float th = 1.f - 2.f * rcp_approx(ex2_approx(x * p.cap_k) + 1.f);
+        sl2 = p.cap_c * kBwdLog2e * th;
+        dcap = 1.f - th * th;
+      } else {
+        sl2 = x * p.scale_log2;
+      }
+      const float pij = ex2_approx(sl2 - l2);
+      float dsij = pij * (y - dl);
+      if constexpr (SOFTCAP) dsij *= dcap;
+      bool keep = true;
+      if constexpr (!FULL) {
+        const int other = a.r0 + a.c0 + cc;
+        const int i = MODE == kModeDkdv ? other : a.my;
+        const int j = MODE == kModeDkdv ? a.my : other;
+        keep = i < p.L && j < p.S;
+        if constexpr (KIND == FA_MASK_CAUSAL) {
+          keep = keep && j <= i;
+        } else if constexpr (KIND == FA_MASK_SLIDING_WINDOW_CAUSAL) {
+          keep = keep && j <= i && i - j < p.window;
+        } else if constexpr (KIND == FA_MASK_DOCUMENT_CAUSAL) {
+          keep = keep && j <= i && a.aux[a.c0 + cc] == a.my_id;
         } else {
-          ldsm_x4(ka, smem_addr(Ks + a_row * LD + kk * 16 + a_col));
-          ldsm_x4(va, smem_addr(Vs + a_row * LD + kk * 16 + a_col));
-        }
-#pragma unroll
-        for (int n2 = 0; n2 < NQ / 2; ++n2) {
-          uint32_t bq[4], bg[4];
-          ldsm_x4(bq, smem_addr(Qt + (n2 * 16 + row) * LD + kk * 16 + col));
-          ldsm_x4(bg, smem_addr(Gt + (n2 * 16 + row) * LD + kk * 16 + col));
-          mma16816<BF>(s[2 * n2], ka, bq[0], bq[1]);
-          mma16816<BF>(s[2 * n2 + 1], ka, bq[2], bq[3]);
-          mma16816<BF>(dp[2 * n2], va, bg[0], bg[1]);
-          mma16816<BF>(dp[2 * n2 + 1], va, bg[2], bg[3]);
+          const uint32_t w = MODE == kModeDkdv
+                                 ? static_cast<uint32_t>(a.aux[(a.c0 + cc) * 4 + ((a.my >> 5) & 3)])
+                                 : a.word;
+          keep = keep && ((w >> (j & 31)) & 1u) != 0u;
         }
       }
+      pv[e] = keep ? pij : 0.f;
+      dv[e] = keep ? dsij : 0.f;
     }
-    // P^T and dS^T in place of S^T and dP^T
-#pragma unroll
-    for (int n = 0; n < NQ; ++n) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int qc = n * 8 + 2 * tq + (c & 1);
-        const int j = kr0 + 8 * (c >> 1), i = i0 + qc;
-        float pij, dsij;
-        pair_grads(p, s[n][c], dp[n][c], Lt[qc], Dt[qc], pij, dsij);
-        bool keep = j < p.S;
-        if (!full) keep = keep && i < p.L && pair_live(p, i, j);
-        s[n][c] = keep ? pij : 0.f;
-        dp[n][c] = keep ? dsij : 0.f;
-      }
-    }
-    // dV += P^T dO, dK += dS^T Q: B operands dO / Q (k = query, n = d) by transposed loads
-    {
-      const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
-      const int col = 8 * (lane >> 4);
-#pragma unroll
-      for (int kq = 0; kq < BR / 16; ++kq) {
-        const uint32_t ap[4] = {pack16<BF>(s[2 * kq][0], s[2 * kq][1]),
-                                pack16<BF>(s[2 * kq][2], s[2 * kq][3]),
-                                pack16<BF>(s[2 * kq + 1][0], s[2 * kq + 1][1]),
-                                pack16<BF>(s[2 * kq + 1][2], s[2 * kq + 1][3])};
-        const uint32_t ad[4] = {pack16<BF>(dp[2 * kq][0], dp[2 * kq][1]),
-                                pack16<BF>(dp[2 * kq][2], dp[2 * kq][3]),
-                                pack16<BF>(dp[2 * kq + 1][0], dp[2 * kq + 1][1]),
-                                pack16<BF>(dp[2 * kq + 1][2], dp[2 * kq + 1][3])};
-#pragma unroll
-        for (int n2 = 0; n2 < ND / 2; ++n2) {
-          uint32_t bg[4], bq[4];
-          ldsm_x4_trans(bg, smem_addr(Gt + (kq * 16 + row) * LD + n2 * 16 + col));
-          ldsm_x4_trans(bq, smem_addr(Qt + (kq * 16 + row) * LD + n2 * 16 + col));
-          mma16816<BF>(dv[2 * n2], ap, bg[0], bg[1]);
-          mma16816<BF>(dv[2 * n2 + 1], ap, bg[2], bg[3]);
-          mma16816<BF>(dk[2 * n2], ad, bq[0], bq[1]);
-          mma16816<BF>(dk[2 * n2 + 1], ad, bq[2], bq[3]);
-        }
-      }
-    }
-    __syncthreads();  // this stage is refilled by the next iteration's prefetch
+    pk_p[c2] = pack16(pv[0], pv[1], bf16);
+    pk_d[c2] = pack16(dv[0], dv[1], bf16);
   }
-  cp_async_wait<0>();
+}
 
-  const bool bf16 = BF;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int j = kr0 + 8 * h;
-    if (j >= p.S) continue;
-    const int64_t off = (kvbh * p.S + j) * D + 2 * tq;
-#pragma unroll
-    for (int n = 0; n < ND; ++n) {
-      store_pair(p.dk + off + n * 8,
-                 make_float2(dk[n][2 * h] * p.scale, dk[n][2 * h + 1] * p.scale), bf16);
-      store_pair(p.dv + off + n * 8, make_float2(dv[n][2 * h], dv[n][2 * h + 1]), bf16);
+template <int MODE, bool SOFTCAP>
+__device__ __forceinline__ void group_dispatch(const BwdParams& p, bool full,
+                                               const uint32_t (&xr)[32], const uint32_t (&yr)[32],
+                                               const GroupArgs& a, bool bf16, uint32_t (&pk_p)[16],
+                                               uint32_t (&pk_d)[16]) {
+  if (full) {
+    group_grads<MODE, true, SOFTCAP, 0>(p, xr, yr, a, bf16, pk_p, pk_d);
+  } else {
+    switch (p.kind) {
+      case FA_MASK_CAUSAL:
+        group_grads<MODE, false, SOFTCAP, FA_MASK_CAUSAL>(p, xr, yr, a, bf16, pk_p, pk_d);
+        break;
+      case FA_MASK_SLIDING_WINDOW_CAUSAL:
+        group_grads<MODE, false, SOFTCAP, FA_MASK_SLIDING_WINDOW_CAUSAL>(p, xr, yr, a, bf16, pk_p, pk_d);
+        break;
+      case FA_MASK_DOCUMENT_CAUSAL:
+        group_grads<MODE, false, SOFTCAP, FA_MASK_DOCUMENT_CAUSAL>(p, xr, yr, a, bf16, pk_p, pk_d);
+        break;
+      default:
+        group_grads<MODE, false, SOFTCAP, FA_MASK_BITMAP>(p, xr, yr, a, bf16, pk_p, pk_d);
+        break;
     }
   }
 }
 
-// dQ of one 128-query tile (b, h, q block), over the kv blocks of its row lists, BC
-// keys at a time.  Warp w owns queries 16 w .. 16 w + 15:
-//   S = Q K^T,  dP = dO V^T  (16 x BC),  then  dQ += dS K.
-// Tiles run in the forward's schedule order (longest rows first).
-template <int D>
-struct DqTile {
-  static constexpr int BC = D == 64 ? 64 : 32;
-  static constexpr int LD = D + 8;
-  static constexpr size_t kSmem = (2 * 128 + 4 * BC) * LD * sizeof(uint16_t);
-};
+// Warps 0-3: thread t owns row t of the stationary tile (TMEM lane t).
+template <int MODE, int D>
+__device__ void tc_compute_role(TcSmem<D>& sm, const BwdParams& p, uint32_t tmem, int64_t tile_bh,
+                                int tile_blk) {
+  const int t = threadIdx.x;
+  const uint32_t lane_off = static_cast<uint32_t>((t >> 5) * 32) << 16;
+  const uint32_t t_x = tmem + lane_off, t_y = tmem + 64 + lane_off;
+  const uint32_t t_acc0 = tmem + 128 + lane_off, t_acc1 = tmem + 128 + D + lane_off;
+  const bool bf16 = p.is_bf16 != 0;
+  // this thread's row: dK/dV key j of K/V head tile_bh; dQ query i of head tile_bh
+  GroupArgs a;
+  a.my = tile_blk * 128 + t;
+  a.my_l2 = INFINITY;
+  a.my_dl = 0.f;
+  if (MODE == kModeDq && a.my < p.L) {
+    const float l = __ldg(p.lse + tile_bh * p.L + a.my);
+    if (l != -INFINITY) {
+      a.my_l2 = l * kBwdLog2e;
+      a.my_dl = p.delta[tile_bh * p.L + a.my];
+    }
+  }
+  StepIter<MODE> it;
+  it.init(p, tile_bh, tile_blk);
+  int s = 0;
+  for (; it.next(p); it.step(), ++s) {
+    const int st = s & 1;
+    if (!tc_wait_warp(sm, &sm.x_full, s & 1, p)) return;
+    tc_fence_after();
+    a.r0 = it.row0();
+    a.lse2 = sm.lse2[st];
+    a.delta = sm.delta[st];
+    a.aux = sm.aux[st];
+    a.my_id = 0;
+    uint32_t w_lo = 0, w_hi = 0;
+    // the thread's own id / words for PARTIAL blocks of document / tabulated masks
+    if (!it.full && p.kind == FA_MASK_DOCUMENT_CAUSAL) {
+      const int n = MODE == kModeDkdv ? p.S : p.L;
+      a.my_id = __ldg(p.doc_id + static_cast<int64_t>(it.inst) * p.doc_len + min(a.my, n - 1));
+    } else if (MODE == kModeDq && !it.full && p.kind == FA_MASK_BITMAP) {
+      const uint32_t* row = p.bitmap + (static_cast<int64_t>(it.inst) * p.L + min(a.my, p.L - 1)) *
+                                           4 * p.n_kv;
+      w_lo = __ldg(row + (a.r0 >> 5));
+      w_hi = __ldg(row + (a.r0 >> 5) + 1);
+    }
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      uint32_t xr[32], yr[32];
+      tmem_ld32(t_x + 32 * h, xr);
+      tmem_ld32(t_y + 32 * h, yr);
+      tmem_wait_ld();
+      reg_fence32(xr);
+      reg_fence32(yr);
+      a.c0 = 32 * h;
+      a.word = h == 0 ? w_lo : w_hi;
+      uint32_t pk_p[16], pk_d[16];
+      if (p.softcap_on)
+        group_dispatch<MODE, true>(p, it.full, xr, yr, a, bf16, pk_p, pk_d);
+      else
+        group_dispatch<MODE, false>(p, it.full, xr, yr, a, bf16, pk_p, pk_d);
+      // 16-bit results over the columns just read: P (dK/dV) at X [16h, 16h + 16),
+      // dS at Y [16h, 16h + 16)
+      if constexpr (MODE == kModeDkdv) tmem_st16(t_x + 16 * h, pk_p);
+      tmem_st16(t_y + 16 * h, pk_d);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if ((t & 31) == 0) mbar_arrive(&sm.comp_done);
+  }
+  // epilogue: the accumulators of this thread's row -> dK, dV or dQ
+  const int my = a.my;
+  const bool valid = MODE == kModeDkdv ? my < p.S : my < p.L;
+  uint16_t* out0 = MODE == kModeDkdv ? p.dv : p.dq;   // dV (unscaled) / dQ (scaled)
+  const size_t orow = static_cast<size_t>(tile_bh) * (MODE == kModeDkdv ? p.S : p.L) + my;
+  if (s > 0) {
+    if (!tc_wait_warp(sm, &sm.acc_full, 0, p)) return;
+    tc_fence_after();
+  }
+#pragma unroll
+  for (int ai = 0; ai < (MODE == kModeDkdv ? 2 : 1); ++ai) {
+    uint16_t* dst = ai == 0 ? out0 : p.dk;
+    const float f = (MODE == kModeDq || ai == 1) ? p.scale : 1.f;
+    const uint32_t t_acc = ai == 0 ? t_acc0 : t_acc1;
+#pragma unroll
+    for (int c0 = 0; c0 < D / 32; ++c0) {
+      uint32_t r[32];
+      if (s > 0) {
+        tmem_ld32(t_acc + 32 * c0, r);
+        tmem_wait_ld();
+        reg_fence32(r);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = 0u;  // no live block: zero gradient
+      }
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        pk[e] = pack16(__uint_as_float(r[2 * e]) * f, __uint_as_float(r[2 * e + 1]) * f, bf16);
+      if (valid) {
+        uint4* o = reinterpret_cast<uint4*>(dst + orow * D + 32 * c0);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      }
+    }
+  }
+}
 
-template <int D, bool BF>
-__global__ void __launch_bounds__(kBwdWarps * 32, 1) bwd_dq_mma_kernel(const BwdParams p) {
-  using T = DqTile<D>;
-  constexpr int BC = T::BC, LD = T::LD, KT = D / 16, NK = BC / 8, ND = D / 8, SUBS = 128 / BC;
-  extern __shared__ __align__(16) uint16_t smem[];
-  uint16_t* Qs = smem;                 // [128][LD]
-  uint16_t* Gs = Qs + 128 * LD;        // [128][LD]  dO
-  uint16_t* Ks = Gs + 128 * LD;        // [2][BC][LD]
-  uint16_t* Vs = Ks + 2 * BC * LD;     // [2][BC][LD]
+template <int MODE, int D>
+__global__ void __launch_bounds__(kTcThreads, TcCfg<D>::kCtasPerSm)
+bwd_tc_kernel(const __grid_constant__ CUtensorMap ts0, const __grid_constant__ CUtensorMap ts1,
+              const __grid_constant__ CUtensorMap tb0, const __grid_constant__ CUtensorMap tb1,
+              const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = smem_u32(smem_raw);
+  TcSmem<D>& sm = *reinterpret_cast<TcSmem<D>*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
+  const int warp = threadIdx.x >> 5;
+  constexpr uint32_t kCols = TcCfg<D>::tmem_cols(MODE);
 
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-  const int64_t n_bh = static_cast<int64_t>(p.B) * p.H;
-  const int rank = static_cast<int>(blockIdx.x / n_bh);
-  const int64_t bh = blockIdx.x - static_cast<int64_t>(rank) * n_bh;
-  const int qb = p.sched != nullptr ? __ldg(p.sched + 2 * rank) : rank;
-  const int64_t kvbh = (bh / p.H) * p.Hkv + (bh % p.H) / p.G;
-  const int i0 = qb * 128;
+  // the CTA's tile.  dK/dV: key tile jb of K/V head kvbh, columns in ascending jb
+  // (the longest causal columns first).  dQ: query tile of head bh at rank `rank` of
+  // its instance's schedule (longest rows first).
+  int64_t tile_bh, stat_z;
+  int tile_blk;
+  if constexpr (MODE == kModeDkdv) {
+    const int64_t n_kvbh = static_cast<int64_t>(p.B) * p.Hkv;
+    tile_blk = static_cast<int>(blockIdx.x / n_kvbh);
+    tile_bh = blockIdx.x - static_cast<int64_t>(tile_blk) * n_kvbh;
+    stat_z = tile_bh;
+  } else {
+    const int64_t n_bh = static_cast<int64_t>(p.B) * p.H;
+    const int rank = static_cast<int>(blockIdx.x / n_bh);
+    tile_bh = blockIdx.x - static_cast<int64_t>(rank) * n_bh;
+    const int64_t inst = bwd_instance(p, tile_bh);
+    tile_blk = __ldg(p.sched + 2 * (inst * p.n_q + rank));
+    stat_z = tile_bh;
+  }
 
-  load_tile<D, 128>(Qs, p.q, bh * p.L + i0, bh * p.L + p.L);
-  load_tile<D, 128>(Gs, p.dout, bh * p.L + i0, bh * p.L + p.L);
-  cp_async_commit();
-
-  const int np = __ldg(p.kv_num + qb), nf = __ldg(p.full_num + qb);
-  const int n_it = (np + nf) * SUBS;
-  const int64_t list_base = static_cast<int64_t>(qb) * p.n_kv;
-  auto decode = [&](int it, int& j0, bool& full) {
-    const int jb = list_entry(p.kv_idx, p.full_idx, np, list_base, it / SUBS, full);
-    j0 = jb * 128 + (it % SUBS) * BC;
-  };
-  auto prefetch = [&](int it, int st) {
-    int j0;
-    bool full;
-    decode(it, j0, full);
-    load_tile<D, BC>(Ks + st * BC * LD, p.k, kvbh * p.S + j0, kvbh * p.S + p.S);
-    load_tile<D, BC>(Vs + st * BC * LD, p.v, kvbh * p.S + j0, kvbh * p.S + p.S);
-  };
-
-  if (n_it > 0) prefetch(0, 0);
-  cp_async_commit();
-  cp_async_wait<1>();  // the Q / dO tile
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.stat_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    mbar_init(&sm.x_full, 1);
+    mbar_init(&sm.comp_done, 4);  // one arrival per compute warp
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kLoadWarp && (threadIdx.x & 31) == 0) {
+    prefetch_tensormap(&ts0);
+    prefetch_tensormap(&ts1);
+    prefetch_tensormap(&tb0);
+    prefetch_tensormap(&tb1);
+  }
+  if (warp == kIssueWarp) {
+    tmem_alloc(&sm.tmem_base, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
 
-  uint32_t qf[KT][4], gf[KT][4];
-  {
-    const int row = 16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1);
-    const int col = 8 * (lane >> 4);
-#pragma unroll
-    for (int kk = 0; kk < KT; ++kk) {
-      ldsm_x4(qf[kk], smem_addr(Qs + row * LD + kk * 16 + col));
-      ldsm_x4(gf[kk], smem_addr(Gs + row * LD + kk * 16 + col));
-    }
+  if (warp < 4) {
+    tc_compute_role<MODE, D>(sm, p, tmem, tile_bh, tile_blk);
+  } else if (warp == kLoadWarp) {
+    tc_load_role<MODE, D>(sm, p, &ts0, &ts1, &tb0, &tb1, tile_bh, tile_blk, stat_z);
+  } else {
+    tc_issue_role<MODE, D>(sm, p, tmem, tile_bh, tile_blk);
   }
-  const int qr0 = i0 + 16 * warp + g;  // query of C rows g; qr0 + 8 for rows g + 8
-  float l2[2], dl[2];
-  row_stats(p, bh, qr0, l2[0], dl[0]);
-  row_stats(p, bh, qr0 + 8, l2[1], dl[1]);
-
-  float dq[ND][4];
-#pragma unroll
-  for (int n = 0; n < ND; ++n)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) dq[n][c] = 0.f;
-
-  for (int it = 0; it < n_it; ++it) {
-    const int st = it & 1;
-    if (it + 1 < n_it) prefetch(it + 1, st ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    int j0;
-    bool full;
-    decode(it, j0, full);
-    const uint16_t* Kt = Ks + st * BC * LD;
-    const uint16_t* Vt = Vs + st * BC * LD;
-
-    float s[NK][4], dp[NK][4];
-#pragma unroll
-    for (int n = 0; n < NK; ++n)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) s[n][c] = dp[n][c] = 0.f;
-    {
-      // B operands: K / V rows (n = key, k = d)
-      const int row = (lane & 7) + 8 * (lane >> 4);
-      const int col = 8 * ((lane >> 3) & 1);
-#pragma unroll
-      for (int kk = 0; kk < KT; ++kk) {
-#pragma unroll
-        for (int n2 = 0; n2 < NK / 2; ++n2) {
-          uint32_t bk[4], bv[4];
-          ldsm_x4(bk, smem_addr(Kt + (n2 * 16 + row) * LD + kk * 16 + col));
-          ldsm_x4(bv, smem_addr(Vt + (n2 * 16 + row) * LD + kk * 16 + col));
-          mma16816<BF>(s[2 * n2], qf[kk], bk[0], bk[1]);
-          mma16816<BF>(s[2 * n2 + 1], qf[kk], bk[2], bk[3]);
-          mma16816<BF>(dp[2 * n2], gf[kk], bv[0], bv[1]);
-          mma16816<BF>(dp[2 * n2 + 1], gf[kk], bv[2], bv[3]);
-        }
-      }
-    }
-#pragma unroll
-    for (int n = 0; n < NK; ++n) {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int h = c >> 1;
-        const int i = qr0 + 8 * h, j = j0 + n * 8 + 2 * tq + (c & 1);
-        float pij, dsij;
-        pair_grads(p, s[n][c], dp[n][c], l2[h], dl[h], pij, dsij);
-        bool keep = j < p.S;
-        if (!full) keep = keep && i < p.L && pair_live(p, i, j);
-        dp[n][c] = keep ? dsij : 0.f;
-      }
-    }
-    // dQ += dS K: B operand K (k = key, n = d) by transposed loads
-    {
-      const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
-      const int col = 8 * (lane >> 4);
-#pragma unroll
-      for (int kq = 0; kq < BC / 16; ++kq) {
-        const uint32_t ad[4] = {pack16<BF>(dp[2 * kq][0], dp[2 * kq][1]),
-                                pack16<BF>(dp[2 * kq][2], dp[2 * kq][3]),
-                                pack16<BF>(dp[2 * kq + 1][0], dp[2 * kq + 1][1]),
-                                pack16<BF>(dp[2 * kq + 1][2], dp[2 * kq + 1][3])};
-#pragma unroll
-        for (int n2 = 0; n2 < ND / 2; ++n2) {
-          uint32_t bk[4];
-          ldsm_x4_trans(bk, smem_addr(Kt + (kq * 16 + row) * LD + n2 * 16 + col));
-          mma16816<BF>(dq[2 * n2], ad, bk[0], bk[1]);
-          mma16816<BF>(dq[2 * n2 + 1], ad, bk[2], bk[3]);
-        }
-      }
-    }
-    __syncthreads();
-  }
-  cp_async_wait<0>();
-
-  const bool bf16 = BF;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int i = qr0 + 8 * h;
-    if (i >= p.L) continue;
-    const int64_t off = (bh * p.L + i) * D + 2 * tq;
-#pragma unroll
-    for (int n = 0; n < ND; ++n)
-      store_pair(p.dq + off + n * 8,
-                 make_float2(dq[n][2 * h] * p.scale, dq[n][2 * h + 1] * p.scale), bf16);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kIssueWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
   }
 }
 
-template <int D, bool BF>
-fa_status bwd_launch(const BwdParams& prm, cudaStream_t s) {
+template <int MODE, int D>
+fa_status tc_launch(const BwdParams& prm, bool bf16, cudaStream_t s) {
+  CUtensorMap ts0, ts1, tb0, tb1;
+  const int64_t BH = static_cast<int64_t>(prm.B) * prm.H, BHkv = static_cast<int64_t>(prm.B) * prm.Hkv;
+  if (MODE == kModeDkdv) {
+    if (!make_tile_map(&ts0, prm.k, bf16, D, prm.S, static_cast<int>(BHkv), 128)) return FA_ERR_CUDA;
+    if (!make_tile_map(&ts1, prm.v, bf16, D, prm.S, static_cast<int>(BHkv), 128)) return FA_ERR_CUDA;
+    if (!make_tile_map(&tb0, prm.q, bf16, D, prm.L, static_cast<int>(BH), kSub)) return FA_ERR_CUDA;
+    if (!make_tile_map(&tb1, prm.dout, bf16, D, prm.L, static_cast<int>(BH), kSub)) return FA_ERR_CUDA;
+  } else {
+    if (!make_tile_map(&ts0, prm.q, bf16, D, prm.L, static_cast<int>(BH), 128)) return FA_ERR_CUDA;
+    if (!make_tile_map(&ts1, prm.dout, bf16, D, prm.L, static_cast<int>(BH), 128)) return FA_ERR_CUDA;
+    if (!make_tile_map(&tb0, prm.k, bf16, D, prm.S, static_cast<int>(BHkv), kSub)) return FA_ERR_CUDA;
+    if (!make_tile_map(&tb1, prm.v, bf16, D, prm.S, static_cast<int>(BHkv), kSub)) return FA_ERR_CUDA;
+  }
+  const size_t smem = sizeof(TcSmem<D>) + 1024;
+  int dev = 0;
+  FA_CUDA_CHECK(cudaGetDevice(&dev));
+  {
+    static std::mutex mu;
+    static bool done[kMaxDevices] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    if (!done[dev]) {
+      FA_CUDA_CHECK(cudaFuncSetAttribute(bwd_tc_kernel<MODE, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem)));
+      done[dev] = true;
+    }
+  }
+  const int64_t grid = MODE == kModeDkdv ? static_cast<int64_t>(prm.n_kv) * BHkv
+                                         : static_cast<int64_t>(prm.n_q) * BH;
+  if (grid == 0) return FA_OK;
+  bwd_tc_kernel<MODE, D><<<static_cast<unsigned>(grid), kTcThreads, smem, s>>>(ts0, ts1, tb0, tb1, prm);
+  FA_CUDA_CHECK(cudaGetLastError());
+  return FA_OK;
+}
+
+template <int D>
+fa_status bwd_launch(const BwdParams& prm, bool bf16, cudaStream_t s) {
   const int64_t rows = static_cast<int64_t>(prm.B) * prm.H * prm.L;
   const int64_t krows = static_cast<int64_t>(prm.B) * prm.Hkv * prm.S;
-  const unsigned threads = kBwdWarps * 32;
   if (rows > 0) {
     const unsigned qgrid = static_cast<unsigned>((rows + kBwdWarps - 1) / kBwdWarps);
-    bwd_delta_kernel<D><<<qgrid, threads, 0, s>>>(prm);
-    FA_CUDA_CHECK(cudaGetLastError());
-    FA_CUDA_CHECK(cudaFuncSetAttribute(bwd_dq_mma_kernel<D, BF>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(DqTile<D>::kSmem)));
-    const unsigned grid = static_cast<unsigned>(static_cast<int64_t>(prm.n_q) * prm.B * prm.H);
-    bwd_dq_mma_kernel<D, BF><<<grid, threads, DqTile<D>::kSmem, s>>>(prm);
+    bwd_delta_kernel<D><<<qgrid, kBwdWarps * 32, 0, s>>>(prm);
     FA_CUDA_CHECK(cudaGetLastError());
   }
+  if (rows > 0) {
+    const fa_status st = tc_launch<kModeDq, D>(prm, bf16, s);
+    if (st != FA_OK) return st;
+  }
   if (krows > 0) {
-    FA_CUDA_CHECK(cudaFuncSetAttribute(bwd_dkdv_mma_kernel<D, BF>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(DkdvTile<D>::kSmem)));
-    const unsigned grid = static_cast<unsigned>(static_cast<int64_t>(prm.n_kv) * prm.B * prm.Hkv);
-    bwd_dkdv_mma_kernel<D, BF><<<grid, threads, DkdvTile<D>::kSmem, s>>>(prm);
-    FA_CUDA_CHECK(cudaGetLastError());
+    const fa_status st = tc_launch<kModeDkdv, D>(prm, bf16, s);
+    if (st != FA_OK) return st;
   }
   return FA_OK;
 }
@@ -602,7 +765,7 @@ fa_status bwd_launch(const BwdParams& prm, cudaStream_t s) {
 
 extern "C" size_t fa_bwd_workspace_bytes(int32_t B, int32_t H, int32_t L) {
   if (B < 0 || H < 0 || L < 0) return 0;
-  return static_cast<size_t>(B) * H * L * sizeof(float) + 256;
+  return fa::kBwdWorkspaceHeader + static_cast<size_t>(B) * H * L * sizeof(float);
 }
 
 extern "C" fa_status fa_flex_attention_bwd(
@@ -622,11 +785,18 @@ extern "C" fa_status fa_flex_attention_bwd(
     return FA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (bm->block != FA_BLOCK || bm->q_len != L || bm->kv_len != S) return FA_ERR_INVALID_ARG;
-  if (bm->mask_batch > 1 || bm->mask_heads > 1) return FA_ERR_UNSUPPORTED;  // broadcast masks only
+  // per-(batch, head) masks: one instance per batch element and / or head (0 reads as 1)
+  const int mb = bm->mask_batch > 1 ? bm->mask_batch : 1;
+  const int mh = bm->mask_heads > 1 ? bm->mask_heads : 1;
+  if ((mb != 1 && mb != B) || (mh != 1 && mh != H)) return FA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(B) * H * L == 0 && static_cast<int64_t>(B) * H_kv * S == 0) return FA_OK;
   if (static_cast<int64_t>(B) * H * L > (int64_t{1} << 33) ||
-      static_cast<int64_t>(B) * H_kv * S > (int64_t{1} << 33))
+      static_cast<int64_t>(B) * H_kv * S > (int64_t{1} << 33) ||
+      static_cast<int64_t>(B) * H > INT32_MAX)
+    return FA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(bm->n_kv_blocks) * B * H_kv > INT32_MAX ||
+      static_cast<int64_t>(bm->n_q_blocks) * B * H > INT32_MAX)
     return FA_ERR_UNSUPPORTED;
   if (workspace == nullptr || workspace_bytes < fa_bwd_workspace_bytes(B, H, L))
     return FA_ERR_INVALID_ARG;
@@ -635,7 +805,8 @@ extern "C" fa_status fa_flex_attention_bwd(
     return FA_ERR_INVALID_ARG;
   if (any_k && (k == nullptr || v == nullptr || dk == nullptr || dv == nullptr))
     return FA_ERR_INVALID_ARG;
-  if (bm->n_q_blocks > 0 && (bm->kv_num_blocks == nullptr || bm->full_kv_num_blocks == nullptr))
+  if (bm->n_q_blocks > 0 && (bm->kv_num_blocks == nullptr || bm->full_kv_num_blocks == nullptr ||
+                             bm->q_order == nullptr))
     return FA_ERR_INVALID_ARG;
   if (bm->n_q_blocks > 0 && bm->n_kv_blocks > 0 &&
       (bm->kv_indices == nullptr || bm->full_kv_indices == nullptr || q_num_blocks == nullptr ||
@@ -643,12 +814,13 @@ extern "C" fa_status fa_flex_attention_bwd(
     return FA_ERR_INVALID_ARG;
   if (bm->kind == FA_MASK_DOCUMENT_CAUSAL && bm->doc_id == nullptr) return FA_ERR_INVALID_ARG;
   if (bm->kind == FA_MASK_BITMAP && S > 0 && bm->bitmap == nullptr) return FA_ERR_INVALID_ARG;
-  // q, k, v, dout are staged by 16-byte cp.async copies; the rest is accessed in
-  // 4-byte pairs / floats
+  // q, k, v, dout are TMA tiles and the gradients are written in 16-byte pieces: 16
+  // bytes; the workspace holds the error word and the row sums: 16 bytes; the rest
+  // is read as 4-byte values (out in 4-byte pairs)
   auto off16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
   auto off4 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) != 0; };
-  if (off16(q) || off16(k) || off16(v) || off16(dout) || off4(out) || off4(dq) || off4(dk) ||
-      off4(dv) || off4(workspace) || off4(lse))
+  if (off16(q) || off16(k) || off16(v) || off16(dout) || off16(dq) || off16(dk) || off16(dv) ||
+      off16(workspace) || off4(out) || off4(lse))
     return FA_ERR_INVALID_ARG;
   if (off4(bm->kv_num_blocks) || off4(bm->full_kv_num_blocks) || off4(bm->kv_indices) ||
       off4(bm->full_kv_indices) || off4(bm->q_order) || off4(bm->doc_id) || off4(bm->bitmap) ||
@@ -662,7 +834,8 @@ extern "C" fa_status fa_flex_attention_bwd(
   prm.out = static_cast<const uint16_t*>(out);
   prm.dout = static_cast<const uint16_t*>(dout);
   prm.lse = lse;
-  prm.delta = static_cast<float*>(workspace);
+  prm.err = static_cast<int32_t*>(workspace);
+  prm.delta = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kBwdWorkspaceHeader);
   prm.dq = static_cast<uint16_t*>(dq);
   prm.dk = static_cast<uint16_t*>(dk);
   prm.dv = static_cast<uint16_t*>(dv);
@@ -687,11 +860,19 @@ extern "C" fa_status fa_flex_attention_bwd(
   prm.n_kv = bm->n_kv_blocks;
   prm.kind = bm->kind;
   prm.window = bm->window;
+  prm.mask_b = mb > 1 ? 1 : 0;
+  prm.mask_h = mh > 1 ? 1 : 0;
+  prm.mask_heads = mh;
+  prm.doc_len = L > S ? L : S;
   prm.softcap_on = score_kind == FA_SCORE_TANH_SOFTCAP ? 1 : 0;
   prm.is_bf16 = dtype == FA_BF16 ? 1 : 0;
   prm.scale = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(D));
+  prm.scale_log2 = prm.scale * kBwdLog2e;
   prm.cap_c = prm.softcap_on ? softcap : 1.f;
+  prm.cap_k = prm.softcap_on ? 2.f * prm.scale * kBwdLog2e / softcap : 0.f;
+  prm.timeout_ns = 2000000000ull;
+  if (debug_stall(&prm.timeout_ns)) prm.stall = 1;
   const cudaStream_t s = as_stream(stream);
-  if (D == 64) return prm.is_bf16 ? bwd_launch<64, true>(prm, s) : bwd_launch<64, false>(prm, s);
-  return prm.is_bf16 ? bwd_launch<128, true>(prm, s) : bwd_launch<128, false>(prm, s);
+  const bool b16 = dtype == FA_BF16;
+  return D == 64 ? bwd_launch<64>(prm, b16, s) : bwd_launch<128>(prm, b16, s);
 }

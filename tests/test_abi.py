@@ -260,6 +260,10 @@ def test_bwd_rejects_bad_arguments_on_host(fa):
     assert _bwd(fa, bm, q=1028) == E                # 4- but not 16-byte aligned (cp.async source)
     assert _bwd(fa, bm, k=1032) == E
     assert _bwd(fa, bm, lse=1026) == E
+    assert _bwd(fa, bm, dq=1032) == E               # gradients are written in 16-byte pieces
+    assert _bwd(fa, bm, dk=1028) == E
+    assert _bwd(fa, bm, dv=1040 + 4) == E
+    assert _bwd(fa, bm, ws=1032) == E               # error word + row sums: 16 bytes
     assert _bwd(fa, bm, cols=4098) == E             # column lists not 4-byte aligned
     bm_doc = fa.fa_block_mask()
     ctypes.pointer(bm_doc)[0] = bm
@@ -267,8 +271,10 @@ def test_bwd_rejects_bad_arguments_on_host(fa):
     assert _bwd(fa, bm_doc) == E
     bm_bh = fa.fa_block_mask()
     ctypes.pointer(bm_bh)[0] = bm
-    bm_bh.mask_heads = 2                            # per-(b, h) tables
-    assert _bwd(fa, bm_bh) == U
+    bm_bh.mask_heads = 3                            # per-head tables for 2 heads
+    assert _bwd(fa, bm_bh) == E
+    bm_bh.mask_heads = 2                            # per-(b, h) tables: past the checks
+    assert _bwd(fa, bm_bh) == fa.FA_ERR_CUDA        # (no GPU here)
     # nothing to do: no query rows and no key rows
     assert _bwd(fa, bm, B=0) == fa.FA_OK
 

@@ -85,3 +85,55 @@ def test_identical_instances_equal_broadcast_bit_for_bit():
     _, ob, lb = _run_bh(q, k, v, OM.DOCUMENT_CAUSAL, doc=one.repeat(B * H, 1), mb=B, mh=H)
     oc, lc = run_gpu(q, k, v, OM.DOCUMENT_CAUSAL, doc_id=one[0])
     assert torch.equal(ob, oc) and torch.equal(lb, lc)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_backward_per_instance_masks(D):
+    """Backward with per-(batch, head) masks: documents per batch element and head,
+    then per-head tabulated masks with grouped heads; every (b, h) against the fp64
+    oracle's gradients with that instance's mask (dk / dv of a K/V head summed over
+    its query heads)."""
+    import block_sparse_attention_create_b200 as fa
+    from oracle import backward as OBW
+
+    def check(got, ref, what):
+        got = got.double().numpy()
+        rms = float(np.sqrt((ref ** 2).mean())) + 1e-6
+        err = np.abs(got - ref)
+        assert (err <= 3e-2 * (np.abs(ref) + rms) + 1e-3).all(), (what, float(err.max()))
+
+    # documents per (b, h)
+    B, H, L = 2, 2, 520
+    q, k, v = W.random_qkv(B, H, L, L, D, torch.bfloat16, seed=91 + D)
+    dout = torch.randn(B, H, L, D, generator=torch.Generator().manual_seed(92)).to(torch.bfloat16)
+    doc = _docs(B * H, L, seed=93)
+    bm = fa.create_block_mask(OM.DOCUMENT_CAUSAL, L, L, doc_id=doc.cuda(), B=B, H=H)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, dout))
+    out, lse = fa.flex_attention(qd, kd, vd, bm, return_lse=True)
+    dq, dk, dv = fa.flex_attention_backward(qd, kd, vd, out, dod, lse, bm, check=True)
+    for b in range(B):
+        for h in range(H):
+            ref = OBW.attention_head_backward(q[b, h], k[b, h], v[b, h], dout[b, h],
+                                              OM.DOCUMENT_CAUSAL, doc_id=doc[b * H + h].numpy())
+            for name, got, want in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+                check(got[b, h].cpu(), want, f"doc b{b} h{h} {name}")
+    # per-head bitmaps, 4 query heads over 2 K/V heads
+    L, S, H, Hkv = 300, 260, 4, 2
+    q, k, v = W.random_qkv(1, H, L, S, D, torch.bfloat16, seed=94 + D, Hkv=Hkv)
+    dout = torch.randn(1, H, L, D, generator=torch.Generator().manual_seed(95)).to(torch.bfloat16)
+    words = np.stack([W.random_bitmap(L, S, seed=96 + h) for h in range(H)])
+    bits = torch.from_numpy(np.ascontiguousarray(words).view(np.int32)).cuda()
+    bm = fa.create_block_mask(OM.BITMAP, L, S, bitmap=bits, H=H)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, dout))
+    out, lse = fa.flex_attention(qd, kd, vd, bm, return_lse=True)
+    dq, dk, dv = fa.flex_attention_backward(qd, kd, vd, out, dod, lse, bm, check=True)
+    G = H // Hkv
+    refs = [OBW.attention_head_backward(q[0, h], k[0, h // G], v[0, h // G], dout[0, h],
+                                        OM.BITMAP, bitmap=words[h]) for h in range(H)]
+    for h in range(H):
+        check(dq[0, h].cpu(), refs[h][0], f"bitmap h{h} dq")
+    for kh in range(Hkv):
+        dk_ref = sum(refs[h][1] for h in range(kh * G, kh * G + G))
+        dv_ref = sum(refs[h][2] for h in range(kh * G, kh * G + G))
+        check(dk[0, kh].cpu(), dk_ref, f"bitmap kv{kh} dk")
+        check(dv[0, kh].cpu(), dv_ref, f"bitmap kv{kh} dv")

@@ -55,7 +55,7 @@ def _run(B, H, Hkv, L, S, D, dtype, kind, window=0, doc=None, words=None, sk=0, 
                               doc_id=doc.cuda() if doc is not None else None, bitmap=bits)
     out, lse = fa.flex_attention(qd, kd, vd, bm, score_mod=sk, softcap=cap, return_lse=True)
     dq, dk, dv = fa.flex_attention_backward(qd, kd, vd, out, dod, lse, bm, score_mod=sk,
-                                            softcap=cap)
+                                            softcap=cap, check=True)
     torch.cuda.synchronize()
     assert fa.last_device_error() == fa.FA_OK
     dq, dk, dv = dq.cpu(), dk.cpu(), dv.cpu()

@@ -75,3 +75,32 @@ def test_decode_bounded_waits_report_timeout_and_context_survives():
         o_ref, l_ref = OA.attention_head(q[b, h], k[b, h // (H // Hkv)], v[b, h // (H // Hkv)],
                                          OM.DECODE_CAUSAL)
         compare(out[b, h].cpu(), lse[b, h].cpu(), o_ref, l_ref, f"b{b} h{h}")
+
+
+def test_backward_bounded_waits_report_timeout_and_context_survives():
+    """The backward's tcgen05 kernels wait on bounded mbarriers as well: with the hook
+    on, no tile is loaded, the waits run out, the error word reads FA_ERR_TIMEOUT,
+    and the next backward on the same context is correct."""
+    import block_sparse_attention_create_b200 as fa
+    from oracle import backward as OB
+    L = 300
+    q, k, v = W.random_qkv(1, 2, L, L, 64, torch.bfloat16, seed=64)
+    g = torch.Generator().manual_seed(65)
+    do = torch.randn(1, 2, L, 64, generator=g).to(torch.bfloat16)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    bm = fa.create_block_mask(OM.CAUSAL, L, L, device="cuda")
+    out, lse = fa.flex_attention(qd, kd, vd, bm, return_lse=True)
+    torch.cuda.synchronize()
+    fa.fa_debug_set_mma_stall(1, 50_000_000)
+    try:
+        with pytest.raises(fa.FAError) as err:
+            fa.flex_attention_backward(qd, kd, vd, out, dod, lse, bm, check=True)
+    finally:
+        fa.fa_debug_set_mma_stall(0, 0)
+    assert err.value.status == fa.FA_ERR_TIMEOUT
+    dq, dk, dv = fa.flex_attention_backward(qd, kd, vd, out, dod, lse, bm, check=True)
+    torch.cuda.synchronize()
+    ref = OB.attention_head_backward(q[0, 1], k[0, 1], v[0, 1], do[0, 1], OM.CAUSAL)
+    for got, want in zip((dq[0, 1], dk[0, 1], dv[0, 1]), ref):
+        err_abs = (got.cpu().double() - torch.as_tensor(want)).abs().max().item()
+        assert err_abs < 0.05 * (float(torch.as_tensor(want).abs().max()) + 1e-3) + 2e-2, err_abs
