@@ -38,6 +38,12 @@ struct DecCfg {
   static constexpr int kCtasPerSm = D == 128 ? 2 : 3;
 };
 constexpr int kBoxBytes = kTile * 128;  // one TMA box: 64 keys x 64 elements
+// K/V tiles in flight per CTA: a ring of stages(D, RM) tiles, plus L2 prefetches
+// of the tiles kPrefetch further on, so that enough bytes are on their way to cover
+// the DRAM latency (one 32 KB tile per CTA was not).  Three stages, except at D =
+// 128 with 32 rows, where two keep two CTAs per SM in shared memory.
+__host__ __device__ constexpr int dec_stages(int D, int RM) { return D == 128 && RM == 32 ? 2 : 3; }
+constexpr int kPrefetch = 4;
 constexpr int kDecWorkspaceHeader = 256;  // word 0: device error flags
 constexpr float kDecLog2e = 1.4426950408889634f;
 constexpr float kDecLn2 = 0.6931471805599453f;
@@ -58,12 +64,13 @@ struct DecParams {
 
 template <int D, int RM>
 struct __align__(1024) DecSmem {
-  uint8_t k[2][D / 64][kBoxBytes];
-  uint8_t v[2][D / 64][kBoxBytes];
+  static constexpr int kStages = dec_stages(D, RM);
+  uint8_t k[kStages][D / 64][kBoxBytes];
+  uint8_t v[kStages][D / 64][kBoxBytes];
   float qs[RM][D];
   float sc[RM][kTile];
   float m[RM], l[RM], alpha[RM];
-  uint64_t full[2];
+  uint64_t full[dec_stages(D, RM)];
   volatile int abort_flag;
 };
 
@@ -124,6 +131,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
   using Sm = DecSmem<D, RM>;
+  constexpr int kStages = Sm::kStages;
   Sm& sm = *reinterpret_cast<Sm*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
   constexpr int kThr = DecCfg<D>::kThreads;
   constexpr int kWarps = kThr / 32;
@@ -145,8 +153,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
   const int ntiles = k_start < c1 ? (c1 - k_start + kTile - 1) / kTile : 0;
 
   if (tid == 0) {
-    mbar_init(&sm.full[0], 1);
-    mbar_init(&sm.full[1], 1);
+    for (int b = 0; b < kStages; ++b) mbar_init(&sm.full[b], 1);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -165,7 +172,7 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
 
   const uint64_t pol = policy_evict_first();
   auto issue = [&](int t) {
-    const int buf = t & 1;
+    const int buf = t % kStages;
     const int k0 = k_start + t * kTile;
     fence_proxy_async_shared();
     mbar_arrive_expect_tx(&sm.full[buf], 2 * (D / 64) * kBoxBytes);
@@ -175,7 +182,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
       tma_load_3d(sm.v[buf][c], &tv, &sm.full[buf], c * 64, k0, bkv, pol);
     }
   };
-  if (tid == 0 && ntiles > 0 && !p.stall_loads) issue(0);
+  auto prefetch = [&](int t) {  // tile t into L2
+    const int k0 = k_start + t * kTile;
+#pragma unroll
+    for (int c = 0; c < D / 64; ++c) {
+      tma_prefetch_3d(&tk, c * 64, k0, bkv);
+      tma_prefetch_3d(&tv, c * 64, k0, bkv);
+    }
+  };
+  if (tid == 0 && !p.stall_loads) {
+    for (int u = 0; u < kStages - 1 && u < ntiles; ++u) issue(u);
+    for (int u = kStages - 1; u < kStages - 1 + kPrefetch && u < ntiles; ++u) prefetch(u);
+  }
 
   const int oc = tid % kChunks, og = tid / kChunks;  // PV: 16-byte chunk, row group
   float o[kRowsPer][8];
@@ -186,15 +204,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
 
   int t = 0;
   for (; t < ntiles; ++t) {
-    const int buf = t & 1;
+    const int buf = t % kStages;
     const int k0 = k_start + t * kTile;
-    // its buffer was released after tile t - 1
-    if (tid == 0 && t + 1 < ntiles && !p.stall_loads) issue(t + 1);
-    const bool ok = dec_wait(sm, &sm.full[buf], (t >> 1) & 1, p);
+    // tile t + kStages - 1 goes to the buffer released after tile t - 1
+    if (tid == 0 && !p.stall_loads) {
+      if (t + kStages - 1 < ntiles) issue(t + kStages - 1);
+      if (t + kStages - 1 + kPrefetch < ntiles) prefetch(t + kStages - 1 + kPrefetch);
+    }
+    const bool ok = dec_wait(sm, &sm.full[buf], (t / kStages) & 1, p);
     if (!__syncthreads_and(ok)) break;
 
-    // scores: thread = (key j, row group rg); rows r = rg, rg + kRowGroups, ...
     {
+      // scores: thread = (key j, row group rg); rows r = rg, rg + kRowGroups, ...
       constexpr int kRowsS = RM / kRowGroups > 0 ? RM / kRowGroups : 1;
       const int j = tid & (kTile - 1), rg = tid / kTile;
       // two independent packed partial sums per row keep the FMA chains short
@@ -262,11 +283,18 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
 
     // O += P V: thread = (16-byte chunk oc of a V row, group og: rows or keys)
     if constexpr (kKeyGroups) {
+      // rescale only when some row's max moved (alpha is exactly 1 otherwise: ex2(0));
+      // the test reads the same shared values in every thread, so it is CTA-uniform
+      bool moved = false;
 #pragma unroll
-      for (int r = 0; r < RM; ++r) {
-        const float a = r < R ? sm.alpha[r] : 0.f;
+      for (int r = 0; r < RM; ++r) moved |= r < R && sm.alpha[r] != 1.f;
+      if (moved) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[r][e] *= a;
+        for (int r = 0; r < RM; ++r) {
+          const float a = r < R ? sm.alpha[r] : 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[r][e] *= a;
+        }
       }
       const int nk = min(kTile, c1 - k0);
       for (int j = og; j < nk; j += kGroups) {
@@ -312,12 +340,12 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
   }
 
   if (t < ntiles) {
-    // aborted: let the copies still in flight (tiles t and t + 1) land, bounded,
-    // before the CTA exits
+    // aborted: let the copies still in flight (tiles t .. t + kStages - 1) land,
+    // bounded, before the CTA exits
     if (tid == 0 && !p.stall_loads) {
       const uint64_t t0 = globaltimer_ns();
-      for (int u = t; u < min(ntiles, t + 2); ++u)
-        while (!mbar_try_wait(&sm.full[u & 1], (u >> 1) & 1) &&
+      for (int u = t; u < min(ntiles, t + kStages); ++u)
+        while (!mbar_try_wait(&sm.full[u % kStages], (u / kStages) & 1) &&
                globaltimer_ns() - t0 < p.timeout_ns) {
         }
     }
@@ -397,16 +425,33 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
 }
 
 // ---------------------------------------------------------------- host side
-// Chunking of the keys: about DecCfg::kCtasPerSm CTAs per SM over the (B * Hkv)
-// groups, whole tiles.
+// Chunking of the keys over the (B * Hkv) groups, whole tiles.  The CTAs run in
+// waves of (SMs x DecCfg::kCtasPerSm); the time is about (waves) x (tiles per chunk
+// + a fixed cost per CTA), so the split count is chosen to minimise that product --
+// a grid just past a whole number of waves leaves most SMs idle in its last wave.
+// The plan is a function of the shape alone (B200: 148 SMs), so the workspace size
+// that depends on it needs no device.
 void decode_plan(int B, int Hkv, int S, int D, int* nsplit, int* chunk) {
-  const int groups = B * Hkv > 0 ? B * Hkv : 1;
+  constexpr int kSms = 148;
+  constexpr int kCtaCost = 2;  // prologue and merge record, in tile units
+  const int64_t groups = static_cast<int64_t>(B) * Hkv > 0 ? static_cast<int64_t>(B) * Hkv : 1;
   const int tiles = S > 0 ? (S + kTile - 1) / kTile : 1;
-  const int target = 148 * (D == 128 ? DecCfg<128>::kCtasPerSm : DecCfg<64>::kCtasPerSm);
-  int n = (target + groups - 1) / groups;
-  n = n < tiles ? n : tiles;
-  const int tiles_per = (tiles + n - 1) / n;
-  *chunk = tiles_per * kTile;
+  const int64_t slots = static_cast<int64_t>(kSms) *
+                        (D == 128 ? DecCfg<128>::kCtasPerSm : DecCfg<64>::kCtasPerSm);
+  int best_tiles = tiles;
+  int64_t best_cost = INT64_MAX;
+  for (int n = 1; n <= tiles && n <= 256; ++n) {
+    const int per = (tiles + n - 1) / n;      // tiles per chunk
+    const int used = (tiles + per - 1) / per; // splits actually used
+    if (used != n) continue;
+    const int64_t waves = (groups * used + slots - 1) / slots;
+    const int64_t cost = waves * (per + kCtaCost);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best_tiles = per;
+    }
+  }
+  *chunk = best_tiles * kTile;
   *nsplit = S > 0 ? (S + *chunk - 1) / *chunk : 1;
 }
 
