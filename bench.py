@@ -57,8 +57,8 @@ NCU_TRAFFIC = {
         "sources_sha256": "24dcbe326e4c71e45960251b4bd663ec11aeabefecacfde0809e516bb7658776",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_launches.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
-        "bytes": 1073943296 + 7651328, "sources": DECODE_SOURCES,
-        "sources_sha256": "7d84849a563dc019493219a78d36bc25086dc5688cd4c99eb537030c4bcbf4f0",
+        "bytes": 1095891200 + 4087808, "sources": DECODE_SOURCES,
+        "sources_sha256": "ed51ef5ef66ae457d6a4887d25400bc121847a78c942bb30900cee34df4f3110",
         "summary": "profiles/decode_split_kernel_L1_S32768_B8_H32_Hkv8_D128_full.md"},
 }
 

@@ -109,6 +109,7 @@ __device__ __forceinline__ bool dec_wait(Sm& sm, uint64_t* bar, uint32_t parity,
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
+#pragma unroll 1  // inlined at every wait site: keep the code small
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (sm.abort_flag) return false;

@@ -233,6 +233,9 @@ template <int D>
 __device__ __forceinline__ bool wait_slow(Smem<D>& sm, uint64_t* bar, uint32_t parity, const Params& p) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
+    // (not unrolled: every wait site inlines this loop, and the kernel's code must
+    // stay small enough for the instruction caches)
+#pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (sm.abort_flag) return false;
@@ -273,8 +276,11 @@ __device__ __forceinline__ bool wait_lane0(Smem<D>& sm, uint64_t* bar, uint32_t 
 // ready.  A slot's blocks run over its non-empty units back to back (block i of
 // the slot's stream); K_i goes to K-ring stage i % kKRing, V_i to V-ring stage
 // i % kVRing, so producer and MMA warp agree on stages without a shared order.
-// Every function that touches per-slot state takes the slot as a template
-// parameter, so that state lives in registers.
+// The MMA warp's per-slot functions take the slot as a template parameter, so that
+// the state of both slots lives in registers; the producer code takes it as a
+// runtime value, so that both producer warps run one copy of it (the kernel's code
+// size is held down for the instruction caches: each instantiation holds only its
+// own mask family and score_mod, and slow paths stay loops).
 
 // Producer-side position in a slot's block stream, with block indices fetched 32
 // at a time (one per lane) and the next unit's first chunk requested early.
@@ -356,8 +362,8 @@ struct ProdCounts {
   int k, v;  // K / V tiles issued on this slot
 };
 
-template <int D, int SLOT, bool BHM>
-__device__ __forceinline__ bool produce_k(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
+template <int D, bool BHM>
+__device__ __forceinline__ bool produce_k(int SLOT, Smem<D>& sm, const Params& p, const CUtensorMap* tq,
                                           const CUtensorMap* tk, ProdCursor<BHM>& c, ProdCounts& n,
                                           int kvb, uint64_t pol_q, uint64_t pol_kv) {
   using C = Cfg<D>;
@@ -376,8 +382,8 @@ __device__ __forceinline__ bool produce_k(Smem<D>& sm, const Params& p, const CU
   return true;
 }
 
-template <int D, int SLOT>
-__device__ __forceinline__ bool produce_v(Smem<D>& sm, const Params& p, const CUtensorMap* tv,
+template <int D>
+__device__ __forceinline__ bool produce_v(int SLOT, Smem<D>& sm, const Params& p, const CUtensorMap* tv,
                                           ProdCounts& n, int kvb, int bh, uint64_t pol_kv) {
   using C = Cfg<D>;
   const int st = n.v % C::kVRing;
@@ -391,8 +397,8 @@ __device__ __forceinline__ bool produce_v(Smem<D>& sm, const Params& p, const CU
 // One producer warp per slot.  Separate-P layout: K runs one block ahead of V
 // (K_0, K_1, V_0, K_2, V_1, ...), matching S_{i+1} being issued during softmax i.
 // Aliased layout: K_i, V_i, K_{i+1}, ...
-template <int D, int SLOT, bool BHM>
-__device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* tq,
+template <int D, bool BHM>
+__device__ void producer_role(int SLOT, Smem<D>& sm, const Params& p, const CUtensorMap* tq,
                               const CUtensorMap* tk, const CUtensorMap* tv) {
   using C = Cfg<D>;
   const int lane = threadIdx.x & 31;
@@ -409,7 +415,7 @@ __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* t
       pend_kvb = pc_block(c, p, lane);
       pend_bh = c.cur.kvbh;
       pend = true;
-      ok = produce_k<D, SLOT>(sm, p, tq, tk, c, n, pend_kvb, pol_q, pol_kv);
+      ok = produce_k<D>(SLOT, sm, p, tq, tk, c, n, pend_kvb, pol_q, pol_kv);
     }
     while (ok && pend) {
       pc_step(c, p, lane);
@@ -418,9 +424,9 @@ __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* t
       if (next) {
         next_kvb = pc_block(c, p, lane);
         next_bh = c.cur.kvbh;
-        ok = produce_k<D, SLOT>(sm, p, tq, tk, c, n, next_kvb, pol_q, pol_kv);
+        ok = produce_k<D>(SLOT, sm, p, tq, tk, c, n, next_kvb, pol_q, pol_kv);
       }
-      if (ok) ok = produce_v<D, SLOT>(sm, p, tv, n, pend_kvb, pend_bh, pol_kv);
+      if (ok) ok = produce_v<D>(SLOT, sm, p, tv, n, pend_kvb, pend_bh, pol_kv);
       pend = next;
       pend_kvb = next_kvb;
       pend_bh = next_bh;
@@ -428,8 +434,8 @@ __device__ void producer_role(Smem<D>& sm, const Params& p, const CUtensorMap* t
   } else {
     while (ok && c.has_cur) {
       const int kvb = pc_block(c, p, lane);
-      ok = produce_k<D, SLOT>(sm, p, tq, tk, c, n, kvb, pol_q, pol_kv);
-      if (ok) ok = produce_v<D, SLOT>(sm, p, tv, n, kvb, c.cur.kvbh, pol_kv);
+      ok = produce_k<D>(SLOT, sm, p, tq, tk, c, n, kvb, pol_q, pol_kv);
+      if (ok) ok = produce_v<D>(SLOT, sm, p, tv, n, kvb, c.cur.kvbh, pol_kv);
       pc_step(c, p, lane);
     }
   }
@@ -721,7 +727,7 @@ struct MaskCols<64> {
 // words `brow` is set (and the key exists).  Dead entries become -inf.
 template <int MK>
 __device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int a, int b, int kv0,
-                                           int dq, bool dq_uniform, const int32_t* docs,
+                                           int dq, const int32_t* docs,
                                            const uint32_t* brow) {
   if constexpr (MK == kMaskBitmap) {
     // the row's two words of keys kv0 .. kv0 + 63 (kv0 is a multiple of 64)
@@ -729,26 +735,27 @@ __device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int 
     MaskCols<0>::doc(x, a, b, static_cast<uint32_t>(w.x));
     MaskCols<32>::doc(x, a, b, static_cast<uint32_t>(w.y));
   } else if constexpr (MK == kMaskDoc) {
-    // bit i of `same`: the document of key kv0 + c*32 + i equals the row's; keys past
-    // S read the last id (in bounds) and are excluded by the range anyway
-    uint32_t same[2];
-    if (dq_uniform) {
-      // every row of the warp is in one document: lane i fetches key i's id and a
-      // ballot gives all rows the same bits
-      const int lane = threadIdx.x & 31;
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-        same[c] = __ballot_sync(0xffffffffu,
-                                ldg_nc(docs + min(kv0 + c * 32 + lane, p.S - 1)) == dq);
-    } else {
-      same[0] = same[1] = 0u;
-#pragma unroll
-      for (int c = 0; c < 2; ++c)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int kv = min(kv0 + c * 32 + i, p.S - 1);
-          same[c] |= (ldg_nc(docs + kv) == dq ? 1u : 0u) << i;
-        }
+    // bit i of `same[c]`: the document of key kv0 + c*32 + i equals the row's; keys
+    // past S read the last id (in bounds) and are excluded by the range anyway.  Lane
+    // i fetches the ids of keys i and 32 + i; then one pass per distinct document
+    // among the warp's rows (one pass unless a document starts inside the warp's 32
+    // rows): the ballot of "key's id == that document" gives its rows their bits.
+    // The loop condition is warp-uniform, so every ballot is taken by all lanes.
+    const int lane = threadIdx.x & 31;
+    const int kid0 = ldg_nc(docs + min(kv0 + lane, p.S - 1));
+    const int kid1 = ldg_nc(docs + min(kv0 + 32 + lane, p.S - 1));
+    uint32_t same[2] = {0u, 0u};
+    uint32_t todo = 0xffffffffu;  // lanes whose document has no pass yet
+    while (todo != 0u) {
+      const int v = __shfl_sync(0xffffffffu, dq, __ffs(todo) - 1);
+      const uint32_t b0 = __ballot_sync(0xffffffffu, kid0 == v);
+      const uint32_t b1 = __ballot_sync(0xffffffffu, kid1 == v);
+      const bool mine = dq == v;
+      if (mine) {
+        same[0] = b0;
+        same[1] = b1;
+      }
+      todo &= ~__ballot_sync(0xffffffffu, mine);
     }
     MaskCols<0>::doc(x, a, b, same[0]);
     MaskCols<32>::doc(x, a, b, same[1]);
@@ -820,7 +827,7 @@ __device__ __forceinline__ float exp_pack64(const float (&x)[64], float xs, floa
 
 // Softmax warpgroup of one slot: thread t owns row t of the slot's 128-row tile
 // (TMEM lane t), so row max and row sum need no shuffles.
-template <int D, int MK, bool BHM>
+template <int D, int MK, bool BHM, bool SC>
 __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int slot) {
   using C = Cfg<D>;
   const int t = threadIdx.x - slot * 128;   // row of the tile this thread owns
@@ -832,7 +839,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
   const bool bf16 = p.is_bf16 != 0;
   // Factor that turns the value kept in x[] into log2 units: the raw score is
   // kept (and scaled inside the exponent's FFMA) unless a score_mod rewrote it.
-  const float xs = p.softcap_on ? 1.f : p.scale_log2;
+  const float xs = SC ? 1.f : p.scale_log2;
   const bool split = p.split_p != 0 && !C::kSepP;
   UnitIter<BHM> it;
   it.init(p, slot);
@@ -855,13 +862,11 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
     // this unit's mask instance: its document ids / bitmap rows
     const int32_t* docs = MK == kMaskDoc ? p.doc_id + static_cast<size_t>(un.inst) * p.doc_len : nullptr;
     const int dq_own = (MK == kMaskDoc && valid) ? __ldg(docs + row) : 0;
-    // all valid rows of this warp in lane 0's document (rows past L do not matter);
-    // the shuffle is taken by every lane, outside any short-circuited expression.
-    // Then every lane, rows past L included, takes lane 0's id: in the ballot of
-    // apply_mask a lane compares the key it fetched for the whole warp.
+    // rows past L (only ever above the valid ones, so lane 0 is valid if any lane is)
+    // take lane 0's document: they add no document to the warp's passes in apply_mask.
+    // The shuffle is taken by every lane, outside any short-circuited expression.
     const int dq0 = __shfl_sync(0xffffffffu, dq_own, 0);
-    const bool dq_uniform = __all_sync(0xffffffffu, !valid || dq_own == dq0);
-    const int dq = dq_uniform ? dq0 : dq_own;
+    const int dq = valid ? dq_own : dq0;
     // tabulated mask: this row's words (rows past L read the last row, unused)
     const uint32_t* brow = MK == kMaskBitmap
                                ? p.bitmap + (static_cast<size_t>(un.inst) * p.L + min(row, p.L - 1)) *
@@ -888,14 +893,14 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         tc_fence_before();
         __syncwarp();
         if ((t & 31) == 0) mbar_arrive(&sm.s_empty[slot]);
-        if (p.softcap_on) softcap64(p, *reinterpret_cast<float(*)[64]>(x)), softcap64(p, *reinterpret_cast<float(*)[64]>(x + 64));
+        if constexpr (SC) softcap64(p, *reinterpret_cast<float(*)[64]>(x)), softcap64(p, *reinterpret_cast<float(*)[64]>(x + 64));
         if (!full) {
           const int a = lo - kvb * kBlockN;
           const int b = hi - kvb * kBlockN;
-          apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x), a, b, kvb * kBlockN, dq, dq_uniform,
-                     docs, brow);
+          apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x), a, b, kvb * kBlockN, dq, docs,
+                     brow);
           apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x + 64), a - 64, b - 64, kvb * kBlockN + 64, dq,
-                     dq_uniform, docs, brow);
+                     docs, brow);
         }
         const float mb = fmaxf(row_max64(*reinterpret_cast<float(*)[64]>(x)),
                                row_max64(*reinterpret_cast<float(*)[64]>(x + 64))) * xs;
@@ -936,13 +941,13 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
           float x[64];
           load_s_half(t_s + h * 64, x);
           if (!full)
-            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, dq_uniform, docs,
+            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, docs,
                            brow);
           rmax = fmaxf(rmax, row_max64(x));
         }
         float mb = rmax;
         if (rmax != -INFINITY) {
-          if (p.softcap_on) {
+          if constexpr (SC) {
             mb = p.cap_a - 2.f * p.cap_a * rcp_approx(ex2_approx(rmax * p.cap_k) + 1.f);
           } else {
             mb = rmax * xs;
@@ -992,7 +997,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
             }
             if (split) tmem_st32(t_p + 64, pl_hold);
           }
-          if (p.softcap_on) {  // x = log2(e) * c * tanh(s * scale / c)
+          if constexpr (SC) {  // x = log2(e) * c * tanh(s * scale / c)
 #pragma unroll
             for (int i = 0; i < 64; i += 2) {
               const float2 e = make_float2(ex2_approx(x[i] * p.cap_k), ex2_approx(x[i + 1] * p.cap_k));
@@ -1004,7 +1009,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
             }
           }
           if (!full)
-            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, dq_uniform, docs,
+            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, docs,
                            brow);
           // P = exp2(x * xs - m) as 16-bit pairs; with the split, P_hi = p truncated to
           // bf16 and P_lo = round(p - P_hi), so P_hi + P_lo carries ~16 significant bits.
@@ -1075,7 +1080,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
   }
 }
 
-template <int D, int MK, bool BHM>
+template <int D, int MK, bool BHM, bool SC>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
            const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ Params p) {
@@ -1129,15 +1134,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
 
   // Role dispatch; the final rendezvous is a named barrier over all threads.
   if (warp < kSoftmaxWarps) {
-    softmax_role<D, MK, BHM>(sm, p, tmem, warp / 4);
+    softmax_role<D, MK, BHM, SC>(sm, p, tmem, warp / 4);
     tc_fence_before();
     named_barrier_sync(1, kThreads);
     return;
   }
-  if (warp == kProducerWarp) {
-    producer_role<D, 0, BHM>(sm, p, &tmap_q, &tmap_k, &tmap_v);
-  } else if (warp == kProducerWarp + 1) {
-    producer_role<D, 1, BHM>(sm, p, &tmap_q, &tmap_k, &tmap_v);
+  if (warp == kProducerWarp || warp == kProducerWarp + 1) {
+    // one copy of the producer code for both slots (the slot is a runtime value)
+    producer_role<D, BHM>(warp - kProducerWarp, sm, p, &tmap_q, &tmap_k, &tmap_v);
   } else if (warp == kMmaWarp) {
     mma_role<D, BHM>(sm, p, tmem);
   }
@@ -1155,7 +1159,7 @@ bool make_map(CUtensorMap* map, const void* ptr, bool bf16, int D, int rows, int
   return make_tile_map(map, ptr, bf16, D, rows, bh, kBlockN);
 }
 
-template <int D, int MK, bool BHM>
+template <int D, int MK, bool BHM, bool SC>
 fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH, int L, int S,
                  const Params& prm, cudaStream_t stream) {
   CUtensorMap tq, tk, tv;
@@ -1173,7 +1177,7 @@ fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH,
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
     if (!done[dev]) {
-      FA_CUDA_CHECK(cudaFuncSetAttribute(fwd_kernel<D, MK, BHM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      FA_CUDA_CHECK(cudaFuncSetAttribute(fwd_kernel<D, MK, BHM, SC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem)));
       done[dev] = true;
     }
@@ -1182,7 +1186,7 @@ fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH,
   if (sms <= 0) return FA_ERR_CUDA;
   const int want = (prm.num_units + kNumSlots - 1) / kNumSlots;
   const int grid = want < sms ? want : sms;
-  FA_CUDA_CHECK(launch_pdl(fwd_kernel<D, MK, BHM>, dim3(grid), dim3(kThreads), smem, stream, tq, tk,
+  FA_CUDA_CHECK(launch_pdl(fwd_kernel<D, MK, BHM, SC>, dim3(grid), dim3(kThreads), smem, stream, tq, tk,
                            tv, prm));
   return FA_OK;
 }
@@ -1195,17 +1199,19 @@ extern "C" size_t fa_fwd_workspace_bytes(void) { return 256; }
 namespace fa {
 namespace {
 
-// The instantiation for a head dim, mask family and (broadcast or per-instance) mask.
-template <bool BHM>
+// The instantiation for a head dim, mask family, (broadcast or per-instance) mask and
+// score_mod: each kernel holds only the code it runs, which keeps it small enough
+// for the instruction caches.
+template <bool BHM, bool SC>
 fa_status launch_family(int kind, int D, const void* q, const void* k, const void* v, bool b16,
                         int L, int S, const Params& prm, cudaStream_t s) {
   switch (mask_family(kind) * 2 + (D == 64 ? 0 : 1)) {
-    case kMaskRange * 2: return launch<64, kMaskRange, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
-    case kMaskRange * 2 + 1: return launch<128, kMaskRange, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
-    case kMaskDoc * 2: return launch<64, kMaskDoc, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
-    case kMaskDoc * 2 + 1: return launch<128, kMaskDoc, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
-    case kMaskBitmap * 2: return launch<64, kMaskBitmap, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
-    default: return launch<128, kMaskBitmap, BHM>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskRange * 2: return launch<64, kMaskRange, BHM, SC>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskRange * 2 + 1: return launch<128, kMaskRange, BHM, SC>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskDoc * 2: return launch<64, kMaskDoc, BHM, SC>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskDoc * 2 + 1: return launch<128, kMaskDoc, BHM, SC>(q, k, v, b16, prm.BH, L, S, prm, s);
+    case kMaskBitmap * 2: return launch<64, kMaskBitmap, BHM, SC>(q, k, v, b16, prm.BH, L, S, prm, s);
+    default: return launch<128, kMaskBitmap, BHM, SC>(q, k, v, b16, prm.BH, L, S, prm, s);
   }
 }
 
@@ -1296,8 +1302,13 @@ fa_status fwd_impl(const void* q, const void* k, const void* v, int32_t dtype, i
   if (debug_stall(&prm.timeout_ns)) prm.stall_mma = 1;
   const cudaStream_t s = as_stream(stream);
   const bool b16 = dtype == FA_BF16;
-  if (prm.mask_b | prm.mask_h) return launch_family<true>(bm->kind, D, q, k, v, b16, L, S, prm, s);
-  return launch_family<false>(bm->kind, D, q, k, v, b16, L, S, prm, s);
+  const bool bhm = (prm.mask_b | prm.mask_h) != 0;
+  if (prm.softcap_on) {
+    return bhm ? launch_family<true, true>(bm->kind, D, q, k, v, b16, L, S, prm, s)
+               : launch_family<false, true>(bm->kind, D, q, k, v, b16, L, S, prm, s);
+  }
+  return bhm ? launch_family<true, false>(bm->kind, D, q, k, v, b16, L, S, prm, s)
+             : launch_family<false, false>(bm->kind, D, q, k, v, b16, L, S, prm, s);
 }
 
 }  // namespace

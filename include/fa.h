@@ -362,21 +362,31 @@ FA_API fa_status fa_flex_attention_decode(const void* q, const void* k, const vo
  * mask, score_mod and scale:
  *   q, out, dout  device (B, H, L, D);  k, v  device (B, H_kv, S, D);  dtype as forward.
  *   lse       device (B, H, L) fp32 from the forward (natural log; -inf rows get no gradient).
- *   bm        the forward's tables (broadcast masks; per-(b, h) tables: FA_ERR_UNSUPPORTED).
+ *   bm        the forward's tables; per-(batch, head) tables (mask_batch 1 or B,
+ *             mask_heads 1 or H, else FA_ERR_INVALID_ARG) as in the forward.
  *   q_num_blocks, q_indices, full_q_num_blocks, full_q_indices
- *             the column lists of bm from fa_block_mask_transpose.
+ *             the column lists of bm from fa_block_mask_transpose (instance-major for
+ *             per-(batch, head) tables, like bm's own arrays).
  *   dq        device (B, H, L, D);  dk, dv  device (B, H_kv, S, D);  in dtype, fully
- *             overwritten.  With H_kv < H, dk and dv of a K/V head are the sums over
- *             the H / H_kv query heads that read it (h / (H / H_kv) == kv head).
- *   workspace device, at least fa_bwd_workspace_bytes(B, H, L) bytes (row sums of
- *             dO * O; no initial contents needed).
- * q, k, v, dout 16-byte aligned, the other pointers 4-byte aligned (else
- * FA_ERR_INVALID_ARG); D 64 or 128; B * H * L and B * H_kv * S at most 2^33
- * (else FA_ERR_UNSUPPORTED).  Three kernels on `stream`: row sums of dO * O; dQ per
- * 128-query tile over its row lists; dK and dV per 128-key tile over its column lists
- * and the query heads sharing its K/V head (each output tile has one owner: no
- * atomics, deterministic).  Returns
- * FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED (nothing launched) or FA_ERR_CUDA.
+ *             overwritten (tiles no row or column list reaches are written as zeros).
+ *             With H_kv < H, dk and dv of a K/V head are the sums over the H / H_kv
+ *             query heads that read it (h / (H / H_kv) == kv head).
+ *   workspace device, at least fa_bwd_workspace_bytes(B, H, L) bytes: a 256-byte
+ *             header whose first 4 bytes are the device error word, then the row sums
+ *             of dO * O.  The caller ZEROES THE HEADER ONCE and may then reuse the
+ *             buffer for every call on one stream; the row sums need no initial
+ *             contents.  Calls that run concurrently need distinct workspaces.
+ * Alignment (checked on the host; a misaligned pointer returns FA_ERR_INVALID_ARG
+ * before any launch): q, k, v, dout, dq, dk, dv and workspace 16 bytes; out, lse and
+ * every table pointer 4 bytes.  D 64 or 128; B * H * L and B * H_kv * S at most 2^33
+ * (else FA_ERR_UNSUPPORTED).  Three kernels on `stream`: row sums of dO * O; dK and dV
+ * per 128-key tile over its column lists and the query heads sharing its K/V head;
+ * dQ per 128-query tile over its row lists.  Both gradient kernels run the products
+ * on the tcgen05 tensor cores with fp32 accumulators in tensor memory; each output
+ * tile has one owner (no atomics, deterministic).  Bounded device waits that run out
+ * set the error word, which fa_get_last_device_error(workspace, stream) reports as
+ * FA_ERR_TIMEOUT.  Returns FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED (nothing
+ * launched) or FA_ERR_CUDA.
  */
 FA_API size_t fa_bwd_workspace_bytes(int32_t B, int32_t H, int32_t L);
 FA_API fa_status fa_flex_attention_bwd(const void* q, const void* k, const void* v, const void* out,
@@ -390,8 +400,8 @@ FA_API fa_status fa_flex_attention_bwd(const void* q, const void* k, const void*
 
 /*
  * Testing hook for failure detection (no counterpart on the pages).  While `on`,
- * the forward kernel's MMA warp issues nothing and the decode kernel loads no K/V
- * tile, so the kernels' bounded waits run out after `wait_limit_ns` (0: the
+ * the forward kernel's MMA warp issues nothing and the decode and backward kernels
+ * load no K/V tile, so the kernels' bounded waits run out after `wait_limit_ns` (0: the
  * default 2 s); each kernel stops, drains what it has in flight, frees TMEM and
  * returns, and fa_get_last_device_error on that call's workspace then reports
  * FA_ERR_TIMEOUT (the outputs of that call are invalid).  Nothing faults, traps or
@@ -399,10 +409,11 @@ FA_API fa_status fa_flex_attention_bwd(const void* q, const void* k, const void*
  */
 FA_API void fa_debug_set_mma_stall(int32_t on, uint64_t wait_limit_ns);
 
-/* Synchronises `stream`, then reads and clears the error word that the forward
- * kernel keeps in `workspace`.  Returns FA_ERR_TIMEOUT if a bounded device wait gave
- * up since the last query (the outputs of that call are then invalid), FA_ERR_CUDA
- * if the stream reports an error, FA_OK otherwise. */
+/* Synchronises `stream`, then reads and clears the error word that the forward,
+ * decode or backward kernels keep at the start of `workspace`.  Returns
+ * FA_ERR_TIMEOUT if a bounded device wait gave up since the last query (the outputs
+ * of that call are then invalid), FA_ERR_CUDA if the stream reports an error,
+ * FA_OK otherwise. */
 FA_API fa_status fa_get_last_device_error(void* workspace, void* stream);
 
 /* Static, human-readable name of a status code. */
