@@ -53,12 +53,12 @@ DECODE_SOURCES = ("block_sparse_attention_create_b200/csrc/decode.cu",
                   "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
 NCU_TRAFFIC = {
     "swa256_L32768_B1_H8_D64_bf16": {
-        "bytes": 101097685 + 2582485, "sources": FWD_SOURCES,
-        "sources_sha256": "24dcbe326e4c71e45960251b4bd663ec11aeabefecacfde0809e516bb7658776",
+        "bytes": 100963840 + 4910336, "sources": FWD_SOURCES,
+        "sources_sha256": "b075d91bfb86d0a0e0f9e4ba0f1cc2955922306600eb73f8d451fd2e923eef5c",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_launches.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
-        "bytes": 1095891200 + 4087808, "sources": DECODE_SOURCES,
-        "sources_sha256": "ed51ef5ef66ae457d6a4887d25400bc121847a78c942bb30900cee34df4f3110",
+        "bytes": 1095234304 + 3778560, "sources": DECODE_SOURCES,
+        "sources_sha256": "3611ac1405d4434173ffc1735da3b2a68ea01a108d306cfba3a397acb93a3dd5",
         "summary": "profiles/decode_split_kernel_L1_S32768_B8_H32_Hkv8_D128_full.md"},
 }
 
