@@ -145,22 +145,37 @@ classify_rows_kernel(int kind, int window, const int32_t* __restrict__ doc_all,
         c = (q_whole && k0 + kBlock <= kv_len) ? 2 : 1;
       } else {
         // Not FULL: that needs one id on both sides.  Live iff some key k has a query
-        // q >= k of its document: lane l takes keys k0 + l + 32 r and scans the
-        // block's query ids (staged in shared memory) from max(q0, k) up, stopping at
-        // the first match.
-        bool any = false;
-        for (int r = 0; r < 4 && !any; ++r) {
+        // q >= k of its document.  One pass per distinct id among the block's keys,
+        // lowest key first: that key k_v is the first of its id v, so the block is
+        // live iff some query q >= k_v has id v (the warp tests the block's query
+        // ids, staged in shared memory, 4 per lane); then every key of id v is done.
+        // Keys past k1 take no pass.  Control flow is warp-uniform (ballots).
+        int kid[4];
+        uint32_t todo[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
           const int64_t kv = k0 + lane + 32 * r;
-          if (kv > k1) break;
-          const int dk = __ldg(doc + kv);
-          for (int64_t q = kv > q0 ? kv : q0; q <= q1; ++q) {
-            if (q_ids[q - q0] == dk) {
-              any = true;
-              break;
-            }
-          }
+          kid[r] = kv <= k1 ? __ldg(doc + kv) : 0;
+          todo[r] = __ballot_sync(0xffffffffu, kv <= k1);
         }
-        c = __any_sync(0xffffffffu, any) ? 1 : 0;
+        bool live = false;
+        while (!live && (todo[0] | todo[1] | todo[2] | todo[3]) != 0u) {
+          const int r0 = todo[0] ? 0 : (todo[1] ? 1 : (todo[2] ? 2 : 3));
+          const int src_lane = __ffs(todo[r0]) - 1;
+          const int kidr = r0 == 0 ? kid[0] : (r0 == 1 ? kid[1] : (r0 == 2 ? kid[2] : kid[3]));
+          const int v = __shfl_sync(0xffffffffu, kidr, src_lane);
+          const int64_t kmin = k0 + src_lane + 32 * r0;
+          bool hit = false;
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int64_t q = q0 + lane + 32 * r;
+            hit |= q <= q1 && q >= kmin && q_ids[q - q0] == v;
+          }
+          live = __any_sync(0xffffffffu, hit);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) todo[r] &= ~__ballot_sync(0xffffffffu, kid[r] == v);
+        }
+        c = live ? 1 : 0;
       }
       if (lane == 0) cls[j] = c;
     }

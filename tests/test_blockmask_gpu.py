@@ -52,6 +52,26 @@ def test_ragged_tables_bit_exact(kind, L, S, window):
     _check(kind, L, S, window, doc)
 
 
+@pytest.mark.parametrize("pattern", ["random300", "descending_runs", "stride37", "one_per_block_end"])
+def test_document_tables_many_ids(pattern):
+    """Document classification with many distinct ids per block (each distinct key id
+    of a block takes one pass in the builder) and with ids whose only matches lie
+    above the causal diagonal (q < k), against the brute-force oracle."""
+    L = S = 1000
+    pos = torch.arange(L, dtype=torch.int32)
+    if pattern == "random300":
+        doc = torch.randint(0, 300, (L,), generator=torch.Generator().manual_seed(7), dtype=torch.int32)
+    elif pattern == "descending_runs":
+        doc = (L - 1 - pos) // 50
+    elif pattern == "stride37":
+        doc = pos % 37
+    else:  # each block's last key shares its id with only the next block's first query
+        doc = pos.clone()
+        doc[127::128] = -1 - (pos[127::128] // 128)
+        doc[128::128] = -1 - (pos[128::128] // 128 - 1)
+    _check(2, L, S, 0, doc.to(torch.int32))
+
+
 def test_page1_densities_from_gpu_tables(golden):
     """The densities printed on page 1, recomputed from the GPU's tables."""
     for pattern, seq, window, _, blk_pct in golden("page1_density_table.txt"):
