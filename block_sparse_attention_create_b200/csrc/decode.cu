@@ -30,19 +30,20 @@ namespace {
 
 constexpr int kTile = 64;            // keys per K/V tile
 constexpr int kMaxRows = FA_DECODE_MAX_ROWS;
-// Threads per CTA and CTAs per SM by head dim: D = 128 runs 8 warps, two CTAs per
-// SM; D = 64 runs 4 warps, three per SM.  The grid is sized for that many CTAs.
+// Threads per CTA and CTAs per SM by head dim and row bound RM: D = 128 runs 8 warps,
+// three CTAs per SM for RM = 4 (two ring stages, 85 registers) and two otherwise;
+// D = 64 runs 4 warps, three per SM.  The grid is sized for that many CTAs.
+__host__ __device__ constexpr int dec_ctas_per_sm(int D, int RM) { return D == 128 && RM > 4 ? 2 : 3; }
 template <int D>
 struct DecCfg {
   static constexpr int kThreads = D == 128 ? 256 : 128;
-  static constexpr int kCtasPerSm = D == 128 ? 2 : 3;
 };
 constexpr int kBoxBytes = kTile * 128;  // one TMA box: 64 keys x 64 elements
 // K/V tiles in flight per CTA: a ring of stages(D, RM) tiles, plus L2 prefetches
 // of the tiles kPrefetch further on, so that enough bytes are on their way to cover
 // the DRAM latency (one 32 KB tile per CTA was not).  Three stages, except at D =
-// 128 with 32 rows, where two keep two CTAs per SM in shared memory.
-__host__ __device__ constexpr int dec_stages(int D, int RM) { return D == 128 && RM == 32 ? 2 : 3; }
+// 128 with 4 rows (three CTAs per SM) or 32 rows (two), where two fit in shared memory.
+__host__ __device__ constexpr int dec_stages(int D, int RM) { return D == 128 && RM != 8 ? 2 : 3; }
 constexpr int kPrefetch = 4;
 constexpr int kDecWorkspaceHeader = 256;  // word 0: device error flags
 constexpr float kDecLog2e = 1.4426950408889634f;
@@ -126,7 +127,7 @@ __device__ __forceinline__ bool dec_wait(Sm& sm, uint64_t* bar, uint32_t parity,
 // the key groups are summed once per CTA at the end; with RM = 32 a thread keeps
 // a few rows over all keys.
 template <int D, int RM>
-__global__ void __launch_bounds__(DecCfg<D>::kThreads, DecCfg<D>::kCtasPerSm)
+__global__ void __launch_bounds__(DecCfg<D>::kThreads, dec_ctas_per_sm(D, RM))
 decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                     const __grid_constant__ DecParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -427,18 +428,18 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
 
 // ---------------------------------------------------------------- host side
 // Chunking of the keys over the (B * Hkv) groups, whole tiles.  The CTAs run in
-// waves of (SMs x DecCfg::kCtasPerSm); the time is about (waves) x (tiles per chunk
+// waves of (SMs x CTAs per SM); the time is about (waves) x (tiles per chunk
 // + a fixed cost per CTA), so the split count is chosen to minimise that product --
 // a grid just past a whole number of waves leaves most SMs idle in its last wave.
 // The plan is a function of the shape alone (B200: 148 SMs), so the workspace size
 // that depends on it needs no device.
-void decode_plan(int B, int Hkv, int S, int D, int* nsplit, int* chunk) {
+void decode_plan(int B, int Hkv, int S, int D, int rows, int* nsplit, int* chunk) {
   constexpr int kSms = 148;
   constexpr int kCtaCost = 2;  // prologue and merge record, in tile units
   const int64_t groups = static_cast<int64_t>(B) * Hkv > 0 ? static_cast<int64_t>(B) * Hkv : 1;
   const int tiles = S > 0 ? (S + kTile - 1) / kTile : 1;
-  const int64_t slots = static_cast<int64_t>(kSms) *
-                        (D == 128 ? DecCfg<128>::kCtasPerSm : DecCfg<64>::kCtasPerSm);
+  const int rm = rows <= 4 ? 4 : (rows <= 8 ? 8 : 32);  // the kernel instantiation
+  const int64_t slots = static_cast<int64_t>(kSms) * dec_ctas_per_sm(D, rm);
   int best_tiles = tiles;
   int64_t best_cost = INT64_MAX;
   for (int n = 1; n <= tiles && n <= 256; ++n) {
@@ -496,7 +497,7 @@ extern "C" size_t fa_decode_workspace_bytes(int32_t B, int32_t H, int32_t H_kv, 
                                             int32_t S, int32_t D) {
   if (B < 0 || H < 0 || H_kv < 1 || L < 0 || S < 0 || D < 0) return 0;
   int nsplit = 0, chunk = 0;
-  fa::decode_plan(B, H_kv, S, D, &nsplit, &chunk);
+  fa::decode_plan(B, H_kv, S, D, H_kv > 0 && H > 0 ? (H / H_kv) * L : L, &nsplit, &chunk);
   return fa::kDecWorkspaceHeader + static_cast<size_t>(B) * H * L * nsplit * (D + 2) * sizeof(float);
 }
 
@@ -548,7 +549,7 @@ extern "C" fa_status fa_flex_attention_decode(const void* q, const void* k, cons
   prm.G = G;
   prm.L = L;
   prm.S = S;
-  decode_plan(B, H_kv, S, D, &prm.nsplit, &prm.chunk);
+  decode_plan(B, H_kv, S, D, G * L, &prm.nsplit, &prm.chunk);
   prm.mask = mask;
   prm.window = mask == FA_DECODE_SLIDING_WINDOW ? window : 0;
   prm.softcap_on = score_kind == FA_SCORE_TANH_SOFTCAP ? 1 : 0;

@@ -22,6 +22,14 @@ def fa():
     return _binding
 
 
+def _gpu_visible():
+    """The calls here pass fake device addresses.  One that passes every host check
+    would launch a kernel on them, so it is made only where no GPU is visible: there
+    it fails with FA_ERR_CUDA before any launch.  With a GPU it is skipped."""
+    import torch
+    return torch.cuda.is_available()
+
+
 def declared_symbols():
     text = open(HEADER).read()
     return sorted(set(re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)))
@@ -274,7 +282,8 @@ def test_bwd_rejects_bad_arguments_on_host(fa):
     bm_bh.mask_heads = 3                            # per-head tables for 2 heads
     assert _bwd(fa, bm_bh) == E
     bm_bh.mask_heads = 2                            # per-(b, h) tables: past the checks
-    assert _bwd(fa, bm_bh) == fa.FA_ERR_CUDA        # (no GPU here)
+    if not _gpu_visible():
+        assert _bwd(fa, bm_bh) == fa.FA_ERR_CUDA    # (no GPU here)
     # nothing to do: no query rows and no key rows
     assert _bwd(fa, bm, B=0) == fa.FA_OK
 
@@ -385,8 +394,9 @@ def test_forward_rejects_each_misaligned_pointer_before_any_launch(fa):
         return fa.fa_flex_attention_fwd(vp(ptrs["q"]), vp(ptrs["k"]), vp(ptrs["v"]), fa.FA_BF16,
                                         1, 2, 256, 256, 64, ctypes.byref(bm), 0, 0.0, 0.0,
                                         vp(ptrs["out"]), vp(ptrs["lse"]), vp(ptrs["ws"]), None)
-    for kind in (0, 2, 3):
-        assert call(good, _fake_mask(fa, kind=kind)) == fa.FA_ERR_CUDA
+    if not _gpu_visible():
+        for kind in (0, 2, 3):
+            assert call(good, _fake_mask(fa, kind=kind)) == fa.FA_ERR_CUDA
     for name, off in (("q", 8), ("k", 4), ("v", 2), ("out", 8), ("lse", 2), ("ws", 1)):
         bad = dict(good)
         bad[name] += off
@@ -409,7 +419,8 @@ def test_decode_rejects_misaligned_pointers_before_any_launch(fa):
         return fa.fa_flex_attention_decode(vp(p["q"]), vp(p["k"]), vp(p["v"]), fa.FA_BF16, 1, 4, 1,
                                            1, 1024, 64, fa.FA_DECODE_CAUSAL, 0, 0, 0.0, 0.0,
                                            vp(p["out"]), vp(p["lse"]), vp(p["ws"]), need, None)
-    assert call(good) == fa.FA_ERR_CUDA
+    if not _gpu_visible():
+        assert call(good) == fa.FA_ERR_CUDA
     for name, off in (("q", 8), ("k", 4), ("v", 2), ("out", 8), ("lse", 2), ("ws", 8)):
         bad = dict(good)
         bad[name] += off
