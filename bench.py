@@ -57,8 +57,8 @@ NCU_TRAFFIC = {
         "sources_sha256": "b075d91bfb86d0a0e0f9e4ba0f1cc2955922306600eb73f8d451fd2e923eef5c",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_launches.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
-        "bytes": 1095234304 + 3778560, "sources": DECODE_SOURCES,
-        "sources_sha256": "3611ac1405d4434173ffc1735da3b2a68ea01a108d306cfba3a397acb93a3dd5",
+        "bytes": 1110748416 + 4076544, "sources": DECODE_SOURCES,
+        "sources_sha256": "8610d608cfd36084d3746d3a9a1b1c5d3acf07ae8bd176a467a52daae35d9e2f",
         "summary": "profiles/decode_split_kernel_L1_S32768_B8_H32_Hkv8_D128_full.md"},
 }
 
