@@ -275,10 +275,10 @@ FA_API fa_status fa_flex_attention_fwd(const void* q, const void* k, const void*
  * file-scope device array of FA_NOALLOC_SCRATCH_BYTES (4 MiB) per device: the
  * tables take about 8 * nQ * nKV bytes, so square problems fit up to
  * L = S = 723 * 128 = 92544 (L = S = 32768 takes 0.5 MiB).  The call allocates
- * nothing and calls no allocating routine.  Each call clears the error word, builds the tables, runs
- * the forward, and, if `device_error` is not NULL (device or pinned host int32),
- * copies the error word there in stream order: 0 = success, nonzero = a bounded
- * device wait gave up and the outputs are invalid.  B*H == 0 or L == 0 is a no-op
+ * nothing and calls no allocating routine.  Each call clears the error word,
+ * builds the tables, runs the forward, and, if `device_error` is not NULL (device
+ * or pinned host int32), copies the error word there in stream order: 0 = success,
+ * nonzero = a bounded device wait gave up and the outputs are invalid.  B*H == 0 or L == 0 is a no-op
  * returning FA_OK (nothing launched, *device_error untouched).
  *
  * Every call on a device shares that one array: calls whose GPU work may overlap
@@ -291,9 +291,10 @@ FA_API fa_status fa_flex_attention_fwd(const void* q, const void* k, const void*
  * device current; in that lookup the CUDA runtime loads the library's device
  * module, which reserves the array's 4 MiB on the device.  Later calls read the
  * cached address.  Make that first call before any stream capture and outside
- * sections that must not wait on the device; after it, calls reserve nothing.  Returns FA_ERR_SCRATCH_TOO_SMALL (nothing launched) when the tables
- * of an (L, S) problem do not fit, the argument errors of the two calls above
- * (nothing launched), or FA_ERR_CUDA.
+ * sections that must not wait on the device; after it, calls reserve nothing.
+ * Returns FA_ERR_SCRATCH_TOO_SMALL (nothing launched) when the tables of an
+ * (L, S) problem do not fit, the argument errors of the two calls above (nothing
+ * launched), or FA_ERR_CUDA.
  */
 #define FA_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
 FA_API fa_status fa_flex_attention_fwd_noalloc(const void* q, const void* k, const void* v,
