@@ -705,21 +705,33 @@ __device__ __forceinline__ float keep_if_in_doc(float v, int a, int b, uint32_t 
   return r;
 }
 
+// Columns I .. I|31 (one 32-column word) with a per-column document / bitmap bit.
 template <int I>
 struct MaskCols {
-  static __device__ __forceinline__ void range(float (&x)[64], int a, int b) {
-    x[I] = keep_if_in<I>(x[I], a, b);
-    MaskCols<I + 1>::range(x, a, b);
-  }
   static __device__ __forceinline__ void doc(float (&x)[64], int a, int b, uint32_t same) {
     x[I] = keep_if_in_doc<I>(x[I], a, b, same);
     if constexpr (I % 32 != 31) MaskCols<I + 1>::doc(x, a, b, same);
   }
 };
-template <>
-struct MaskCols<64> {
-  static __device__ __forceinline__ void range(float (&)[64], int, int) {}
+
+// Columns I .. E-1 against the interval [a, b].
+template <int I, int E>
+struct RangeCols {
+  static __device__ __forceinline__ void apply(float (&x)[64], int a, int b) {
+    x[I] = keep_if_in<I>(x[I], a, b);
+    if constexpr (I + 1 < E) RangeCols<I + 1, E>::apply(x, a, b);
+  }
 };
+
+// Interval rule on the 32 columns C0 .. C0+31, decided once for the warp where it
+// can be: every row of the warp keeps them (amax <= C0 and bmin >= C0 + 31), or
+// every row drops them (bmax < C0 or amin > C0 + 31); otherwise each row tests its
+// columns.  The bounds are the warp's extremes of a and b (warp-uniform branches).
+template <int C0>
+__device__ __forceinline__ void range_chunk(float (&x)[64], int a, int b, int amin, int amax,
+                                            int bmin, int bmax) {
+  if (!(amax <= C0 && bmin >= C0 + 31)) RangeCols<C0, C0 + 32>::apply(x, a, b);
+}
 
 // Mask rule on 64 columns of a PARTIAL block: column i (key kv0 + i) is live iff
 // a <= i <= b (causal / window interval, clipped to the keys that exist) and, for
@@ -760,7 +772,10 @@ __device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int 
     MaskCols<0>::doc(x, a, b, same[0]);
     MaskCols<32>::doc(x, a, b, same[1]);
   } else {
-    MaskCols<0>::range(x, a, b);
+    const int amin = __reduce_min_sync(0xffffffffu, a), amax = __reduce_max_sync(0xffffffffu, a);
+    const int bmin = __reduce_min_sync(0xffffffffu, b), bmax = __reduce_max_sync(0xffffffffu, b);
+    range_chunk<0>(x, a, b, amin, amax, bmin, bmax);
+    range_chunk<32>(x, a, b, amin, amax, bmin, bmax);
   }
 }
 
