@@ -57,9 +57,9 @@ NCU_TRAFFIC = {
         "sources_sha256": "241e471ad0698b045586e1b945537b4434067834ee93939e5e93d87ec87aa45d",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_launches.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
-        "bytes": 1110748416 + 4076544, "sources": DECODE_SOURCES,
-        "sources_sha256": "8610d608cfd36084d3746d3a9a1b1c5d3acf07ae8bd176a467a52daae35d9e2f",
-        "summary": "profiles/decode_split_kernel_L1_S32768_B8_H32_Hkv8_D128_full.md"},
+        "bytes": 1073846272 + 3377152, "sources": DECODE_SOURCES,
+        "sources_sha256": "341606de9e93c984068ada4eb45c9edef0382c4efdc6268e54ce65985197534a",
+        "summary": "profiles/decode_mma_kernel_L1_S32768_B8_H32_Hkv8_D128_full.md"},
 }
 
 
@@ -607,8 +607,13 @@ def main():
         roof = {"bound": "tensor", "achieved": fwd_tflops, "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": tensor_frac, "traffic": ncu_traffic(w)}
     roof["peak_source"] = f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"
-    roof["kernel"] = ("decode_split_kernel (fa_flex_attention_decode)" if is_decode(w)
-                      else "fwd_kernel (fa_flex_attention_fwd)")
+    if is_decode(w):
+        # the chunk kernel for at most 8 query rows per K/V head, else the CUDA-core one
+        rows = (w.H // w.n_kv_heads) * w.L
+        roof["kernel"] = (("decode_mma_kernel" if rows <= 8 else "decode_split_kernel")
+                          + " + decode_combine_kernel (fa_flex_attention_decode)")
+    else:
+        roof["kernel"] = "fwd_kernel (fa_flex_attention_fwd)"
     page_ms = PAGE_FWD_MS.get(w.name)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": r["total_ms"] / args.steps,

@@ -2,17 +2,19 @@
 // after S - L cached keys, the causal mask aligned to the lower right (query i sits
 // at key position S - L + i), optionally within a window of W keys, or no mask.
 // L is small (a token or a short chunk), S long, so the work is reading K and V
-// once: the path is bound by HBM, not by the tensor cores, and runs on the CUDA
-// cores.
+// once: the path is bound by HBM.
 //
 // Split-KV: CTA (split, b * Hkv + kvh) takes every query row that reads K/V head
 // kvh -- the H / Hkv query heads of the group times the L queries, R <= 32 rows --
 // against one contiguous chunk of keys, streamed through shared memory in 64-key
-// tiles by TMA (128-byte swizzle, double-buffered, bounded mbarrier waits).  It
+// tiles by TMA (128-byte swizzle, a ring of stages, bounded mbarrier waits).  It
 // leaves the chunk's running max, sum and unnormalised output per row in the
 // workspace; a second kernel merges the chunks of each row (rescaling each by
 // 2^(m_chunk - m)) into out and LSE.  Chunks no row can see (sliding window) load
-// nothing.
+// nothing.  Two kernels do the chunk: for R <= 8 rows (grouped-query decode of one
+// or a few tokens) `decode_mma_kernel`, whose warps keep private softmax states and
+// run both products on warp-level tensor-core tiles, so the instruction stream stays
+// well below the HBM time; for more rows `decode_split_kernel` on the CUDA cores.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -30,10 +32,13 @@ namespace {
 
 constexpr int kTile = 64;            // keys per K/V tile
 constexpr int kMaxRows = FA_DECODE_MAX_ROWS;
-// Threads per CTA and CTAs per SM by head dim and row bound RM: D = 128 runs 8 warps,
-// three CTAs per SM for RM = 4 (two ring stages, 85 registers) and two otherwise;
-// D = 64 runs 4 warps, three per SM.  The grid is sized for that many CTAs.
-__host__ __device__ constexpr int dec_ctas_per_sm(int D, int RM) { return D == 128 && RM > 4 ? 2 : 3; }
+// CTAs per SM of the chunk kernel for R rows: the tensor-core kernel (R <= 8) runs
+// three; the CUDA-core kernel runs 8 warps, two CTAs per SM, at D = 128 and 4 warps,
+// three per SM, at D = 64.  The grid is sized for that many CTAs.
+__host__ __device__ constexpr int split_ctas_per_sm(int D) { return D == 128 ? 2 : 3; }
+__host__ __device__ constexpr int dec_ctas_per_sm(int D, int rows) {
+  return rows <= 8 ? 3 : split_ctas_per_sm(D);
+}
 template <int D>
 struct DecCfg {
   static constexpr int kThreads = D == 128 ? 256 : 128;
@@ -42,8 +47,8 @@ constexpr int kBoxBytes = kTile * 128;  // one TMA box: 64 keys x 64 elements
 // K/V tiles in flight per CTA: a ring of stages(D, RM) tiles, plus L2 prefetches
 // of the tiles kPrefetch further on, so that enough bytes are on their way to cover
 // the DRAM latency (one 32 KB tile per CTA was not).  Three stages, except at D =
-// 128 with 4 rows (three CTAs per SM) or 32 rows (two), where two fit in shared memory.
-__host__ __device__ constexpr int dec_stages(int D, int RM) { return D == 128 && RM != 8 ? 2 : 3; }
+// 128 with 32 rows, where two keep two CTAs per SM in shared memory.
+__host__ __device__ constexpr int dec_stages(int D, int RM) { return D == 128 && RM == 32 ? 2 : 3; }
 constexpr int kPrefetch = 4;
 constexpr int kDecWorkspaceHeader = 256;  // word 0: device error flags
 constexpr float kDecLog2e = 1.4426950408889634f;
@@ -122,12 +127,13 @@ __device__ __forceinline__ bool dec_wait(Sm& sm, uint64_t* bar, uint32_t parity,
   }
 }
 
-// RM: bound on the rows R, 4, 8 or 32.  With RM <= 8 every PV thread keeps all rows
+// RM: bound on the rows R (the path launches it with RM = 32 for R > 8; at most 8
+// rows take decode_mma_kernel).  With RM <= 8 every PV thread keeps all rows
 // for one 16-byte column chunk over a subset of the tile's keys (key group), and
 // the key groups are summed once per CTA at the end; with RM = 32 a thread keeps
 // a few rows over all keys.
 template <int D, int RM>
-__global__ void __launch_bounds__(DecCfg<D>::kThreads, dec_ctas_per_sm(D, RM))
+__global__ void __launch_bounds__(DecCfg<D>::kThreads, split_ctas_per_sm(D))
 decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                     const __grid_constant__ DecParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -399,6 +405,299 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
   }
 }
 
+// ---------------------------------------------------------------- at most 8 rows
+// The common grouped-query decode (R = (H / H_kv) * L <= 8 rows per K/V head) on
+// warp-level tensor-core tiles (16 x 8 x 16), with each warp keeping its own online
+// softmax state over its keys, so that a tile needs no barrier across the CTA.
+// Warp w of the 4 compute warps takes keys 16w .. 16w + 15 of every 64-key tile:
+//   S^T (16 keys x 8 rows) = K_w Q^T      (A = K rows by ldmatrix from the swizzled
+//                                          TMA tile, B = Q^T held in registers for
+//                                          the whole chunk; rows R .. 7 are zero)
+//   O^T (D x 8 rows)      += V_w^T P      (A = V^T by transposing ldmatrix, B = P:
+//                                          the S^T fragment rounded to 16 bits and
+//                                          transposed in registers by movmatrix)
+// Lane l holds rows 2(l % 4) and 2(l % 4) + 1 of both fragments, so its online
+// softmax state and its share of O belong to the same two rows.  A fifth warp
+// keeps the ring of tiles full; the 4 warps' states are merged at the end.  The
+// score is the fp32 accumulation of 16-bit products, scaled in fp32.
+constexpr int kMdWarps = 4;                      // compute warps
+constexpr int kMdThreads = (kMdWarps + 1) * 32;  // + the producer warp
+constexpr int kMdRows = 8;                       // the MMA's N: rows R .. 7 are padding
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ uint32_t movm_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+// d += a b: m16n8k16, 16-bit A and B of one type, fp32 accumulators
+template <bool BF16>
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  if constexpr (BF16) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+// Shared-memory address of 16-byte chunk c (elements 8c .. 8c + 7) of key row j of a
+// swizzled tile: box c / 8, position (c % 8) ^ (j % 8) inside the row's 128 bytes.
+template <int NB>
+__device__ __forceinline__ uint32_t chunk_addr(const uint8_t (&tile)[NB][kBoxBytes], int j, int c) {
+  return smem_u32(&tile[c >> 3][j * 128 + (((c & 7) ^ (j & 7)) << 4)]);
+}
+__device__ __forceinline__ uint32_t pack_16(float lo, float hi, bool bf16) {
+  if (bf16) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int D>
+struct __align__(1024) MdSmem {
+  static constexpr int kStages = D == 128 ? 2 : 3;
+  uint8_t k[kStages][D / 64][kBoxBytes];
+  uint8_t v[kStages][D / 64][kBoxBytes];
+  float wm[kMdWarps][kMdRows], wl[kMdWarps][kMdRows];
+  uint64_t full[kStages], empty[kStages];
+  volatile int abort_flag;
+};
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kMdThreads, 3)
+decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                  const __grid_constant__ DecParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t base = smem_u32(smem_raw);
+  using Sm = MdSmem<D>;
+  constexpr int kStages = Sm::kStages;
+  constexpr int kKs = D / 16;  // k-steps of S = 16-dim slices; m-tiles of O^T
+  Sm& sm = *reinterpret_cast<Sm*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int split = blockIdx.x, bkv = blockIdx.y;
+  const int b = bkv / p.Hkv, kvh = bkv - b * p.Hkv;
+  const int R = p.G * p.L;
+
+  int k_start = split * p.chunk;
+  const int c1 = min(p.S, k_start + p.chunk);
+  if (p.mask == FA_DECODE_SLIDING_WINDOW) k_start = max(k_start, p.S - p.L - p.window + 1);
+  const int ntiles = k_start < c1 ? (c1 - k_start + kTile - 1) / kTile : 0;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kMdWarps);
+    }
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  // this lane's rows in both fragments (2q, 2q + 1) and its key / dim row (l / 4)
+  const int q4 = lane & 3, g8 = lane >> 2;
+  const int n0 = 2 * q4, n1 = 2 * q4 + 1;
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+  float o[kKs][4];
+#pragma unroll
+  for (int t = 0; t < kKs; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[t][e] = 0.f;
+
+  if (warp == kMdWarps) {
+    // producer: tile t into stage t % kStages once the warps have released the tile
+    // that used it.  No L2 prefetch here: with the tiles consumed at this rate the
+    // prefetched tiles of the CTAs in flight outgrew L2 and were read twice (16% over
+    // K + V with four tiles ahead, 4% with none).
+    if (lane == 0 && !p.stall_loads) {
+      const uint64_t pol = policy_evict_first();
+      int t = 0;
+      for (; t < ntiles; ++t) {
+        const int buf = t % kStages;
+        if (t >= kStages && !dec_wait(sm, &sm.empty[buf], ((t / kStages) - 1) & 1, p)) break;
+        const int k0 = k_start + t * kTile;
+        fence_proxy_async_shared();
+        mbar_arrive_expect_tx(&sm.full[buf], 2 * (D / 64) * kBoxBytes);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(sm.k[buf][c], &tk, &sm.full[buf], c * 64, k0, bkv, pol);
+          tma_load_3d(sm.v[buf][c], &tv, &sm.full[buf], c * 64, k0, bkv, pol);
+        }
+      }
+      // the last kStages tiles issued may still be in flight if the compute warps
+      // stopped early: let them land (bounded) before the CTA exits
+      const uint64_t t0 = globaltimer_ns();
+      for (int u = max(0, t - kStages); u < t; ++u)
+        while (!mbar_try_wait(&sm.full[u % kStages], (u / kStages) & 1) &&
+               globaltimer_ns() - t0 < p.timeout_ns) {
+        }
+    }
+  } else {
+    // Q^T as the B fragments of S^T: slice ks, lane holds Q[row g8][16 ks + 2 q4 + {0, 1}]
+    // and the same 8 dims further on; rows past R are zero
+    uint32_t qb[kKs][2];
+    {
+      const bool live = g8 < R;
+      const int g = live ? g8 / p.L : 0, i = live ? g8 - g * p.L : 0;
+      const uint16_t* qrow = p.q + (static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i) * D;
+#pragma unroll
+      for (int ks = 0; ks < kKs; ++ks) {
+        qb[ks][0] = live ? __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * ks + 2 * q4)) : 0u;
+        qb[ks][1] = live ? __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * ks + 8 + 2 * q4)) : 0u;
+      }
+    }
+    const int pos0 = p.S - p.L + (n0 < R ? n0 % p.L : 0);
+    const int pos1 = p.S - p.L + (n1 < R ? n1 % p.L : 0);
+    // ldmatrix row of this lane: matrix lane / 8, row lane % 8
+    const int mi = lane >> 3, mr = lane & 7;
+    for (int t = 0; t < ntiles; ++t) {
+      const int buf = t % kStages;
+      if (!__all_sync(0xffffffffu, dec_wait(sm, &sm.full[buf], (t / kStages) & 1, p))) break;
+      const int k0 = k_start + t * kTile;
+      // S^T = K_w Q^T: A = keys 16 warp + (0..15) x dims 16 ks + (0..15); the four 8x8
+      // matrices are (keys 0-7, dims 0-7), (keys 8-15, dims 0-7), (keys 0-7, dims
+      // 8-15), (keys 8-15, dims 8-15)
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int key = 16 * warp + mr + 8 * (mi & 1);
+#pragma unroll
+        for (int ks = 0; ks < kKs; ++ks) {
+          uint32_t a[4];
+          ldsm_x4(chunk_addr(sm.k[buf], key, 2 * ks + (mi >> 1)), a);
+          mma16816<BF16>(s, a, qb[ks][0], qb[ks][1]);
+        }
+      }
+      // s[0], s[1]: key 16 warp + g8, rows n0, n1; s[2], s[3]: key + 8
+      const int kva = k0 + 16 * warp + g8, kvb = kva + 8;
+      float x[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kv = e < 2 ? kva : kvb;
+        const int n = (e & 1) ? n1 : n0;
+        const int pos = (e & 1) ? pos1 : pos0;
+        float v = s[e] * p.q_scale;
+        if (p.softcap_on) v = p.cap_a * tanhf(v / p.cap_c);
+        bool keep = n < R && kv < c1;
+        if (p.mask != FA_DECODE_FULL) keep = keep && kv <= pos;
+        if (p.mask == FA_DECODE_SLIDING_WINDOW) keep = keep && pos - kv < p.window;
+        x[e] = keep ? v : -INFINITY;
+      }
+      // online softmax per row over the warp's 16 keys (lanes with the same l % 4)
+      float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+      }
+      const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
+      const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
+      const float p0 = ex2_approx(x[0] - mu0), p1 = ex2_approx(x[1] - mu1);
+      const float p2 = ex2_approx(x[2] - mu0), p3 = ex2_approx(x[3] - mu1);
+      float sm0 = p0 + p2, sm1 = p1 + p3;
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        sm0 += __shfl_xor_sync(0xffffffffu, sm0, off);
+        sm1 += __shfl_xor_sync(0xffffffffu, sm1, off);
+      }
+      const float al0 = ex2_approx(m[0] - mu0), al1 = ex2_approx(m[1] - mu1);
+      l[0] = l[0] * al0 + sm0;
+      l[1] = l[1] * al1 + sm1;
+      m[0] = mn0;
+      m[1] = mn1;
+      if (al0 != 1.f || al1 != 1.f) {
+#pragma unroll
+        for (int mt = 0; mt < kKs; ++mt) {
+          o[mt][0] *= al0;
+          o[mt][1] *= al1;
+          o[mt][2] *= al0;
+          o[mt][3] *= al1;
+        }
+      }
+      // P as the B fragment of O^T += V^T P: transpose the two 8x8 halves
+      const uint32_t pb0 = movm_trans(pack_16(p0, p1, BF16));
+      const uint32_t pb1 = movm_trans(pack_16(p2, p3, BF16));
+      // A = V^T: dims 16 mt + (0..15) x keys 16 warp + (0..15); matrices (dims 0-7,
+      // keys 0-7), (dims 8-15, keys 0-7), (dims 0-7, keys 8-15), (dims 8-15, keys
+      // 8-15), each the transpose of 8 key rows x 8 dims of the tile
+      {
+        const int key = 16 * warp + mr + 8 * (mi >> 1);
+#pragma unroll
+        for (int mt = 0; mt < kKs; ++mt) {
+          uint32_t a[4];
+          ldsm_x4_trans(chunk_addr(sm.v[buf], key, 2 * mt + (mi & 1)), a);
+          mma16816<BF16>(o[mt], a, pb0, pb1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[buf]);
+    }
+  }
+  __syncthreads();
+  if (sm.abort_flag) return;
+
+  // merge the 4 warps' states per row.  The tile buffers are free now and hold the
+  // warps' O^T: red[warp][row][D]
+  float* red = reinterpret_cast<float*>(&sm.k[0][0][0]);
+  static_assert(sizeof(Sm::k) + sizeof(Sm::v) >= sizeof(float) * kMdWarps * kMdRows * D,
+                "reduction space");
+  if (warp < kMdWarps) {
+#pragma unroll
+    for (int mt = 0; mt < kKs; ++mt) {
+      const int d = 16 * mt + g8;
+      red[(warp * kMdRows + n0) * D + d] = o[mt][0];
+      red[(warp * kMdRows + n1) * D + d] = o[mt][1];
+      red[(warp * kMdRows + n0) * D + d + 8] = o[mt][2];
+      red[(warp * kMdRows + n1) * D + d + 8] = o[mt][3];
+    }
+    if (g8 == 0) {
+      sm.wm[warp][n0] = m[0];
+      sm.wm[warp][n1] = m[1];
+      sm.wl[warp][n0] = l[0];
+      sm.wl[warp][n1] = l[1];
+    }
+  }
+  __syncthreads();
+  for (int xi = tid; xi < R * D; xi += kMdThreads) {
+    const int rr = xi / D, d = xi - (xi / D) * D;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kMdWarps; ++w) mx = fmaxf(mx, sm.wm[w][rr]);
+    float lsum = 0.f, acc = 0.f;
+    if (mx != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kMdWarps; ++w) {
+        const float a = ex2_approx(sm.wm[w][rr] - mx);  // 0 for a warp that saw no key
+        lsum = fmaf(a, sm.wl[w][rr], lsum);
+        acc = fmaf(a, red[(w * kMdRows + rr) * D + d], acc);
+      }
+    }
+    const int g = rr / p.L, i = rr - g * p.L;
+    const size_t row = static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i;
+    float* rec = p.part + (row * p.nsplit + split) * (D + 2);
+    if (d == 0) {
+      rec[0] = mx;
+      rec[1] = lsum;
+    }
+    rec[2 + d] = acc;
+  }
+}
+
 // One CTA per query row, one thread per output column: merge the chunks.
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant__ DecParams p) {
@@ -438,8 +737,7 @@ void decode_plan(int B, int Hkv, int S, int D, int rows, int* nsplit, int* chunk
   constexpr int kCtaCost = 2;  // prologue and merge record, in tile units
   const int64_t groups = static_cast<int64_t>(B) * Hkv > 0 ? static_cast<int64_t>(B) * Hkv : 1;
   const int tiles = S > 0 ? (S + kTile - 1) / kTile : 1;
-  const int rm = rows <= 4 ? 4 : (rows <= 8 ? 8 : 32);  // the kernel instantiation
-  const int64_t slots = static_cast<int64_t>(kSms) * dec_ctas_per_sm(D, rm);
+  const int64_t slots = static_cast<int64_t>(kSms) * dec_ctas_per_sm(D, rows);
   int best_tiles = tiles;
   int64_t best_cost = INT64_MAX;
   for (int n = 1; n <= tiles && n <= 256; ++n) {
@@ -455,6 +753,39 @@ void decode_plan(int B, int Hkv, int S, int D, int rows, int* nsplit, int* chunk
   }
   *chunk = best_tiles * kTile;
   *nsplit = S > 0 ? (S + *chunk - 1) / *chunk : 1;
+}
+
+template <int D, bool BF16>
+fa_status decode_mma_launch(const void* k, const void* v, int B, int S, const DecParams& prm,
+                            cudaStream_t stream) {
+  CUtensorMap tk, tv;
+  // With S == 0 no tile is loaded; the maps only need to be well formed.
+  const void* kp = S > 0 ? k : prm.q;
+  const void* vp = S > 0 ? v : prm.q;
+  const int rows = S > 0 ? S : 1, bh = S > 0 ? B * prm.Hkv : 1;
+  if (!make_tile_map(&tk, kp, BF16, D, rows, bh, kTile)) return FA_ERR_CUDA;
+  if (!make_tile_map(&tv, vp, BF16, D, rows, bh, kTile)) return FA_ERR_CUDA;
+  const size_t smem = sizeof(MdSmem<D>) + 1024;
+  int dev = 0;
+  FA_CUDA_CHECK(cudaGetDevice(&dev));
+  {
+    static std::mutex mu;
+    static bool done[kMaxDevices] = {};
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+    if (!done[dev]) {
+      FA_CUDA_CHECK(cudaFuncSetAttribute(decode_mma_kernel<D, BF16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem)));
+      done[dev] = true;
+    }
+  }
+  const dim3 grid(prm.nsplit, B * prm.Hkv);
+  decode_mma_kernel<D, BF16><<<grid, kMdThreads, smem, stream>>>(tk, tv, prm);
+  FA_CUDA_CHECK(cudaGetLastError());
+  decode_combine_kernel<D><<<B * prm.H * prm.L, D, 0, stream>>>(prm);
+  FA_CUDA_CHECK(cudaGetLastError());
+  return FA_OK;
 }
 
 template <int D, int RM>
@@ -563,12 +894,15 @@ extern "C" fa_status fa_flex_attention_decode(const void* q, const void* k, cons
   const cudaStream_t s = as_stream(stream);
   const bool b16 = dtype == FA_BF16;
   const int rows = G * L;
+  // up to 8 rows (the MMA's N): the tensor-core chunk kernel; more: the CUDA-core one
   if (D == 64) {
-    if (rows <= 4) return decode_launch<64, 4>(k, v, b16, B, S, prm, s);
-    if (rows <= 8) return decode_launch<64, 8>(k, v, b16, B, S, prm, s);
+    if (rows <= kMdRows)
+      return b16 ? decode_mma_launch<64, true>(k, v, B, S, prm, s)
+                 : decode_mma_launch<64, false>(k, v, B, S, prm, s);
     return decode_launch<64, 32>(k, v, b16, B, S, prm, s);
   }
-  if (rows <= 4) return decode_launch<128, 4>(k, v, b16, B, S, prm, s);
-  if (rows <= 8) return decode_launch<128, 8>(k, v, b16, B, S, prm, s);
+  if (rows <= kMdRows)
+    return b16 ? decode_mma_launch<128, true>(k, v, B, S, prm, s)
+               : decode_mma_launch<128, false>(k, v, B, S, prm, s);
   return decode_launch<128, 32>(k, v, b16, B, S, prm, s);
 }

@@ -71,3 +71,21 @@ def test_decode_window_skips_far_chunks_and_matches():
     """A small window over a long cache: most chunks load nothing."""
     q, k, v = W.random_qkv(2, 8, 1, 20000, 64, torch.bfloat16, seed=54, Hkv=8)
     _check(q, k, v, 2, window=100)
+
+
+@pytest.mark.parametrize("B,H,Hkv,L,S,D,mask,window,dtype,xs", [
+    (1, 3, 3, 1, 1000, 128, 1, 0, torch.bfloat16, 1.0),     # one row per K/V head
+    (2, 6, 2, 1, 999, 64, 0, 0, torch.bfloat16, 1.0),       # three rows, ragged tail
+    (1, 2, 1, 2, 4097, 128, 2, 500, torch.float16, 1.0),    # four rows, window
+    (1, 1, 1, 4, 3, 64, 1, 0, torch.bfloat16, 1.0),         # L > S: a row sees nothing
+    (1, 8, 2, 1, 6000, 128, 1, 0, torch.bfloat16, 2.0),     # x2 inputs: peaked rows
+    (1, 8, 1, 1, 2500, 64, 1, 0, torch.bfloat16, 1.0),      # eight rows (the MMA's N)
+    (2, 6, 2, 2, 1500, 128, 2, 400, torch.float16, 1.0),    # six rows, window
+])
+def test_decode_tensor_core_path(B, H, Hkv, L, S, D, mask, window, dtype, xs):
+    """At most 8 rows per K/V head take the warp-level tensor-core kernel (16-bit P
+    against each warp's exact running max): element by element against the oracle."""
+    q, k, v = W.random_qkv(B, H, L, S, D, dtype, seed=B * 1000 + S + L, scale=xs, Hkv=Hkv)
+    out, lse = _check(q, k, v, mask, window)
+    if L > S:
+        assert torch.all(out[:, :, :L - S] == 0) and torch.all(torch.isneginf(lse[:, :, :L - S]))
