@@ -81,34 +81,43 @@ struct BwdParams {
   int stall;  // testing hook: nothing is loaded, the waits run out
 };
 
-__device__ __forceinline__ float2 load_pair(const uint16_t* ptr, bool bf16) {
-  const uint32_t u = __ldg(reinterpret_cast<const unsigned int*>(ptr));
-  if (bf16) return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
-  return __half22float2(*reinterpret_cast<const __half2*>(&u));
-}
-
-__device__ __forceinline__ float warp_sum(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  return x;
-}
-
-// delta_i = rowsum(dO_i * O_i): one warp per row of (B * H * L).
+// delta_i = rowsum(dO_i * O_i) over the B * H * L rows: D / 8 lanes per row, each
+// reading 16 bytes of O and of dO (so a warp covers 32 * 8 / D rows per pass), the
+// partial sums combined by shuffles within the row's lanes; grid-stride over rows.
 template <int D>
 __global__ void __launch_bounds__(kBwdWarps * 32) bwd_delta_kernel(const BwdParams p) {
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * kBwdWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= static_cast<int64_t>(p.B) * p.H * p.L) return;
+  constexpr int kLanes = D / 8;                // lanes per row
+  constexpr int kRowsPerBlock = kBwdWarps * 32 / kLanes;
+  const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.L;
   const bool bf16 = p.is_bf16 != 0;
-  float acc = 0.f;
+  const int sub = threadIdx.x % kLanes;
+  // the loop runs while the block's first row is in range (uniform over the block),
+  // so every lane reaches the shuffles; rows past the end load and store nothing
+  for (int64_t first = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock; first < rows;
+       first += static_cast<int64_t>(gridDim.x) * kRowsPerBlock) {
+    const int64_t row = first + threadIdx.x / kLanes;
+    const bool in = row < rows;
+    const int64_t off = (in ? row : 0) * D + sub * 8;
+    const uint4 o4 = __ldg(reinterpret_cast<const uint4*>(p.out + off));
+    const uint4 g4 = __ldg(reinterpret_cast<const uint4*>(p.dout + off));
+    const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w}, gw[4] = {g4.x, g4.y, g4.z, g4.w};
+    float acc = 0.f;
 #pragma unroll
-  for (int e = 0; e < D / 64; ++e) {
-    const int64_t off = row * D + 2 * lane + 64 * e;
-    const float2 o = load_pair(p.out + off, bf16), g = load_pair(p.dout + off, bf16);
-    acc = fmaf(o.x, g.x, fmaf(o.y, g.y, acc));
+    for (int i = 0; i < 4; ++i) {
+      float2 o, g;
+      if (bf16) {
+        o = make_float2(__uint_as_float(ow[i] << 16), __uint_as_float(ow[i] & 0xFFFF0000u));
+        g = make_float2(__uint_as_float(gw[i] << 16), __uint_as_float(gw[i] & 0xFFFF0000u));
+      } else {
+        o = __half22float2(*reinterpret_cast<const __half2*>(&ow[i]));
+        g = __half22float2(*reinterpret_cast<const __half2*>(&gw[i]));
+      }
+      acc = fmaf(o.x, g.x, fmaf(o.y, g.y, acc));
+    }
+#pragma unroll
+    for (int s = kLanes / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s, kLanes);
+    if (in && sub == 0) p.delta[row] = acc;
   }
-  acc = warp_sum(acc);
-  if (lane == 0) p.delta[row] = acc;
 }
 
 // ---------------------------------------------------------------- tcgen05 kernels
@@ -745,7 +754,12 @@ fa_status bwd_launch(const BwdParams& prm, bool bf16, cudaStream_t s) {
   const int64_t rows = static_cast<int64_t>(prm.B) * prm.H * prm.L;
   const int64_t krows = static_cast<int64_t>(prm.B) * prm.Hkv * prm.S;
   if (rows > 0) {
-    const unsigned qgrid = static_cast<unsigned>((rows + kBwdWarps - 1) / kBwdWarps);
+    // grid-stride: a few blocks per SM cover any row count
+    const int64_t per_block = kBwdWarps * 32 / (D / 8);
+    const int64_t want = (rows + per_block - 1) / per_block;
+    const int sms = num_sms_current_device();
+    const int64_t cap = static_cast<int64_t>(sms > 0 ? sms : 148) * 8;
+    const unsigned qgrid = static_cast<unsigned>(want < cap ? want : cap);
     bwd_delta_kernel<D><<<qgrid, kBwdWarps * 32, 0, s>>>(prm);
     FA_CUDA_CHECK(cudaGetLastError());
   }
@@ -814,13 +828,13 @@ extern "C" fa_status fa_flex_attention_bwd(
     return FA_ERR_INVALID_ARG;
   if (bm->kind == FA_MASK_DOCUMENT_CAUSAL && bm->doc_id == nullptr) return FA_ERR_INVALID_ARG;
   if (bm->kind == FA_MASK_BITMAP && S > 0 && bm->bitmap == nullptr) return FA_ERR_INVALID_ARG;
-  // q, k, v, dout are TMA tiles and the gradients are written in 16-byte pieces: 16
-  // bytes; the workspace holds the error word and the row sums: 16 bytes; the rest
-  // is read as 4-byte values (out in 4-byte pairs)
+  // q, k, v, dout are TMA tiles, out and dout are read in 16-byte pieces and the
+  // gradients written in 16-byte pieces: 16 bytes; the workspace holds the error word
+  // and the row sums: 16 bytes; the rest is read as 4-byte values
   auto off16 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
   auto off4 = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) != 0; };
-  if (off16(q) || off16(k) || off16(v) || off16(dout) || off16(dq) || off16(dk) || off16(dv) ||
-      off16(workspace) || off4(out) || off4(lse))
+  if (off16(q) || off16(k) || off16(v) || off16(out) || off16(dout) || off16(dq) || off16(dk) ||
+      off16(dv) || off16(workspace) || off4(lse))
     return FA_ERR_INVALID_ARG;
   if (off4(bm->kv_num_blocks) || off4(bm->full_kv_num_blocks) || off4(bm->kv_indices) ||
       off4(bm->full_kv_indices) || off4(bm->q_order) || off4(bm->doc_id) || off4(bm->bitmap) ||

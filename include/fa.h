@@ -378,8 +378,8 @@ FA_API fa_status fa_flex_attention_decode(const void* q, const void* k, const vo
  *             buffer for every call on one stream; the row sums need no initial
  *             contents.  Calls that run concurrently need distinct workspaces.
  * Alignment (checked on the host; a misaligned pointer returns FA_ERR_INVALID_ARG
- * before any launch): q, k, v, dout, dq, dk, dv and workspace 16 bytes; out, lse and
- * every table pointer 4 bytes.  D 64 or 128; B * H * L and B * H_kv * S at most 2^33
+ * before any launch): q, k, v, out, dout, dq, dk, dv and workspace 16 bytes; lse
+ * and every table pointer 4 bytes.  D 64 or 128; B * H * L and B * H_kv * S at most 2^33
  * (else FA_ERR_UNSUPPORTED).  Three kernels on `stream`: row sums of dO * O; dK and dV
  * per 128-key tile over its column lists and the query heads sharing its K/V head;
  * dQ per 128-query tile over its row lists.  Both gradient kernels run the products

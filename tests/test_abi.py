@@ -265,6 +265,7 @@ def test_bwd_rejects_bad_arguments_on_host(fa):
     assert _bwd(fa, bm, dv=0) == E
     assert _bwd(fa, bm, cols=0) == E                # column lists missing
     assert _bwd(fa, bm, dout=1026) == E             # not 4-byte aligned
+    assert _bwd(fa, bm, out=1032) == E              # 8- but not 16-byte aligned (16-byte loads)
     assert _bwd(fa, bm, q=1028) == E                # 4- but not 16-byte aligned (cp.async source)
     assert _bwd(fa, bm, k=1032) == E
     assert _bwd(fa, bm, lse=1026) == E
