@@ -57,8 +57,8 @@ NCU_TRAFFIC = {
         "sources_sha256": "241e471ad0698b045586e1b945537b4434067834ee93939e5e93d87ec87aa45d",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_launches.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
-        "bytes": 1073846272 + 3377152, "sources": DECODE_SOURCES,
-        "sources_sha256": "341606de9e93c984068ada4eb45c9edef0382c4efdc6268e54ce65985197534a",
+        "bytes": 1073887488 + 3557632, "sources": DECODE_SOURCES,
+        "sources_sha256": "78393a08231b16ebe651a9b3434ca4a91b22c2c9d64c50879e73c979fc893e80",
         "summary": "profiles/decode_mma_kernel_L1_S32768_B8_H32_Hkv8_D128_full.md"},
 }
 
