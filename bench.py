@@ -53,8 +53,8 @@ DECODE_SOURCES = ("block_sparse_attention_create_b200/csrc/decode.cu",
                   "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
 NCU_TRAFFIC = {
     "swa256_L32768_B1_H8_D64_bf16": {
-        "bytes": 100959232 + 5034752, "sources": FWD_SOURCES,
-        "sources_sha256": "241e471ad0698b045586e1b945537b4434067834ee93939e5e93d87ec87aa45d",
+        "bytes": 101026560 + 5083136, "sources": FWD_SOURCES,
+        "sources_sha256": "6f30b4f50f85a426533ccfe9e2671dd40b905625c210f1b9a6b0fdebb260cb9d",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_launches.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
         "bytes": 1073887488 + 3557632, "sources": DECODE_SOURCES,

@@ -500,11 +500,10 @@ struct MmaShared {
   bool split;
 };
 
-// Probe shared by lanes: lane 0 tests the phase, the warp gets the answer.
+// Probe by the whole warp: every lane tests the phase (one shared-memory access for
+// the warp) and the vote makes the answer warp-uniform; no shuffle from a leader lane.
 __device__ __forceinline__ bool probe(uint64_t* bar, uint32_t parity) {
-  uint32_t ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_test_wait(bar, parity) ? 1u : 0u;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  return __all_sync(0xffffffffu, mbar_test_wait(bar, parity));
 }
 
 // S_i = Q K_i^T for the slot's stream position `c`, if its inputs are ready.
@@ -583,13 +582,20 @@ __device__ __forceinline__ bool try_pv(Smem<D>& sm, const Params& p, MmaStream<B
 
 // Per slot: its S stream and its PV stream (the PV stream trails).  In the aliased
 // layout S_{i+1} may only follow PV_i (the MMAs of one thread run in issue order,
-// so PV_i has read P before S_{i+1} overwrites it).
+// so PV_i has read P before S_{i+1} overwrites it); there the PV is tried first, so
+// that S_{i+1} can follow it in the same pass (a pass later cost the D = 128
+// softcap workload 15%).  In the separate-P layout the S goes first.
 template <int D, int SLOT, bool BHM>
 __device__ __forceinline__ bool mma_slot(Smem<D>& sm, const Params& p, MmaStream<BHM>& cs,
                                          MmaStream<BHM>& cp, MmaShared& ms) {
   bool progress = false;
+  if constexpr (!Cfg<D>::kSepP) {
+    if (cp.active && (!cs.active || cp.i < cs.i)) progress |= try_pv<D, SLOT>(sm, p, cp, ms);
+  }
   if (cs.active && (Cfg<D>::kSepP || cs.i == cp.i)) progress |= try_s<D, SLOT>(sm, p, cs, ms);
-  if (cp.active && (!cs.active || cp.i < cs.i)) progress |= try_pv<D, SLOT>(sm, p, cp, ms);
+  if constexpr (Cfg<D>::kSepP) {
+    if (cp.active && (!cs.active || cp.i < cs.i)) progress |= try_pv<D, SLOT>(sm, p, cp, ms);
+  }
   return progress;
 }
 
