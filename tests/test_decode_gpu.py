@@ -81,6 +81,8 @@ def test_decode_window_skips_far_chunks_and_matches():
     (1, 8, 2, 1, 6000, 128, 1, 0, torch.bfloat16, 2.0),     # x2 inputs: peaked rows
     (1, 8, 1, 1, 2500, 64, 1, 0, torch.bfloat16, 1.0),      # eight rows (the MMA's N)
     (2, 6, 2, 2, 1500, 128, 2, 400, torch.float16, 1.0),    # six rows, window
+    (1, 4, 1, 1, 1000, 64, 0, 0, torch.float16, 2.0),       # fp16 at D = 64, no mask
+    (1, 2, 2, 3, 0, 64, 1, 0, torch.bfloat16, 1.0),         # empty cache: no key at all
 ])
 def test_decode_tensor_core_path(B, H, Hkv, L, S, D, mask, window, dtype, xs):
     """At most 8 rows per K/V head take the warp-level tensor-core kernel (16-bit P
