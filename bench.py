@@ -310,6 +310,50 @@ def run_ours(args, w: W.Workload, rank, world, device):
             "mask_ms": mask_ms, "clocks": clk.summary(), "e2e": e2e}
 
 
+def config_sweep(device, steps=10, warmup=3):
+    """The forward kernel alone on the other configurations of the benchmark set
+    (causal 256, the 8192 sweep, both document workloads, the D = 128 softcap
+    workload): mask built once, `warmup` launches, then `steps` launches each
+    bracketed by CUDA events with a 512 MiB L2 flush between them (untimed).
+    Reported beside the main line so that these figures come from the same run."""
+    import block_sparse_attention_create_b200 as fa
+    peaks, _ = load_peaks()
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    res = {}
+    for w in (W.C1_CAUSAL_256, W.C2_CAUSAL_8192) + W.C2_WINDOWS + (
+            W.C4_DOC_FIXED, W.C4_DOC_SEEDED, W.C5_SWA1024_SOFTCAP):
+        q, k, v = (t.to(device) for t in W.make_qkv(w))
+        doc = W.make_doc_id(w)
+        dd = doc.to(device) if doc is not None else None
+        out = torch.empty_like(q)
+        lse = torch.empty(w.B, w.H, w.L, dtype=torch.float32, device=device)
+        build, attend, dev_error = step_calls(fa, w, q, k, v, dd, None, out, lse, device, stream)
+        build()
+        for _ in range(warmup):
+            attend()
+        torch.cuda.synchronize()
+        t = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            attend()
+            e1.record(stream)
+            t.append((e0, e1))
+        torch.cuda.synchronize()
+        assert dev_error() == fa.FA_OK
+        ms = sum(a.elapsed_time(b) for a, b in t) / steps
+        fig = work_figures(w)
+        tflops = fig["flops"] / (ms * 1e-3) / 1e12
+        gbs = fig["bytes"] / (ms * 1e-3) / 1e9
+        tf, hf = tflops / peaks["bf16_tflops"], gbs / peaks["hbm_gbs"]
+        res[w.name] = {"fwd_us": round(ms * 1e3, 2), "live_tflops": round(tflops, 1),
+                       "bound": "tensor" if tf >= hf else "hbm", "frac": round(max(tf, hf), 4)}
+        del q, k, v, out, lse
+    return res
+
+
 def run_backward(args, w: W.Workload, world, device, fig):
     """Backward step timed like the forward: the mask's column lists and
     fa_flex_attention_bwd, L2 flushed between steps, CUDA events, max over ranks.
@@ -651,6 +695,9 @@ def main():
                                            if is_decode(w) else
                                            f"{len(rows)} random query rows of head (0,0), "
                                            f"{dt:.1f} s; live-block FLOPs of those rows credited")}
+    if world == 1 and not args.profile and args.workload == W.C3_SWA256_32K.name:
+        # the other configurations of the benchmark set, forward kernel only, same run
+        line["configs"] = config_sweep(device)
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank == 0:
