@@ -60,11 +60,24 @@ classify_rows_kernel(int kind, int window, const int32_t* __restrict__ doc_all,
   const bool q_whole = q0 + kBlock <= q_len;
 
   if (kind == FA_MASK_BITMAP) {
-    // a warp per kv block: lane l reads rows q0 + l + 32 r (r < 4), all four words;
-    // bits past kv_len do not count, rows past q_len neither
+    // Rows are read whole, coalesced: lane l of a warp takes kv blocks l, l + 32, ...
+    // (each block's 4 words of a row are one 16-byte load), the warps take the
+    // block's rows in turn.  Per group of 32 blocks a warp folds its rows into an
+    // "any bit set" and an "all bits set" flag per block, ballots them into two
+    // words and merges those into the CTA's words in shared memory (OR / AND).
+    // Bits past kv_len do not count, rows past q_len are not read.
     const int nwarps = blockDim.x >> 5;
+    const int nwords = (n_kv + 31) / 32;
+    uint32_t* any_bits = reinterpret_cast<uint32_t*>(cls + ((n_kv + 15) & ~15));
+    uint32_t* all_bits = any_bits + nwords;
+    for (int t = threadIdx.x; t < nwords; t += blockDim.x) {
+      any_bits[t] = 0u;
+      all_bits[t] = 0xFFFFFFFFu;
+    }
+    __syncthreads();
     const size_t wpr = static_cast<size_t>(n_kv) * 4;  // words per bitmap row
-    for (int j = warp; j < n_kv; j += nwarps) {
+    for (int m = 0; m < nwords; ++m) {
+      const int j = 32 * m + lane;
       const int64_t k0 = static_cast<int64_t>(j) * kBlock;
       uint32_t valid[4];
 #pragma unroll
@@ -72,22 +85,32 @@ classify_rows_kernel(int kind, int window, const int32_t* __restrict__ doc_all,
         const int64_t nk = kv_len - (k0 + 32 * w);  // keys of word w that exist
         valid[w] = nk >= 32 ? 0xFFFFFFFFu : (nk <= 0 ? 0u : ((1u << nk) - 1u));
       }
-      bool any = false, all = q_whole && k0 + kBlock <= kv_len;
+      bool any = false, all = true;
+      if (j < n_kv) {
+#pragma unroll 4
+        for (int64_t q = q0 + warp; q <= q1; q += nwarps) {
+          const uint4 v4 = __ldg(reinterpret_cast<const uint4*>(bitmap + q * wpr + 4 * j));
+          const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int64_t q = q0 + lane + 32 * r;
-        if (q >= q_len) continue;
-        const uint4 v4 = __ldg(reinterpret_cast<const uint4*>(bitmap + q * wpr + 4 * j));
-        const uint32_t wv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          any |= (wv[w] & valid[w]) != 0u;
-          all &= (wv[w] & valid[w]) == valid[w];
+          for (int w = 0; w < 4; ++w) {
+            any |= (wv[w] & valid[w]) != 0u;
+            all &= (wv[w] & valid[w]) == valid[w];
+          }
         }
       }
-      any = __any_sync(0xffffffffu, any);
-      all = __all_sync(0xffffffffu, all);
-      if (lane == 0) cls[j] = any ? (all ? 2 : 1) : 0;
+      const uint32_t any_w = __ballot_sync(0xffffffffu, any);
+      const uint32_t all_w = __ballot_sync(0xffffffffu, all);
+      if (lane == 0) {
+        atomicOr(&any_bits[m], any_w);
+        atomicAnd(&all_bits[m], all_w);
+      }
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < n_kv; j += blockDim.x) {
+      const bool whole = q_whole && static_cast<int64_t>(j + 1) * kBlock <= kv_len;
+      const bool any = (any_bits[j >> 5] >> (j & 31)) & 1u;
+      const bool all = (all_bits[j >> 5] >> (j & 31)) & 1u;
+      cls[j] = any ? (all && whole ? 2 : 1) : 0;
     }
   } else if (kind != FA_MASK_DOCUMENT_CAUSAL) {
     for (int j = threadIdx.x; j < n_kv; j += blockDim.x) {
@@ -473,8 +496,12 @@ fa_status build_tables(int32_t kind, int32_t window, const int32_t* doc_id, cons
                              bm->full_kv_indices, bm->q_order));
     return FA_OK;
   }
+  // shared memory: a class byte per kv block, and for tabulated masks two bit words
+  // per 32 blocks (any / all bits set)
+  const size_t cls_smem = static_cast<size_t>((nkv + 15) & ~15) + 16 +
+                          (kind == FA_MASK_BITMAP ? 8 * static_cast<size_t>((nkv + 31) / 32) : 0);
   FA_CUDA_CHECK(launch_pdl(classify_rows_kernel, dim3(nq, inst), dim3(kClassifyThreads),
-                           static_cast<size_t>(nkv > 0 ? nkv : 1), s, kind, bm->window, bm->doc_id,
+                           cls_smem, s, kind, bm->window, bm->doc_id,
                            bm->bitmap, q_len, kv_len, nkv, bm->kv_num_blocks, bm->kv_indices,
                            bm->full_kv_num_blocks, bm->full_kv_indices));
   int n_pow2 = 1;
