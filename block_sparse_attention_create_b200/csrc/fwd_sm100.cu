@@ -30,6 +30,10 @@
 // overwrites the S it came from (TMEM holds no more), S_{j+1} is issued after PV_j
 // (tcgen05 operations of one thread run in issue order), and the commit that
 // signals S_{j+1} also means PV_j is done.
+// Epilogue of a unit, O / l: at D = 64, for a unit of at most kStageMaxBlocks
+// blocks, each softmax warp writes its 32 rows into the unit's Q tile and one lane
+// stores them with a TMA tensor store, so the LSU carries no output traffic; longer
+// units and D = 128 store from registers.
 //
 // Every mbarrier wait is bounded: after `timeout_ns` the waiting warp sets an abort
 // flag and the device error word, all roles stop, in-flight copies and MMAs are
@@ -59,6 +63,13 @@ constexpr int kThreads = (kSoftmaxWarps + kNumSlots + 1) * 32;  // + 2 producers
 // three per sub-partition here, and each sub-partition has a quarter of the
 // register file (16384): 3 x 32 x 168 fits, 3 x 32 x 176 does not.
 constexpr int kBlockN = 128;                 // rows of a Q tile / K,V tile
+// Units of at most this many blocks store O through the staging tile (TMA store);
+// longer ones store it from registers.  Measured at D = 64: short units end every
+// few blocks, and their direct stores queued behind one another in the load/store
+// unit (window 256, 32k: 77 -> 74 us staged); a long unit's stores drain during
+// its successor, and there the staging (proxy fence, release of the tile) cost
+// 2-3% (causal 8192, window 4096).
+constexpr int kStageMaxBlocks = 4;
 constexpr int kChunkBytes = 128 * 128;       // one TMA box: 128 rows x 64 elems x 2 B
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -88,6 +99,13 @@ struct Cfg {
   // Q tiles per slot: two at D=64, so the next unit's Q loads while this one runs.
   static constexpr int kQBuf = (D == 64) ? 2 : 1;
   static constexpr bool kSepP = (D == 64);
+  // D = 64: O of a short unit leaves through shared memory, one TMA store per warp
+  // (its 32 rows), so the epilogue issues no global stores of its own.  The staging
+  // tile is the unit's own Q tile (same size and swizzle, no longer read once the
+  // unit's MMAs are done), which the softmax warps then release together with the
+  // MMA warp.  D = 128 (one Q buffer, reloaded at once for the next unit) stores
+  // from registers.
+  static constexpr bool kStageO = (D == 64);
   static constexpr uint32_t kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t s_col(int slot) { return 128u * slot; }
   __host__ __device__ static constexpr uint32_t p_col(int slot) {
@@ -119,6 +137,11 @@ struct __align__(1024) Smem {
   uint32_t tmem_base;
   volatile int abort_flag;
 };
+
+// Dynamic shared memory of a CTA (the struct plus 1024 bytes to align it) within the
+// 227 KB a block may use.
+static_assert(sizeof(Smem<64>) + 1024 <= 232448, "shared memory of the D = 64 forward");
+static_assert(sizeof(Smem<128>) + 1024 <= 232448, "shared memory of the D = 128 forward");
 
 struct Params {
   const int32_t* kv_idx;
@@ -849,7 +872,8 @@ __device__ __forceinline__ float exp_pack64(const float (&x)[64], float xs, floa
 // Softmax warpgroup of one slot: thread t owns row t of the slot's 128-row tile
 // (TMEM lane t), so row max and row sum need no shuffles.
 template <int D, int MK, bool BHM, bool SC>
-__device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int slot) {
+__device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int slot,
+                             const CUtensorMap* tmap_o) {
   using C = Cfg<D>;
   const int t = threadIdx.x - slot * 128;   // row of the tile this thread owns
   const int wq = t >> 5;                    // TMEM lane quarter of this warp
@@ -870,9 +894,9 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
   while (it.pop(p, un)) {
     const int row = un.qblk * kBlockN + t;
     const bool valid = row < p.L;
-    const size_t orow = static_cast<size_t>(un.bh) * p.L + row;
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow * D);
     if (un.n == 0) {
+      const size_t orow = static_cast<size_t>(un.bh) * p.L + row;
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow * D);
       if (valid) {
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0, 0, 0, 0);
@@ -880,23 +904,33 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
       }
       continue;
     }
-    // this unit's mask instance: its document ids / bitmap rows
-    const int32_t* docs = MK == kMaskDoc ? p.doc_id + static_cast<size_t>(un.inst) * p.doc_len : nullptr;
-    const int dq_own = (MK == kMaskDoc && valid) ? __ldg(docs + row) : 0;
+    // this unit's mask instance: its document ids / bitmap rows (pointers formed
+    // where they are used, like the key range below)
+    auto docs_of = [&]() {
+      return MK == kMaskDoc ? p.doc_id + static_cast<size_t>(un.inst) * p.doc_len : nullptr;
+    };
+    const int dq_own = (MK == kMaskDoc && valid) ? __ldg(docs_of() + row) : 0;
     // rows past L (only ever above the valid ones, so lane 0 is valid if any lane is)
     // take lane 0's document: they add no document to the warp's passes in apply_mask.
     // The shuffle is taken by every lane, outside any short-circuited expression.
     const int dq0 = __shfl_sync(0xffffffffu, dq_own, 0);
     const int dq = valid ? dq_own : dq0;
     // tabulated mask: this row's words (rows past L read the last row, unused)
-    const uint32_t* brow = MK == kMaskBitmap
-                               ? p.bitmap + (static_cast<size_t>(un.inst) * p.L + min(row, p.L - 1)) *
+    auto brow_of = [&]() {
+      return MK == kMaskBitmap ? p.bitmap + (static_cast<size_t>(un.inst) * p.L +
+                                             min(un.qblk * kBlockN + t, p.L - 1)) *
                                                 p.bitmap_words
                                : nullptr;
+    };
     // live keys of this row: kv in [lo, hi] (and, for documents, doc_id[kv] == dq;
-    // for a tabulated mask, its bit); only the causal rules bound hi by the row
-    const int hi = MK == kMaskBitmap ? p.S - 1 : min(row, p.S - 1);
-    const int lo = p.mask_kind == FA_MASK_SLIDING_WINDOW_CAUSAL ? max(row - p.window + 1, 0) : 0;
+    // for a tabulated mask, its bit); only the causal rules bound hi by the row.
+    // Formed where a PARTIAL block needs them, so that no register holds them
+    // through the block loop.
+    auto key_range = [&](int& lo, int& hi) {
+      const int r = un.qblk * kBlockN + t;
+      hi = MK == kMaskBitmap ? p.S - 1 : min(r, p.S - 1);
+      lo = p.mask_kind == FA_MASK_SLIDING_WINDOW_CAUSAL ? max(r - p.window + 1, 0) : 0;
+    };
     float m = -INFINITY, l = 0.f;  // running max (log2 units) and running sum
     int kvb = block_index(p, un, 0);
 
@@ -905,6 +939,15 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
       const int kvb_next = j + 1 < un.n ? block_index(p, un, j + 1) : 0;
       if (!wait_warp(sm, &sm.s_full[slot], blk & 1, p)) return;
       tc_fence_after();
+      if constexpr (C::kStageO) {
+        // The previous unit's TMA store has had a block's wait to read its staging
+        // tile (that unit's Q buffer): once it has, the tile goes back to the
+        // producer.
+        if (j == 0 && units > 0 && (t & 31) == 0) {
+          bulk_wait_read_all();
+          mbar_arrive(&sm.q_empty[slot][(units - 1) % C::kQBuf]);
+        }
+      }
       if constexpr (C::kSepP) {
         // Separate-P layout: the whole row of S (128 columns) comes into registers at
         // once, S is released to the MMA warp right away, and P is written per half.
@@ -916,12 +959,14 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         if ((t & 31) == 0) mbar_arrive(&sm.s_empty[slot]);
         if constexpr (SC) softcap64(p, *reinterpret_cast<float(*)[64]>(x)), softcap64(p, *reinterpret_cast<float(*)[64]>(x + 64));
         if (!full) {
+          int lo, hi;
+          key_range(lo, hi);
           const int a = lo - kvb * kBlockN;
           const int b = hi - kvb * kBlockN;
-          apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x), a, b, kvb * kBlockN, dq, docs,
-                     brow);
+          apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x), a, b, kvb * kBlockN, dq, docs_of(),
+                     brow_of());
           apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x + 64), a - 64, b - 64, kvb * kBlockN + 64, dq,
-                     docs, brow);
+                     docs_of(), brow_of());
         }
         const float mb = fmaxf(row_max64(*reinterpret_cast<float(*)[64]>(x)),
                                row_max64(*reinterpret_cast<float(*)[64]>(x + 64))) * xs;
@@ -954,6 +999,8 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         // that one max: P_hi of half h goes to P columns [32h, 32h + 32); with the
         // split, P_lo goes to columns 64 + [32h, 32h + 32), held in registers until
         // half 1 has been read (in the aliased layout those columns are still S).
+        int lo, hi;
+        key_range(lo, hi);
         const int a = lo - kvb * kBlockN;  // live columns of the block: a <= i <= b
         const int b = hi - kvb * kBlockN;
         float rmax = -INFINITY;
@@ -962,8 +1009,8 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
           float x[64];
           load_s_half(t_s + h * 64, x);
           if (!full)
-            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, docs,
-                           brow);
+            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, docs_of(),
+                           brow_of());
           rmax = fmaxf(rmax, row_max64(x));
         }
         float mb = rmax;
@@ -1030,8 +1077,8 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
             }
           }
           if (!full)
-            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, docs,
-                           brow);
+            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, docs_of(),
+                           brow_of());
           // P = exp2(x * xs - m) as 16-bit pairs; with the split, P_hi = p truncated to
           // bf16 and P_lo = round(p - P_hi), so P_hi + P_lo carries ~16 significant bits.
           float2 sums[4];
@@ -1073,29 +1120,74 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
       kvb = kvb_next;
     }
 
-    // epilogue: O / l -> out, LSE
+    // epilogue: O / l -> out, LSE (the output row is formed here, not kept in
+    // registers through the block loop)
     if (!wait_warp(sm, &sm.o_full[slot], units & 1, p)) return;
     tc_fence_after();
+    const size_t orow = static_cast<size_t>(un.bh) * p.L + un.qblk * kBlockN + t;
     const float inv = l > 0.f ? 1.f / l : 0.f;
+    if (C::kStageO && un.n <= kStageMaxBlocks) {
+      // O comes into registers and is released to the next unit's PV at once; the
+      // warp writes its 32 rows into the staging tile (128-byte rows, 16-byte chunk
+      // c of row r at chunk c ^ (r % 8): the layout of the map's 128-byte swizzle,
+      // and conflict-free for one row per thread) and lane 0 stores them with TMA.
+      // Rows past L are clipped by the map's extent.
+      uint32_t pk[32];  // the row as 16-bit pairs
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t r[32];
-      tmem_ld32(t_o + c * 32, r);
-      tmem_wait_ld();
-      reg_fence32(r);
-      uint32_t pk[16];
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_o + c * 32, r);
+        tmem_wait_ld();
+        reg_fence32(r);
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        pk[i] = pack2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv, bf16);
-      if (valid) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          dst[c * 4 + i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        for (int i = 0; i < 16; ++i)
+          pk[16 * c + i] = pack2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv, bf16);
       }
+      tc_fence_before();
+      __syncwarp();
+      // The lane index is read here (a volatile read), so that the staging
+      // addresses below are formed here and not kept in registers across the
+      // block loop, where every register is taken.
+      const int lane = lane_id_volatile();
+      if (lane == 0) mbar_arrive(&sm.o_empty[slot]);
+      // the unit's Q tile: its MMAs are done (o_full), and the producer refills it
+      // only after this warp releases it, in the next unit's first block
+      const int qb = units % C::kQBuf;
+      uint8_t* rowp = sm.q[slot][qb] + (wq * 32 + lane) * 128;
+      uint8_t* tile = rowp - lane * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_proxy_async_shared();
+      __syncwarp();
+      const int row0 = un.qblk * kBlockN + wq * 32;
+      if (lane == 0 && row0 < p.L) {
+        tma_store_3d(tmap_o, tile, 0, row0, un.bh);
+        bulk_commit_group();
+      }
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow * D);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_o + c * 32, r);
+        tmem_wait_ld();
+        reg_fence32(r);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv, bf16);
+        if (valid) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[c * 4 + i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if ((t & 31) == 0) mbar_arrive(&sm.o_empty[slot]);
     }
-    tc_fence_before();
-    __syncwarp();
-    if ((t & 31) == 0) mbar_arrive(&sm.o_empty[slot]);
     if (valid && p.lse) p.lse[orow] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
     ++units;
   }
@@ -1104,7 +1196,8 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
 template <int D, int MK, bool BHM, bool SC>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-           const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ Params p) {
+           const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o,
+           const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
   Smem<D>& sm = *reinterpret_cast<Smem<D>*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
@@ -1114,7 +1207,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
     for (int s = 0; s < kNumSlots; ++s) {
       for (int b = 0; b < Cfg<D>::kQBuf; ++b) {
         mbar_init(&sm.q_full[s][b], 1);
-        mbar_init(&sm.q_empty[s][b], 1);
+        // the MMA warp's commit, and with O staged in it, one arrival per softmax warp
+        mbar_init(&sm.q_empty[s][b], Cfg<D>::kStageO ? 1 + 4 : 1);
       }
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.s_empty[s], 4);
@@ -1139,6 +1233,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
     prefetch_tensormap(&tmap_q);  // the other producer warp shares the cached maps
     prefetch_tensormap(&tmap_k);
     prefetch_tensormap(&tmap_v);
+    if (Cfg<D>::kStageO) prefetch_tensormap(&tmap_o);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem_base, Cfg<D>::kTmemCols);
@@ -1155,7 +1250,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ C
 
   // Role dispatch; the final rendezvous is a named barrier over all threads.
   if (warp < kSoftmaxWarps) {
-    softmax_role<D, MK, BHM, SC>(sm, p, tmem, warp / 4);
+    softmax_role<D, MK, BHM, SC>(sm, p, tmem, warp / 4, &tmap_o);
+    // the warp's TMA stores of O (issued by lane 0) complete before the CTA exits
+    if (Cfg<D>::kStageO && (threadIdx.x & 31) == 0) bulk_wait_all();
     tc_fence_before();
     named_barrier_sync(1, kThreads);
     return;
@@ -1189,6 +1286,9 @@ fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH,
   const int BHkv = BH / prm.kv_group;
   if (!make_map(&tk, S > 0 ? k : q, bf16, D, S > 0 ? S : L, S > 0 ? BHkv : BH)) return FA_ERR_CUDA;
   if (!make_map(&tv, S > 0 ? v : q, bf16, D, S > 0 ? S : L, S > 0 ? BHkv : BH)) return FA_ERR_CUDA;
+  // out, stored by the softmax warps 32 rows at a time (D = 64)
+  CUtensorMap to;
+  if (!make_tile_map(&to, prm.out, bf16, D, L, BH, 32)) return FA_ERR_CUDA;
   const size_t smem = sizeof(Smem<D>) + 1024;
   int dev = 0;
   FA_CUDA_CHECK(cudaGetDevice(&dev));
@@ -1208,7 +1308,7 @@ fa_status launch(const void* q, const void* k, const void* v, bool bf16, int BH,
   const int want = (prm.num_units + kNumSlots - 1) / kNumSlots;
   const int grid = want < sms ? want : sms;
   FA_CUDA_CHECK(launch_pdl(fwd_kernel<D, MK, BHM, SC>, dim3(grid), dim3(kThreads), smem, stream, tq, tk,
-                           tv, prm));
+                           tv, to, prm));
   return FA_OK;
 }
 

@@ -71,6 +71,14 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) 
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// The lane index, read with a volatile instruction: values derived from it are
+// computed where it is read, not hoisted out of enclosing loops.
+__device__ __forceinline__ int lane_id_volatile() {
+  int lane;
+  asm volatile("mov.u32 %0, %%laneid;" : "=r"(lane));
+  return lane;
+}
+
 // ------------------------------------------------------------------ TMA
 // 3-D tiled load global -> shared, completion signalled on `bar` (tx bytes).
 // No multicast.
@@ -92,6 +100,29 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int32_t 
                    reinterpret_cast<uint64_t>(map)),
                "r"(x), "r"(y), "r"(z)
                : "memory");
+}
+
+// 3-D tiled store shared -> global, in the issuing thread's current bulk async-group.
+// Rows of the box past the tensor's extent are not written.  The start coordinates
+// must not be negative.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int32_t x,
+                                             int32_t y, int32_t z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+// Close the issuing thread's current bulk async-group.
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until none of this thread's bulk async-groups still reads shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until all of this thread's bulk async-groups have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Order this thread's generic-proxy shared-memory accesses before later
