@@ -603,22 +603,19 @@ __device__ __forceinline__ bool try_pv(Smem<D>& sm, const Params& p, MmaStream<B
   return true;
 }
 
-// Per slot: its S stream and its PV stream (the PV stream trails).  In the aliased
-// layout S_{i+1} may only follow PV_i (the MMAs of one thread run in issue order,
-// so PV_i has read P before S_{i+1} overwrites it); there the PV is tried first, so
-// that S_{i+1} can follow it in the same pass (a pass later cost the D = 128
-// softcap workload 15%).  In the separate-P layout the S goes first.
+// Per slot: its S stream and its PV stream (the PV stream trails).  The PV is tried
+// first.  In the aliased layout S_{i+1} may only follow PV_i (the MMAs of one thread
+// run in issue order, so PV_i has read P before S_{i+1} overwrites it), and this
+// lets S_{i+1} follow it in the same pass (a pass later cost the D = 128 softcap
+// workload 15%).  In the separate-P layout a PV ahead of an S that is also ready
+// lets the softmax, which waits for PV_{i-1} before it writes P_i, go on sooner
+// (causal 8192: 131 -> 123 us; window 4096: 121 -> 116 us).
 template <int D, int SLOT, bool BHM>
 __device__ __forceinline__ bool mma_slot(Smem<D>& sm, const Params& p, MmaStream<BHM>& cs,
                                          MmaStream<BHM>& cp, MmaShared& ms) {
   bool progress = false;
-  if constexpr (!Cfg<D>::kSepP) {
-    if (cp.active && (!cs.active || cp.i < cs.i)) progress |= try_pv<D, SLOT>(sm, p, cp, ms);
-  }
+  if (cp.active && (!cs.active || cp.i < cs.i)) progress |= try_pv<D, SLOT>(sm, p, cp, ms);
   if (cs.active && (Cfg<D>::kSepP || cs.i == cp.i)) progress |= try_s<D, SLOT>(sm, p, cs, ms);
-  if constexpr (Cfg<D>::kSepP) {
-    if (cp.active && (!cs.active || cp.i < cs.i)) progress |= try_pv<D, SLOT>(sm, p, cp, ms);
-  }
   return progress;
 }
 
@@ -766,9 +763,10 @@ __device__ __forceinline__ void range_chunk(float (&x)[64], int a, int b, int am
 // a <= i <= b (causal / window interval, clipped to the keys that exist) and, for
 // documents, doc_id[kv0 + i] == dq; for a tabulated mask, iff its bit in the row's
 // words `brow` is set (and the key exists).  Dead entries become -inf.
+// `ext` = (min a, max a, min b, max b) over the warp's 32 rows (interval rule).
 template <int MK>
-__device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int a, int b, int kv0,
-                                           int dq, const int32_t* docs,
+__device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int a, int b, int4 ext,
+                                           int kv0, int dq, const int32_t* docs,
                                            const uint32_t* brow) {
   if constexpr (MK == kMaskBitmap) {
     // the row's two words of keys kv0 .. kv0 + 63 (kv0 is a multiple of 64)
@@ -801,10 +799,8 @@ __device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int 
     MaskCols<0>::doc(x, a, b, same[0]);
     MaskCols<32>::doc(x, a, b, same[1]);
   } else {
-    const int amin = __reduce_min_sync(0xffffffffu, a), amax = __reduce_max_sync(0xffffffffu, a);
-    const int bmin = __reduce_min_sync(0xffffffffu, b), bmax = __reduce_max_sync(0xffffffffu, b);
-    range_chunk<0>(x, a, b, amin, amax, bmin, bmax);
-    range_chunk<32>(x, a, b, amin, amax, bmin, bmax);
+    range_chunk<0>(x, a, b, ext.x, ext.y, ext.z, ext.w);
+    range_chunk<32>(x, a, b, ext.x, ext.y, ext.z, ext.w);
   }
 }
 
@@ -926,10 +922,27 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
     // for a tabulated mask, its bit); only the causal rules bound hi by the row.
     // Formed where a PARTIAL block needs them, so that no register holds them
     // through the block loop.
-    auto key_range = [&](int& lo, int& hi) {
-      const int r = un.qblk * kBlockN + t;
+    // Both bounds are non-decreasing in the row, so over the warp's 32 rows their
+    // extremes are those of its first and last row: `mask_span` forms a block's
+    // bounds for this row (a, b) and the warp's extremes without a warp reduction.
+    auto key_range = [&](int r, int& lo, int& hi) {
       hi = MK == kMaskBitmap ? p.S - 1 : min(r, p.S - 1);
       lo = p.mask_kind == FA_MASK_SLIDING_WINDOW_CAUSAL ? max(r - p.window + 1, 0) : 0;
+    };
+    auto mask_span = [&](int kv0, int& a, int& b, int4& ext) {
+      const int r = un.qblk * kBlockN + t;
+      int lo, hi;
+      key_range(r, lo, hi);
+      a = lo - kv0;
+      b = hi - kv0;
+      ext = make_int4(0, 0, 0, 0);
+      if constexpr (MK == kMaskRange) {
+        const int rw = r - (t & 31);
+        int lo0, hi0, lo1, hi1;
+        key_range(rw, lo0, hi0);
+        key_range(rw + 31, lo1, hi1);
+        ext = make_int4(lo0 - kv0, lo1 - kv0, hi0 - kv0, hi1 - kv0);
+      }
     };
     float m = -INFINITY, l = 0.f;  // running max (log2 units) and running sum
     int kvb = block_index(p, un, 0);
@@ -959,14 +972,14 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         if ((t & 31) == 0) mbar_arrive(&sm.s_empty[slot]);
         if constexpr (SC) softcap64(p, *reinterpret_cast<float(*)[64]>(x)), softcap64(p, *reinterpret_cast<float(*)[64]>(x + 64));
         if (!full) {
-          int lo, hi;
-          key_range(lo, hi);
-          const int a = lo - kvb * kBlockN;
-          const int b = hi - kvb * kBlockN;
-          apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x), a, b, kvb * kBlockN, dq, docs_of(),
-                     brow_of());
-          apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x + 64), a - 64, b - 64, kvb * kBlockN + 64, dq,
-                     docs_of(), brow_of());
+          int a, b;
+          int4 e;
+          mask_span(kvb * kBlockN, a, b, e);
+          apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x), a, b, e, kvb * kBlockN, dq, docs_of(),
+                         brow_of());
+          apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x + 64), a - 64, b - 64,
+                         make_int4(e.x - 64, e.y - 64, e.z - 64, e.w - 64), kvb * kBlockN + 64, dq,
+                         docs_of(), brow_of());
         }
         const float mb = fmaxf(row_max64(*reinterpret_cast<float(*)[64]>(x)),
                                row_max64(*reinterpret_cast<float(*)[64]>(x + 64))) * xs;
@@ -999,18 +1012,18 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
         // that one max: P_hi of half h goes to P columns [32h, 32h + 32); with the
         // split, P_lo goes to columns 64 + [32h, 32h + 32), held in registers until
         // half 1 has been read (in the aliased layout those columns are still S).
-        int lo, hi;
-        key_range(lo, hi);
-        const int a = lo - kvb * kBlockN;  // live columns of the block: a <= i <= b
-        const int b = hi - kvb * kBlockN;
+        int a, b;  // live columns of the block: a <= i <= b
+        int4 e;
+        mask_span(kvb * kBlockN, a, b, e);
         float rmax = -INFINITY;
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           float x[64];
           load_s_half(t_s + h * 64, x);
           if (!full)
-            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, docs_of(),
-                           brow_of());
+            apply_mask<MK>(p, x, a - h * 64, b - h * 64,
+                           make_int4(e.x - h * 64, e.y - h * 64, e.z - h * 64, e.w - h * 64),
+                           kvb * kBlockN + h * 64, dq, docs_of(), brow_of());
           rmax = fmaxf(rmax, row_max64(x));
         }
         float mb = rmax;
@@ -1077,8 +1090,9 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
             }
           }
           if (!full)
-            apply_mask<MK>(p, x, a - h * 64, b - h * 64, kvb * kBlockN + h * 64, dq, docs_of(),
-                           brow_of());
+            apply_mask<MK>(p, x, a - h * 64, b - h * 64,
+                           make_int4(e.x - h * 64, e.y - h * 64, e.z - h * 64, e.w - h * 64),
+                           kvb * kBlockN + h * 64, dq, docs_of(), brow_of());
           // P = exp2(x * xs - m) as 16-bit pairs; with the split, P_hi = p truncated to
           // bf16 and P_lo = round(p - P_hi), so P_hi + P_lo carries ~16 significant bits.
           float2 sums[4];
