@@ -53,12 +53,12 @@ DECODE_SOURCES = ("block_sparse_attention_create_b200/csrc/decode.cu",
                   "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
 NCU_TRAFFIC = {
     "swa256_L32768_B1_H8_D64_bf16": {
-        "bytes": 101026560 + 5083136, "sources": FWD_SOURCES,
-        "sources_sha256": "6f30b4f50f85a426533ccfe9e2671dd40b905625c210f1b9a6b0fdebb260cb9d",
+        "bytes": 101149440 + 7180544, "sources": FWD_SOURCES,
+        "sources_sha256": "5454ccb6e0329a5d1ceaae47f34c47d023e96b0ff524260b3a90862d1c8d2949",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_launches.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
-        "bytes": 1073887488 + 3557632, "sources": DECODE_SOURCES,
-        "sources_sha256": "78393a08231b16ebe651a9b3434ca4a91b22c2c9d64c50879e73c979fc893e80",
+        "bytes": 1073843200 + 3553792, "sources": DECODE_SOURCES,
+        "sources_sha256": "aac525e8048b62fb3872f57170f7c86ae2904fb865c82a5577d15bafd2eac08f",
         "summary": "profiles/decode_mma_kernel_L1_S32768_B8_H32_Hkv8_D128_full.md"},
 }
 

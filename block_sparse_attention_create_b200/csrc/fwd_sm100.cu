@@ -30,7 +30,7 @@
 // overwrites the S it came from (TMEM holds no more), S_{j+1} is issued after PV_j
 // (tcgen05 operations of one thread run in issue order), and the commit that
 // signals S_{j+1} also means PV_j is done.
-// Epilogue of a unit, O / l: at D = 64, for a unit of at most kStageMaxBlocks
+// Epilogue of a unit, O / l: at D = 64, for a unit of at most stage_max_blocks()
 // blocks, each softmax warp writes its 32 rows into the unit's Q tile and one lane
 // stores them with a TMA tensor store, so the LSU carries no output traffic; longer
 // units and D = 128 store from registers.
@@ -63,13 +63,6 @@ constexpr int kThreads = (kSoftmaxWarps + kNumSlots + 1) * 32;  // + 2 producers
 // three per sub-partition here, and each sub-partition has a quarter of the
 // register file (16384): 3 x 32 x 168 fits, 3 x 32 x 176 does not.
 constexpr int kBlockN = 128;                 // rows of a Q tile / K,V tile
-// Units of at most this many blocks store O through the staging tile (TMA store);
-// longer ones store it from registers.  Measured at D = 64: short units end every
-// few blocks, and their direct stores queued behind one another in the load/store
-// unit (window 256, 32k: 77 -> 74 us staged); a long unit's stores drain during
-// its successor, and there the staging (proxy fence, release of the tile) cost
-// 2-3% (causal 8192, window 4096).
-constexpr int kStageMaxBlocks = 4;
 constexpr int kChunkBytes = 128 * 128;       // one TMA box: 128 rows x 64 elems x 2 B
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -80,6 +73,19 @@ constexpr int kMaskDoc = 1;
 constexpr int kMaskBitmap = 2;
 __host__ __device__ constexpr int mask_family(int kind) {
   return kind == FA_MASK_DOCUMENT_CAUSAL ? kMaskDoc : (kind == FA_MASK_BITMAP ? kMaskBitmap : kMaskRange);
+}
+// Units of at most this many blocks store O through the staging tile (TMA store);
+// longer ones store it from registers.  Measured at D = 64: short units end every
+// few blocks, and their direct stores queued behind one another in the load/store
+// unit (window 256, 32k: 77 -> 74 us staged); a long unit's stores drain during
+// its successor, and there the staging cost 3-11% (window 4096; causal 8192:
+// 127 -> 142 us with every unit staged).  The tabulated-mask kernel stages every
+// unit: with both epilogues compiled in, its register allocation spills in the
+// block loop, and the bitmap loads there wait on the spilled values (8192, random
+// block classes: 305 us mixed, 259 us all staged, 262 us all direct).
+template <int MK>
+__host__ __device__ constexpr int stage_max_blocks() {
+  return MK == kMaskBitmap ? (1 << 30) : 4;
 }
 
 // TMEM layouts (512 columns, lanes = the 128 rows of a tile):
@@ -759,20 +765,38 @@ __device__ __forceinline__ void range_chunk(float (&x)[64], int a, int b, int am
   if (!(amax <= C0 && bmin >= C0 + 31)) RangeCols<C0, C0 + 32>::apply(x, a, b);
 }
 
+// Tabulated rule: the row's four mask words of a PARTIAL block, keys kv0 .. kv0+127
+// (bit i of w[c]: key kv0 + 32c + i), loaded before the block's S is waited for,
+// so that the load's latency overlaps that wait (kv0 is a multiple of 128; the
+// words are read in 8-byte pairs, the alignment the bitmap is checked for).
+template <int MK>
+__device__ __forceinline__ void mask_fetch(const uint32_t* brow, int kv0, uint32_t (&w)[4]) {
+  if constexpr (MK == kMaskBitmap) {
+    const int2 w01 = ldg_nc_v2(reinterpret_cast<const int32_t*>(brow + (kv0 >> 5)));
+    const int2 w23 = ldg_nc_v2(reinterpret_cast<const int32_t*>(brow + (kv0 >> 5) + 2));
+    w[0] = static_cast<uint32_t>(w01.x);
+    w[1] = static_cast<uint32_t>(w01.y);
+    w[2] = static_cast<uint32_t>(w23.x);
+    w[3] = static_cast<uint32_t>(w23.y);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) w[c] = 0u;
+  }
+}
+
 // Mask rule on 64 columns of a PARTIAL block: column i (key kv0 + i) is live iff
 // a <= i <= b (causal / window interval, clipped to the keys that exist) and, for
-// documents, doc_id[kv0 + i] == dq; for a tabulated mask, iff its bit in the row's
-// words `brow` is set (and the key exists).  Dead entries become -inf.
-// `ext` = (min a, max a, min b, max b) over the warp's 32 rows (interval rule).
+// documents, doc_id[kv0 + i] == dq; for a tabulated mask, iff its bit in the words
+// w0 (columns 0-31) and w1 (32-63) from mask_fetch is set.  Dead entries become
+// -inf.  `ext` = (min a, max a, min b, max b) over the warp's 32 rows (interval
+// rule).
 template <int MK>
 __device__ __forceinline__ void apply_mask(const Params& p, float (&x)[64], int a, int b, int4 ext,
-                                           int kv0, int dq, const int32_t* docs,
-                                           const uint32_t* brow) {
+                                           int kv0, int dq, const int32_t* docs, uint32_t w0,
+                                           uint32_t w1) {
   if constexpr (MK == kMaskBitmap) {
-    // the row's two words of keys kv0 .. kv0 + 63 (kv0 is a multiple of 64)
-    const int2 w = ldg_nc_v2(reinterpret_cast<const int32_t*>(brow + (kv0 >> 5)));
-    MaskCols<0>::doc(x, a, b, static_cast<uint32_t>(w.x));
-    MaskCols<32>::doc(x, a, b, static_cast<uint32_t>(w.y));
+    MaskCols<0>::doc(x, a, b, w0);
+    MaskCols<32>::doc(x, a, b, w1);
   } else if constexpr (MK == kMaskDoc) {
     // bit i of `same[c]`: the document of key kv0 + c*32 + i equals the row's; keys
     // past S read the last id (in bounds) and are excluded by the range anyway.  Lane
@@ -950,6 +974,9 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
     for (int j = 0; j < un.n; ++j) {
       const bool full = j >= un.np;
       const int kvb_next = j + 1 < un.n ? block_index(p, un, j + 1) : 0;
+      // a PARTIAL block's tabulated-mask words, loaded before S is waited for
+      uint32_t mw[4] = {0u, 0u, 0u, 0u};
+      if (!full) mask_fetch<MK>(brow_of(), kvb * kBlockN, mw);
       if (!wait_warp(sm, &sm.s_full[slot], blk & 1, p)) return;
       tc_fence_after();
       if constexpr (C::kStageO) {
@@ -976,10 +1003,10 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
           int4 e;
           mask_span(kvb * kBlockN, a, b, e);
           apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x), a, b, e, kvb * kBlockN, dq, docs_of(),
-                         brow_of());
+                         mw[0], mw[1]);
           apply_mask<MK>(p, *reinterpret_cast<float(*)[64]>(x + 64), a - 64, b - 64,
                          make_int4(e.x - 64, e.y - 64, e.z - 64, e.w - 64), kvb * kBlockN + 64, dq,
-                         docs_of(), brow_of());
+                         docs_of(), mw[2], mw[3]);
         }
         const float mb = fmaxf(row_max64(*reinterpret_cast<float(*)[64]>(x)),
                                row_max64(*reinterpret_cast<float(*)[64]>(x + 64))) * xs;
@@ -1023,7 +1050,8 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
           if (!full)
             apply_mask<MK>(p, x, a - h * 64, b - h * 64,
                            make_int4(e.x - h * 64, e.y - h * 64, e.z - h * 64, e.w - h * 64),
-                           kvb * kBlockN + h * 64, dq, docs_of(), brow_of());
+                           kvb * kBlockN + h * 64, dq, docs_of(), h ? mw[2] : mw[0],
+                           h ? mw[3] : mw[1]);
           rmax = fmaxf(rmax, row_max64(x));
         }
         float mb = rmax;
@@ -1092,7 +1120,8 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
           if (!full)
             apply_mask<MK>(p, x, a - h * 64, b - h * 64,
                            make_int4(e.x - h * 64, e.y - h * 64, e.z - h * 64, e.w - h * 64),
-                           kvb * kBlockN + h * 64, dq, docs_of(), brow_of());
+                           kvb * kBlockN + h * 64, dq, docs_of(), h ? mw[2] : mw[0],
+                           h ? mw[3] : mw[1]);
           // P = exp2(x * xs - m) as 16-bit pairs; with the split, P_hi = p truncated to
           // bf16 and P_lo = round(p - P_hi), so P_hi + P_lo carries ~16 significant bits.
           float2 sums[4];
@@ -1140,7 +1169,7 @@ __device__ void softmax_role(Smem<D>& sm, const Params& p, uint32_t tmem, int sl
     tc_fence_after();
     const size_t orow = static_cast<size_t>(un.bh) * p.L + un.qblk * kBlockN + t;
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    if (C::kStageO && un.n <= kStageMaxBlocks) {
+    if (C::kStageO && un.n <= stage_max_blocks<MK>()) {
       // O comes into registers and is released to the next unit's PV at once; the
       // warp writes its 32 rows into the staging tile (128-byte rows, 16-byte chunk
       // c of row r at chunk c ^ (r % 8): the layout of the map's 128-byte swizzle,
