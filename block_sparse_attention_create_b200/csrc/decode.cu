@@ -32,12 +32,13 @@ namespace {
 
 constexpr int kTile = 64;            // keys per K/V tile
 constexpr int kMaxRows = FA_DECODE_MAX_ROWS;
-// CTAs per SM of the chunk kernel for R rows: the tensor-core kernel (R <= 8) runs
-// three; the CUDA-core kernel runs 8 warps, two CTAs per SM, at D = 128 and 4 warps,
-// three per SM, at D = 64.  The grid is sized for that many CTAs.
+// CTAs per SM of the chunk kernel for R rows: the tensor-core kernel runs three
+// (two at D = 128 for R > 8, twice the accumulators); the CUDA-core kernel
+// (R <= 32) runs 8 warps, two CTAs per SM, at D = 128 and 4 warps, three per SM, at
+// D = 64.  The grid is sized for that many CTAs.
 __host__ __device__ constexpr int split_ctas_per_sm(int D) { return D == 128 ? 2 : 3; }
 __host__ __device__ constexpr int dec_ctas_per_sm(int D, int rows) {
-  return rows <= 8 ? 3 : split_ctas_per_sm(D);
+  return rows <= 8 ? 3 : (rows <= 16 ? (D == 128 ? 2 : 3) : split_ctas_per_sm(D));
 }
 template <int D>
 struct DecCfg {
@@ -405,24 +406,27 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
   }
 }
 
-// ---------------------------------------------------------------- at most 8 rows
-// The common grouped-query decode (R = (H / H_kv) * L <= 8 rows per K/V head) on
+// ---------------------------------------------------------------- at most 16 rows
+// The common grouped-query decode (R = (H / H_kv) * L <= 16 rows per K/V head) on
 // warp-level tensor-core tiles (16 x 8 x 16), with each warp keeping its own online
 // softmax state over its keys, so that a tile needs no barrier across the CTA.
-// Warp w of the 4 compute warps takes keys 16w .. 16w + 15 of every 64-key tile:
+// Warp w of the 4 compute warps takes keys 16w .. 16w + 15 of every 64-key tile;
+// the rows come in NT = ceil(R / 8) column tiles of 8 (the MMA's N), each sharing
+// the A fragments loaded for the others:
 //   S^T (16 keys x 8 rows) = K_w Q^T      (A = K rows by ldmatrix from the swizzled
 //                                          TMA tile, B = Q^T held in registers for
-//                                          the whole chunk; rows R .. 7 are zero)
+//                                          the whole chunk; rows past R are zero)
 //   O^T (D x 8 rows)      += V_w^T P      (A = V^T by transposing ldmatrix, B = P:
 //                                          the S^T fragment rounded to 16 bits and
 //                                          transposed in registers by movmatrix)
-// Lane l holds rows 2(l % 4) and 2(l % 4) + 1 of both fragments, so its online
-// softmax state and its share of O belong to the same two rows.  A fifth warp
-// keeps the ring of tiles full; the 4 warps' states are merged at the end.  The
-// score is the fp32 accumulation of 16-bit products, scaled in fp32.
+// Lane l holds rows 8t + 2(l % 4) and 8t + 2(l % 4) + 1 of tile t of both
+// fragments, so its online softmax state and its share of O belong to the same
+// rows.  A fifth warp keeps the ring of tiles full; the 4 warps' states are merged
+// at the end.  The score is the fp32 accumulation of 16-bit products, scaled in
+// fp32.
 constexpr int kMdWarps = 4;                      // compute warps
 constexpr int kMdThreads = (kMdWarps + 1) * 32;  // + the producer warp
-constexpr int kMdRows = 8;                       // the MMA's N: rows R .. 7 are padding
+constexpr int kMdRows = 16;                      // rows this kernel takes (NT <= 2)
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -470,23 +474,24 @@ __device__ __forceinline__ uint32_t pack_16(float lo, float hi, bool bf16) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int D>
+template <int D, int NT>
 struct __align__(1024) MdSmem {
   static constexpr int kStages = D == 128 ? 2 : 3;
   uint8_t k[kStages][D / 64][kBoxBytes];
   uint8_t v[kStages][D / 64][kBoxBytes];
-  float wm[kMdWarps][kMdRows], wl[kMdWarps][kMdRows];
+  float wm[kMdWarps][8 * NT], wl[kMdWarps][8 * NT];
   uint64_t full[kStages], empty[kStages];
   volatile int abort_flag;
 };
 
-template <int D, bool BF16>
-__global__ void __launch_bounds__(kMdThreads, 3)
+template <int D, bool BF16, int NT>
+__global__ void __launch_bounds__(kMdThreads, dec_ctas_per_sm(D, 8 * NT))
 decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                   const __grid_constant__ DecParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
-  using Sm = MdSmem<D>;
+  using Sm = MdSmem<D, NT>;
+  constexpr int kRows = 8 * NT;
   constexpr int kStages = Sm::kStages;
   constexpr int kKs = D / 16;  // k-steps of S = 16-dim slices; m-tiles of O^T
   Sm& sm = *reinterpret_cast<Sm*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
@@ -510,15 +515,21 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
   }
   __syncthreads();
 
-  // this lane's rows in both fragments (2q, 2q + 1) and its key / dim row (l / 4)
+  // this lane's rows in both fragments (8t + 2q, 8t + 2q + 1 of tile t) and its key /
+  // dim row (l / 4)
   const int q4 = lane & 3, g8 = lane >> 2;
-  const int n0 = 2 * q4, n1 = 2 * q4 + 1;
-  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
-  float o[kKs][4];
+  const int n0 = 2 * q4, n1 = 2 * q4 + 1;  // rows within a tile
+  float m[NT][2], l[NT][2];
+  float o[NT][kKs][4];
 #pragma unroll
-  for (int t = 0; t < kKs; ++t)
+  for (int nt = 0; nt < NT; ++nt) {
+    m[nt][0] = m[nt][1] = -INFINITY;
+    l[nt][0] = l[nt][1] = 0.f;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[t][e] = 0.f;
+    for (int t = 0; t < kKs; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[nt][t][e] = 0.f;
+  }
 
   if (warp == kMdWarps) {
     // producer: tile t into stage t % kStages once the warps have released the tile
@@ -549,21 +560,21 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
         }
     }
   } else {
-    // Q^T as the B fragments of S^T: slice ks, lane holds Q[row g8][16 ks + 2 q4 + {0, 1}]
-    // and the same 8 dims further on; rows past R are zero
-    uint32_t qb[kKs][2];
-    {
-      const bool live = g8 < R;
-      const int g = live ? g8 / p.L : 0, i = live ? g8 - g * p.L : 0;
+    // Q^T as the B fragments of S^T: tile nt, slice ks, lane holds Q[row 8 nt + g8]
+    // [16 ks + 2 q4 + {0, 1}] and the same 8 dims further on; rows past R are zero
+    uint32_t qb[NT][kKs][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int r = 8 * nt + g8;
+      const bool live = r < R;
+      const int g = live ? r / p.L : 0, i = live ? r - g * p.L : 0;
       const uint16_t* qrow = p.q + (static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i) * D;
 #pragma unroll
       for (int ks = 0; ks < kKs; ++ks) {
-        qb[ks][0] = live ? __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * ks + 2 * q4)) : 0u;
-        qb[ks][1] = live ? __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * ks + 8 + 2 * q4)) : 0u;
+        qb[nt][ks][0] = live ? __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * ks + 2 * q4)) : 0u;
+        qb[nt][ks][1] = live ? __ldg(reinterpret_cast<const unsigned int*>(qrow + 16 * ks + 8 + 2 * q4)) : 0u;
       }
     }
-    const int pos0 = p.S - p.L + (n0 < R ? n0 % p.L : 0);
-    const int pos1 = p.S - p.L + (n1 < R ? n1 % p.L : 0);
     // ldmatrix row of this lane: matrix lane / 8, row lane % 8
     const int mi = lane >> 3, mr = lane & 7;
     for (int t = 0; t < ntiles; ++t) {
@@ -572,66 +583,78 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
       const int k0 = k_start + t * kTile;
       // S^T = K_w Q^T: A = keys 16 warp + (0..15) x dims 16 ks + (0..15); the four 8x8
       // matrices are (keys 0-7, dims 0-7), (keys 8-15, dims 0-7), (keys 0-7, dims
-      // 8-15), (keys 8-15, dims 8-15)
-      float s[4] = {0.f, 0.f, 0.f, 0.f};
+      // 8-15), (keys 8-15, dims 8-15); one A fragment serves every row tile
+      float s[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
       {
         const int key = 16 * warp + mr + 8 * (mi & 1);
 #pragma unroll
         for (int ks = 0; ks < kKs; ++ks) {
           uint32_t a[4];
           ldsm_x4(chunk_addr(sm.k[buf], key, 2 * ks + (mi >> 1)), a);
-          mma16816<BF16>(s, a, qb[ks][0], qb[ks][1]);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma16816<BF16>(s[nt], a, qb[nt][ks][0], qb[nt][ks][1]);
         }
       }
-      // s[0], s[1]: key 16 warp + g8, rows n0, n1; s[2], s[3]: key + 8
+      // s[nt][0], s[nt][1]: key 16 warp + g8, rows 8 nt + n0, n1; s[nt][2], s[nt][3]: key + 8
       const int kva = k0 + 16 * warp + g8, kvb = kva + 8;
-      float x[4];
+      uint32_t pb[NT][2];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int kv = e < 2 ? kva : kvb;
-        const int n = (e & 1) ? n1 : n0;
-        const int pos = (e & 1) ? pos1 : pos0;
-        float v = s[e] * p.q_scale;
-        if (p.softcap_on) v = p.cap_a * tanhf(v / p.cap_c);
-        bool keep = n < R && kv < c1;
-        if (p.mask != FA_DECODE_FULL) keep = keep && kv <= pos;
-        if (p.mask == FA_DECODE_SLIDING_WINDOW) keep = keep && pos - kv < p.window;
-        x[e] = keep ? v : -INFINITY;
-      }
-      // online softmax per row over the warp's 16 keys (lanes with the same l % 4)
-      float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
+      for (int nt = 0; nt < NT; ++nt) {
+        const int r0 = 8 * nt + n0, r1 = 8 * nt + n1;
+        const int pos0 = p.S - p.L + (r0 < R ? r0 % p.L : 0);
+        const int pos1 = p.S - p.L + (r1 < R ? r1 % p.L : 0);
+        float x[4];
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-      }
-      const float mn0 = fmaxf(m[0], mx0), mn1 = fmaxf(m[1], mx1);
-      const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
-      const float p0 = ex2_approx(x[0] - mu0), p1 = ex2_approx(x[1] - mu1);
-      const float p2 = ex2_approx(x[2] - mu0), p3 = ex2_approx(x[3] - mu1);
-      float sm0 = p0 + p2, sm1 = p1 + p3;
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        sm0 += __shfl_xor_sync(0xffffffffu, sm0, off);
-        sm1 += __shfl_xor_sync(0xffffffffu, sm1, off);
-      }
-      const float al0 = ex2_approx(m[0] - mu0), al1 = ex2_approx(m[1] - mu1);
-      l[0] = l[0] * al0 + sm0;
-      l[1] = l[1] * al1 + sm1;
-      m[0] = mn0;
-      m[1] = mn1;
-      if (al0 != 1.f || al1 != 1.f) {
-#pragma unroll
-        for (int mt = 0; mt < kKs; ++mt) {
-          o[mt][0] *= al0;
-          o[mt][1] *= al1;
-          o[mt][2] *= al0;
-          o[mt][3] *= al1;
+        for (int e = 0; e < 4; ++e) {
+          const int kv = e < 2 ? kva : kvb;
+          const int n = (e & 1) ? r1 : r0;
+          const int pos = (e & 1) ? pos1 : pos0;
+          float v = s[nt][e] * p.q_scale;
+          if (p.softcap_on) v = p.cap_a * tanhf(v / p.cap_c);
+          bool keep = n < R && kv < c1;
+          if (p.mask != FA_DECODE_FULL) keep = keep && kv <= pos;
+          if (p.mask == FA_DECODE_SLIDING_WINDOW) keep = keep && pos - kv < p.window;
+          x[e] = keep ? v : -INFINITY;
         }
+        // online softmax per row over the warp's 16 keys (lanes with the same l % 4)
+        float mx0 = fmaxf(x[0], x[2]), mx1 = fmaxf(x[1], x[3]);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        const float mn0 = fmaxf(m[nt][0], mx0), mn1 = fmaxf(m[nt][1], mx1);
+        const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
+        const float p0 = ex2_approx(x[0] - mu0), p1 = ex2_approx(x[1] - mu1);
+        const float p2 = ex2_approx(x[2] - mu0), p3 = ex2_approx(x[3] - mu1);
+        float sm0 = p0 + p2, sm1 = p1 + p3;
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          sm0 += __shfl_xor_sync(0xffffffffu, sm0, off);
+          sm1 += __shfl_xor_sync(0xffffffffu, sm1, off);
+        }
+        const float al0 = ex2_approx(m[nt][0] - mu0), al1 = ex2_approx(m[nt][1] - mu1);
+        l[nt][0] = l[nt][0] * al0 + sm0;
+        l[nt][1] = l[nt][1] * al1 + sm1;
+        m[nt][0] = mn0;
+        m[nt][1] = mn1;
+        if (al0 != 1.f || al1 != 1.f) {
+#pragma unroll
+          for (int mt = 0; mt < kKs; ++mt) {
+            o[nt][mt][0] *= al0;
+            o[nt][mt][1] *= al1;
+            o[nt][mt][2] *= al0;
+            o[nt][mt][3] *= al1;
+          }
+        }
+        // P as the B fragment of O^T += V^T P: transpose the two 8x8 halves
+        pb[nt][0] = movm_trans(pack_16(p0, p1, BF16));
+        pb[nt][1] = movm_trans(pack_16(p2, p3, BF16));
       }
-      // P as the B fragment of O^T += V^T P: transpose the two 8x8 halves
-      const uint32_t pb0 = movm_trans(pack_16(p0, p1, BF16));
-      const uint32_t pb1 = movm_trans(pack_16(p2, p3, BF16));
       // A = V^T: dims 16 mt + (0..15) x keys 16 warp + (0..15); matrices (dims 0-7,
       // keys 0-7), (dims 8-15, keys 0-7), (dims 0-7, keys 8-15), (dims 8-15, keys
       // 8-15), each the transpose of 8 key rows x 8 dims of the tile
@@ -641,7 +664,8 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
         for (int mt = 0; mt < kKs; ++mt) {
           uint32_t a[4];
           ldsm_x4_trans(chunk_addr(sm.v[buf], key, 2 * mt + (mi & 1)), a);
-          mma16816<BF16>(o[mt], a, pb0, pb1);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) mma16816<BF16>(o[nt][mt], a, pb[nt][0], pb[nt][1]);
         }
       }
       __syncwarp();
@@ -654,22 +678,26 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
   // merge the 4 warps' states per row.  The tile buffers are free now and hold the
   // warps' O^T: red[warp][row][D]
   float* red = reinterpret_cast<float*>(&sm.k[0][0][0]);
-  static_assert(sizeof(Sm::k) + sizeof(Sm::v) >= sizeof(float) * kMdWarps * kMdRows * D,
+  static_assert(sizeof(Sm::k) + sizeof(Sm::v) >= sizeof(float) * kMdWarps * kRows * D,
                 "reduction space");
   if (warp < kMdWarps) {
 #pragma unroll
-    for (int mt = 0; mt < kKs; ++mt) {
-      const int d = 16 * mt + g8;
-      red[(warp * kMdRows + n0) * D + d] = o[mt][0];
-      red[(warp * kMdRows + n1) * D + d] = o[mt][1];
-      red[(warp * kMdRows + n0) * D + d + 8] = o[mt][2];
-      red[(warp * kMdRows + n1) * D + d + 8] = o[mt][3];
-    }
-    if (g8 == 0) {
-      sm.wm[warp][n0] = m[0];
-      sm.wm[warp][n1] = m[1];
-      sm.wl[warp][n0] = l[0];
-      sm.wl[warp][n1] = l[1];
+    for (int nt = 0; nt < NT; ++nt) {
+      const int r0 = 8 * nt + n0, r1 = 8 * nt + n1;
+#pragma unroll
+      for (int mt = 0; mt < kKs; ++mt) {
+        const int d = 16 * mt + g8;
+        red[(warp * kRows + r0) * D + d] = o[nt][mt][0];
+        red[(warp * kRows + r1) * D + d] = o[nt][mt][1];
+        red[(warp * kRows + r0) * D + d + 8] = o[nt][mt][2];
+        red[(warp * kRows + r1) * D + d + 8] = o[nt][mt][3];
+      }
+      if (g8 == 0) {
+        sm.wm[warp][r0] = m[nt][0];
+        sm.wm[warp][r1] = m[nt][1];
+        sm.wl[warp][r0] = l[nt][0];
+        sm.wl[warp][r1] = l[nt][1];
+      }
     }
   }
   __syncthreads();
@@ -684,7 +712,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
       for (int w = 0; w < kMdWarps; ++w) {
         const float a = ex2_approx(sm.wm[w][rr] - mx);  // 0 for a warp that saw no key
         lsum = fmaf(a, sm.wl[w][rr], lsum);
-        acc = fmaf(a, red[(w * kMdRows + rr) * D + d], acc);
+        acc = fmaf(a, red[(w * kRows + rr) * D + d], acc);
       }
     }
     const int g = rr / p.L, i = rr - g * p.L;
@@ -755,7 +783,7 @@ void decode_plan(int B, int Hkv, int S, int D, int rows, int* nsplit, int* chunk
   *nsplit = S > 0 ? (S + *chunk - 1) / *chunk : 1;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, int NT>
 fa_status decode_mma_launch(const void* k, const void* v, int B, int S, const DecParams& prm,
                             cudaStream_t stream) {
   CUtensorMap tk, tv;
@@ -765,7 +793,7 @@ fa_status decode_mma_launch(const void* k, const void* v, int B, int S, const De
   const int rows = S > 0 ? S : 1, bh = S > 0 ? B * prm.Hkv : 1;
   if (!make_tile_map(&tk, kp, BF16, D, rows, bh, kTile)) return FA_ERR_CUDA;
   if (!make_tile_map(&tv, vp, BF16, D, rows, bh, kTile)) return FA_ERR_CUDA;
-  const size_t smem = sizeof(MdSmem<D>) + 1024;
+  const size_t smem = sizeof(MdSmem<D, NT>) + 1024;
   int dev = 0;
   FA_CUDA_CHECK(cudaGetDevice(&dev));
   {
@@ -774,14 +802,14 @@ fa_status decode_mma_launch(const void* k, const void* v, int B, int S, const De
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
     if (!done[dev]) {
-      FA_CUDA_CHECK(cudaFuncSetAttribute(decode_mma_kernel<D, BF16>,
+      FA_CUDA_CHECK(cudaFuncSetAttribute(decode_mma_kernel<D, BF16, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem)));
       done[dev] = true;
     }
   }
   const dim3 grid(prm.nsplit, B * prm.Hkv);
-  decode_mma_kernel<D, BF16><<<grid, kMdThreads, smem, stream>>>(tk, tv, prm);
+  decode_mma_kernel<D, BF16, NT><<<grid, kMdThreads, smem, stream>>>(tk, tv, prm);
   FA_CUDA_CHECK(cudaGetLastError());
   decode_combine_kernel<D><<<B * prm.H * prm.L, D, 0, stream>>>(prm);
   FA_CUDA_CHECK(cudaGetLastError());
@@ -894,15 +922,22 @@ extern "C" fa_status fa_flex_attention_decode(const void* q, const void* k, cons
   const cudaStream_t s = as_stream(stream);
   const bool b16 = dtype == FA_BF16;
   const int rows = G * L;
-  // up to 8 rows (the MMA's N): the tensor-core chunk kernel; more: the CUDA-core one
+  // up to 16 rows (one or two of the MMA's 8-row N tiles): the tensor-core chunk
+  // kernel; more: the CUDA-core one
   if (D == 64) {
+    if (rows <= 8)
+      return b16 ? decode_mma_launch<64, true, 1>(k, v, B, S, prm, s)
+                 : decode_mma_launch<64, false, 1>(k, v, B, S, prm, s);
     if (rows <= kMdRows)
-      return b16 ? decode_mma_launch<64, true>(k, v, B, S, prm, s)
-                 : decode_mma_launch<64, false>(k, v, B, S, prm, s);
+      return b16 ? decode_mma_launch<64, true, 2>(k, v, B, S, prm, s)
+                 : decode_mma_launch<64, false, 2>(k, v, B, S, prm, s);
     return decode_launch<64, 32>(k, v, b16, B, S, prm, s);
   }
+  if (rows <= 8)
+    return b16 ? decode_mma_launch<128, true, 1>(k, v, B, S, prm, s)
+               : decode_mma_launch<128, false, 1>(k, v, B, S, prm, s);
   if (rows <= kMdRows)
-    return b16 ? decode_mma_launch<128, true>(k, v, B, S, prm, s)
-               : decode_mma_launch<128, false>(k, v, B, S, prm, s);
+    return b16 ? decode_mma_launch<128, true, 2>(k, v, B, S, prm, s)
+               : decode_mma_launch<128, false, 2>(k, v, B, S, prm, s);
   return decode_launch<128, 32>(k, v, b16, B, S, prm, s);
 }

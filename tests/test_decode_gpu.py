@@ -83,10 +83,15 @@ def test_decode_window_skips_far_chunks_and_matches():
     (2, 6, 2, 2, 1500, 128, 2, 400, torch.float16, 1.0),    # six rows, window
     (1, 4, 1, 1, 1000, 64, 0, 0, torch.float16, 2.0),       # fp16 at D = 64, no mask
     (1, 2, 2, 3, 0, 64, 1, 0, torch.bfloat16, 1.0),         # empty cache: no key at all
+    (1, 3, 1, 3, 2049, 64, 1, 0, torch.bfloat16, 1.0),      # nine rows: a second row tile
+    (1, 8, 1, 2, 3000, 128, 1, 0, torch.bfloat16, 2.0),     # sixteen rows, x2 inputs
+    (2, 4, 1, 3, 1700, 64, 2, 350, torch.float16, 1.0),     # twelve rows, window, fp16
+    (1, 4, 1, 4, 2, 128, 1, 0, torch.bfloat16, 1.0),        # sixteen rows, L > S
 ])
 def test_decode_tensor_core_path(B, H, Hkv, L, S, D, mask, window, dtype, xs):
-    """At most 8 rows per K/V head take the warp-level tensor-core kernel (16-bit P
-    against each warp's exact running max): element by element against the oracle."""
+    """At most 16 rows per K/V head take the warp-level tensor-core kernel (one or two
+    8-row column tiles; 16-bit P against each warp's exact running max): element by
+    element against the oracle."""
     q, k, v = W.random_qkv(B, H, L, S, D, dtype, seed=B * 1000 + S + L, scale=xs, Hkv=Hkv)
     out, lse = _check(q, k, v, mask, window)
     if L > S:

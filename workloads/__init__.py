@@ -128,7 +128,12 @@ GQA_CAUSAL_8192 = _w("gqa_causal_L8192_B1_H32_Hkv8_D64_bf16", 1, 32, 8192, 64, t
 DECODE_32K = Workload(name="decode_L1_S32768_B8_H32_Hkv8_D128_bf16", B=8, H=32, L=1, S=32768,
                       D=128, dtype=torch.bfloat16, mask_kind=MASK_DECODE_CAUSAL, seed=14, Hkv=8)
 
-EXTRA = (BITMAP_8192, GQA_CAUSAL_8192, DECODE_32K)
+# The same cache with 4 new tokens per sequence (speculative decoding): 16 query
+# rows per K/V head.
+DECODE_32K_L4 = Workload(name="decode_L4_S32768_B8_H32_Hkv8_D128_bf16", B=8, H=32, L=4, S=32768,
+                         D=128, dtype=torch.bfloat16, mask_kind=MASK_DECODE_CAUSAL, seed=15, Hkv=8)
+
+EXTRA = (BITMAP_8192, GQA_CAUSAL_8192, DECODE_32K, DECODE_32K_L4)
 BY_NAME = {w.name: w for w in ALL + EXTRA}
 
 
