@@ -57,8 +57,8 @@ NCU_TRAFFIC = {
         "sources_sha256": "5454ccb6e0329a5d1ceaae47f34c47d023e96b0ff524260b3a90862d1c8d2949",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_launches.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
-        "bytes": 1073866496 + 3301888, "sources": DECODE_SOURCES,
-        "sources_sha256": "edbbcc5c01565c786478a0f380b48e80ec29934bbe7f8c64dace463ffb09136e",
+        "bytes": 1073843200 + 3686912, "sources": DECODE_SOURCES,
+        "sources_sha256": "ac7775954e81c51e6f33526a9d8387a32e00fc345b53f9632b5a6b6914123be1",
         "summary": "profiles/decode_mma_kernel_L1_S32768_B8_H32_Hkv8_D128_full.md"},
 }
 
@@ -652,11 +652,7 @@ def main():
                 "frac": tensor_frac, "traffic": ncu_traffic(w)}
     roof["peak_source"] = f"{peaks_src} (MEASURED_PEAKS.json)" if peaks_src == "measured" else "fallback"
     if is_decode(w):
-        # the tensor-core chunk kernel for at most 16 query rows per K/V head, else the
-        # CUDA-core one
-        rows = (w.H // w.n_kv_heads) * w.L
-        roof["kernel"] = (("decode_mma_kernel" if rows <= 16 else "decode_split_kernel")
-                          + " + decode_combine_kernel (fa_flex_attention_decode)")
+        roof["kernel"] = "decode_mma_kernel + decode_combine_kernel (fa_flex_attention_decode)"
     else:
         roof["kernel"] = "fwd_kernel (fa_flex_attention_fwd)"
     page_ms = PAGE_FWD_MS.get(w.name)

@@ -11,10 +11,11 @@
 // leaves the chunk's running max, sum and unnormalised output per row in the
 // workspace; a second kernel merges the chunks of each row (rescaling each by
 // 2^(m_chunk - m)) into out and LSE.  Chunks no row can see (sliding window) load
-// nothing.  Two kernels do the chunk: for R <= 8 rows (grouped-query decode of one
-// or a few tokens) `decode_mma_kernel`, whose warps keep private softmax states and
-// run both products on warp-level tensor-core tiles, so the instruction stream stays
-// well below the HBM time; for more rows `decode_split_kernel` on the CUDA cores.
+// nothing.  The chunk kernel, `decode_mma_kernel`, gives its warps private softmax
+// states and runs both products on warp-level tensor-core tiles, so the instruction
+// stream stays well below the HBM time; up to 16 rows one CTA takes them all, beyond
+// that one CTA per 16 rows, neighbours in launch order, so K and V still come from
+// DRAM about once.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -32,25 +33,15 @@ namespace {
 
 constexpr int kTile = 64;            // keys per K/V tile
 constexpr int kMaxRows = FA_DECODE_MAX_ROWS;
-// CTAs per SM of the chunk kernel for R rows: the tensor-core kernel runs three
-// (two at D = 128 for R > 8, twice the accumulators); the CUDA-core kernel
-// (R <= 32) runs 8 warps, two CTAs per SM, at D = 128 and 4 warps, three per SM, at
-// D = 64.  The grid is sized for that many CTAs.
-__host__ __device__ constexpr int split_ctas_per_sm(int D) { return D == 128 ? 2 : 3; }
+// CTAs per SM of the chunk kernel for R rows: three (two at D = 128 for R > 8, with
+// twice the accumulators).  The grid is sized for that many CTAs.
 __host__ __device__ constexpr int dec_ctas_per_sm(int D, int rows) {
-  return rows <= 8 ? 3 : (rows <= 16 ? (D == 128 ? 2 : 3) : split_ctas_per_sm(D));
+  return rows <= 8 ? 3 : (D == 128 ? 2 : 3);
 }
-template <int D>
-struct DecCfg {
-  static constexpr int kThreads = D == 128 ? 256 : 128;
-};
+// Tensor-core kernel: CTAs per (chunk, K/V head), each taking 16 of the R rows (one
+// for R <= 16).
+__host__ __device__ constexpr int dec_row_tiles(int rows) { return rows <= 16 ? 1 : (rows + 15) / 16; }
 constexpr int kBoxBytes = kTile * 128;  // one TMA box: 64 keys x 64 elements
-// K/V tiles in flight per CTA: a ring of stages(D, RM) tiles, plus L2 prefetches
-// of the tiles kPrefetch further on, so that enough bytes are on their way to cover
-// the DRAM latency (one 32 KB tile per CTA was not).  Three stages, except at D =
-// 128 with 32 rows, where two keep two CTAs per SM in shared memory.
-__host__ __device__ constexpr int dec_stages(int D, int RM) { return D == 128 && RM == 32 ? 2 : 3; }
-constexpr int kPrefetch = 4;
 constexpr int kDecWorkspaceHeader = 256;  // word 0: device error flags
 constexpr float kDecLog2e = 1.4426950408889634f;
 constexpr float kDecLn2 = 0.6931471805599453f;
@@ -62,53 +53,13 @@ struct DecParams {
   float* part;        // per (b, h, i, split): m, l, O[D]
   int32_t* err;
   int H, Hkv, G, L, S, nsplit, chunk, mask, window, softcap_on, is_bf16;
+  int row_tiles;  // tensor-core kernel: CTAs per (chunk, K/V head), each taking 16 rows
   float q_scale;  // folded into Q: scale * log2(e), or scale alone under the softcap
   float cap_c;    // softcap c
   float cap_a;    // c * log2(e)
   unsigned long long timeout_ns;
   int stall_loads;  // testing hook: no K/V tile is loaded (see fa_debug_set_mma_stall)
 };
-
-template <int D, int RM>
-struct __align__(1024) DecSmem {
-  static constexpr int kStages = dec_stages(D, RM);
-  uint8_t k[kStages][D / 64][kBoxBytes];
-  uint8_t v[kStages][D / 64][kBoxBytes];
-  float qs[RM][D];
-  float sc[RM][kTile];
-  float m[RM], l[RM], alpha[RM];
-  uint64_t full[dec_stages(D, RM)];
-  volatile int abort_flag;
-};
-
-__device__ __forceinline__ float load16(const uint16_t* ptr, bool bf16) {
-  const uint16_t u = __ldg(ptr);
-  return bf16 ? __uint_as_float(static_cast<uint32_t>(u) << 16)
-              : __half2float(__ushort_as_half(u));
-}
-
-// 8 consecutive 16-bit values -> fp32.
-__device__ __forceinline__ void unpack8(const uint4 raw, bool bf16, float (&f)[8]) {
-  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (bf16) {
-      f[2 * i] = __uint_as_float(w[i] << 16);
-      f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    } else {
-      const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
-      f[2 * i] = h.x;
-      f[2 * i + 1] = h.y;
-    }
-  }
-}
-
-// 16-byte chunk c (elements 8c .. 8c+7) of key row j of a tile: box c / 8, swizzled
-// position (c % 8) ^ (j % 8) inside the row's 128 bytes.
-template <int NB>
-__device__ __forceinline__ uint4 tile_chunk(const uint8_t (&tile)[NB][kBoxBytes], int j, int c) {
-  return *reinterpret_cast<const uint4*>(&tile[c >> 3][j * 128 + (((c & 7) ^ (j & 7)) << 4)]);
-}
 
 template <class Sm>
 __device__ __forceinline__ bool dec_wait(Sm& sm, uint64_t* bar, uint32_t parity,
@@ -128,290 +79,12 @@ __device__ __forceinline__ bool dec_wait(Sm& sm, uint64_t* bar, uint32_t parity,
   }
 }
 
-// RM: bound on the rows R (the path launches it with RM = 32 for R > 8; at most 8
-// rows take decode_mma_kernel).  With RM <= 8 every PV thread keeps all rows
-// for one 16-byte column chunk over a subset of the tile's keys (key group), and
-// the key groups are summed once per CTA at the end; with RM = 32 a thread keeps
-// a few rows over all keys.
-template <int D, int RM>
-__global__ void __launch_bounds__(DecCfg<D>::kThreads, split_ctas_per_sm(D))
-decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-                    const __grid_constant__ DecParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t base = smem_u32(smem_raw);
-  using Sm = DecSmem<D, RM>;
-  constexpr int kStages = Sm::kStages;
-  Sm& sm = *reinterpret_cast<Sm*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
-  constexpr int kThr = DecCfg<D>::kThreads;
-  constexpr int kWarps = kThr / 32;
-  constexpr int kRowGroups = kThr / kTile;        // score threads per key
-  constexpr int kChunks = D / 8;                  // 16-byte chunks of a row
-  constexpr int kGroups = kThr / kChunks;         // PV thread groups (rows or keys)
-  constexpr bool kKeyGroups = RM <= 8;
-  constexpr int kRowsPer = kKeyGroups ? RM : RM / kGroups;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int split = blockIdx.x, bkv = blockIdx.y;
-  const int b = bkv / p.Hkv, kvh = bkv - b * p.Hkv;
-  const int R = p.G * p.L;
-  const bool bf16 = p.is_bf16 != 0;
-
-  // keys of this chunk that some row can see: the window's lower edge for row 0
-  int k_start = split * p.chunk;
-  const int c1 = min(p.S, k_start + p.chunk);
-  if (p.mask == FA_DECODE_SLIDING_WINDOW) k_start = max(k_start, p.S - p.L - p.window + 1);
-  const int ntiles = k_start < c1 ? (c1 - k_start + kTile - 1) / kTile : 0;
-
-  if (tid == 0) {
-    for (int b = 0; b < kStages; ++b) mbar_init(&sm.full[b], 1);
-    sm.abort_flag = 0;
-    fence_barrier_init();
-  }
-  // query rows r = g * L + i (query head kvh * G + g, query i), scaled
-  for (int e = tid; e < R * D; e += kThr) {
-    const int r = e / D, d = e - (e / D) * D;
-    const int g = r / p.L, i = r - g * p.L;
-    const size_t qi = (static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i) * D + d;
-    sm.qs[r][d] = load16(p.q + qi, bf16) * p.q_scale;
-  }
-  for (int r = tid; r < R; r += kThr) {
-    sm.m[r] = -INFINITY;
-    sm.l[r] = 0.f;
-  }
-  __syncthreads();
-
-  const uint64_t pol = policy_evict_first();
-  auto issue = [&](int t) {
-    const int buf = t % kStages;
-    const int k0 = k_start + t * kTile;
-    fence_proxy_async_shared();
-    mbar_arrive_expect_tx(&sm.full[buf], 2 * (D / 64) * kBoxBytes);
-#pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      tma_load_3d(sm.k[buf][c], &tk, &sm.full[buf], c * 64, k0, bkv, pol);
-      tma_load_3d(sm.v[buf][c], &tv, &sm.full[buf], c * 64, k0, bkv, pol);
-    }
-  };
-  auto prefetch = [&](int t) {  // tile t into L2
-    const int k0 = k_start + t * kTile;
-#pragma unroll
-    for (int c = 0; c < D / 64; ++c) {
-      tma_prefetch_3d(&tk, c * 64, k0, bkv);
-      tma_prefetch_3d(&tv, c * 64, k0, bkv);
-    }
-  };
-  if (tid == 0 && !p.stall_loads) {
-    for (int u = 0; u < kStages - 1 && u < ntiles; ++u) issue(u);
-    for (int u = kStages - 1; u < kStages - 1 + kPrefetch && u < ntiles; ++u) prefetch(u);
-  }
-
-  const int oc = tid % kChunks, og = tid / kChunks;  // PV: 16-byte chunk, row group
-  float o[kRowsPer][8];
-#pragma unroll
-  for (int k = 0; k < kRowsPer; ++k)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) o[k][e] = 0.f;
-
-  int t = 0;
-  for (; t < ntiles; ++t) {
-    const int buf = t % kStages;
-    const int k0 = k_start + t * kTile;
-    // tile t + kStages - 1 goes to the buffer released after tile t - 1
-    if (tid == 0 && !p.stall_loads) {
-      if (t + kStages - 1 < ntiles) issue(t + kStages - 1);
-      if (t + kStages - 1 + kPrefetch < ntiles) prefetch(t + kStages - 1 + kPrefetch);
-    }
-    const bool ok = dec_wait(sm, &sm.full[buf], (t / kStages) & 1, p);
-    if (!__syncthreads_and(ok)) break;
-
-    {
-      // scores: thread = (key j, row group rg); rows r = rg, rg + kRowGroups, ...
-      constexpr int kRowsS = RM / kRowGroups > 0 ? RM / kRowGroups : 1;
-      const int j = tid & (kTile - 1), rg = tid / kTile;
-      // two independent packed partial sums per row keep the FMA chains short
-      float2 acc[kRowsS][2];
-#pragma unroll
-      for (int k = 0; k < kRowsS; ++k) acc[k][0] = acc[k][1] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < kChunks; ++c) {
-        float kf[8];
-        unpack8(tile_chunk(sm.k[buf], j, c), bf16, kf);
-#pragma unroll
-        for (int k = 0; k < kRowsS; ++k) {
-          const int r = rg + kRowGroups * k;
-          if (r < R) {
-            const float4 qa = *reinterpret_cast<const float4*>(&sm.qs[r][c * 8]);
-            const float4 qb = *reinterpret_cast<const float4*>(&sm.qs[r][c * 8 + 4]);
-            acc[k][0] = fma2(make_float2(qa.x, qa.y), make_float2(kf[0], kf[1]), acc[k][0]);
-            acc[k][1] = fma2(make_float2(qa.z, qa.w), make_float2(kf[2], kf[3]), acc[k][1]);
-            acc[k][0] = fma2(make_float2(qb.x, qb.y), make_float2(kf[4], kf[5]), acc[k][0]);
-            acc[k][1] = fma2(make_float2(qb.z, qb.w), make_float2(kf[6], kf[7]), acc[k][1]);
-          }
-        }
-      }
-      const int kv = k0 + j;
-#pragma unroll
-      for (int k = 0; k < kRowsS; ++k) {
-        const int r = rg + kRowGroups * k;
-        if (r < R) {
-          const int pos = p.S - p.L + (r % p.L);  // the query's key position
-          bool keep = kv < c1;
-          if (p.mask != FA_DECODE_FULL) keep = keep && kv <= pos;
-          if (p.mask == FA_DECODE_SLIDING_WINDOW) keep = keep && pos - kv < p.window;
-          float s = (acc[k][0].x + acc[k][0].y) + (acc[k][1].x + acc[k][1].y);
-          if (p.softcap_on) s = p.cap_a * tanhf(s / p.cap_c);
-          sm.sc[r][j] = keep ? s : -INFINITY;
-        }
-      }
-    }
-    __syncthreads();
-
-    // online softmax: warp w takes rows w, w + 4, ...; lane holds keys lane, lane + 32
-    for (int r = warp; r < R; r += kWarps) {
-      const float s0 = sm.sc[r][lane], s1 = sm.sc[r][lane + 32];
-      float mx = fmaxf(s0, s1);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      const float m_old = sm.m[r];
-      const float m_new = fmaxf(m_old, mx);
-      const float mu = m_new == -INFINITY ? 0.f : m_new;  // a row with no key yet: p = 0
-      const float p0 = ex2_approx(s0 - mu), p1 = ex2_approx(s1 - mu);
-      float sum = p0 + p1;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      sm.sc[r][lane] = p0;
-      sm.sc[r][lane + 32] = p1;
-      __syncwarp();
-      if (lane == 0) {
-        const float a = ex2_approx(m_old - mu);  // 0 while the row had no key
-        sm.alpha[r] = a;
-        sm.l[r] = sm.l[r] * a + sum;
-        sm.m[r] = m_new;
-      }
-    }
-    __syncthreads();
-
-    // O += P V: thread = (16-byte chunk oc of a V row, group og: rows or keys)
-    if constexpr (kKeyGroups) {
-      // rescale only when some row's max moved (alpha is exactly 1 otherwise: ex2(0));
-      // the test reads the same shared values in every thread, so it is CTA-uniform
-      bool moved = false;
-#pragma unroll
-      for (int r = 0; r < RM; ++r) moved |= r < R && sm.alpha[r] != 1.f;
-      if (moved) {
-#pragma unroll
-        for (int r = 0; r < RM; ++r) {
-          const float a = r < R ? sm.alpha[r] : 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) o[r][e] *= a;
-        }
-      }
-      const int nk = min(kTile, c1 - k0);
-      for (int j = og; j < nk; j += kGroups) {
-        float vf[8];
-        unpack8(tile_chunk(sm.v[buf], j, oc), bf16, vf);
-#pragma unroll
-        for (int r = 0; r < RM; ++r) {
-          const float pj = r < R ? sm.sc[r][j] : 0.f;
-          const float2 p2 = make_float2(pj, pj);
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            const float2 acc2 = fma2(p2, make_float2(vf[e], vf[e + 1]), make_float2(o[r][e], o[r][e + 1]));
-            o[r][e] = acc2.x;
-            o[r][e + 1] = acc2.y;
-          }
-        }
-      }
-    } else {
-      float al[kRowsPer];
-#pragma unroll
-      for (int k = 0; k < kRowsPer; ++k) {
-        const int r = og + kGroups * k;
-        al[k] = r < R ? sm.alpha[r] : 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o[k][e] *= al[k];
-      }
-      const int nk = min(kTile, c1 - k0);
-      for (int j = 0; j < nk; ++j) {
-        float vf[8];
-        unpack8(tile_chunk(sm.v[buf], j, oc), bf16, vf);
-#pragma unroll
-        for (int k = 0; k < kRowsPer; ++k) {
-          const int r = og + kGroups * k;
-          if (r < R) {
-            const float pj = sm.sc[r][j];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) o[k][e] = fmaf(pj, vf[e], o[k][e]);
-          }
-        }
-      }
-    }
-    __syncthreads();  // tile buffer and scores free
-  }
-
-  if (t < ntiles) {
-    // aborted: let the copies still in flight (tiles t .. t + kStages - 1) land,
-    // bounded, before the CTA exits
-    if (tid == 0 && !p.stall_loads) {
-      const uint64_t t0 = globaltimer_ns();
-      for (int u = t; u < min(ntiles, t + kStages); ++u)
-        while (!mbar_try_wait(&sm.full[u % kStages], (u / kStages) & 1) &&
-               globaltimer_ns() - t0 < p.timeout_ns) {
-        }
-    }
-    return;
-  }
-
-  // this chunk's partial result per row
-  if constexpr (kKeyGroups) {
-    // sum the key groups through shared memory: the K and V tile buffers (adjacent,
-    // free now) hold [kGroups][RM][D] floats
-    float* red = reinterpret_cast<float*>(&sm.k[0][0][0]);
-    static_assert(sizeof(Sm::k) + sizeof(Sm::v) >= sizeof(float) * kGroups * RM * D,
-                  "reduction space");
-#pragma unroll
-    for (int r = 0; r < RM; ++r)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) red[(og * RM + r) * D + oc * 8 + e] = o[r][e];
-    __syncthreads();
-    for (int x = tid; x < R * D; x += kThr) {
-      const int r = x / D, d = x - (x / D) * D;
-      float sum = 0.f;
-#pragma unroll
-      for (int gk = 0; gk < kGroups; ++gk) sum += red[(gk * RM + r) * D + d];
-      const int g = r / p.L, i = r - g * p.L;
-      const size_t row = static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i;
-      float* rec = p.part + (row * p.nsplit + split) * (D + 2);
-      if (d == 0) {
-        rec[0] = sm.m[r];
-        rec[1] = sm.l[r];
-      }
-      rec[2 + d] = sum;
-    }
-  } else {
-#pragma unroll
-    for (int k = 0; k < kRowsPer; ++k) {
-      const int r = og + kGroups * k;
-      if (r < R) {
-        const int g = r / p.L, i = r - g * p.L;
-        const size_t row = static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i;
-        float* rec = p.part + (row * p.nsplit + split) * (D + 2);
-        if (oc == 0) {
-          rec[0] = sm.m[r];
-          rec[1] = sm.l[r];
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) rec[2 + oc * 8 + e] = o[k][e];
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------- at most 16 rows
-// The common grouped-query decode (R = (H / H_kv) * L <= 16 rows per K/V head) on
+// ---------------------------------------------------------------- chunk kernel
+// Grouped-query decode (R = (H / H_kv) * L <= 32 rows per K/V head, 16 per CTA) on
 // warp-level tensor-core tiles (16 x 8 x 16), with each warp keeping its own online
 // softmax state over its keys, so that a tile needs no barrier across the CTA.
 // Warp w of the 4 compute warps takes keys 16w .. 16w + 15 of every 64-key tile;
-// the rows come in NT = ceil(R / 8) column tiles of 8 (the MMA's N), each sharing
+// the CTA's rows come in NT = 1 or 2 column tiles of 8 (the MMA's N), each sharing
 // the A fragments loaded for the others:
 //   S^T (16 keys x 8 rows) = K_w Q^T      (A = K rows by ldmatrix from the swizzled
 //                                          TMA tile, B = Q^T held in registers for
@@ -426,7 +99,6 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constan
 // fp32.
 constexpr int kMdWarps = 4;                      // compute warps
 constexpr int kMdThreads = (kMdWarps + 1) * 32;  // + the producer warp
-constexpr int kMdRows = 16;                      // rows this kernel takes (NT <= 2)
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -496,9 +168,13 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
   constexpr int kKs = D / 16;  // k-steps of S = 16-dim slices; m-tiles of O^T
   Sm& sm = *reinterpret_cast<Sm*>(smem_raw + ((1024u - (base & 1023u)) & 1023u));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int split = blockIdx.x, bkv = blockIdx.y;
+  // blockIdx.x = chunk * row_tiles + row tile: the CTAs of one chunk's row tiles are
+  // neighbours in launch order, so they read the same K / V tiles at about the same
+  // time and all but the first find them in L2
+  const int split = blockIdx.x / p.row_tiles, bkv = blockIdx.y;
+  const int rbase = (blockIdx.x - split * p.row_tiles) * kRows;  // first row of this CTA
   const int b = bkv / p.Hkv, kvh = bkv - b * p.Hkv;
-  const int R = p.G * p.L;
+  const int R = min(p.G * p.L - rbase, kRows);  // rows of this CTA: rbase .. rbase + R - 1
 
   int k_start = split * p.chunk;
   const int c1 = min(p.S, k_start + p.chunk);
@@ -567,7 +243,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
     for (int nt = 0; nt < NT; ++nt) {
       const int r = 8 * nt + g8;
       const bool live = r < R;
-      const int g = live ? r / p.L : 0, i = live ? r - g * p.L : 0;
+      const int g = live ? (rbase + r) / p.L : 0, i = live ? rbase + r - g * p.L : 0;
       const uint16_t* qrow = p.q + (static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i) * D;
 #pragma unroll
       for (int ks = 0; ks < kKs; ++ks) {
@@ -605,8 +281,8 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int r0 = 8 * nt + n0, r1 = 8 * nt + n1;
-        const int pos0 = p.S - p.L + (r0 < R ? r0 % p.L : 0);
-        const int pos1 = p.S - p.L + (r1 < R ? r1 % p.L : 0);
+        const int pos0 = p.S - p.L + (r0 < R ? (rbase + r0) % p.L : 0);
+        const int pos1 = p.S - p.L + (r1 < R ? (rbase + r1) % p.L : 0);
         float x[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -715,7 +391,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
         acc = fmaf(a, red[(w * kRows + rr) * D + d], acc);
       }
     }
-    const int g = rr / p.L, i = rr - g * p.L;
+    const int g = (rbase + rr) / p.L, i = rbase + rr - g * p.L;
     const size_t row = static_cast<size_t>(b * p.H + kvh * p.G + g) * p.L + i;
     float* rec = p.part + (row * p.nsplit + split) * (D + 2);
     if (d == 0) {
@@ -763,7 +439,8 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
 void decode_plan(int B, int Hkv, int S, int D, int rows, int* nsplit, int* chunk) {
   constexpr int kSms = 148;
   constexpr int kCtaCost = 2;  // prologue and merge record, in tile units
-  const int64_t groups = static_cast<int64_t>(B) * Hkv > 0 ? static_cast<int64_t>(B) * Hkv : 1;
+  const int64_t groups = (static_cast<int64_t>(B) * Hkv > 0 ? static_cast<int64_t>(B) * Hkv : 1) *
+                        dec_row_tiles(rows);
   const int tiles = S > 0 ? (S + kTile - 1) / kTile : 1;
   const int64_t slots = static_cast<int64_t>(kSms) * dec_ctas_per_sm(D, rows);
   int best_tiles = tiles;
@@ -808,41 +485,8 @@ fa_status decode_mma_launch(const void* k, const void* v, int B, int S, const De
       done[dev] = true;
     }
   }
-  const dim3 grid(prm.nsplit, B * prm.Hkv);
+  const dim3 grid(prm.nsplit * prm.row_tiles, B * prm.Hkv);
   decode_mma_kernel<D, BF16, NT><<<grid, kMdThreads, smem, stream>>>(tk, tv, prm);
-  FA_CUDA_CHECK(cudaGetLastError());
-  decode_combine_kernel<D><<<B * prm.H * prm.L, D, 0, stream>>>(prm);
-  FA_CUDA_CHECK(cudaGetLastError());
-  return FA_OK;
-}
-
-template <int D, int RM>
-fa_status decode_launch(const void* k, const void* v, bool bf16, int B, int S, const DecParams& prm,
-                        cudaStream_t stream) {
-  CUtensorMap tk, tv;
-  // With S == 0 no tile is loaded; the maps only need to be well formed.
-  const void* kp = S > 0 ? k : prm.q;
-  const void* vp = S > 0 ? v : prm.q;
-  const int rows = S > 0 ? S : 1, bh = S > 0 ? B * prm.Hkv : 1;
-  if (!make_tile_map(&tk, kp, bf16, D, rows, bh, kTile)) return FA_ERR_CUDA;
-  if (!make_tile_map(&tv, vp, bf16, D, rows, bh, kTile)) return FA_ERR_CUDA;
-  const size_t smem = sizeof(DecSmem<D, RM>) + 1024;
-  int dev = 0;
-  FA_CUDA_CHECK(cudaGetDevice(&dev));
-  {
-    static std::mutex mu;
-    static bool done[kMaxDevices] = {};
-    std::lock_guard<std::mutex> lock(mu);
-    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
-    if (!done[dev]) {
-      FA_CUDA_CHECK(cudaFuncSetAttribute(decode_split_kernel<D, RM>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem)));
-      done[dev] = true;
-    }
-  }
-  const dim3 grid(prm.nsplit, B * prm.Hkv);
-  decode_split_kernel<D, RM><<<grid, DecCfg<D>::kThreads, smem, stream>>>(tk, tv, prm);
   FA_CUDA_CHECK(cudaGetLastError());
   decode_combine_kernel<D><<<B * prm.H * prm.L, D, 0, stream>>>(prm);
   FA_CUDA_CHECK(cudaGetLastError());
@@ -909,6 +553,7 @@ extern "C" fa_status fa_flex_attention_decode(const void* q, const void* k, cons
   prm.L = L;
   prm.S = S;
   decode_plan(B, H_kv, S, D, G * L, &prm.nsplit, &prm.chunk);
+  prm.row_tiles = dec_row_tiles(G * L);
   prm.mask = mask;
   prm.window = mask == FA_DECODE_SLIDING_WINDOW ? window : 0;
   prm.softcap_on = score_kind == FA_SCORE_TANH_SOFTCAP ? 1 : 0;
@@ -922,22 +567,18 @@ extern "C" fa_status fa_flex_attention_decode(const void* q, const void* k, cons
   const cudaStream_t s = as_stream(stream);
   const bool b16 = dtype == FA_BF16;
   const int rows = G * L;
-  // up to 16 rows (one or two of the MMA's 8-row N tiles): the tensor-core chunk
-  // kernel; more: the CUDA-core one
+  // the tensor-core chunk kernel: one 8-row column tile up to 8 rows, else two,
+  // with a CTA per 16 rows beyond 16
   if (D == 64) {
     if (rows <= 8)
       return b16 ? decode_mma_launch<64, true, 1>(k, v, B, S, prm, s)
                  : decode_mma_launch<64, false, 1>(k, v, B, S, prm, s);
-    if (rows <= kMdRows)
-      return b16 ? decode_mma_launch<64, true, 2>(k, v, B, S, prm, s)
-                 : decode_mma_launch<64, false, 2>(k, v, B, S, prm, s);
-    return decode_launch<64, 32>(k, v, b16, B, S, prm, s);
+    return b16 ? decode_mma_launch<64, true, 2>(k, v, B, S, prm, s)
+               : decode_mma_launch<64, false, 2>(k, v, B, S, prm, s);
   }
   if (rows <= 8)
     return b16 ? decode_mma_launch<128, true, 1>(k, v, B, S, prm, s)
                : decode_mma_launch<128, false, 1>(k, v, B, S, prm, s);
-  if (rows <= kMdRows)
-    return b16 ? decode_mma_launch<128, true, 2>(k, v, B, S, prm, s)
-               : decode_mma_launch<128, false, 2>(k, v, B, S, prm, s);
-  return decode_launch<128, 32>(k, v, b16, B, S, prm, s);
+  return b16 ? decode_mma_launch<128, true, 2>(k, v, B, S, prm, s)
+             : decode_mma_launch<128, false, 2>(k, v, B, S, prm, s);
 }

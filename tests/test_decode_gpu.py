@@ -1,4 +1,4 @@
-"""Decode against a KV cache on the GPU (split-KV kernel + merge), against the fp64
+"""Decode against a KV cache on the GPU (split-KV tensor-core kernel + merge), against the fp64
 CPU oracle: the lower-right causal, sliding-window and unmasked cases, grouped
 query heads, softcap, ragged cache lengths, and rows that see no key."""
 import numpy as np
@@ -87,11 +87,14 @@ def test_decode_window_skips_far_chunks_and_matches():
     (1, 8, 1, 2, 3000, 128, 1, 0, torch.bfloat16, 2.0),     # sixteen rows, x2 inputs
     (2, 4, 1, 3, 1700, 64, 2, 350, torch.float16, 1.0),     # twelve rows, window, fp16
     (1, 4, 1, 4, 2, 128, 1, 0, torch.bfloat16, 1.0),        # sixteen rows, L > S
+    (1, 8, 1, 3, 2500, 128, 1, 0, torch.bfloat16, 1.0),     # 24 rows: CTAs of 16 and 8 rows
+    (1, 4, 1, 8, 1800, 64, 2, 300, torch.float16, 1.0),     # 32 rows, window
+    (1, 1, 1, 17, 900, 64, 1, 0, torch.bfloat16, 1.0),      # 17 rows: a CTA with one row
 ])
 def test_decode_tensor_core_path(B, H, Hkv, L, S, D, mask, window, dtype, xs):
-    """At most 16 rows per K/V head take the warp-level tensor-core kernel (one or two
-    8-row column tiles; 16-bit P against each warp's exact running max): element by
-    element against the oracle."""
+    """Every decode runs on the warp-level tensor-core kernel: one or two 8-row column
+    tiles, and a CTA per 16 rows beyond 16 (16-bit P against each warp's exact
+    running max): element by element against the oracle."""
     q, k, v = W.random_qkv(B, H, L, S, D, dtype, seed=B * 1000 + S + L, scale=xs, Hkv=Hkv)
     out, lse = _check(q, k, v, mask, window)
     if L > S:

@@ -133,7 +133,11 @@ DECODE_32K = Workload(name="decode_L1_S32768_B8_H32_Hkv8_D128_bf16", B=8, H=32, 
 DECODE_32K_L4 = Workload(name="decode_L4_S32768_B8_H32_Hkv8_D128_bf16", B=8, H=32, L=4, S=32768,
                          D=128, dtype=torch.bfloat16, mask_kind=MASK_DECODE_CAUSAL, seed=15, Hkv=8)
 
-EXTRA = (BITMAP_8192, GQA_CAUSAL_8192, DECODE_32K, DECODE_32K_L4)
+# 8 new tokens: 32 query rows per K/V head, the most one decode call takes.
+DECODE_32K_L8 = Workload(name="decode_L8_S32768_B8_H32_Hkv8_D128_bf16", B=8, H=32, L=8, S=32768,
+                         D=128, dtype=torch.bfloat16, mask_kind=MASK_DECODE_CAUSAL, seed=16, Hkv=8)
+
+EXTRA = (BITMAP_8192, GQA_CAUSAL_8192, DECODE_32K, DECODE_32K_L4, DECODE_32K_L8)
 BY_NAME = {w.name: w for w in ALL + EXTRA}
 
 
