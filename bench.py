@@ -325,22 +325,26 @@ def run_ours(args, w: W.Workload, rank, world, device):
 def config_sweep(device, steps=10, warmup=3):
     """The forward kernel alone on the other configurations of the benchmark set
     (causal 256, the 8192 sweep, both document workloads, the D = 128 softcap
-    workload): mask built once, `warmup` launches, then `steps` launches each
-    bracketed by CUDA events with a 512 MiB L2 flush between them (untimed).
-    Reported beside the main line so that these figures come from the same run."""
+    workload) and on the workloads of the wider calls (tabulated mask, grouped-query
+    heads; decode, whose call is its whole step): mask built once, `warmup`
+    launches, then `steps` launches each bracketed by CUDA events with a 512 MiB L2
+    flush between them (untimed).  Reported beside the main line so that these
+    figures come from the same run."""
     import block_sparse_attention_create_b200 as fa
     peaks, _ = load_peaks()
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
     res = {}
     for w in (W.C1_CAUSAL_256, W.C2_CAUSAL_8192) + W.C2_WINDOWS + (
-            W.C4_DOC_FIXED, W.C4_DOC_SEEDED, W.C5_SWA1024_SOFTCAP):
+            W.C4_DOC_FIXED, W.C4_DOC_SEEDED, W.C5_SWA1024_SOFTCAP) + W.EXTRA:
         q, k, v = (t.to(device) for t in W.make_qkv(w))
         doc = W.make_doc_id(w)
         dd = doc.to(device) if doc is not None else None
+        words = W.make_bitmap(w)
+        bd = torch.from_numpy(words.view(np.int32)).to(device) if words is not None else None
         out = torch.empty_like(q)
         lse = torch.empty(w.B, w.H, w.L, dtype=torch.float32, device=device)
-        build, attend, dev_error = step_calls(fa, w, q, k, v, dd, None, out, lse, device, stream)
+        build, attend, dev_error = step_calls(fa, w, q, k, v, dd, bd, out, lse, device, stream)
         build()
         for _ in range(warmup):
             attend()
@@ -362,7 +366,7 @@ def config_sweep(device, steps=10, warmup=3):
         tf, hf = tflops / peaks["bf16_tflops"], gbs / peaks["hbm_gbs"]
         res[w.name] = {"fwd_us": round(ms * 1e3, 2), "live_tflops": round(tflops, 1),
                        "bound": "tensor" if tf >= hf else "hbm", "frac": round(max(tf, hf), 4)}
-        del q, k, v, out, lse
+        del q, k, v, out, lse, bd
     return res
 
 
