@@ -52,7 +52,7 @@ extern "C" {
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1,  /* bad pointer, size, enum value or mismatched shapes */
-  FA_ERR_UNSUPPORTED = 2,  /* valid request outside what this build implements (e.g. D=96) */
+  FA_ERR_UNSUPPORTED = 2,  /* valid request outside what this library implements (e.g. D=96) */
   FA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (no device, launch error ...) */
   FA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (reported by
                               fa_get_last_device_error) */
@@ -75,7 +75,7 @@ typedef enum {
 
 typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
 
-/* Block size of the mask tables; the only value this build accepts. */
+/* Block size of the mask tables; the only value this library accepts. */
 #define FA_BLOCK 128
 /* Largest Q_LEN / KV_LEN accepted (8192 blocks of 128). */
 #define FA_MAX_LEN (8192 * 128)
