@@ -53,8 +53,8 @@ DECODE_SOURCES = ("block_sparse_attention_create_b200/csrc/decode.cu",
                   "block_sparse_attention_create_b200/csrc/sm100_ptx.cuh")
 NCU_TRAFFIC = {
     "swa256_L32768_B1_H8_D64_bf16": {
-        "bytes": 101149440 + 7180544, "sources": FWD_SOURCES,
-        "sources_sha256": "5454ccb6e0329a5d1ceaae47f34c47d023e96b0ff524260b3a90862d1c8d2949",
+        "bytes": 101080576 + 7429376, "sources": FWD_SOURCES,
+        "sources_sha256": "0e33e5c29e978af55a7630c50c2c7c1d314fa86b85e0778dde788592b50e0683",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_launches.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
         "bytes": 1073843200 + 3686912, "sources": DECODE_SOURCES,
