@@ -67,6 +67,13 @@ def test_decode_rows_before_the_cache_see_nothing():
     assert torch.all(out[:, :, :3] == 0) and torch.all(torch.isneginf(lse[:, :, :3]))
 
 
+def test_decode_long_cache_32_rows_sampled_heads():
+    """8 new tokens for 32 query heads over 8 K/V heads (32 rows per K/V head, two
+    CTAs per chunk), 32768 cached keys."""
+    q, k, v = W.random_qkv(1, 32, 8, 32768, 128, torch.bfloat16, seed=53, Hkv=8)
+    _check(q, k, v, 1, heads=[(0, 0), (0, 5), (0, 31)])
+
+
 def test_decode_window_skips_far_chunks_and_matches():
     """A small window over a long cache: most chunks load nothing."""
     q, k, v = W.random_qkv(2, 8, 1, 20000, 64, torch.bfloat16, seed=54, Hkv=8)
