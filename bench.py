@@ -57,8 +57,8 @@ NCU_TRAFFIC = {
         "sources_sha256": "0e33e5c29e978af55a7630c50c2c7c1d314fa86b85e0778dde788592b50e0683",
         "summary": "profiles/fwd_kernel_swa256_L32768_B1_H8_D64_launches.md"},
     "decode_L1_S32768_B8_H32_Hkv8_D128_bf16": {
-        "bytes": 1073843200 + 3686912, "sources": DECODE_SOURCES,
-        "sources_sha256": "ac7775954e81c51e6f33526a9d8387a32e00fc345b53f9632b5a6b6914123be1",
+        "bytes": 1073856512 + 3907840, "sources": DECODE_SOURCES,
+        "sources_sha256": "7a50235ad66ea70215c719a32ac78bf42221f867fdc26866fef91ca8c4df4d1a",
         "summary": "profiles/decode_mma_kernel_L1_S32768_B8_H32_Hkv8_D128_full.md"},
 }
 

@@ -190,6 +190,11 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
     fence_barrier_init();
   }
   __syncthreads();
+  // Launched as a programmatic dependent: nothing in global memory is read before
+  // the previous kernel on the stream has finished.  The merge kernel may launch
+  // as soon as every CTA is running (it waits for this grid before reading).
+  grid_dep_wait();
+  grid_dep_launch_dependents();
 
   // this lane's rows in both fragments (8t + 2q, 8t + 2q + 1 of tile t) and its key /
   // dim row (l / 4)
@@ -405,6 +410,7 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant_
 // One CTA per query row, one thread per output column: merge the chunks.
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant__ DecParams p) {
+  grid_dep_wait();  // the chunk kernel's records are complete
   const size_t row = blockIdx.x;
   const int d = threadIdx.x;
   const float* rec0 = p.part + row * p.nsplit * (D + 2);
@@ -486,10 +492,10 @@ fa_status decode_mma_launch(const void* k, const void* v, int B, int S, const De
     }
   }
   const dim3 grid(prm.nsplit * prm.row_tiles, B * prm.Hkv);
-  decode_mma_kernel<D, BF16, NT><<<grid, kMdThreads, smem, stream>>>(tk, tv, prm);
-  FA_CUDA_CHECK(cudaGetLastError());
-  decode_combine_kernel<D><<<B * prm.H * prm.L, D, 0, stream>>>(prm);
-  FA_CUDA_CHECK(cudaGetLastError());
+  FA_CUDA_CHECK(launch_pdl(decode_mma_kernel<D, BF16, NT>, grid, dim3(kMdThreads), smem, stream,
+                           tk, tv, prm));
+  FA_CUDA_CHECK(launch_pdl(decode_combine_kernel<D>, dim3(B * prm.H * prm.L), dim3(D), 0, stream,
+                           prm));
   return FA_OK;
 }
 
