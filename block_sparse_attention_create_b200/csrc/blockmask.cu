@@ -398,6 +398,9 @@ transpose_kernel(int n_q, int n_kv, const int32_t* __restrict__ kv_num,
                  int32_t* __restrict__ q_idx, int32_t* __restrict__ full_q_num,
                  int32_t* __restrict__ full_q_idx) {
   extern __shared__ uint8_t cls[];
+  // programmatic dependent launch: the tables are complete before they are read
+  grid_dep_wait();
+  grid_dep_launch_dependents();
   const int j = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   {  // this instance's tables and column lists
@@ -592,9 +595,9 @@ extern "C" fa_status fa_block_mask_transpose(const fa_block_mask* bm, int32_t* q
       full_q_num_blocks == nullptr || full_q_indices == nullptr)
     return FA_ERR_INVALID_ARG;
   const int inst = (bm->mask_batch > 1 ? bm->mask_batch : 1) * (bm->mask_heads > 1 ? bm->mask_heads : 1);
-  transpose_kernel<<<dim3(nkv, inst), kClassifyThreads, nq, as_stream(stream)>>>(
-      nq, nkv, bm->kv_num_blocks, bm->kv_indices, bm->full_kv_num_blocks, bm->full_kv_indices,
-      q_num_blocks, q_indices, full_q_num_blocks, full_q_indices);
-  FA_CUDA_CHECK(cudaGetLastError());
+  FA_CUDA_CHECK(launch_pdl(transpose_kernel, dim3(nkv, inst), dim3(kClassifyThreads),
+                           static_cast<size_t>(nq), as_stream(stream), nq, nkv, bm->kv_num_blocks,
+                           bm->kv_indices, bm->full_kv_num_blocks, bm->full_kv_indices,
+                           q_num_blocks, q_indices, full_q_num_blocks, full_q_indices));
   return FA_OK;
 }

@@ -79,6 +79,7 @@ struct BwdParams {
   float scale, scale_log2, cap_c, cap_k;
   unsigned long long timeout_ns;
   int stall;  // testing hook: nothing is loaded, the waits run out
+  int dkdv_overlaps_dq;  // dK/dV launched right after dQ (see bwd_tc_kernel)
 };
 
 // delta_i = rowsum(dO_i * O_i) over the B * H * L rows: D / 8 lanes per row, each
@@ -86,6 +87,9 @@ struct BwdParams {
 // partial sums combined by shuffles within the row's lanes; grid-stride over rows.
 template <int D>
 __global__ void __launch_bounds__(kBwdWarps * 32) bwd_delta_kernel(const BwdParams p) {
+  // programmatic dependent launch: O and dO are complete; dQ may start its prologue
+  grid_dep_wait();
+  grid_dep_launch_dependents();
   constexpr int kLanes = D / 8;                // lanes per row
   constexpr int kRowsPerBlock = kBwdWarps * 32 / kLanes;
   const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.L;
@@ -695,6 +699,14 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap ts0, const __grid_constant__ C
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  // Programmatic dependent launch.  dQ waits here for the row sums.  dK/dV launched
+  // right after dQ reads nothing dQ writes, and its inputs (row sums, column lists)
+  // were complete before any dQ CTA could let it launch, so it runs beside dQ's
+  // last CTAs and waits for dQ only before it exits, which keeps the stream's
+  // order; launched after anything else, it waits here.
+  const bool overlap = MODE == kModeDkdv && p.dkdv_overlaps_dq != 0;
+  if (!overlap) grid_dep_wait();
+  grid_dep_launch_dependents();
 
   if (warp < 4) {
     tc_compute_role<MODE, D>(sm, p, tmem, tile_bh, tile_blk);
@@ -709,6 +721,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap ts0, const __grid_constant__ C
     tc_fence_after();
     tmem_dealloc(tmem, kCols);
   }
+  if (overlap) grid_dep_wait();  // dQ has finished before this grid does
 }
 
 template <int MODE, int D>
@@ -744,13 +757,14 @@ fa_status tc_launch(const BwdParams& prm, bool bf16, cudaStream_t s) {
   const int64_t grid = MODE == kModeDkdv ? static_cast<int64_t>(prm.n_kv) * BHkv
                                          : static_cast<int64_t>(prm.n_q) * BH;
   if (grid == 0) return FA_OK;
-  bwd_tc_kernel<MODE, D><<<static_cast<unsigned>(grid), kTcThreads, smem, s>>>(ts0, ts1, tb0, tb1, prm);
-  FA_CUDA_CHECK(cudaGetLastError());
+  FA_CUDA_CHECK(launch_pdl(bwd_tc_kernel<MODE, D>, dim3(static_cast<unsigned>(grid)), dim3(kTcThreads),
+                           smem, s, ts0, ts1, tb0, tb1, prm));
   return FA_OK;
 }
 
 template <int D>
-fa_status bwd_launch(const BwdParams& prm, bool bf16, cudaStream_t s) {
+fa_status bwd_launch(const BwdParams& prm_in, bool bf16, cudaStream_t s) {
+  BwdParams prm = prm_in;
   const int64_t rows = static_cast<int64_t>(prm.B) * prm.H * prm.L;
   const int64_t krows = static_cast<int64_t>(prm.B) * prm.Hkv * prm.S;
   if (rows > 0) {
@@ -760,14 +774,14 @@ fa_status bwd_launch(const BwdParams& prm, bool bf16, cudaStream_t s) {
     const int sms = num_sms_current_device();
     const int64_t cap = static_cast<int64_t>(sms > 0 ? sms : 148) * 8;
     const unsigned qgrid = static_cast<unsigned>(want < cap ? want : cap);
-    bwd_delta_kernel<D><<<qgrid, kBwdWarps * 32, 0, s>>>(prm);
-    FA_CUDA_CHECK(cudaGetLastError());
+    FA_CUDA_CHECK(launch_pdl(bwd_delta_kernel<D>, dim3(qgrid), dim3(kBwdWarps * 32), 0, s, prm));
   }
   if (rows > 0) {
     const fa_status st = tc_launch<kModeDq, D>(prm, bf16, s);
     if (st != FA_OK) return st;
   }
   if (krows > 0) {
+    prm.dkdv_overlaps_dq = rows > 0 ? 1 : 0;  // dQ was launched just before
     const fa_status st = tc_launch<kModeDkdv, D>(prm, bf16, s);
     if (st != FA_OK) return st;
   }
